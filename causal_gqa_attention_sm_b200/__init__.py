@@ -1,0 +1,164 @@
+"""Causal grouped-query attention with RoPE for NVIDIA B200 (sm_100a).
+
+Thin ctypes binding over ``libnea.so`` (C ABI in ``include/nea_attn.h``).
+This module only checks and marshals arguments; every step of the
+computation runs in the library's CUDA kernels.  There is no fallback: if the
+library is missing, importing this package raises.
+
+Tensors are torch CUDA tensors, contiguous, in the library layout:
+``q, o, do, dq: [B, T, Hq, D]``, ``k, v, dk, dv: [B, T, Hkv, D]``,
+``lse: [B, Hq, T]`` (float32); dtype float32 or bfloat16.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "nea_attn_fwd", "nea_attn_bwd", "nea_device_status", "nea_set_wait_limit_ns", "nea_debug_inject",
+    "nea_status_string", "nea_version", "NeaError", "LIB_PATH", "NEA_OK", "NEA_ERR_ARG", "NEA_ERR_CUDA",
+    "NEA_ERR_TIMEOUT", "NEA_ERR_UNSUPPORTED", "NEA_ERR_NOMEM", "NEA_F32", "NEA_BF16",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnea.so")
+
+NEA_F32, NEA_BF16 = 0, 1
+NEA_OK, NEA_ERR_ARG, NEA_ERR_CUDA, NEA_ERR_TIMEOUT, NEA_ERR_UNSUPPORTED, NEA_ERR_NOMEM = range(6)
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libnea.so not built ({LIB_PATH}); run `python -m causal_gqa_attention_sm_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_vp, _i, _f, _ll = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_longlong
+_lib.nea_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp]
+_lib.nea_attn_fwd.restype = _i
+_lib.nea_attn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp]
+_lib.nea_attn_bwd.restype = _i
+_lib.nea_device_status.argtypes = [_vp]
+_lib.nea_device_status.restype = _i
+_lib.nea_set_wait_limit_ns.argtypes = [_ll]
+_lib.nea_set_wait_limit_ns.restype = _ll
+_lib.nea_debug_inject.argtypes = [_i]
+_lib.nea_debug_inject.restype = None
+_lib.nea_status_string.argtypes = [_i]
+_lib.nea_status_string.restype = ctypes.c_char_p
+_lib.nea_version.argtypes = []
+_lib.nea_version.restype = _i
+
+
+class NeaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {nea_status_string(status)}")
+        self.status = status
+
+
+def nea_status_string(status: int) -> str:
+    return _lib.nea_status_string(int(status)).decode()
+
+
+def nea_version() -> int:
+    return int(_lib.nea_version())
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None and t.numel() > 0 else None
+
+
+def _stream(stream):
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t):
+    import torch
+
+    if t.dtype == torch.float32:
+        return NEA_F32
+    if t.dtype == torch.bfloat16:
+        return NEA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; expected float32 or bfloat16")
+
+
+def _check(t, name, shape, dtype, device):
+    if not t.is_cuda or t.device != device:
+        raise ValueError(f"{name} must be a CUDA tensor on {device}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _shapes(q, k, v):
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q, k, v must be [B, T, H, D]")
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    return B, T, Hq, Hkv, D
+
+
+def nea_attn_fwd(q, k, v, rope_base: float = 10000.0, causal: bool = True, o=None, lse=None, stream=None):
+    """Forward: returns ``(o, lse)``.  ``o``/``lse`` may be passed preallocated."""
+    import torch
+
+    B, T, Hq, Hkv, D = _shapes(q, k, v)
+    dev, dt = q.device, q.dtype
+    code = _dtype_code(q)
+    _check(q, "q", (B, T, Hq, D), dt, dev)
+    _check(k, "k", (B, T, Hkv, D), dt, dev)
+    _check(v, "v", (B, T, Hkv, D), dt, dev)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, T), dtype=torch.float32, device=dev)
+    _check(o, "o", (B, T, Hq, D), dt, dev)
+    _check(lse, "lse", (B, Hq, T), torch.float32, dev)
+    rc = _lib.nea_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, T, Hq, Hkv, D, code,
+                           float(rope_base), int(bool(causal)), _stream(stream))
+    if rc != NEA_OK:
+        raise NeaError(rc, "nea_attn_fwd")
+    return o, lse
+
+
+def nea_attn_bwd(q, k, v, o, lse, do, rope_base: float = 10000.0, causal: bool = True,
+                 dq=None, dk=None, dv=None, stream=None):
+    """Backward: returns ``(dq, dk, dv)`` (gradients w.r.t. un-rotated q, k and v)."""
+    import torch
+
+    B, T, Hq, Hkv, D = _shapes(q, k, v)
+    dev, dt = q.device, q.dtype
+    code = _dtype_code(q)
+    _check(q, "q", (B, T, Hq, D), dt, dev)
+    _check(k, "k", (B, T, Hkv, D), dt, dev)
+    _check(v, "v", (B, T, Hkv, D), dt, dev)
+    _check(o, "o", (B, T, Hq, D), dt, dev)
+    _check(do, "do", (B, T, Hq, D), dt, dev)
+    _check(lse, "lse", (B, Hq, T), torch.float32, dev)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check(dq, "dq", (B, T, Hq, D), dt, dev)
+    _check(dk, "dk", (B, T, Hkv, D), dt, dev)
+    _check(dv, "dv", (B, T, Hkv, D), dt, dev)
+    rc = _lib.nea_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
+                           B, T, Hq, Hkv, D, code, float(rope_base), int(bool(causal)), _stream(stream))
+    if rc != NEA_OK:
+        raise NeaError(rc, "nea_attn_bwd")
+    return dq, dk, dv
+
+
+def nea_device_status(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device status."""
+    return int(_lib.nea_device_status(_stream(stream)))
+
+
+def nea_set_wait_limit_ns(ns: int) -> int:
+    return int(_lib.nea_set_wait_limit_ns(int(ns)))
+
+
+def nea_debug_inject(flags: int) -> None:
+    _lib.nea_debug_inject(int(flags))

@@ -1,0 +1,285 @@
+// Device-side building blocks for the sm_100a attention kernels: mbarriers
+// with bounded waits, tensor-memory (TMEM) allocation and access, tcgen05 MMA
+// issue, UMMA shared-memory / instruction descriptors, and the swizzled
+// shared-memory operand layout those descriptors describe.
+//
+// Everything here is written against the public PTX ISA for sm_100a
+// (tcgen05.*, mbarrier.*).  Operand tiles are bf16, one row of a [rows][D]
+// tile per 2*D bytes, stored with the hardware swizzle whose atom width equals
+// the row (128 B for D = 64, 64 B for D = 32); the same bytes serve as a
+// K-major operand (contraction over D) and as an MN-major operand
+// (contraction over rows).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace nea {
+
+constexpr uint32_t kFullMask = 0xffffffffu;
+
+// ------------------------------------------------------------------ status
+// Device error codes written (first writer wins) into the library's error
+// word; the host maps any nonzero value to NEA_ERR_TIMEOUT.
+enum : int {
+  kErrNone = 0,
+  kErrWaitProducer = 0x100,  // a consumer gave up waiting for loaded tiles
+  kErrWaitMma = 0x200,       // a consumer gave up waiting for an MMA commit
+  kErrWaitSoftmax = 0x300,   // the MMA issuer gave up waiting for P / dS
+  kErrWaitEmpty = 0x400,     // the producer gave up waiting for a free stage
+};
+
+struct WaitCtl {
+  int* err;                  // global error word
+  unsigned long long limit;  // per-wait limit, nanoseconds of %globaltimer
+  volatile int* abort;       // shared-memory abort flag of this CTA
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// ------------------------------------------------------------------ mbarrier
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+// Makes barrier initialisation visible to the async proxy (tcgen05.commit).
+__device__ __forceinline__ void mbar_init_fence() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ void raise_error(const WaitCtl& c, int code) {
+  atomicCAS(c.err, 0, code);
+  *c.abort = 1;
+}
+
+// Wait of a single thread for the phase of `bar` with the given parity to
+// complete.  Returns false, after recording `code`, once the CTA aborted or
+// the wait exceeded its limit.
+__device__ __noinline__ bool wait_thread(uint64_t* bar, uint32_t parity, const WaitCtl& c, int code) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*c.abort) return false;
+    if (global_timer_ns() - t0 > c.limit) {
+      raise_error(c, code);
+      return false;
+    }
+  }
+}
+
+// Same wait, taken by all 32 lanes of a warp with a warp-uniform outcome, so
+// that warp-collective tcgen05 loads/stores after it stay converged.  Every
+// lane performs its own successful try_wait (acquire) before proceeding.
+__device__ __noinline__ bool wait_warp(uint64_t* bar, uint32_t parity, const WaitCtl& c, int code) {
+  bool done = mbar_try_wait(bar, parity);
+  if (__all_sync(kFullMask, done)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+    done = done || mbar_try_wait(bar, parity);
+    if (__all_sync(kFullMask, done)) return true;
+    const bool quit = (*c.abort != 0) || (global_timer_ns() - t0 > c.limit);
+    if (__any_sync(kFullMask, quit)) {
+      if ((threadIdx.x & 31) == 0 && *c.abort == 0) raise_error(c, code);
+      __syncwarp();
+      return false;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ proxies
+// Generic-proxy shared-memory writes -> visible to tcgen05.mma operand reads.
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ------------------------------------------------------------------ TMEM
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Arrives on `bar` once every tcgen05 operation this thread issued so far has
+// completed.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+// TMEM address of (lane, column).
+__device__ __forceinline__ uint32_t tmem_addr(uint32_t base, uint32_t lane, uint32_t col) {
+  return base + (lane << 16) + col;
+}
+
+#define NEA_R8(i) "=r"(r[i + 0]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), \
+                  "=r"(r[i + 4]), "=r"(r[i + 5]), "=r"(r[i + 6]), "=r"(r[i + 7])
+#define NEA_W8(i) "r"(r[i + 0]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), \
+                  "r"(r[i + 4]), "r"(r[i + 5]), "r"(r[i + 6]), "r"(r[i + 7])
+
+// Loads 32 consecutive 32-bit columns of this thread's lane (warp-collective,
+// 32x32b shape: lane = warp's quarter base + lane id) and waits for them.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : NEA_R8(0), NEA_R8(8), NEA_R8(16), NEA_R8(24)
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : NEA_R8(0), NEA_R8(8)
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n"
+      ::"r"(taddr), NEA_W8(0), NEA_W8(8), NEA_W8(16), NEA_W8(24)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n"
+      ::"r"(taddr), NEA_W8(0), NEA_W8(8)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+#undef NEA_R8
+#undef NEA_W8
+
+// ------------------------------------------------------------------ UMMA
+// Instruction descriptor, kind::f16 with bf16 A and B, fp32 accumulator.
+// a_mn / b_mn select MN-major (1) instead of K-major (0) operands.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
+  return (1u << 4)                        // D format: f32
+         | (1u << 7)                      // A format: bf16
+         | (1u << 10)                     // B format: bf16
+         | (uint32_t(a_mn) << 15) | (uint32_t(b_mn) << 16) |
+         (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+
+// Shared-memory descriptor of a swizzled operand whose rows are `row_bytes`
+// (64 or 128) wide, i.e. exactly one swizzle atom: 8 rows form an atom of
+// 8*row_bytes bytes.  For a K-major operand the leading offset is unused
+// (encoded 16 B); for an MN-major operand it is the distance between
+// consecutive atom columns along MN, which these tiles never have.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t row_bytes, uint32_t lbo_bytes) {
+  const uint64_t layout = (row_bytes == 128) ? 2ull : 4ull;  // SWIZZLE_128B : SWIZZLE_64B
+  uint64_t d = 0;
+  d |= uint64_t((saddr >> 4) & 0x3FFF);
+  d |= uint64_t((lbo_bytes >> 4) & 0x3FFF) << 16;
+  d |= uint64_t(((8 * row_bytes) >> 4) & 0x3FFF) << 32;  // stride between 8-row groups
+  d |= 1ull << 46;                                        // descriptor version (sm_100)
+  d |= layout << 61;
+  return d;
+}
+
+// D[tmem] (+)= A[smem] * B[smem]
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Byte offset, inside a 1024-aligned tile, of logical offset `off` under the
+// swizzle whose atom row is `row_bytes` wide (XOR of the 16-byte chunk index
+// with the row index inside the atom, as the hardware addresses it).
+__host__ __device__ __forceinline__ uint32_t swizzle(uint32_t off, uint32_t row_bytes) {
+  return row_bytes == 128 ? (off ^ (((off >> 7) & 7u) << 4)) : (off ^ (((off >> 7) & 3u) << 4));
+}
+
+// ------------------------------------------------------------------ numerics
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Packs two floats into bf16x2 (round to nearest even); `lo` in the low half.
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float bf16_lo_f(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi_f(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+// Splits (a, b) into bf16 high parts and bf16 residuals so that
+// a ~= hi.lo + lo.lo and b ~= hi.hi + lo.hi to about 2^-17 relative.
+__device__ __forceinline__ void split_bf16(float a, float b, uint32_t& hi, uint32_t& lo) {
+  hi = pack_bf16(a, b);
+  lo = pack_bf16(a - bf16_lo_f(hi), b - bf16_hi_f(hi));
+}
+
+}  // namespace nea

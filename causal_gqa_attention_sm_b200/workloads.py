@@ -1,0 +1,91 @@
+"""Seeded synthetic inputs shaped like the source pages' models.
+
+Holds no attention arithmetic: only the workload table and a seeded Gaussian
+generator, shared by the tests and the benchmark.  Shapes follow the GPU and
+CPU model configurations of the NanoEuler pages (agentlenshq.com summary,
+model-configuration table: 768-dim / 12 query and 4 key-value heads / context
+512 for the GPU model, 128-dim / 4 and 2 heads / context 128 for the CPU
+model; smartinfralog.com post, config listing and benchmark table: batch 4,
+sequence 1024).  No corpus or checkpoint is used anywhere; activations are
+i.i.d. Gaussians with the stated spreads.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, replace
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    T: int
+    Hq: int
+    Hkv: int
+    D: int
+    dtype: str          # "f32" (float32 storage) or "bf16"
+    qk_std: float = 1.0
+    v_std: float = 1.0
+    do_std: float = 1.0
+    causal: bool = True
+    rope_base: float = 10000.0
+    layers: int = 1     # independent attention layers per step
+    seed: int = 0
+
+    @property
+    def torch_dtype(self):
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+    @property
+    def G(self) -> int:
+        return self.Hq // self.Hkv
+
+    def flops(self) -> float:
+        """Algorithmic FLOPs of one causal fwd+bwd pass: 7 * B * Hq * T^2 * D per
+        layer (forward 2, backward 5; half of the 4/10 of a full square)."""
+        f = 7.0 * self.B * self.Hq * self.T * self.T * self.D
+        if not self.causal:
+            f *= 2.0
+        return f * self.layers
+
+    def tokens(self) -> int:
+        return self.B * self.T * self.layers
+
+
+WORKLOADS = {
+    # small CPU model shape: dim 128, 4/2 heads, context 128
+    "tiny": Workload("tiny", 1, 128, 4, 2, 32, "f32", seed=1000),
+    # GPU model layer: dim 768 = 12 heads x 64, 4 kv heads, context 512; dO ~ N(0, 1e-2)
+    "layer": Workload("layer", 8, 512, 12, 4, 64, "f32", do_std=0.1, seed=2000),
+    # longer context, peaked softmax: Q, K ~ N(0, 3^2)
+    "long": Workload("long", 4, 1024, 12, 4, 64, "f32", qk_std=3.0, seed=3000),
+    # full stack: 16 independent layers of the GPU model shape
+    "stack": Workload("stack", 8, 512, 12, 4, 64, "f32", do_std=0.1, layers=16, seed=4000),
+    # bf16 sweep at B*T = 16384 tokens
+    "sweep512": Workload("sweep512", 32, 512, 12, 4, 64, "bf16", seed=5000),
+    "sweep1024": Workload("sweep1024", 16, 1024, 12, 4, 64, "bf16", seed=5001),
+    "sweep2048": Workload("sweep2048", 8, 2048, 12, 4, 64, "bf16", seed=5002),
+    "sweep4096": Workload("sweep4096", 4, 4096, 12, 4, 64, "bf16", seed=5003),
+}
+
+
+def make_inputs(w: Workload, layer: int = 0, device="cpu"):
+    """Returns ``dict(q, k, v, do)`` for one layer: float32 Gaussians drawn from
+    a CPU generator seeded with ``w.seed + layer``, scaled, then cast to the
+    workload's dtype (the cast values are the exact inputs both sides see)."""
+    g = torch.Generator(device="cpu").manual_seed(int(w.seed) + int(layer))
+    shp_q = (w.B, w.T, w.Hq, w.D)
+    shp_k = (w.B, w.T, w.Hkv, w.D)
+    q = torch.randn(shp_q, generator=g, dtype=torch.float32) * w.qk_std
+    k = torch.randn(shp_k, generator=g, dtype=torch.float32) * w.qk_std
+    v = torch.randn(shp_k, generator=g, dtype=torch.float32) * w.v_std
+    do = torch.randn(shp_q, generator=g, dtype=torch.float32) * w.do_std
+    out = {"q": q, "k": k, "v": v, "do": do}
+    return {n: t.to(w.torch_dtype).to(device).contiguous() for n, t in out.items()}
+
+
+def custom(name="custom", **kw) -> Workload:
+    """A workload with explicit fields (edge-case tests)."""
+    base = Workload(name, 1, 1, 1, 1, 64, "f32")
+    return replace(base, **kw)

@@ -1,0 +1,138 @@
+/*
+ * nea_attn.h -- C ABI of the B200 (sm_100a) causal grouped-query attention
+ * library: forward and backward of softmax attention with rotary position
+ * embeddings on queries and keys.
+ *
+ * Operation (the tiled FlashAttention of a bias-free decoder-only
+ * transformer: "NanoEuler" write-up, aimsg.uk, section 4 "GPU version",
+ * FlashAttention bullet -- tiled, online softmax, the T x T matrix never kept
+ * in memory; section 2 "Model components": RoPE on queries and keys, GQA,
+ * no bias terms; "Tiny Hackable CUDA LM", aimsg.uk, section 1: causal
+ * scaled dot-product attention):
+ *
+ *   q'_t = R_t q_t,  k'_t = R_t k_t   (R_t turns each interleaved pair
+ *                                      (x[2i], x[2i+1]) by t * base^(-2i/D);
+ *                                      t = 0 .. T-1; V is not rotated)
+ *   s_ij = q'_i . k'_j / sqrt(D),     masked for j > i when causal
+ *   LSE_i = ln sum_j exp(s_ij),  P_ij = exp(s_ij - LSE_i),  O_i = sum_j P_ij v_j
+ *
+ * Query head h reads key/value head floor(h / (Hq / Hkv)).
+ *
+ * Layouts (row-major, contiguous, element type given by `dtype`):
+ *   Q, O, dO, dQ : [B][T][Hq][D]
+ *   K, V, dK, dV : [B][T][Hkv][D]
+ *   LSE          : [B][Hq][T], always float32
+ *
+ * Ownership: every pointer is a device pointer owned by the caller; the
+ * library never frees or retains them.  The library keeps, per device, a
+ * cached workspace (the rotary cos/sin table and the backward's row term
+ * D_i = sum_d dO_id O_id), allocated on first use and grown only when a call
+ * needs more; steady-state calls allocate nothing.
+ *
+ * Streams: work is enqueued on `stream` (a cudaStream_t, NULL for the legacy
+ * default stream) and the call returns without synchronising.  Device-side
+ * wait limits are reported asynchronously: see nea_device_status().
+ *
+ * Errors: a call returns NEA_OK or one of the codes below; on NEA_ERR_ARG
+ * nothing is launched and no output is touched.  Kernels never trap.
+ */
+#ifndef NEA_ATTN_H
+#define NEA_ATTN_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element type of Q, K, V, O, dO, dQ, dK, dV. */
+typedef enum {
+  NEA_F32 = 0,  /* float32 storage; contractions in split bf16 (see below) */
+  NEA_BF16 = 1  /* bfloat16 storage; bf16 tensor-core operands, fp32 accumulation */
+} nea_dtype;
+
+enum {
+  NEA_OK = 0,
+  NEA_ERR_ARG = 1,         /* invalid pointer, shape, alignment or dtype */
+  NEA_ERR_CUDA = 2,        /* a CUDA runtime call or kernel launch failed */
+  NEA_ERR_TIMEOUT = 3,     /* a kernel gave up a bounded device-side wait */
+  NEA_ERR_UNSUPPORTED = 4, /* current device is not sm_100 */
+  NEA_ERR_NOMEM = 5        /* workspace allocation failed */
+};
+
+/*
+ * Forward.  Writes O and LSE.
+ *
+ *   Q, K, V     inputs, see layouts above; 16-byte aligned
+ *   O           output, same shape and dtype as Q
+ *   LSE         output, float32 [B][Hq][T], natural-log log-sum-exp of the
+ *               scaled, masked scores of each query row
+ *   B, T        batch and sequence length, >= 0 (B*T == 0 is a no-op)
+ *   Hq, Hkv     query and key/value heads, Hq % Hkv == 0
+ *   D           head dimension, 32 or 64
+ *   dtype       NEA_F32 or NEA_BF16
+ *   rope_base   rotary base (10000 for the workloads here); <= 0 disables
+ *               the rotation
+ *   causal      1: key j visible to query i iff j <= i; 0: all keys visible
+ *   stream      cudaStream_t to enqueue on
+ *
+ * NEA_F32: each score and output contraction is formed from bf16 high and
+ * low parts of its fp32 operands (hi*hi + hi*lo + lo*hi, fp32 accumulation),
+ * about 2^-16 relative per product.  NEA_BF16: plain bf16 products.
+ */
+int nea_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int T, int Hq,
+                 int Hkv, int D, int dtype, float rope_base, int causal, void* stream);
+
+/*
+ * Backward.  Given the forward's inputs, its outputs O and LSE, and the
+ * upstream gradient dO, writes dQ, dK, dV: gradients with respect to the
+ * un-rotated Q and K and to V, with dK and dV summed over the query heads of
+ * each group.  Arguments as for nea_attn_fwd; dQ has the shape of Q, dK and
+ * dV the shape of K.  O and LSE must be the forward's results for the same
+ * Q, K, V, rope_base and causal.
+ *
+ * Runs three kernels on `stream`: the row term D_i = sum_d dO_id O_id, the
+ * dK/dV kernel (one CTA per key tile and kv head, looping over the query
+ * heads of the group), and the dQ kernel (one CTA per query tile and head);
+ * both recompute P from LSE.
+ *
+ * NEA_F32: the score product and dO V^T use split bf16 (as in the forward);
+ * the three gradient products use single bf16 operands with fp32
+ * accumulation.
+ */
+int nea_attn_bwd(const void* Q, const void* K, const void* V, const void* O, const float* LSE, const void* dO,
+                 void* dQ, void* dK, void* dV, int B, int T, int Hq, int Hkv, int D, int dtype, float rope_base,
+                 int causal, void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device error word of the
+ * current device.  Returns NEA_OK, NEA_ERR_TIMEOUT when a kernel since the
+ * last call abandoned a bounded wait (its outputs are then undefined), or
+ * NEA_ERR_CUDA when the synchronisation itself failed.
+ */
+int nea_device_status(void* stream);
+
+/*
+ * Sets the per-wait device limit in nanoseconds for later launches on this
+ * host thread (default 2e9; values < 1e6 are raised to 1e6).  Returns the
+ * previous value.
+ */
+long long nea_set_wait_limit_ns(long long ns);
+
+/*
+ * Fault-injection hook for tests: when `flags` & 1, the next forward launch
+ * on this host thread withholds the query-tile arrival its MMA issuer waits
+ * for, so every dependent wait runs into its limit and the kernel returns
+ * with NEA_ERR_TIMEOUT pending.  Cleared after one launch.
+ */
+void nea_debug_inject(int flags);
+
+/* Human-readable name of a status code (static storage). */
+const char* nea_status_string(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int nea_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NEA_ATTN_H */
