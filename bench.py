@@ -1,0 +1,412 @@
+"""Throughput of causal GQA attention forward+backward on B200.
+
+One step = nea_attn_fwd + nea_attn_bwd (four kernels: forward, row term,
+dK/dV, dQ) over one batch of synthetic inputs already resident in HBM.
+Default workload: B=4, T=1024, Hq=12, Hkv=4, D=64, float32 storage, causal,
+RoPE base 10000, Q,K ~ N(0, 9), V, dO ~ N(0, 1) -- the longer-context
+configuration of the NanoEuler GPU model shape.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload long]
+    python bench.py --impl reference ...   # the fp64 CPU oracle, timed on host cores
+
+Prints one JSON line (rank 0).  value = algorithmic TFLOP/s of the whole job
+(7 * B * Hq * T^2 * D per causal step and layer, summed over ranks, divided by
+the slowest rank's device time of the K timed steps).  L2 is flushed (a 256 MiB
+write) before every timed step, outside the step's events.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "causal GQA attention fwd+bwd TFLOP/s (% of tensor-core peak) and tokens/s"
+KERNELS = ("attn_fwd", "attn_bwd_rowterm", "attn_bwd_dkdv", "attn_bwd_dq")
+# Algorithmic work per kernel in units of B*Hq*T^2*D (causal): the forward's
+# two products; the dK/dV kernel's S, dP, dV, dK products; the dQ kernel's S,
+# dP, dQ products (S and dP are recomputed there, so the two backward kernels
+# together are credited 5 units, the conventional backward count, split 3:2 by
+# their distinct outputs: dK/dV gets dP, dV, dK; dQ gets S and dQ).
+UNITS = {"attn_fwd": 2.0, "attn_bwd_dkdv": 3.0, "attn_bwd_dq": 2.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="long")
+    ap.add_argument("--impl", default="nea", choices=["nea", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    a = ap.parse_args()
+    a.warmup = max(a.warmup, 3)
+    return a
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------- distributed plumbing
+def dist_init(n):
+    if n <= 1 and "WORLD_SIZE" not in os.environ:
+        return 0, 1, 0
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    rank, world = int(os.environ["RANK"]), int(os.environ["WORLD_SIZE"])
+    local = int(os.environ.get("LOCAL_RANK", rank))
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            self.proc.wait(timeout=10)
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+        load = [s for s in sm if s > 0.5 * mx] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows
+                                                         if r[3].replace(".", "").isdigit())}
+
+
+# ---------------------------------------------------------------- ncu traffic records
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "causal_gqa_attention_sm_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, or None when absent
+    or when the kernel sources changed since it was captured."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    if rec.get("source_hash") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------- CPU baseline (oracle)
+def run_oracle_sample(w, max_units=None):
+    """Times the fp64 oracle on (batch, kv-group) slices of the workload (each
+    slice: one batch element, the G query heads of one kv head), all slices in
+    one call so OpenMP spreads them over the host cores.  Returns (seconds,
+    flops, threads, description)."""
+    import numpy as np
+
+    import oracle
+    from causal_gqa_attention_sm_b200.workloads import make_inputs
+
+    cores = len(os.sched_getaffinity(0))
+    units = w.B * w.Hkv
+    n = min(units, max_units or units)
+    inp = make_inputs(w)
+    G = w.G
+    pairs = [(i // w.Hkv, i % w.Hkv) for i in range(n)]
+    arr = {k: v.float().double().numpy() for k, v in inp.items()}
+    qs = np.concatenate([arr["q"][b:b + 1, :, g * G:(g + 1) * G] for b, g in pairs])
+    dos = np.concatenate([arr["do"][b:b + 1, :, g * G:(g + 1) * G] for b, g in pairs])
+    ks = np.concatenate([arr["k"][b:b + 1, :, g:g + 1] for b, g in pairs])
+    vs = np.concatenate([arr["v"][b:b + 1, :, g:g + 1] for b, g in pairs])
+    threads = min(cores, n)
+    oracle.set_threads(threads)
+    t0 = time.perf_counter()
+    oracle.attn_fwd(qs, ks, vs, w.rope_base, w.causal)
+    oracle.attn_bwd(qs, ks, vs, dos, w.rope_base, w.causal)
+    dt = time.perf_counter() - t0
+    flops = w.flops() / w.layers * n / units
+    desc = f"{n} of {units} (batch, kv-group) slices of one layer, fwd+bwd, fp64, {threads} threads"
+    return dt, flops, threads, desc
+
+
+def reference_arm(a, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    for _ in range(a.warmup):
+        pass  # the oracle has no state to warm; each step is a full independent run
+    secs, flops = 0.0, 0.0
+    threads = desc = None
+    per_step_units = max(1, min(w.B * w.Hkv, len(os.sched_getaffinity(0))))
+    for _ in range(a.steps):
+        dt, fl, threads, desc = run_oracle_sample(w, per_step_units)
+        secs += dt
+        flops += fl
+    value = flops / secs / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": a.gpus,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": secs / a.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+                   "storage": w.dtype, "causal": w.causal, "rope_base": w.rope_base, "layers": w.layers},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU arm
+def main():
+    a = parse()
+    from causal_gqa_attention_sm_b200.workloads import WORKLOADS
+
+    w = WORKLOADS[a.workload]
+    if a.impl == "reference":
+        return reference_arm(a, w)
+
+    import torch
+
+    import causal_gqa_attention_sm_b200 as nea
+    from causal_gqa_attention_sm_b200.workloads import make_inputs
+
+    rank, world, local = dist_init(a.gpus)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+
+    # per-rank independent data: each rank processes its own batch (weak scaling)
+    layers = []
+    for layer in range(w.layers):
+        inp = make_inputs(w, layer + 1000 * rank)
+        layers.append({n: t.to(dev) for n, t in inp.items()})
+    outs = []
+    for L in layers:
+        o = torch.empty_like(L["q"])
+        lse = torch.empty((w.B, w.Hq, w.T), dtype=torch.float32, device=dev)
+        outs.append({"o": o, "lse": lse, "dq": torch.empty_like(L["q"]), "dk": torch.empty_like(L["k"]),
+                     "dv": torch.empty_like(L["v"])})
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        for L, O in zip(layers, outs):
+            nea.nea_attn_fwd(L["q"], L["k"], L["v"], w.rope_base, w.causal, o=O["o"], lse=O["lse"])
+            nea.nea_attn_bwd(L["q"], L["k"], L["v"], O["o"], O["lse"], L["do"], w.rope_base, w.causal,
+                             dq=O["dq"], dk=O["dk"], dv=O["dv"])
+
+    for _ in range(a.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize(dev)
+    status = nea.nea_device_status()
+    if status != nea.NEA_OK:
+        raise SystemExit(f"device status after warm-up: {nea.nea_status_string(status)}")
+
+    K = a.steps
+    ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    # per-layer kernel-boundary events of every step (6 per layer)
+    ev_k = [[[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(w.layers)] for _ in range(K)]
+    for evs in ev_k:
+        for row in evs:
+            for e in row:
+                e.record(stream)  # materialise the CUDA events
+    torch.cuda.synchronize(dev)
+
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with clocks:
+        wall0 = time.perf_counter()
+        for i in range(K):
+            flush.fill_(float(i))
+            ev_step[i][0].record(stream)
+            for li, (L, O) in enumerate(zip(layers, outs)):
+                nea.nea_set_profile_events(ev_k[i][li])
+                nea.nea_attn_fwd(L["q"], L["k"], L["v"], w.rope_base, w.causal, o=O["o"], lse=O["lse"])
+                nea.nea_attn_bwd(L["q"], L["k"], L["v"], O["o"], O["lse"], L["do"], w.rope_base, w.causal,
+                                 dq=O["dq"], dk=O["dk"], dv=O["dv"])
+            nea.nea_set_profile_events(None)
+            ev_step[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        wall = time.perf_counter() - wall0
+    barrier(world)
+    status = nea.nea_device_status()
+    if status != nea.NEA_OK:
+        raise SystemExit(f"device status after timing: {nea.nea_status_string(status)}")
+
+    step_ms = [s.elapsed_time(e) for s, e in ev_step]
+    total_ms = max_over_ranks(sum(step_ms), world)
+    kern_ms = {k: 0.0 for k in KERNELS}
+    for i in range(K):
+        for li in range(w.layers):
+            ev = ev_k[i][li]
+            kern_ms["attn_fwd"] += ev[0].elapsed_time(ev[1])
+            kern_ms["attn_bwd_rowterm"] += ev[2].elapsed_time(ev[3])
+            kern_ms["attn_bwd_dkdv"] += ev[3].elapsed_time(ev[4])
+            kern_ms["attn_bwd_dq"] += ev[4].elapsed_time(ev[5])
+    launches_per_kernel = K * w.layers
+
+    flops_step = w.flops()
+    value = flops_step * K * world / (total_ms * 1e-3) / 1e12
+    tokens_s = w.tokens() * K * world / (total_ms * 1e-3)
+
+    # roofline of the dominant kernel
+    pk = peaks()
+    dominant = max(kern_ms, key=kern_ms.get)
+    per_launch_ms = kern_ms[dominant] / launches_per_kernel
+    unit_flops = w.B * w.Hq * w.T * w.T * w.D * (1.0 if w.causal else 2.0)
+    if dominant in UNITS:
+        achieved = UNITS[dominant] * unit_flops / (per_launch_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / pk["bf16_tflops"], "traffic": ncu_traffic(dominant, w.name),
+                "kernel": dominant, "peak_kind": f"bf16 dense burst ({pk['source']})"}
+    else:
+        e = 2 if w.dtype == "bf16" else 4
+        byts = 2 * w.B * w.T * w.Hq * w.D * e + 4 * w.B * w.Hq * w.T
+        achieved = byts / (per_launch_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / pk["hbm_gbs"], "traffic": ncu_traffic(dominant, w.name), "kernel": dominant}
+    kernels = {k: {"ms_per_launch": kern_ms[k] / launches_per_kernel,
+                   "share": kern_ms[k] / max(sum(kern_ms.values()), 1e-12)} for k in KERNELS}
+    for k, u in UNITS.items():
+        kernels[k]["tflops"] = u * unit_flops / (kernels[k]["ms_per_launch"] * 1e-3) / 1e12
+
+    # end to end through the public API with pinned host buffers
+    e2e = None
+    if not a.no_e2e:
+        host_in = [{n: t.cpu().pin_memory() for n, t in L.items()} for L in layers]
+        host_out = [{n: torch.empty(O[n].shape, dtype=O[n].dtype, pin_memory=True) for n in ("o", "dq", "dk", "dv")}
+                    for O in outs]
+        dev_in = [{n: torch.empty_like(t) for n, t in L.items()} for L in layers]
+        h2d = sum(t.numel() * t.element_size() for H in host_in for t in H.values())
+        d2h = sum(t.numel() * t.element_size() for H in host_out for t in H.values())
+
+        def e2e_step():
+            for H, Dv, HO in zip(host_in, dev_in, host_out):
+                for n in Dv:
+                    Dv[n].copy_(H[n], non_blocking=True)
+                o, lse = nea.nea_attn_fwd(Dv["q"], Dv["k"], Dv["v"], w.rope_base, w.causal)
+                dq, dk, dv = nea.nea_attn_bwd(Dv["q"], Dv["k"], Dv["v"], o, lse, Dv["do"], w.rope_base, w.causal)
+                for n, t in (("o", o), ("dq", dq), ("dk", dk), ("dv", dv)):
+                    HO[n].copy_(t, non_blocking=True)
+
+        for _ in range(a.warmup):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(K):
+            e2e_step()
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(s0.elapsed_time(s1), world)
+        e2e = {"value": flops_step * K * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "tokens_per_s": w.tokens() * K * world / (e2e_ms * 1e-3)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        dt, fl, threads, desc = run_oracle_sample(w)
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc,
+               "seconds": dt}
+
+    if rank == 0:
+        storage = {"f32": "float32", "bf16": "bfloat16"}[w.dtype]
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": a.warmup,
+            "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16x3" if w.dtype == "f32" else "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+                       "storage": storage, "causal": w.causal, "rope_base": w.rope_base, "layers": w.layers,
+                       "qk_std": w.qk_std, "l2": "flushed (256 MiB write) before every timed step",
+                       "parallelism": f"dp{world} (independent batches per GPU)"},
+            "tokens_per_s": tokens_s,
+            "frac_of_bf16_peak": value / pk["bf16_tflops"],
+            "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+            "clocks": clocks.summary(), "gpu_launches": 4 * K * w.layers, "wall_s_timed": wall,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

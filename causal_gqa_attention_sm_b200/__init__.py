@@ -16,7 +16,7 @@ import os
 
 __all__ = [
     "nea_attn_fwd", "nea_attn_bwd", "nea_device_status", "nea_set_wait_limit_ns", "nea_debug_inject",
-    "nea_status_string", "nea_version", "NeaError", "LIB_PATH", "NEA_OK", "NEA_ERR_ARG", "NEA_ERR_CUDA",
+    "nea_status_string", "nea_version", "nea_set_profile_events", "NeaError", "LIB_PATH", "NEA_OK", "NEA_ERR_ARG", "NEA_ERR_CUDA",
     "NEA_ERR_TIMEOUT", "NEA_ERR_UNSUPPORTED", "NEA_ERR_NOMEM", "NEA_F32", "NEA_BF16",
 ]
 
@@ -26,7 +26,7 @@ NEA_F32, NEA_BF16 = 0, 1
 NEA_OK, NEA_ERR_ARG, NEA_ERR_CUDA, NEA_ERR_TIMEOUT, NEA_ERR_UNSUPPORTED, NEA_ERR_NOMEM = range(6)
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"libnea.so not built ({LIB_PATH}); run `python -m causal_gqa_attention_sm_b200.build`")
+    raise ImportError(f"libnea.so not built ({LIB_PATH}); run `python causal_gqa_attention_sm_b200/build.py`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 _vp, _i, _f, _ll = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_longlong
@@ -42,6 +42,8 @@ _lib.nea_debug_inject.argtypes = [_i]
 _lib.nea_debug_inject.restype = None
 _lib.nea_status_string.argtypes = [_i]
 _lib.nea_status_string.restype = ctypes.c_char_p
+_lib.nea_set_profile_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), _i]
+_lib.nea_set_profile_events.restype = None
 _lib.nea_version.argtypes = []
 _lib.nea_version.restype = _i
 
@@ -162,3 +164,19 @@ def nea_set_wait_limit_ns(ns: int) -> int:
 
 def nea_debug_inject(flags: int) -> None:
     _lib.nea_debug_inject(int(flags))
+
+
+_prof_keep = None
+
+
+def nea_set_profile_events(events) -> None:
+    """Records the given torch.cuda.Event objects at kernel boundaries of later
+    calls (see include/nea_attn.h); ``None`` disables."""
+    global _prof_keep
+    if not events:
+        _prof_keep = None
+        _lib.nea_set_profile_events(None, 0)
+        return
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _prof_keep = (arr, list(events))
+    _lib.nea_set_profile_events(arr, len(events))

@@ -1,5 +1,7 @@
 """Builds ``libnea.so`` (the sm_100a kernels and their C ABI) in the package
-directory with nvcc.  ``python -m causal_gqa_attention_sm_b200.build``."""
+directory with nvcc: ``python causal_gqa_attention_sm_b200/build.py``.  Run it
+as a script (or load it by path): the package's ``__init__`` needs the built
+library, so this file must not be imported through the package."""
 from __future__ import annotations
 
 import os

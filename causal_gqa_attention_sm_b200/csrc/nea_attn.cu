@@ -21,6 +21,13 @@ constexpr int kVersion = 100;  // 0.1.0
 
 thread_local long long t_wait_limit_ns = 2000000000LL;
 thread_local int t_debug_flags = 0;
+thread_local void* const* t_prof_events = nullptr;
+thread_local int t_prof_n = 0;
+
+void prof_record(int i, cudaStream_t stream) {
+  if (t_prof_events && i < t_prof_n && t_prof_events[i])
+    cudaEventRecord(static_cast<cudaEvent_t>(t_prof_events[i]), stream);
+}
 
 struct DeviceState {
   bool probed = false;
@@ -147,8 +154,10 @@ int launch_fwd(DeviceState& st, const nea::FwdParams& p, cudaStream_t stream) {
   auto kern = nea::attn_fwd_kernel<D, F32IO>;
   int rc = set_smem(st, (D == 64) * 2 + F32IO, kern, L::kAlloc);
   if (rc) return rc;
+  prof_record(0, stream);
   kern<<<p.B * p.Hq * p.n_tiles, 288, L::kAlloc, stream>>>(p);
   cudaError_t e = cudaGetLastError();
+  prof_record(1, stream);
   return e == cudaSuccess ? NEA_OK : cuda_fail(e);
 }
 
@@ -157,10 +166,12 @@ int launch_bwd(DeviceState& st, const nea::BwdParams& p, const void* O, cudaStre
   const int rows = p.B * p.T * p.Hq;
   constexpr int kLanes = D / (F32IO ? 4 : 8);
   const long long threads = static_cast<long long>(rows) * kLanes;
+  prof_record(2, stream);
   nea::attn_bwd_rowterm_kernel<D, F32IO>
       <<<unsigned((threads + 255) / 256), 256, 0, stream>>>(O, p.dO, const_cast<float*>(p.Dv), rows, p.T, p.Hq);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
+  prof_record(3, stream);
 
   using LK = nea::BwdSmem<D, F32IO, true>;
   auto kk = nea::attn_bwd_kernel<D, F32IO, true>;
@@ -168,6 +179,7 @@ int launch_bwd(DeviceState& st, const nea::BwdParams& p, const void* O, cudaStre
   if (rc) return rc;
   kk<<<p.B * p.Hkv * p.n_tiles, 288, LK::kAlloc, stream>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+  prof_record(4, stream);
 
   using LQ = nea::BwdSmem<D, F32IO, false>;
   auto kq = nea::attn_bwd_kernel<D, F32IO, false>;
@@ -175,6 +187,7 @@ int launch_bwd(DeviceState& st, const nea::BwdParams& p, const void* O, cudaStre
   if (rc) return rc;
   kq<<<p.B * p.Hq * p.n_tiles, 288, LQ::kAlloc, stream>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+  prof_record(5, stream);
   return NEA_OK;
 }
 
@@ -286,6 +299,11 @@ long long nea_set_wait_limit_ns(long long ns) {
 }
 
 void nea_debug_inject(int flags) { t_debug_flags = flags; }
+
+void nea_set_profile_events(void* const* events, int n) {
+  t_prof_events = (events && n > 0) ? events : nullptr;
+  t_prof_n = t_prof_events ? n : 0;
+}
 
 const char* nea_status_string(int status) {
   switch (status) {

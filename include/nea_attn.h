@@ -125,6 +125,17 @@ long long nea_set_wait_limit_ns(long long ns);
  */
 void nea_debug_inject(int flags);
 
+/*
+ * Profiling hook.  `events` points at `n` cudaEvent_t handles owned by the
+ * caller (NULL / 0 disables).  While set, later calls on this host thread
+ * record them on their stream at kernel boundaries:
+ *   nea_attn_fwd: events[0] before, events[1] after the forward kernel;
+ *   nea_attn_bwd: events[2] before the row-term kernel, events[3] after it,
+ *                 events[4] after the dK/dV kernel, events[5] after the dQ kernel.
+ * Indices >= n are skipped.  The array must stay valid while set.
+ */
+void nea_set_profile_events(void* const* events, int n);
+
 /* Human-readable name of a status code (static storage). */
 const char* nea_status_string(int status);
 

@@ -14,9 +14,9 @@ LIB = os.path.join(ROOT, "causal_gqa_attention_sm_b200", "libnea.so")
 
 @pytest.fixture(scope="module")
 def lib():
-    from causal_gqa_attention_sm_b200 import build
+    import __graft_entry__
 
-    build.build()
+    __graft_entry__.build()
     return ctypes.CDLL(LIB)
 
 
