@@ -85,13 +85,21 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(x, world):
+def batch_shard(B, world, rank):
+    """Rows [lo, hi) of a batch of B that `rank` owns: contiguous, sizes differ
+    by at most one.  Batches are independent, so shards exchange nothing."""
+    base, extra = divmod(B, world)
+    lo = rank * base + min(rank, extra)
+    return lo, lo + base + (1 if rank < extra else 0)
+
+
+def max_over_ranks(x, world, device="cuda"):
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
