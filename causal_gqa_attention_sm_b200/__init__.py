@@ -17,13 +17,14 @@ import os
 __all__ = [
     "nea_attn_fwd", "nea_attn_bwd", "nea_device_status", "nea_set_wait_limit_ns", "nea_debug_inject",
     "nea_status_string", "nea_version", "nea_set_profile_events", "NeaError", "LIB_PATH", "NEA_OK", "NEA_ERR_ARG", "NEA_ERR_CUDA",
-    "NEA_ERR_TIMEOUT", "NEA_ERR_UNSUPPORTED", "NEA_ERR_NOMEM", "NEA_F32", "NEA_BF16",
+    "NEA_ERR_TIMEOUT", "NEA_ERR_UNSUPPORTED", "NEA_ERR_NOMEM", "NEA_ERR_SCRATCH_LIMIT", "NEA_F32", "NEA_BF16",
+    "nea_attn_bwd_noalloc",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnea.so")
 
 NEA_F32, NEA_BF16 = 0, 1
-NEA_OK, NEA_ERR_ARG, NEA_ERR_CUDA, NEA_ERR_TIMEOUT, NEA_ERR_UNSUPPORTED, NEA_ERR_NOMEM = range(6)
+NEA_OK, NEA_ERR_ARG, NEA_ERR_CUDA, NEA_ERR_TIMEOUT, NEA_ERR_UNSUPPORTED, NEA_ERR_NOMEM, NEA_ERR_SCRATCH_LIMIT = range(7)
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"libnea.so not built ({LIB_PATH}); run `python causal_gqa_attention_sm_b200/build.py`")
@@ -44,6 +45,8 @@ _lib.nea_status_string.argtypes = [_i]
 _lib.nea_status_string.restype = ctypes.c_char_p
 _lib.nea_set_profile_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), _i]
 _lib.nea_set_profile_events.restype = None
+_lib.nea_attn_bwd_noalloc.argtypes = list(_lib.nea_attn_bwd.argtypes)
+_lib.nea_attn_bwd_noalloc.restype = _i
 _lib.nea_version.argtypes = []
 _lib.nea_version.restype = _i
 
@@ -150,6 +153,30 @@ def nea_attn_bwd(q, k, v, o, lse, do, rope_base: float = 10000.0, causal: bool =
                            B, T, Hq, Hkv, D, code, float(rope_base), int(bool(causal)), _stream(stream))
     if rc != NEA_OK:
         raise NeaError(rc, "nea_attn_bwd")
+    return dq, dk, dv
+
+
+def nea_attn_bwd_noalloc(q, k, v, o, lse, do, dq, dk, dv, rope_base: float = 10000.0, causal: bool = True,
+                         stream=None):
+    """Backward that allocates no device memory (for callers that may not call
+    cudaMalloc): the outputs ``dq, dk, dv`` must be passed preallocated; the
+    scratch is a fixed 4 MiB array inside the library (see include/nea_attn.h
+    for its limit and the rule that concurrent calls must be serialised)."""
+    import torch
+
+    B, T, Hq, Hkv, D = _shapes(q, k, v)
+    dev, dt = q.device, q.dtype
+    code = _dtype_code(q)
+    for t, n, shp in ((q, "q", (B, T, Hq, D)), (k, "k", (B, T, Hkv, D)), (v, "v", (B, T, Hkv, D)),
+                      (o, "o", (B, T, Hq, D)), (do, "do", (B, T, Hq, D)), (dq, "dq", (B, T, Hq, D)),
+                      (dk, "dk", (B, T, Hkv, D)), (dv, "dv", (B, T, Hkv, D))):
+        _check(t, n, shp, dt, dev)
+    _check(lse, "lse", (B, Hq, T), torch.float32, dev)
+    rc = _lib.nea_attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk),
+                                   _ptr(dv), B, T, Hq, Hkv, D, code, float(rope_base), int(bool(causal)),
+                                   _stream(stream))
+    if rc != NEA_OK:
+        raise NeaError(rc, "nea_attn_bwd_noalloc")
     return dq, dk, dv
 
 

@@ -313,6 +313,8 @@ const char* nea_status_string(int status) {
     case NEA_ERR_TIMEOUT: return "NEA_ERR_TIMEOUT: a kernel abandoned a bounded device-side wait";
     case NEA_ERR_UNSUPPORTED: return "NEA_ERR_UNSUPPORTED: current device is not sm_100";
     case NEA_ERR_NOMEM: return "NEA_ERR_NOMEM: workspace allocation failed";
+    case NEA_ERR_SCRATCH_LIMIT:
+      return "NEA_ERR_SCRATCH_LIMIT: problem exceeds the fixed scratch of nea_attn_bwd_noalloc";
     default: return "unknown status";
   }
 }
@@ -320,3 +322,154 @@ const char* nea_status_string(int status) {
 int nea_version(void) { return kVersion; }
 
 }  // extern "C"
+
+// ===================================================================== no-allocation backward
+// A second way into the same backward kernels for callers that may not
+// allocate device memory.  Its scratch is this fixed array instead of the
+// per-device workspace above; nothing here calls cudaMalloc/cudaFree.
+namespace {
+
+constexpr size_t kNoAllocScratchFloats = size_t(1) << 20;  // 4 MiB
+constexpr size_t kNoAllocStatusFloats = 64;                 // status word, padded to 256 bytes
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
+
+// Host-side state per device: the array's device address (the host-side name
+// `g_noalloc_scratch` is only a stand-in and must never reach a kernel) and
+// which kernel attributes are set.  Fixed-size, so no host allocation either.
+struct NoAllocDevice {
+  bool ready = false;
+  bool sm100 = false;
+  float* scratch = nullptr;
+  uint32_t attr_done = 0;
+};
+NoAllocDevice g_noalloc_dev[kNoAllocMaxDevices];
+std::mutex g_noalloc_mu;
+
+// Rotary table [T][D/2] of (cos, sin) of t * base^(-2i/D), angles in double.
+__global__ void noalloc_rope_table_kernel(float2* out, int T, int D, double base) {
+  const long idx = long(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int half = D / 2;
+  if (idx >= long(T) * half) return;
+  const int t = int(idx / half), i = int(idx % half);
+  const double a = double(t) * pow(base, -2.0 * double(i) / double(D));
+  double sn, cs;
+  sincos(a, &sn, &cs);
+  out[idx] = make_float2(float(cs), float(sn));
+}
+
+size_t round4(size_t n) { return (n + 3) & ~size_t(3); }
+
+template <typename Kern>
+int noalloc_smem(NoAllocDevice& st, int bit, Kern kern, uint32_t bytes) {
+  if (st.attr_done & (1u << bit)) return NEA_OK;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes));
+  if (e != cudaSuccess) return cuda_fail(e);
+  st.attr_done |= 1u << bit;
+  return NEA_OK;
+}
+
+template <int D, bool F32IO>
+int noalloc_launch(NoAllocDevice& st, const nea::BwdParams& p, const void* O, cudaStream_t stream) {
+  const int rows = p.B * p.T * p.Hq;
+  constexpr int kLanes = D / (F32IO ? 4 : 8);
+  const long long threads = static_cast<long long>(rows) * kLanes;
+  nea::attn_bwd_rowterm_kernel<D, F32IO>
+      <<<unsigned((threads + 255) / 256), 256, 0, stream>>>(O, p.dO, const_cast<float*>(p.Dv), rows, p.T, p.Hq);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  using LK = nea::BwdSmem<D, F32IO, true>;
+  auto kk = nea::attn_bwd_kernel<D, F32IO, true>;
+  int rc = noalloc_smem(st, (D == 64) * 2 + F32IO, kk, LK::kAlloc);
+  if (rc) return rc;
+  kk<<<p.B * p.Hkv * p.n_tiles, 288, LK::kAlloc, stream>>>(p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+  using LQ = nea::BwdSmem<D, F32IO, false>;
+  auto kq = nea::attn_bwd_kernel<D, F32IO, false>;
+  rc = noalloc_smem(st, 4 + (D == 64) * 2 + F32IO, kq, LQ::kAlloc);
+  if (rc) return rc;
+  kq<<<p.B * p.Hq * p.n_tiles, 288, LQ::kAlloc, stream>>>(p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+  return NEA_OK;
+}
+
+}  // namespace
+
+extern "C" int nea_attn_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O, const float* LSE,
+                                    const void* dO, void* dQ, void* dK, void* dV, int B, int T, int Hq, int Hkv,
+                                    int D, int dtype, float rope_base, int causal, void* stream_) {
+  bool empty = false;
+  int rc = check_shape(B, T, Hq, Hkv, D, dtype, causal, &empty);
+  if (rc) return rc;
+  if (empty) return NEA_OK;
+  if (!Q || !K || !V || !O || !LSE || !dO || !dQ || !dK || !dV) return NEA_ERR_ARG;
+  for (const void* ptr : {Q, K, V, O, static_cast<const void*>(LSE), dO, static_cast<const void*>(dQ),
+                          static_cast<const void*>(dK), static_cast<const void*>(dV)})
+    if (!aligned16(ptr)) return NEA_ERR_ARG;
+  if (!std::isfinite(rope_base)) return NEA_ERR_ARG;
+  const size_t dv_floats = round4(size_t(B) * Hq * T);
+  const size_t rope_floats = (rope_base > 0.f) ? round4(size_t(T) * D) : 0;
+  if (kNoAllocStatusFloats + dv_floats + rope_floats > kNoAllocScratchFloats) return NEA_ERR_SCRATCH_LIMIT;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return NEA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  NoAllocDevice& st = g_noalloc_dev[dev];
+  if (!st.ready) {
+    // one-time set-up on this device (it is current): resolve the array's
+    // device address; the symbol itself is only a host-side placeholder
+    int major = 0, minor = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+      return cuda_fail(e);
+    st.sm100 = (major == 10 && minor == 0);
+    if (st.sm100) {
+      void* ptr = nullptr;
+      if ((e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch)) != cudaSuccess) return cuda_fail(e);
+      st.scratch = static_cast<float*>(ptr);
+    }
+    st.ready = true;
+  }
+  if (!st.sm100) return NEA_ERR_UNSUPPORTED;
+
+  int* status = reinterpret_cast<int*>(st.scratch);
+  float* dv = st.scratch + kNoAllocStatusFloats;
+  float2* rope = rope_floats ? reinterpret_cast<float2*>(dv + dv_floats) : nullptr;
+  // the status word must start at zero; Dv is fully rewritten by the row-term
+  // kernel and the table by its own kernel, so neither needs clearing
+  if ((e = cudaMemsetAsync(status, 0, sizeof(int), stream)) != cudaSuccess) return cuda_fail(e);
+  if (rope) {
+    const long n = long(T) * (D / 2);
+    noalloc_rope_table_kernel<<<unsigned((n + 255) / 256), 256, 0, stream>>>(rope, T, D, double(rope_base));
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+  }
+  nea::BwdParams p{};
+  p.Q = Q;
+  p.K = K;
+  p.V = V;
+  p.dO = dO;
+  p.LSE = LSE;
+  p.Dv = dv;
+  p.dQ = dQ;
+  p.dK = dK;
+  p.dV = dV;
+  p.rope = rope;
+  p.B = B;
+  p.T = T;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.n_tiles = (T + 127) / 128;
+  p.causal = causal;
+  p.scale = float(1.0 / std::sqrt(double(D)));
+  p.scale_log2 = float(1.4426950408889634 / std::sqrt(double(D)));
+  p.err = status;
+  p.wait_limit = static_cast<unsigned long long>(t_wait_limit_ns);
+  const bool f32 = dtype == NEA_F32;
+  if (D == 64) return f32 ? noalloc_launch<64, true>(st, p, O, stream) : noalloc_launch<64, false>(st, p, O, stream);
+  return f32 ? noalloc_launch<32, true>(st, p, O, stream) : noalloc_launch<32, false>(st, p, O, stream);
+}

@@ -55,7 +55,8 @@ enum {
   NEA_ERR_CUDA = 2,        /* a CUDA runtime call or kernel launch failed */
   NEA_ERR_TIMEOUT = 3,     /* a kernel gave up a bounded device-side wait */
   NEA_ERR_UNSUPPORTED = 4, /* current device is not sm_100 */
-  NEA_ERR_NOMEM = 5        /* workspace allocation failed */
+  NEA_ERR_NOMEM = 5,       /* workspace allocation failed */
+  NEA_ERR_SCRATCH_LIMIT = 6 /* problem too large for nea_attn_bwd_noalloc's fixed scratch */
 };
 
 /*
@@ -135,6 +136,37 @@ void nea_debug_inject(int flags);
  * Indices >= n are skipped.  The array must stay valid while set.
  */
 void nea_set_profile_events(void* const* events, int n);
+
+/*
+ * Backward without any device allocation.  The source pages have no
+ * counterpart; this entry point exists for callers that must not call
+ * cudaMalloc or cudaFree themselves or through a library -- code that runs
+ * under a host-side memory manager that owns every device buffer (custom
+ * allocators, pre-planned arenas, some embedded or real-time hosts), or code
+ * whose allocations would synchronise or fragment the device at a bad time.
+ *
+ * Same arguments, layouts and results as nea_attn_bwd.  The caller passes all
+ * inputs and outputs; everything else the backward needs (the row term
+ * D_i = sum_d dO_id O_id, the rotary cos/sin table, computed on the device in
+ * double precision, and a device status word) lives in one fixed array of
+ * 4 MiB (1048576 floats) compiled into the library: every GPU that loads the
+ * library keeps it until the process exits.  A call needs
+ * 64 + B*Hq*T + T*D floats of it (rounded up to multiples of 4); larger
+ * problems return NEA_ERR_SCRATCH_LIMIT before anything is launched.
+ *
+ * The first call on a device does a one-time set-up with that device
+ * current (it looks up the array's device address and sets kernel
+ * attributes); make that first call before any stream capture.  All calls
+ * share the one array and it keeps the last call's contents, so calls whose
+ * work may overlap on the GPU (different streams without ordering, or
+ * several host threads) race and must be serialised by the caller.  Each
+ * call clears the status word it uses; a device-side wait that runs into its
+ * limit is recorded only there (outputs are then undefined) and is not
+ * reported by nea_device_status.
+ */
+int nea_attn_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O, const float* LSE,
+                         const void* dO, void* dQ, void* dK, void* dV, int B, int T, int Hq, int Hkv, int D,
+                         int dtype, float rope_base, int causal, void* stream);
 
 /* Human-readable name of a status code (static storage). */
 const char* nea_status_string(int status);
