@@ -1,28 +1,40 @@
 // C ABI of the attention library: argument checks, the per-device workspace
-// (rotary table, backward row term, device error word) and kernel launches.
-// Declarations and contracts: include/nea_attn.h.
+// (rotary table, backward row terms, fp32 operand planes, device error word),
+// TMA descriptors and kernel launches.  Declarations and contracts:
+// include/nea_attn.h.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <map>
 #include <mutex>
 #include <tuple>
+#include <type_traits>
 #include <vector>
 
 #include "nea_attn.h"
 #include "nea_bwd.cuh"
 #include "nea_fwd.cuh"
+#include "nea_prep.cuh"
 
 namespace {
 
-constexpr int kVersion = 100;  // 0.1.0
+constexpr int kVersion = 300;  // 0.3.0
 
 thread_local long long t_wait_limit_ns = 2000000000LL;
 thread_local int t_debug_flags = 0;
 thread_local void* const* t_prof_events = nullptr;
 thread_local int t_prof_n = 0;
+
+#ifdef NEA_TRACE
+// Performance-analysis builds only: destination of the forward kernel's phase
+// stamps (80 per CTA), set through nea_debug_set_trace.
+thread_local unsigned long long* t_trace = nullptr;
+#endif
 
 void prof_record(int i, cudaStream_t stream) {
   if (t_prof_events && i < t_prof_n && t_prof_events[i])
@@ -33,8 +45,8 @@ struct DeviceState {
   bool probed = false;
   bool sm100 = false;
   int* err = nullptr;          // device error word
-  float* dvec = nullptr;       // backward row term [B][Hq][T]
-  size_t dvec_elems = 0;
+  uint8_t* ws = nullptr;       // row terms and fp32 operand planes of the current call
+  size_t ws_bytes = 0;
   // rotary tables keyed by (T, D, base bits); never freed while the process
   // runs, so in-flight kernels on any stream keep valid pointers
   std::map<std::tuple<int, int, uint32_t>, float2*> rope;
@@ -47,6 +59,57 @@ std::map<int, DeviceState> g_dev;
 int cuda_fail(cudaError_t e) {
   (void)cudaGetLastError();
   return e == cudaErrorMemoryAllocation ? NEA_ERR_NOMEM : NEA_ERR_CUDA;
+}
+
+size_t round_up(size_t n, size_t a) { return (n + a - 1) / a * a; }
+
+// ----------------------------------------------------------------- TMA descriptors
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    (void)cudaGetLastError();
+  });
+  return fn;
+}
+
+// Descriptor of a [B][T][H][D] tensor read as 128-row tiles of one head:
+// dimensions (innermost first) {D, H, T, B}, box {D, 1, 128, 1}; rows past T
+// read as zero.  bf16 tiles land in the operand swizzle (row = atom).
+int make_tile_map(CUtensorMap* m, const void* base, int B, int T, int H, int D) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return NEA_ERR_CUDA;
+  const cuuint64_t e = 2;
+  const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(H), cuuint64_t(T), cuuint64_t(B)};
+  const cuuint64_t strides[3] = {D * e, cuuint64_t(H) * D * e, cuuint64_t(T) * H * D * e};
+  const cuuint32_t box[4] = {cuuint32_t(D), 1, cuuint32_t(nea::kTileRows), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUtensorMapSwizzle sw = D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? NEA_OK : NEA_ERR_CUDA;
+}
+
+// Descriptor of the backward row terms ws[B*Hq][2][Tp], box {128, 2, 1}:
+// one box is a column tile's LSE*log2e followed by its Dv.
+int make_rowterm_map(CUtensorMap* m, const float* base, int BH, int Tp) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return NEA_ERR_CUDA;
+  const cuuint64_t dims[3] = {cuuint64_t(Tp), 2, cuuint64_t(BH)};
+  const cuuint64_t strides[2] = {cuuint64_t(Tp) * 4, cuuint64_t(Tp) * 8};
+  const cuuint32_t box[3] = {cuuint32_t(nea::kTileRows), 2, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? NEA_OK : NEA_ERR_CUDA;
 }
 
 // Returns the state of the current device, probing it once.
@@ -72,7 +135,13 @@ int device_state(DeviceState** out) {
   return NEA_OK;
 }
 
-// Rotary table [T][D/2] of (cos, sin) of t * base^(-2i/D), computed in double.
+// Rows of the rotary table: T positions, then two block-start rows per tile.
+size_t rope_rows(int T) { return size_t(T) + 2 * ((size_t(T) + nea::kTileRows - 1) / nea::kTileRows); }
+
+// Rotary table [T][D/2] of (cos, sin) of t * base^(-2i/D), computed in double,
+// followed by, per 128-row tile j, the rows of its two 64-row block starts
+// (j*128 and j*128+64, clamped to T-1), contiguous so a kernel can bulk-copy
+// a tile's bases in one piece.
 int rope_table(DeviceState& st, int T, int D, float base, cudaStream_t stream, const float2** out) {
   if (!(base > 0.f)) {
     *out = nullptr;
@@ -86,12 +155,16 @@ int rope_table(DeviceState& st, int T, int D, float base, cudaStream_t stream, c
     *out = it->second;
     return NEA_OK;
   }
-  std::vector<float2> h(size_t(T) * (D / 2));
+  std::vector<float2> h(rope_rows(T) * (D / 2));
   for (int t = 0; t < T; ++t)
     for (int i = 0; i < D / 2; ++i) {
       const double a = double(t) * std::pow(double(base), -2.0 * i / double(D));
       h[size_t(t) * (D / 2) + i] = make_float2(float(std::cos(a)), float(std::sin(a)));
     }
+  for (size_t r = 0; r + T < rope_rows(T); ++r) {
+    const int t = std::min(int(r) * nea::kRopeRows, T - 1);
+    std::memcpy(&h[(T + r) * (D / 2)], &h[size_t(t) * (D / 2)], sizeof(float2) * (D / 2));
+  }
   float2* d = nullptr;
   cudaError_t e = cudaMalloc(&d, h.size() * sizeof(float2));
   if (e != cudaSuccess) return cuda_fail(e);
@@ -106,25 +179,24 @@ int rope_table(DeviceState& st, int T, int D, float base, cudaStream_t stream, c
   return NEA_OK;
 }
 
-int ensure_dvec(DeviceState& st, size_t elems, cudaStream_t stream) {
-  if (elems <= st.dvec_elems) return NEA_OK;
+int ensure_ws(DeviceState& st, size_t bytes) {
+  if (bytes <= st.ws_bytes) return NEA_OK;
   cudaError_t e;
-  if (st.dvec) {
+  if (st.ws) {
     // kernels on any stream may still read the old buffer
     if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cuda_fail(e);
-    cudaFree(st.dvec);
-    st.dvec = nullptr;
-    st.dvec_elems = 0;
+    cudaFree(st.ws);
+    st.ws = nullptr;
+    st.ws_bytes = 0;
   }
-  (void)stream;
-  if ((e = cudaMalloc(&st.dvec, elems * sizeof(float))) != cudaSuccess) return cuda_fail(e);
-  st.dvec_elems = elems;
+  if ((e = cudaMalloc(&st.ws, bytes)) != cudaSuccess) return cuda_fail(e);
+  st.ws_bytes = bytes;
   return NEA_OK;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Shape/dtype checks shared by both entry points.  `empty` is set when
+// Shape/dtype checks shared by the entry points.  `empty` is set when
 // B*T == 0 (nothing to do, pointers may be null).
 int check_shape(int B, int T, int Hq, int Hkv, int D, int dtype, int causal, bool* empty) {
   if (B < 0 || T < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return NEA_ERR_ARG;
@@ -134,61 +206,193 @@ int check_shape(int B, int T, int Hq, int Hkv, int D, int dtype, int causal, boo
   // 32-bit grid and tile indices: keep every launch well inside them
   const long long tiles = (static_cast<long long>(T) + 127) / 128;
   if (tiles * B * Hq > (1LL << 30) || static_cast<long long>(T) > (1LL << 24)) return NEA_ERR_ARG;
-  if (static_cast<long long>(B) * T * Hq > (1LL << 30)) return NEA_ERR_ARG;
+  if (static_cast<long long>(B) * (tiles * 128) * Hq > (1LL << 30)) return NEA_ERR_ARG;
   *empty = (static_cast<long long>(B) * T == 0);
   return NEA_OK;
 }
 
 template <typename Kern>
-int set_smem(DeviceState& st, int bit, Kern kern, uint32_t bytes) {
-  if (st.attr_done & (1u << bit)) return NEA_OK;
+int set_smem(uint32_t& attr_done, int bit, Kern kern, uint32_t bytes) {
+  if (attr_done & (1u << bit)) return NEA_OK;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes));
   if (e != cudaSuccess) return cuda_fail(e);
-  st.attr_done |= 1u << bit;
+  attr_done |= 1u << bit;
   return NEA_OK;
 }
 
-template <int D, bool F32IO>
-int launch_fwd(DeviceState& st, const nea::FwdParams& p, cudaStream_t stream) {
-  using L = nea::FwdSmem<D, F32IO>;
-  auto kern = nea::attn_fwd_kernel<D, F32IO>;
-  int rc = set_smem(st, (D == 64) * 2 + F32IO, kern, L::kAlloc);
-  if (rc) return rc;
-  prof_record(0, stream);
-  kern<<<p.B * p.Hq * p.n_tiles, 288, L::kAlloc, stream>>>(p);
-  cudaError_t e = cudaGetLastError();
-  prof_record(1, stream);
+// Calls f(std::integral_constant<int, D>, std::bool_constant<F32IO>).
+template <typename F>
+int dispatch(int D, int dtype, F&& f) {
+  const bool f32 = dtype == NEA_F32;
+  if (D == 64)
+    return f32 ? f(std::integral_constant<int, 64>{}, std::true_type{})
+               : f(std::integral_constant<int, 64>{}, std::false_type{});
+  return f32 ? f(std::integral_constant<int, 32>{}, std::true_type{})
+             : f(std::integral_constant<int, 32>{}, std::false_type{});
+}
+
+// ----------------------------------------------------------------- fp32 operand planes
+// Byte layout of the planes of `n` tensors of `elems[i]` elements: hi, then
+// lo, each 256-byte aligned.
+size_t planes_bytes(const size_t* elems, int n) {
+  size_t b = 0;
+  for (int i = 0; i < n; ++i) b += 2 * round_up(elems[i] * 2, 256);
+  return b;
+}
+
+// Carves the planes out of `base` and runs the operand prologue over the
+// tensors (rotating those with rope[i] set).
+int run_prep(uint8_t* base, const float* const* src, const size_t* elems, const int* H, const int* rope, int n,
+             int T, int D, const float2* table, nea::PrepJob* jobs_out, cudaStream_t stream) {
+  nea::PrepParams pp{};
+  size_t off = 0;
+  pp.n_jobs = n;
+  pp.T = T;
+  pp.rope = table;
+  for (int i = 0; i < n; ++i) {
+    nea::PrepJob& j = pp.job[i];
+    j.src = src[i];
+    j.hi = reinterpret_cast<__nv_bfloat16*>(base + off);
+    off += round_up(elems[i] * 2, 256);
+    j.lo = reinterpret_cast<__nv_bfloat16*>(base + off);
+    off += round_up(elems[i] * 2, 256);
+    j.chunks = static_cast<long long>(elems[i] / 4);
+    j.H = H[i];
+    j.rope = rope[i] && table != nullptr;
+    pp.total += j.chunks;
+    jobs_out[i] = j;
+  }
+  const long long blocks = std::min<long long>((pp.total + 255) / 256, 148LL * 16);
+  if (D == 64)
+    nea::attn_prep_split_kernel<64><<<unsigned(blocks), 256, 0, stream>>>(pp);
+  else
+    nea::attn_prep_split_kernel<32><<<unsigned(blocks), 256, 0, stream>>>(pp);
+  const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? NEA_OK : cuda_fail(e);
 }
 
+// ----------------------------------------------------------------- forward
 template <int D, bool F32IO>
-int launch_bwd(DeviceState& st, const nea::BwdParams& p, const void* O, cudaStream_t stream) {
-  const int rows = p.B * p.T * p.Hq;
+int launch_fwd(uint32_t& attr_done, const nea::FwdParams& p, cudaStream_t stream) {
+  using L = nea::FwdSmem<D, F32IO>;
+  auto kern = nea::attn_fwd_kernel<D, F32IO>;
+  int rc = set_smem(attr_done, (D == 64) * 2 + F32IO, kern, L::kAlloc);
+  if (rc) return rc;
+  kern<<<p.B * p.Hq * p.n_pairs, L::kThreads, L::kAlloc, stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? NEA_OK : cuda_fail(e);
+}
+
+// ----------------------------------------------------------------- backward
+// Row terms, dK/dV kernel, dQ kernel.  `ev` selects profiling events (the
+// regular backward records them, the allocation-free one does not).
+template <int D, bool F32IO>
+int launch_bwd(uint32_t& attr_done, const nea::BwdParams& p, const void* O, const void* dO, const float* LSE,
+               cudaStream_t stream, bool ev) {
   constexpr int kLanes = D / (F32IO ? 4 : 8);
-  const long long threads = static_cast<long long>(rows) * kLanes;
-  prof_record(2, stream);
-  nea::attn_bwd_rowterm_kernel<D, F32IO>
-      <<<unsigned((threads + 255) / 256), 256, 0, stream>>>(O, p.dO, const_cast<float*>(p.Dv), rows, p.T, p.Hq);
+  const long long threads = static_cast<long long>(p.B) * p.Tp * p.Hq * kLanes;
+  nea::attn_bwd_rowterm_kernel<D, F32IO><<<unsigned((threads + 255) / 256), 256, 0, stream>>>(
+      O, dO, LSE, const_cast<float*>(p.ws), p.B, p.T, p.Tp, p.Hq);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
-  prof_record(3, stream);
+  if (ev) prof_record(3, stream);
 
   using LK = nea::BwdSmem<D, F32IO, true>;
   auto kk = nea::attn_bwd_kernel<D, F32IO, true>;
-  int rc = set_smem(st, 4 + (D == 64) * 2 + F32IO, kk, LK::kAlloc);
+  int rc = set_smem(attr_done, 4 + (D == 64) * 2 + F32IO, kk, LK::kAlloc);
   if (rc) return rc;
-  kk<<<p.B * p.Hkv * p.n_tiles, 288, LK::kAlloc, stream>>>(p);
+  kk<<<p.B * p.Hkv * p.n_tiles, LK::kThreads, LK::kAlloc, stream>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
-  prof_record(4, stream);
+  if (ev) prof_record(4, stream);
 
   using LQ = nea::BwdSmem<D, F32IO, false>;
   auto kq = nea::attn_bwd_kernel<D, F32IO, false>;
-  rc = set_smem(st, 8 + (D == 64) * 2 + F32IO, kq, LQ::kAlloc);
+  rc = set_smem(attr_done, 8 + (D == 64) * 2 + F32IO, kq, LQ::kAlloc);
   if (rc) return rc;
-  kq<<<p.B * p.Hq * p.n_tiles, 288, LQ::kAlloc, stream>>>(p);
+  kq<<<p.B * p.Hq * p.n_tiles, LQ::kThreads, LQ::kAlloc, stream>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
-  prof_record(5, stream);
+  if (ev) prof_record(5, stream);
   return NEA_OK;
+}
+
+int check_bwd_args(const void* Q, const void* K, const void* V, const void* O, const float* LSE, const void* dO,
+                   void* dQ, void* dK, void* dV, int B, int T, int Hq, int Hkv, int D, int dtype, float rope_base,
+                   int causal, bool* empty) {
+  int rc = check_shape(B, T, Hq, Hkv, D, dtype, causal, empty);
+  if (rc || *empty) return rc;
+  if (!Q || !K || !V || !O || !LSE || !dO || !dQ || !dK || !dV) return NEA_ERR_ARG;
+  for (const void* ptr : {Q, K, V, O, static_cast<const void*>(LSE), dO, static_cast<const void*>(dQ),
+                          static_cast<const void*>(dK), static_cast<const void*>(dV)})
+    if (!aligned16(ptr)) return NEA_ERR_ARG;
+  if (!std::isfinite(rope_base)) return NEA_ERR_ARG;
+  return NEA_OK;
+}
+
+// Bytes of backward workspace: the padded row terms, then (fp32) the planes
+// of Q, K, V, dO.
+size_t bwd_ws_bytes(int B, int T, int Hq, int Hkv, int D, bool f32, size_t* rowterm_bytes) {
+  const size_t Tp = round_up(size_t(T), nea::kTileRows);
+  *rowterm_bytes = round_up(size_t(B) * Hq * 2 * Tp * sizeof(float), 256);
+  if (!f32) return *rowterm_bytes;
+  const size_t nq = size_t(B) * T * Hq * D, nk = size_t(B) * T * Hkv * D;
+  const size_t elems[4] = {nq, nk, nk, nq};
+  return *rowterm_bytes + planes_bytes(elems, 4);
+}
+
+// The backward after argument checks, given a workspace of bwd_ws_bytes()
+// bytes, a rotary table (or nullptr) and a status word.
+int run_bwd(uint32_t& attr_done, uint8_t* ws, const float2* rope, int* status, const void* Q, const void* K,
+            const void* V, const void* O, const float* LSE, const void* dO, void* dQ, void* dK, void* dV, int B,
+            int T, int Hq, int Hkv, int D, int dtype, int causal, cudaStream_t stream, bool ev) {
+  const bool f32 = dtype == NEA_F32;
+  size_t rowterm_bytes = 0;
+  (void)bwd_ws_bytes(B, T, Hq, Hkv, D, f32, &rowterm_bytes);
+  nea::BwdParams p{};
+  p.Tp = int(round_up(size_t(T), nea::kTileRows));
+  p.ws = reinterpret_cast<const float*>(ws);
+  int rc;
+  if (ev) prof_record(2, stream);
+  if (f32) {
+    const size_t nq = size_t(B) * T * Hq * D, nk = size_t(B) * T * Hkv * D;
+    const float* src[4] = {static_cast<const float*>(Q), static_cast<const float*>(K),
+                           static_cast<const float*>(V), static_cast<const float*>(dO)};
+    const size_t elems[4] = {nq, nk, nk, nq};
+    const int H[4] = {Hq, Hkv, Hkv, Hq}, rot[4] = {1, 1, 0, 0};
+    nea::PrepJob jobs[4];
+    if ((rc = run_prep(ws + rowterm_bytes, src, elems, H, rot, 4, T, D, rope, jobs, stream))) return rc;
+    if ((rc = make_tile_map(&p.tm_q, jobs[0].hi, B, T, Hq, D)) ||
+        (rc = make_tile_map(&p.tm_q_lo, jobs[0].lo, B, T, Hq, D)) ||
+        (rc = make_tile_map(&p.tm_k, jobs[1].hi, B, T, Hkv, D)) ||
+        (rc = make_tile_map(&p.tm_k_lo, jobs[1].lo, B, T, Hkv, D)) ||
+        (rc = make_tile_map(&p.tm_v, jobs[2].hi, B, T, Hkv, D)) ||
+        (rc = make_tile_map(&p.tm_v_lo, jobs[2].lo, B, T, Hkv, D)) ||
+        (rc = make_tile_map(&p.tm_do, jobs[3].hi, B, T, Hq, D)) ||
+        (rc = make_tile_map(&p.tm_do_lo, jobs[3].lo, B, T, Hq, D)))
+      return rc;
+  } else {
+    if ((rc = make_tile_map(&p.tm_q, Q, B, T, Hq, D)) || (rc = make_tile_map(&p.tm_k, K, B, T, Hkv, D)) ||
+        (rc = make_tile_map(&p.tm_v, V, B, T, Hkv, D)) || (rc = make_tile_map(&p.tm_do, dO, B, T, Hq, D)))
+      return rc;
+  }
+  if ((rc = make_rowterm_map(&p.tm_ws, p.ws, B * Hq, p.Tp))) return rc;
+  p.dQ = dQ;
+  p.dK = dK;
+  p.dV = dV;
+  p.rope = rope;
+  p.B = B;
+  p.T = T;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.n_tiles = (T + 127) / 128;
+  p.causal = causal;
+  p.scale = float(1.0 / std::sqrt(double(D)));
+  p.scale_log2 = float(1.4426950408889634 / std::sqrt(double(D)));
+  p.err = status;
+  p.wait_limit = static_cast<unsigned long long>(t_wait_limit_ns);
+  return dispatch(D, dtype, [&](auto d, auto f) {
+    return launch_bwd<decltype(d)::value, decltype(f)::value>(attr_done, p, O, dO, LSE, stream, ev);
+  });
 }
 
 }  // namespace
@@ -205,15 +409,36 @@ int nea_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE)) return NEA_ERR_ARG;
   if (!std::isfinite(rope_base)) return NEA_ERR_ARG;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  const bool f32 = dtype == NEA_F32;
 
   std::lock_guard<std::mutex> lock(g_mu);
   DeviceState* st = nullptr;
   if ((rc = device_state(&st))) return rc;
   nea::FwdParams p{};
   if ((rc = rope_table(*st, T, D, rope_base, stream, &p.rope))) return rc;
-  p.Q = Q;
-  p.K = K;
-  p.V = V;
+  prof_record(0, stream);
+  if (f32) {
+    // operand prologue: rotated, split Q and K; split V
+    const size_t nq = size_t(B) * T * Hq * D, nk = size_t(B) * T * Hkv * D;
+    const float* src[3] = {static_cast<const float*>(Q), static_cast<const float*>(K),
+                           static_cast<const float*>(V)};
+    const size_t elems[3] = {nq, nk, nk};
+    const int H[3] = {Hq, Hkv, Hkv}, rot[3] = {1, 1, 0};
+    if ((rc = ensure_ws(*st, planes_bytes(elems, 3)))) return rc;
+    nea::PrepJob jobs[3];
+    if ((rc = run_prep(st->ws, src, elems, H, rot, 3, T, D, p.rope, jobs, stream))) return rc;
+    if ((rc = make_tile_map(&p.tm_q, jobs[0].hi, B, T, Hq, D)) ||
+        (rc = make_tile_map(&p.tm_q_lo, jobs[0].lo, B, T, Hq, D)) ||
+        (rc = make_tile_map(&p.tm_k, jobs[1].hi, B, T, Hkv, D)) ||
+        (rc = make_tile_map(&p.tm_k_lo, jobs[1].lo, B, T, Hkv, D)) ||
+        (rc = make_tile_map(&p.tm_v, jobs[2].hi, B, T, Hkv, D)) ||
+        (rc = make_tile_map(&p.tm_v_lo, jobs[2].lo, B, T, Hkv, D)))
+      return rc;
+  } else {
+    if ((rc = make_tile_map(&p.tm_q, Q, B, T, Hq, D)) || (rc = make_tile_map(&p.tm_k, K, B, T, Hkv, D)) ||
+        (rc = make_tile_map(&p.tm_v, V, B, T, Hkv, D)))
+      return rc;
+  }
   p.O = O;
   p.LSE = LSE;
   p.B = B;
@@ -222,60 +447,40 @@ int nea_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
   p.Hkv = Hkv;
   p.G = Hq / Hkv;
   p.n_tiles = (T + 127) / 128;
+  p.n_pairs = (p.n_tiles + 1) / 2;
   p.causal = causal;
   p.scale_log2 = float(1.4426950408889634 / std::sqrt(double(D)));
   p.err = st->err;
   p.wait_limit = static_cast<unsigned long long>(t_wait_limit_ns);
   p.debug = t_debug_flags;
   t_debug_flags = 0;
-  const bool f32 = dtype == NEA_F32;
-  if (D == 64) return f32 ? launch_fwd<64, true>(*st, p, stream) : launch_fwd<64, false>(*st, p, stream);
-  return f32 ? launch_fwd<32, true>(*st, p, stream) : launch_fwd<32, false>(*st, p, stream);
+#ifdef NEA_TRACE
+  p.trace = t_trace;
+#endif
+  rc = dispatch(D, dtype, [&](auto d, auto f) {
+    return launch_fwd<decltype(d)::value, decltype(f)::value>(st->attr_done, p, stream);
+  });
+  prof_record(1, stream);
+  return rc;
 }
 
 int nea_attn_bwd(const void* Q, const void* K, const void* V, const void* O, const float* LSE, const void* dO,
                  void* dQ, void* dK, void* dV, int B, int T, int Hq, int Hkv, int D, int dtype, float rope_base,
                  int causal, void* stream_) {
   bool empty = false;
-  int rc = check_shape(B, T, Hq, Hkv, D, dtype, causal, &empty);
-  if (rc) return rc;
-  if (empty) return NEA_OK;
-  if (!Q || !K || !V || !O || !LSE || !dO || !dQ || !dK || !dV) return NEA_ERR_ARG;
-  for (const void* ptr : {Q, K, V, O, static_cast<const void*>(LSE), dO, static_cast<const void*>(dQ),
-                          static_cast<const void*>(dK), static_cast<const void*>(dV)})
-    if (!aligned16(ptr)) return NEA_ERR_ARG;
-  if (!std::isfinite(rope_base)) return NEA_ERR_ARG;
+  int rc = check_bwd_args(Q, K, V, O, LSE, dO, dQ, dK, dV, B, T, Hq, Hkv, D, dtype, rope_base, causal, &empty);
+  if (rc || empty) return rc;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
 
   std::lock_guard<std::mutex> lock(g_mu);
   DeviceState* st = nullptr;
   if ((rc = device_state(&st))) return rc;
-  nea::BwdParams p{};
-  if ((rc = rope_table(*st, T, D, rope_base, stream, &p.rope))) return rc;
-  if ((rc = ensure_dvec(*st, size_t(B) * Hq * T, stream))) return rc;
-  p.Q = Q;
-  p.K = K;
-  p.V = V;
-  p.dO = dO;
-  p.LSE = LSE;
-  p.Dv = st->dvec;
-  p.dQ = dQ;
-  p.dK = dK;
-  p.dV = dV;
-  p.B = B;
-  p.T = T;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.G = Hq / Hkv;
-  p.n_tiles = (T + 127) / 128;
-  p.causal = causal;
-  p.scale = float(1.0 / std::sqrt(double(D)));
-  p.scale_log2 = float(1.4426950408889634 / std::sqrt(double(D)));
-  p.err = st->err;
-  p.wait_limit = static_cast<unsigned long long>(t_wait_limit_ns);
-  const bool f32 = dtype == NEA_F32;
-  if (D == 64) return f32 ? launch_bwd<64, true>(*st, p, O, stream) : launch_bwd<64, false>(*st, p, O, stream);
-  return f32 ? launch_bwd<32, true>(*st, p, O, stream) : launch_bwd<32, false>(*st, p, O, stream);
+  const float2* rope = nullptr;
+  if ((rc = rope_table(*st, T, D, rope_base, stream, &rope))) return rc;
+  size_t rowterm_bytes = 0;
+  if ((rc = ensure_ws(*st, bwd_ws_bytes(B, T, Hq, Hkv, D, dtype == NEA_F32, &rowterm_bytes)))) return rc;
+  return run_bwd(st->attr_done, st->ws, rope, st->err, Q, K, V, O, LSE, dO, dQ, dK, dV, B, T, Hq, Hkv, D, dtype,
+                 causal, stream, true);
 }
 
 int nea_device_status(void* stream_) {
@@ -299,6 +504,10 @@ long long nea_set_wait_limit_ns(long long ns) {
 }
 
 void nea_debug_inject(int flags) { t_debug_flags = flags; }
+
+#ifdef NEA_TRACE
+void nea_debug_set_trace(void* buffer) { t_trace = static_cast<unsigned long long*>(buffer); }
+#endif
 
 void nea_set_profile_events(void* const* events, int n) {
   t_prof_events = (events && n > 0) ? events : nullptr;
@@ -330,7 +539,7 @@ int nea_version(void) { return kVersion; }
 namespace {
 
 constexpr size_t kNoAllocScratchFloats = size_t(1) << 20;  // 4 MiB
-constexpr size_t kNoAllocStatusFloats = 64;                 // status word, padded to 256 bytes
+constexpr size_t kNoAllocStatusBytes = 256;                 // status word, padded
 constexpr int kNoAllocMaxDevices = 64;
 
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
@@ -341,57 +550,26 @@ static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
 struct NoAllocDevice {
   bool ready = false;
   bool sm100 = false;
-  float* scratch = nullptr;
+  uint8_t* scratch = nullptr;
   uint32_t attr_done = 0;
 };
 NoAllocDevice g_noalloc_dev[kNoAllocMaxDevices];
 std::mutex g_noalloc_mu;
 
-// Rotary table [T][D/2] of (cos, sin) of t * base^(-2i/D), angles in double.
+// Rotary table [T][D/2] of (cos, sin) of t * base^(-2i/D), angles in double;
+// rows T .. rope_rows(T)-1 repeat the rows of the 64-row block starts
+// (row r -> position min(64 (r - T), T - 1)), as in the regular table.
 __global__ void noalloc_rope_table_kernel(float2* out, int T, int D, double base) {
   const long idx = long(blockIdx.x) * blockDim.x + threadIdx.x;
   const int half = D / 2;
-  if (idx >= long(T) * half) return;
-  const int t = int(idx / half), i = int(idx % half);
+  const int rows = T + 2 * ((T + nea::kTileRows - 1) / nea::kTileRows);
+  if (idx >= long(rows) * half) return;
+  const int row = int(idx / half), i = int(idx % half);
+  const int t = row < T ? row : min((row - T) * nea::kRopeRows, T - 1);
   const double a = double(t) * pow(base, -2.0 * double(i) / double(D));
   double sn, cs;
   sincos(a, &sn, &cs);
   out[idx] = make_float2(float(cs), float(sn));
-}
-
-size_t round4(size_t n) { return (n + 3) & ~size_t(3); }
-
-template <typename Kern>
-int noalloc_smem(NoAllocDevice& st, int bit, Kern kern, uint32_t bytes) {
-  if (st.attr_done & (1u << bit)) return NEA_OK;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes));
-  if (e != cudaSuccess) return cuda_fail(e);
-  st.attr_done |= 1u << bit;
-  return NEA_OK;
-}
-
-template <int D, bool F32IO>
-int noalloc_launch(NoAllocDevice& st, const nea::BwdParams& p, const void* O, cudaStream_t stream) {
-  const int rows = p.B * p.T * p.Hq;
-  constexpr int kLanes = D / (F32IO ? 4 : 8);
-  const long long threads = static_cast<long long>(rows) * kLanes;
-  nea::attn_bwd_rowterm_kernel<D, F32IO>
-      <<<unsigned((threads + 255) / 256), 256, 0, stream>>>(O, p.dO, const_cast<float*>(p.Dv), rows, p.T, p.Hq);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e);
-  using LK = nea::BwdSmem<D, F32IO, true>;
-  auto kk = nea::attn_bwd_kernel<D, F32IO, true>;
-  int rc = noalloc_smem(st, (D == 64) * 2 + F32IO, kk, LK::kAlloc);
-  if (rc) return rc;
-  kk<<<p.B * p.Hkv * p.n_tiles, 288, LK::kAlloc, stream>>>(p);
-  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
-  using LQ = nea::BwdSmem<D, F32IO, false>;
-  auto kq = nea::attn_bwd_kernel<D, F32IO, false>;
-  rc = noalloc_smem(st, 4 + (D == 64) * 2 + F32IO, kq, LQ::kAlloc);
-  if (rc) return rc;
-  kq<<<p.B * p.Hq * p.n_tiles, 288, LQ::kAlloc, stream>>>(p);
-  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
-  return NEA_OK;
 }
 
 }  // namespace
@@ -400,17 +578,13 @@ extern "C" int nea_attn_bwd_noalloc(const void* Q, const void* K, const void* V,
                                     const void* dO, void* dQ, void* dK, void* dV, int B, int T, int Hq, int Hkv,
                                     int D, int dtype, float rope_base, int causal, void* stream_) {
   bool empty = false;
-  int rc = check_shape(B, T, Hq, Hkv, D, dtype, causal, &empty);
-  if (rc) return rc;
-  if (empty) return NEA_OK;
-  if (!Q || !K || !V || !O || !LSE || !dO || !dQ || !dK || !dV) return NEA_ERR_ARG;
-  for (const void* ptr : {Q, K, V, O, static_cast<const void*>(LSE), dO, static_cast<const void*>(dQ),
-                          static_cast<const void*>(dK), static_cast<const void*>(dV)})
-    if (!aligned16(ptr)) return NEA_ERR_ARG;
-  if (!std::isfinite(rope_base)) return NEA_ERR_ARG;
-  const size_t dv_floats = round4(size_t(B) * Hq * T);
-  const size_t rope_floats = (rope_base > 0.f) ? round4(size_t(T) * D) : 0;
-  if (kNoAllocStatusFloats + dv_floats + rope_floats > kNoAllocScratchFloats) return NEA_ERR_SCRATCH_LIMIT;
+  int rc = check_bwd_args(Q, K, V, O, LSE, dO, dQ, dK, dV, B, T, Hq, Hkv, D, dtype, rope_base, causal, &empty);
+  if (rc || empty) return rc;
+  size_t rowterm_bytes = 0;
+  const size_t ws_bytes = bwd_ws_bytes(B, T, Hq, Hkv, D, dtype == NEA_F32, &rowterm_bytes);
+  const size_t rope_bytes = (rope_base > 0.f) ? round_up(rope_rows(T) * D * sizeof(float), 256) : 0;
+  if (kNoAllocStatusBytes + ws_bytes + rope_bytes > kNoAllocScratchFloats * sizeof(float))
+    return NEA_ERR_SCRATCH_LIMIT;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
 
   int dev = 0;
@@ -430,46 +604,24 @@ extern "C" int nea_attn_bwd_noalloc(const void* Q, const void* K, const void* V,
     if (st.sm100) {
       void* ptr = nullptr;
       if ((e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch)) != cudaSuccess) return cuda_fail(e);
-      st.scratch = static_cast<float*>(ptr);
+      st.scratch = static_cast<uint8_t*>(ptr);
     }
     st.ready = true;
   }
   if (!st.sm100) return NEA_ERR_UNSUPPORTED;
 
+  // scratch: status word | row terms (+ fp32 operand planes) | rotary table
   int* status = reinterpret_cast<int*>(st.scratch);
-  float* dv = st.scratch + kNoAllocStatusFloats;
-  float2* rope = rope_floats ? reinterpret_cast<float2*>(dv + dv_floats) : nullptr;
-  // the status word must start at zero; Dv is fully rewritten by the row-term
-  // kernel and the table by its own kernel, so neither needs clearing
+  uint8_t* ws = st.scratch + kNoAllocStatusBytes;
+  float2* rope = rope_bytes ? reinterpret_cast<float2*>(ws + ws_bytes) : nullptr;
+  // the status word must start at zero; the row terms, planes and table are
+  // fully rewritten by their kernels, so they need no clearing
   if ((e = cudaMemsetAsync(status, 0, sizeof(int), stream)) != cudaSuccess) return cuda_fail(e);
   if (rope) {
-    const long n = long(T) * (D / 2);
+    const long n = long(rope_rows(T)) * (D / 2);
     noalloc_rope_table_kernel<<<unsigned((n + 255) / 256), 256, 0, stream>>>(rope, T, D, double(rope_base));
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
   }
-  nea::BwdParams p{};
-  p.Q = Q;
-  p.K = K;
-  p.V = V;
-  p.dO = dO;
-  p.LSE = LSE;
-  p.Dv = dv;
-  p.dQ = dQ;
-  p.dK = dK;
-  p.dV = dV;
-  p.rope = rope;
-  p.B = B;
-  p.T = T;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.G = Hq / Hkv;
-  p.n_tiles = (T + 127) / 128;
-  p.causal = causal;
-  p.scale = float(1.0 / std::sqrt(double(D)));
-  p.scale_log2 = float(1.4426950408889634 / std::sqrt(double(D)));
-  p.err = status;
-  p.wait_limit = static_cast<unsigned long long>(t_wait_limit_ns);
-  const bool f32 = dtype == NEA_F32;
-  if (D == 64) return f32 ? noalloc_launch<64, true>(st, p, O, stream) : noalloc_launch<64, false>(st, p, O, stream);
-  return f32 ? noalloc_launch<32, true>(st, p, O, stream) : noalloc_launch<32, false>(st, p, O, stream);
+  return run_bwd(st.attr_done, ws, rope, status, Q, K, V, O, LSE, dO, dQ, dK, dV, B, T, Hq, Hkv, D, dtype, causal,
+                 stream, false);
 }

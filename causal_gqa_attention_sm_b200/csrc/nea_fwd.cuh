@@ -4,99 +4,179 @@
 // the pages' own kernel stages K/V tiles in shared memory and loops over them
 // per query block -- smartinfralog.com post, "Tiled FlashAttention" section).
 //
-// One CTA computes a 128-row query tile of one (batch, query head):
-//   warps 0-3  softmax: thread r owns query row r = TMEM lane r; reads S from
-//              TMEM, masks, keeps the running max m and sum l, writes
-//              P = exp(s - m) back into the same TMEM columns as bf16 (hi and
-//              lo parts for float32 storage), rescales O in TMEM when m grows
-//              by more than 2^8, and writes O / l and LSE at the end.
-//   warps 4-7  producer: loads the query tile once, then key/value tiles into
-//              a two-stage ring, applying RoPE to Q and K on the way.
-//   warp 8     MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM
-//              score buffers, then O += P_j V_j with P_j read from TMEM.
+// One CTA computes two adjacent 128-row query tiles (A = 2m, B = 2m + 1) of
+// one (batch, query head); both read the same key/value tiles, so every K/V
+// tile is loaded (and rotated) once per pair.
+//
+// Operands.  bf16 storage: TMA lands each tile already in the swizzled
+// tensor-core layout and the converter warps rotate queries and keys in place
+// (RoPE fused into the tile load).  float32 storage: the tiles come from the
+// bf16 hi/lo planes written by the operand prologue (nea_prep.cuh, queries and
+// keys already rotated); TMA lands the hi and lo halves of each tile and every
+// product is formed from three bf16 products (hi*hi + hi*lo + lo*hi).
+//
+// Warps:
+//   0-3, 4-7   softmax of tile A, of tile B: thread r owns row r (TMEM lane
+//              r); pass 1 over S finds the row max, pass 2 writes
+//              P = exp(s - m) back as bf16 (hi over S, lo in its own columns
+//              for float32 storage); the running max m moves only when it
+//              grows by more than 2^8 (O rescaled in TMEM then); the epilogue
+//              writes O / l and LSE.
+//   8          MMA issuer (one thread): S_X = Q_X K_j^T, O_X += P_X V_j for X
+//              in {A, B}, ping-ponging so one tile's softmax overlaps the
+//              other tile's MMAs.
+//   9          TMA: query tiles, then K and V tiles into two rings (K stages
+//              free as soon as S is computed, V stages after PV).
+//   10-13      (bf16 only) converter: in-place RoPE of the Q and K tiles.
+// TMEM per tile X: S [256X, 256X+128), O [256X+128, +D), P lo [256X+192, +64).
 // Causal tiles above the diagonal are never visited; only the diagonal tile
-// and a ragged last tile are masked.  Key/value tiles are visited in order, so
-// the issue of S_{j+1} overlaps the softmax of tile j.
+// and a ragged last tile are masked.
 #pragma once
 
+#include <cuda.h>
+
 #include "nea_tiles.cuh"
+
+// Phase stamps for performance analysis: compiled only with -DNEA_TRACE, when
+// `p.trace` receives per CTA 80 %globaltimer values (slot 79: SM id).
+#ifdef NEA_TRACE
+#define NEA_TRACE_STAMP(p, slot, cond)                                                  \
+  do {                                                                                  \
+    if ((p).trace && (cond)) {                                                          \
+      (p).trace[size_t(blockIdx.x) * 80 + (slot)] = nea::global_timer_ns();             \
+      if ((slot) == 0) {                                                                \
+        unsigned smid_;                                                                 \
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid_));                              \
+        (p).trace[size_t(blockIdx.x) * 80 + 79] = smid_;                                \
+      }                                                                                 \
+    }                                                                                   \
+  } while (0)
+#else
+#define NEA_TRACE_STAMP(p, slot, cond) \
+  do {                                 \
+  } while (0)
+#endif
 
 namespace nea {
 
 struct FwdParams {
-  const void* Q;
-  const void* K;
-  const void* V;
+  // bf16 storage: the inputs.  float32 storage: the hi planes.
+  CUtensorMap tm_q;  // [B][T][Hq][D], box {D, 1, 128, 1}
+  CUtensorMap tm_k;  // [B][T][Hkv][D]
+  CUtensorMap tm_v;
+  // float32 storage: the lo planes
+  CUtensorMap tm_q_lo;
+  CUtensorMap tm_k_lo;
+  CUtensorMap tm_v_lo;
   void* O;
   float* LSE;
-  const float2* rope;  // [T][D/2] (cos, sin) or nullptr when the rotation is off
+  // [T][D/2] (cos, sin), then [2*n_tiles][D/2] block-start rows; nullptr
+  // when the rotation is off (bf16 storage only; fp32 planes are pre-rotated)
+  const float2* rope;
   int B, T, Hq, Hkv, G;
   int n_tiles;         // ceil(T / 128)
+  int n_pairs;         // ceil(n_tiles / 2)
   int causal;
   float scale_log2;    // log2(e) / sqrt(D)
   int* err;
   unsigned long long wait_limit;
   int debug;
+  unsigned long long* trace;  // per-CTA phase stamps (NEA_TRACE builds only)
 };
 
 template <int D, bool F32IO>
 struct FwdSmem {
-  static constexpr int kParts = F32IO ? 2 : 1;
-  static constexpr int kStages = 2;
-  static constexpr uint32_t kTile = TileGeom<D>::kTileBytes;
-  static constexpr uint32_t kQ = 0;
-  static constexpr uint32_t kStage0 = kQ + kParts * kTile;
-  static constexpr uint32_t kStageBytes = 2 * kParts * kTile;  // K parts, then V parts
-  static constexpr uint32_t kBars = kStage0 + kStages * kStageBytes;
-  static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 1 + 1;
+  static constexpr bool kConv = !F32IO;        // converter warps (in-place RoPE)
+  static constexpr int kNK = F32IO ? 3 : 4;    // K ring stages
+  static constexpr int kNV = F32IO ? 2 : 3;    // V ring stages
+  static constexpr uint32_t kTile = Stage<D, F32IO>::kBytes;  // one tile: hi (+ lo)
+  static constexpr uint32_t kBase = RopeBaseRows<D>::kBytes;
+  static constexpr uint32_t kSide = kConv ? 1024 : 0;          // per-tile rotary base rows
+  static constexpr uint32_t kQA = 0;
+  static constexpr uint32_t kQB = kTile;
+  static constexpr uint32_t kQBase = 2 * kTile;  // base rows of A then B
+  static constexpr uint32_t kRope = kQBase + kSide;
+  static constexpr uint32_t kK0 = kRope + (kConv ? TileGeom<D>::kRopeBytes : 0);
+  static constexpr uint32_t kKStage = kTile + kSide;  // tile, then its base rows
+  static constexpr uint32_t kV0 = kK0 + kNK * kKStage;
+  static constexpr uint32_t kVStage = kTile;
+  static constexpr uint32_t kBars = kV0 + kNV * kVStage;
+  // qtma, qready, K tma/full/empty, V tma/empty, s[2], p[2], o[2], fin
+  static constexpr int kNumBars = 2 + 3 * kNK + 2 * kNV + 6 + 1;
   static constexpr uint32_t kMisc = kBars + 8 * kNumBars;
   static constexpr uint32_t kUsed = kMisc + 16;
-  // +1024 for manual alignment; at least 120 KB so two CTAs never share an SM
-  // (each allocates all 512 TMEM columns).
-  static constexpr uint32_t kAlloc = (kUsed + 1024 > 120u * 1024u) ? kUsed + 1024 : 120u * 1024u;
+  // +1024 for manual alignment; at least 116 KB so two CTAs never share an SM
+  // (each takes all 512 TMEM columns)
+  static constexpr uint32_t kAlloc = kUsed + 1024 > 116u * 1024u ? kUsed + 1024 : 116u * 1024u;
+  static constexpr int kThreads = kConv ? 448 : 320;
+  static_assert(kK0 % 1024 == 0 && kKStage % 1024 == 0 && kV0 % 1024 == 0 && kVStage % 1024 == 0,
+                "operand tiles need 1024-byte alignment");
+  static_assert(2 * kBase <= 1024, "query base rows");
+  static_assert(kAlloc <= 232448, "shared memory");
 };
 
 template <int D, bool F32IO>
-__global__ void __launch_bounds__(288, 1) attn_fwd_kernel(const __grid_constant__ FwdParams p) {
+__global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ FwdParams p) {
   using L = FwdSmem<D, F32IO>;
   constexpr uint32_t RB = TileGeom<D>::kRowBytes;
-  constexpr int NS = L::kStages;
+  constexpr uint32_t OPB = TileGeom<D>::kOpBytes;
+  constexpr int NK = L::kNK, NV = L::kNV;
   constexpr int kTerms = F32IO ? 3 : 1;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
-  uint64_t* bar_q = bars + 0;
-  uint64_t* bar_full = bars + 1;             // [NS]
-  uint64_t* bar_empty = bars + 1 + NS;       // [NS]
-  uint64_t* bar_s = bars + 1 + 2 * NS;       // [2]
-  uint64_t* bar_p = bars + 3 + 2 * NS;       // [2]
-  uint64_t* bar_o = bars + 5 + 2 * NS;
-  uint64_t* bar_fin = bars + 6 + 2 * NS;
+  uint64_t* bar_qtma = bars + 0;
+  uint64_t* bar_qconv = bars + 1;                       // Q tiles rotated (count 128)
+  uint64_t* bar_ktma = bars + 2;                        // [NK]
+  uint64_t* bar_kconv = bars + 2 + NK;                  // [NK] (count 128)
+  uint64_t* bar_kempty = bars + 2 + 2 * NK;             // [NK]
+  uint64_t* bar_vtma = bars + 2 + 3 * NK;               // [NV]
+  uint64_t* bar_vempty = bars + 2 + 3 * NK + NV;        // [NV]
+  uint64_t* bar_s = bars + 2 + 3 * NK + 2 * NV;         // [2] S_X landed
+  uint64_t* bar_p = bar_s + 2;                          // [2] P_X written (count 128)
+  uint64_t* bar_o = bar_s + 4;                          // [2] PV_X done
+  uint64_t* bar_fin = bar_s + 6;
+  // what the MMA issuer waits for: converted tiles (bf16) or landed planes (fp32)
+  uint64_t* bar_qready = L::kConv ? bar_qconv : bar_qtma;
+  uint64_t* bar_kready = L::kConv ? bar_kconv : bar_ktma;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  const float2* rope_off = reinterpret_cast<const float2*>(smem + L::kRope);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int n_bh = p.B * p.Hq;
-  const int qt = p.n_tiles - 1 - int(blockIdx.x) / n_bh;  // longest causal rows first
+  const int m = p.n_pairs - 1 - int(blockIdx.x) / n_bh;  // longest causal rows first
   const int bh = int(blockIdx.x) % n_bh;
   const int b = bh / p.Hq, h = bh % p.Hq, g = h / p.G;
-  const int n_kv = p.causal ? qt + 1 : p.n_tiles;
+  const int qt_a = 2 * m, qt_b = 2 * m + 1;
+  const bool has_b = qt_b < p.n_tiles;
+  const int nkv_a = p.causal ? qt_a + 1 : p.n_tiles, nkv_b = has_b ? (p.causal ? qt_b + 1 : p.n_tiles) : 0;
+  const int n_kv = has_b ? nkv_b : nkv_a;
+  auto active = [&](int x, int j) { return j < (x ? nkv_b : nkv_a); };
   const WaitCtl wc{p.err, p.wait_limit, abort_flag};
+  NEA_TRACE_STAMP(p, 0, tid == 0);
 
   if (tid == 0) {
     *abort_flag = 0;
-    mbar_init(bar_q, 128);
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(&bar_full[s], 128);
-      mbar_init(&bar_empty[s], 1);
+    mbar_init(bar_qtma, 1);
+    mbar_init(bar_qconv, 128);
+    for (int s = 0; s < NK; ++s) {
+      mbar_init(&bar_ktma[s], 1);
+      mbar_init(&bar_kconv[s], 128);
+      mbar_init(&bar_kempty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bar_s[s], 1);
-      mbar_init(&bar_p[s], 128);
+    for (int s = 0; s < NV; ++s) {
+      mbar_init(&bar_vtma[s], 1);
+      mbar_init(&bar_vempty[s], 1);
     }
-    mbar_init(bar_o, 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bar_s[x], 1);
+      mbar_init(&bar_p[x], 128);
+      mbar_init(&bar_o[x], 1);
+    }
     mbar_init(bar_fin, 1);
     mbar_init_fence();
   }
@@ -105,159 +185,254 @@ __global__ void __launch_bounds__(288, 1) attn_fwd_kernel(const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_holder;
-  constexpr uint32_t kColO = 256;
+  NEA_TRACE_STAMP(p, 1, tid == 0);
 
-  if (warp >= 4 && warp < 8) {
-    // ------------------------------------------------------------ producer
-    const int pt = tid - 128;
-    load_tile<D, F32IO, true>(smem + L::kQ, p.Q, b, qt * kTileRows, h, p.T, p.Hq, p.rope, pt);
-    fence_async_smem();
-    if (!(p.debug & 1)) mbar_arrive(bar_q);
-    for (int j = 0; j < n_kv; ++j) {
-      const int s = j % NS;
-      if (j >= NS && !wait_warp(&bar_empty[s], ((j / NS) - 1) & 1, wc, kErrWaitEmpty)) break;
-      uint8_t* st = smem + L::kStage0 + s * L::kStageBytes;
-      load_tile<D, F32IO, true>(st, p.K, b, j * kTileRows, g, p.T, p.Hkv, p.rope, pt);
-      load_tile<D, F32IO, false>(st + L::kParts * L::kTile, p.V, b, j * kTileRows, g, p.T, p.Hkv, nullptr, pt);
+  if (warp == 9) {
+    // ------------------------------------------------------------ TMA
+    if ((tid & 31) == 0) {
+      prefetch_tmap(&p.tm_q);
+      prefetch_tmap(&p.tm_k);
+      prefetch_tmap(&p.tm_v);
+      const int nq = has_b ? 2 : 1;
+      const bool rot = L::kConv && p.rope != nullptr;
+      const uint32_t rope_bytes = rot ? uint32_t(min(p.T, kRopeRows)) * (D / 2) * 8 : 0;
+      const uint32_t qbase_bytes = rot ? nq * L::kBase : 0;
+      const float2* base_table = rot ? p.rope + size_t(p.T) * (D / 2) : nullptr;
+      // a load of `row0` of tensor X: the tile (bf16) or its hi and lo planes
+      auto load_tile = [&](uint8_t* dst, const CUtensorMap* hi, const CUtensorMap* lo, int head, int row0,
+                           uint64_t* bar) {
+        tma_load_4d(dst, hi, 0, head, row0, b, bar);
+        if (F32IO) tma_load_4d(dst + OPB, lo, 0, head, row0, b, bar);
+      };
+      // fault-injection hook: withhold the query tiles so every wait on them
+      // runs into its limit
+      const bool q_armed = !(p.debug & 1);
+      if (q_armed) {
+        mbar_arrive_expect_tx(bar_qtma, nq * L::kTile + rope_bytes + qbase_bytes);
+        load_tile(smem + L::kQA, &p.tm_q, &p.tm_q_lo, h, qt_a * kTileRows, bar_qtma);
+        if (has_b) load_tile(smem + L::kQB, &p.tm_q, &p.tm_q_lo, h, qt_b * kTileRows, bar_qtma);
+        if (rot) {
+          bulk_load(smem + L::kRope, p.rope, rope_bytes, bar_qtma);
+          bulk_load(smem + L::kQBase, base_table + size_t(2 * qt_a) * (D / 2), qbase_bytes, bar_qtma);
+        }
+      }
+      int armed_k = 0, armed_v = 0;
+      for (int j = 0; j < n_kv; ++j) {
+        const int sk = j % NK, sv = j % NV;
+        if (j >= NK && !wait_thread(&bar_kempty[sk], ((j / NK) - 1) & 1, wc, kErrWaitEmpty)) break;
+        uint8_t* kst = smem + L::kK0 + sk * L::kKStage;
+        mbar_arrive_expect_tx(&bar_ktma[sk], L::kTile + (rot ? L::kBase : 0));
+        load_tile(kst, &p.tm_k, &p.tm_k_lo, g, j * kTileRows, &bar_ktma[sk]);
+        if (rot) bulk_load(kst + L::kTile, base_table + size_t(2 * j) * (D / 2), L::kBase, &bar_ktma[sk]);
+        NEA_TRACE_STAMP(p, 52 + min(j, 7), true);
+        armed_k = j + 1;
+        if (j >= NV && !wait_thread(&bar_vempty[sv], ((j / NV) - 1) & 1, wc, kErrWaitEmpty)) break;
+        mbar_arrive_expect_tx(&bar_vtma[sv], L::kTile);
+        load_tile(smem + L::kV0 + sv * L::kVStage, &p.tm_v, &p.tm_v_lo, g, j * kTileRows, &bar_vtma[sv]);
+        NEA_TRACE_STAMP(p, 60 + min(j, 7), true);
+        armed_v = j + 1;
+      }
+      // never leave copies in flight: on an abort, wait (bounded) for every
+      // load still outstanding before the CTA exits
+      if (*abort_flag) {
+        for (int j = max(0, armed_k - NK); j < armed_k; ++j) drain_wait(&bar_ktma[j % NK], (j / NK) & 1, wc);
+        for (int j = max(0, armed_v - NV); j < armed_v; ++j) drain_wait(&bar_vtma[j % NV], (j / NV) & 1, wc);
+        if (q_armed) drain_wait(bar_qtma, 0, wc);
+      }
+    }
+    __syncwarp();
+  } else if (L::kConv && warp >= 10) {
+    // ------------------------------------------------------------ converter (bf16: in-place RoPE)
+    const int pt = tid - 320;
+    uint32_t conv_count = 0;  // unused: bf16 tiles need no rendezvous
+    const float2* qbase = p.rope ? reinterpret_cast<const float2*>(smem + L::kQBase) : nullptr;
+    bool ok = wait_warp(bar_qtma, 0, wc, kErrWaitProducer);
+    if (ok) {
+      prepare_tile<D, false, true>(smem + L::kQA, rope_off, qbase, qt_a * kTileRows, p.T, nullptr, conv_count,
+                                   wc, pt);
+      if (has_b)
+        prepare_tile<D, false, true>(smem + L::kQB, rope_off, qbase ? qbase + 2 * (D / 2) : nullptr,
+                                     qt_b * kTileRows, p.T, nullptr, conv_count, wc, pt);
       fence_async_smem();
-      mbar_arrive(&bar_full[s]);
+      mbar_arrive(bar_qconv);
+      NEA_TRACE_STAMP(p, 2, pt == 0);
+    }
+    for (int j = 0; ok && j < n_kv; ++j) {
+      const int sk = j % NK;
+      if (!wait_warp(&bar_ktma[sk], (j / NK) & 1, wc, kErrWaitProducer)) break;
+      uint8_t* kst = smem + L::kK0 + sk * L::kKStage;
+      const float2* kbase = p.rope ? reinterpret_cast<const float2*>(kst + L::kTile) : nullptr;
+      prepare_tile<D, false, true>(kst, rope_off, kbase, j * kTileRows, p.T, nullptr, conv_count, wc, pt);
+      fence_async_smem();
+      mbar_arrive(&bar_kconv[sk]);
+      NEA_TRACE_STAMP(p, 36 + min(j, 7), pt == 0);
     }
   } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issuer
     if ((tid & 31) == 0) {
       constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
       constexpr uint32_t idO = idesc_bf16(128, D, 0, 1);
-      const uint32_t sQ = smem_u32(smem + L::kQ);
-      auto issue_s = [&](int j) -> bool {
-        const int s = j % NS;
-        if (!wait_thread(&bar_full[s], (j / NS) & 1, wc, kErrWaitProducer)) return false;
-        tc_fence_after();
-        const uint32_t sK = smem_u32(smem + L::kStage0 + s * L::kStageBytes);
-        const uint32_t dS = tbase + (j & 1) * 128;
+      const uint32_t sQ[2] = {smem_u32(smem + L::kQA), smem_u32(smem + L::kQB)};
+      auto issue_s = [&](int x, int j) {
+        const uint32_t sK = smem_u32(smem + L::kK0 + (j % NK) * L::kKStage);
+        const uint32_t dS = tbase + 256 * x;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
 #pragma unroll
           for (int term = 0; term < kTerms; ++term) {
             // float32 storage: hi*hi + hi*lo + lo*hi
-            const uint32_t qa = sQ + (term == 2 ? L::kTile : 0) + kk * 32;
-            const uint32_t kb = sK + (term == 1 ? L::kTile : 0) + kk * 32;
+            const uint32_t qa = sQ[x] + (term == 2 ? OPB : 0) + kk * 32;
+            const uint32_t kb = sK + (term == 1 ? OPB : 0) + kk * 32;
             mma_ss(dS, smem_desc(qa, RB, 16), smem_desc(kb, RB, 16), idS, (kk | term) != 0);
           }
         }
-        tc_commit(&bar_s[j & 1]);
-        return true;
+        tc_commit(&bar_s[x]);
       };
-      bool ok = wait_thread(bar_q, 0, wc, kErrWaitProducer) && issue_s(0);
-      for (int j = 0; ok && j < n_kv; ++j) {
-        if (j + 1 < n_kv) {
-          // the score buffer of tile j+1 still holds P_{j-1}: wait for PV_{j-1}
-          if (j >= 1 && !wait_thread(bar_o, (j - 1) & 1, wc, kErrWaitMma)) break;
-          if (!issue_s(j + 1)) break;
-        }
-        if (!wait_thread(&bar_p[j & 1], (j >> 1) & 1, wc, kErrWaitSoftmax)) break;
+      bool ok = wait_thread(bar_qready, 0, wc, kErrWaitProducer) &&
+                wait_thread(&bar_kready[0], 0, wc, kErrWaitProducer);
+      if (ok) {
         tc_fence_after();
-        const int s = j % NS;
-        const uint32_t sV = smem_u32(smem + L::kStage0 + s * L::kStageBytes + L::kParts * L::kTile);
-        const uint32_t pcol = tbase + (j & 1) * 128;
+        issue_s(0, 0);
+        if (has_b) issue_s(1, 0);
+        tc_commit(&bar_kempty[0]);
+      }
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const int sv = j % NV;
+        if (!wait_thread(&bar_vtma[sv], (j / NV) & 1, wc, kErrWaitProducer)) break;
+        const uint32_t sV = smem_u32(smem + L::kV0 + sv * L::kVStage);
+        bool next_k = false;
+        for (int x = 0; ok && x < 2; ++x) {
+          if (!active(x, j)) continue;
+          if (!wait_thread(&bar_p[x], j & 1, wc, kErrWaitSoftmax)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t phi = tbase + 256 * x, plo = tbase + 256 * x + 192, dO = tbase + 256 * x + 128;
 #pragma unroll
-        for (int kk = 0; kk < kTileRows / 16; ++kk) {
+          for (int kk = 0; kk < kTileRows / 16; ++kk) {
 #pragma unroll
-          for (int term = 0; term < kTerms; ++term) {
-            // float32 storage: Phi*Vhi + Phi*Vlo + Plo*Vhi
-            const uint32_t pa = pcol + (term == 2 ? 64 : 0) + kk * 8;
-            const uint32_t vb = sV + (term == 1 ? L::kTile : 0) + kk * 16 * RB;
-            mma_ts(tbase + kColO, pa, smem_desc(vb, RB, kTileRows * RB), idO, (j | kk | term) != 0);
+            for (int term = 0; term < kTerms; ++term) {
+              // float32 storage: Phi*Vhi + Phi*Vlo + Plo*Vhi
+              const uint32_t pa = (term == 2 ? plo : phi) + kk * 8;
+              const uint32_t vb = sV + (term == 1 ? OPB : 0) + kk * 16 * RB;
+              mma_ts(dO, pa, smem_desc(vb, RB, kTileRows * RB), idO, (j | kk | term) != 0);
+            }
+          }
+          tc_commit(&bar_o[x]);
+          NEA_TRACE_STAMP(p, 68 + min(j, 7), x == 0);
+          if (active(x, j + 1)) {
+            if (!next_k) {
+              const int sk = (j + 1) % NK;
+              if (!wait_thread(&bar_kready[sk], ((j + 1) / NK) & 1, wc, kErrWaitProducer)) { ok = false; break; }
+              next_k = true;
+            }
+            // S_X(j+1) overwrites P_X(j): wait until PV_X(j) has read it
+            if (!wait_thread(&bar_o[x], j & 1, wc, kErrWaitMma)) { ok = false; break; }
+            tc_fence_after();
+            issue_s(x, j + 1);
           }
         }
-        tc_commit(bar_o);
-        tc_commit(&bar_empty[s]);
+        if (!ok) break;
+        tc_commit(&bar_vempty[sv]);
+        if (next_k) tc_commit(&bar_kempty[(j + 1) % NK]);
       }
       tc_commit(bar_fin);
-      wait_thread(bar_fin, 0, wc, kErrWaitMma);
+      drain_wait(bar_fin, 0, wc);
     }
     __syncwarp();
-  } else {
-    // ------------------------------------------------------------ softmax
-    const int r = tid;  // query row inside the tile, TMEM lane
-    const int q = qt * kTileRows + r;
-    const uint32_t lane_base = tmem_addr(tbase, uint32_t(warp) * 32, 0);
-    float m_run = -INFINITY, l_run = 0.f;
-    bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      if (!wait_warp(&bar_s[j & 1], (j >> 1) & 1, wc, kErrWaitMma)) { ok = false; break; }
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ softmax (warps 0-7)
+    const int x = warp >> 2;   // query tile A or B
+    const int r = tid & 127;   // row inside the tile, TMEM lane
+    const int my_qt = x ? qt_b : qt_a, my_nkv = x ? nkv_b : nkv_a;
+    const int q = my_qt * kTileRows + r;
+    const uint32_t lane_base = tmem_addr(tbase, uint32_t(warp & 3) * 32, 0);
+    const uint32_t scol = lane_base + 256 * x, ocol = scol + 128, plocol = scol + 192;
+    float m_run = -INFINITY, l0 = 0.f, l1 = 0.f;
+    bool ok = x == 0 || has_b;
+    for (int j = 0; ok && j < my_nkv; ++j) {
+      if (!wait_warp(&bar_s[x], j & 1, wc, kErrWaitMma)) { ok = false; break; }
+      NEA_TRACE_STAMP(p, 4 + 16 * x + 2 * min(j, 7), r == 0);
       tc_fence_after();
-      const uint32_t scol = lane_base + (j & 1) * 128;
-      float s[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(scol + 32 * c, rr);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(rr[i]);
-      }
       const int kv0 = j * kTileRows;
-      if ((p.causal && j == qt) || kv0 + kTileRows > p.T) {
-        const int lim = p.causal ? min(q, p.T - 1) : p.T - 1;  // last visible key
+      const bool need_mask = (p.causal && j == my_qt) || kv0 + kTileRows > p.T;
+      const int lim = (p.causal ? min(q, p.T - 1) : p.T - 1) - kv0;  // last visible column
+      // pass 1: row maximum
+      float mx = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (kv0 + c > lim) s[c] = -INFINITY;
+      for (int c = 0; c < 2; ++c) {
+        uint32_t rr[64];
+        tmem_ld64(scol + 64 * c, rr);
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const float v = __uint_as_float(rr[i]);
+          mx = fmaxf(mx, (need_mask && 64 * c + i > lim) ? -INFINITY : v);
+        }
       }
-      float mx = s[0];
-#pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
       const float m_tile = mx * p.scale_log2;
       float alpha = 1.f;
       if (m_tile > m_run + 8.f) {  // keep a stale max unless it grew by > 2^8
         alpha = ex2(m_run - m_tile);
         m_run = m_tile;
       }
-      l_run *= alpha;
+      l0 *= alpha;
+      l1 *= alpha;
+      // pass 2: P = exp2(s * scale_log2 - m) -> bf16 (hi over S, lo apart)
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(scol + 32 * c, rr);
         uint32_t hi[16], lo[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2(fmaf(s[32 * c + 2 * i], p.scale_log2, -m_run));
-          const float p1 = ex2(fmaf(s[32 * c + 2 * i + 1], p.scale_log2, -m_run));
-          l_run += p0 + p1;
+          const int c0 = 32 * c + 2 * i;
+          float p0 = ex2(fmaf(__uint_as_float(rr[2 * i]), p.scale_log2, -m_run));
+          float p1 = ex2(fmaf(__uint_as_float(rr[2 * i + 1]), p.scale_log2, -m_run));
+          if (need_mask) {
+            p0 = (c0 > lim) ? 0.f : p0;
+            p1 = (c0 + 1 > lim) ? 0.f : p1;
+          }
+          l0 += p0;
+          l1 += p1;
           if (F32IO) {
             split_bf16(p0, p1, hi[i], lo[i]);
           } else {
             hi[i] = pack_bf16(p0, p1);
           }
         }
+        // columns [16c, 16c+16) of S were read in chunk c/2 <= c already
         tmem_st16(scol + 16 * c, hi);
-        if (F32IO) tmem_st16(scol + 64 + 16 * c, lo);
+        if (F32IO) tmem_st16(plocol + 16 * c, lo);
       }
       if (__any_sync(kFullMask, alpha != 1.f && j > 0)) {
-        // O holds sum over tiles < j: wait until PV_{j-1} has landed, rescale
-        if (!wait_warp(bar_o, (j - 1) & 1, wc, kErrWaitMma)) { ok = false; break; }
+        // O holds the sum over tiles < j: PV_X(j-1) has landed (S_X(j) was
+        // issued after it); rescale
+        if (!wait_warp(&bar_o[x], (j - 1) & 1, wc, kErrWaitMma)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t rr[32];
-          tmem_ld32(lane_base + kColO + 32 * c, rr);
+          tmem_ld32(ocol + 32 * c, rr);
 #pragma unroll
           for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
-          tmem_st32(lane_base + kColO + 32 * c, rr);
+          tmem_st32(ocol + 32 * c, rr);
         }
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bar_p[j & 1]);
+      mbar_arrive(&bar_p[x]);
+      NEA_TRACE_STAMP(p, 5 + 16 * x + 2 * min(j, 7), r == 0);
     }
-    // bar_o can trail by two phases here; the issuer's final commit cannot.
-    if (ok && wait_warp(bar_fin, 0, wc, kErrWaitMma)) {
+    if (ok && (x == 0 || has_b) && wait_warp(&bar_o[x], (my_nkv - 1) & 1, wc, kErrWaitMma)) {
       tc_fence_after();
       float o[D];
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t rr[32];
-        tmem_ld32(lane_base + kColO + 32 * c, rr);
+        tmem_ld32(ocol + 32 * c, rr);
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[32 * c + i] = __uint_as_float(rr[i]);
       }
       if (q < p.T) {
+        const float l_run = l0 + l1;
         const float inv = 1.f / l_run;
 #pragma unroll
         for (int i = 0; i < D; ++i) o[i] *= inv;
@@ -265,6 +440,7 @@ __global__ void __launch_bounds__(288, 1) attn_fwd_kernel(const __grid_constant_
         // LSE = ln(2^m * l) with m in log2 units of the scaled scores
         p.LSE[(size_t(b) * p.Hq + h) * p.T + q] = (m_run + log2f(l_run)) * 0.69314718055994531f;
       }
+      NEA_TRACE_STAMP(p, 76 + x, r == 0);
     }
   }
   tc_fence_before();
@@ -273,6 +449,7 @@ __global__ void __launch_bounds__(288, 1) attn_fwd_kernel(const __grid_constant_
     tc_fence_after();
     tmem_dealloc(tbase, 512);
   }
+  NEA_TRACE_STAMP(p, 78, tid == 0);
 }
 
 }  // namespace nea

@@ -25,13 +25,15 @@
  *
  * Ownership: every pointer is a device pointer owned by the caller; the
  * library never frees or retains them.  The library keeps, per device, a
- * cached workspace (the rotary cos/sin table and the backward's row term
- * D_i = sum_d dO_id O_id), allocated on first use and grown only when a call
- * needs more; steady-state calls allocate nothing.
+ * cached workspace (the rotary cos/sin tables, the backward's per-row terms
+ * and, for NEA_F32, the bf16 hi/lo operand planes), allocated on first use and
+ * grown only when a call needs more; steady-state calls allocate nothing.
  *
  * Streams: work is enqueued on `stream` (a cudaStream_t, NULL for the legacy
- * default stream) and the call returns without synchronising.  Device-side
- * wait limits are reported asynchronously: see nea_device_status().
+ * default stream) and the call returns without synchronising.  Calls on one
+ * device share its workspace, so calls on different streams must not overlap
+ * in time.  Device-side wait limits are reported asynchronously: see
+ * nea_device_status().
  *
  * Errors: a call returns NEA_OK or one of the codes below; on NEA_ERR_ARG
  * nothing is launched and no output is touched.  Kernels never trap.
@@ -75,9 +77,12 @@ enum {
  *   causal      1: key j visible to query i iff j <= i; 0: all keys visible
  *   stream      cudaStream_t to enqueue on
  *
- * NEA_F32: each score and output contraction is formed from bf16 high and
- * low parts of its fp32 operands (hi*hi + hi*lo + lo*hi, fp32 accumulation),
- * about 2^-16 relative per product.  NEA_BF16: plain bf16 products.
+ * NEA_BF16: plain bf16 tensor-core products, fp32 accumulation; the rotation
+ * is applied to each Q/K tile as it is staged in shared memory.
+ * NEA_F32: an operand prologue kernel first rotates Q and K and writes Q, K,
+ * V as bf16 high and low planes in the workspace; each score and output
+ * contraction is then formed from them as hi*hi + hi*lo + lo*hi (fp32
+ * accumulation), about 2^-16 relative per product.
  */
 int nea_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int T, int Hq,
                  int Hkv, int D, int dtype, float rope_base, int causal, void* stream);
@@ -90,13 +95,13 @@ int nea_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
  * dV the shape of K.  O and LSE must be the forward's results for the same
  * Q, K, V, rope_base and causal.
  *
- * Runs three kernels on `stream`: the row term D_i = sum_d dO_id O_id, the
- * dK/dV kernel (one CTA per key tile and kv head, looping over the query
- * heads of the group), and the dQ kernel (one CTA per query tile and head);
- * both recompute P from LSE.
+ * Runs on `stream`: (NEA_F32) the operand prologue over Q, K, V, dO; the row
+ * terms LSE*log2(e) and D_i = sum_d dO_id O_id; the dK/dV kernel (one CTA per
+ * key tile and kv head, looping over the query heads of the group); the dQ
+ * kernel (one CTA per query tile and head); both recompute P from LSE.
  *
  * NEA_F32: the score product and dO V^T use split bf16 (as in the forward);
- * the three gradient products use single bf16 operands with fp32
+ * the three gradient products use the bf16 high parts with fp32
  * accumulation.
  */
 int nea_attn_bwd(const void* Q, const void* K, const void* V, const void* O, const float* LSE, const void* dO,
@@ -130,9 +135,13 @@ void nea_debug_inject(int flags);
  * Profiling hook.  `events` points at `n` cudaEvent_t handles owned by the
  * caller (NULL / 0 disables).  While set, later calls on this host thread
  * record them on their stream at kernel boundaries:
- *   nea_attn_fwd: events[0] before, events[1] after the forward kernel;
- *   nea_attn_bwd: events[2] before the row-term kernel, events[3] after it,
- *                 events[4] after the dK/dV kernel, events[5] after the dQ kernel.
+ *   nea_attn_fwd: events[0] before the first kernel (the NEA_F32 operand
+ *                 prologue, else the forward kernel), events[1] after the
+ *                 forward kernel;
+ *   nea_attn_bwd: events[2] before the first kernel (NEA_F32 operand
+ *                 prologue, else the row-term kernel), events[3] after the
+ *                 row-term kernel, events[4] after the dK/dV kernel,
+ *                 events[5] after the dQ kernel.
  * Indices >= n are skipped.  The array must stay valid while set.
  */
 void nea_set_profile_events(void* const* events, int n);
@@ -146,13 +155,15 @@ void nea_set_profile_events(void* const* events, int n);
  * whose allocations would synchronise or fragment the device at a bad time.
  *
  * Same arguments, layouts and results as nea_attn_bwd.  The caller passes all
- * inputs and outputs; everything else the backward needs (the row term
- * D_i = sum_d dO_id O_id, the rotary cos/sin table, computed on the device in
- * double precision, and a device status word) lives in one fixed array of
- * 4 MiB (1048576 floats) compiled into the library: every GPU that loads the
- * library keeps it until the process exits.  A call needs
- * 64 + B*Hq*T + T*D floats of it (rounded up to multiples of 4); larger
- * problems return NEA_ERR_SCRATCH_LIMIT before anything is launched.
+ * inputs and outputs; everything else the backward needs (the per-row terms
+ * LSE*log2(e) and D_i = sum_d dO_id O_id, the rotary cos/sin table, computed
+ * on the device in double precision, a device status word and, for NEA_F32,
+ * the bf16 hi/lo planes of Q, K, V, dO) lives in one fixed array of 4 MiB
+ * compiled into the library: every GPU that loads the library keeps it until
+ * the process exits.  With Tp = 128*ceil(T/128), a call needs about
+ * 256 + 8*B*Hq*Tp + 4*(T + 2*ceil(T/128))*D bytes of it, plus
+ * 8*B*T*(Hq + Hkv)*D bytes for NEA_F32 (each part rounded up to 256 bytes);
+ * larger problems return NEA_ERR_SCRATCH_LIMIT before anything is launched.
  *
  * The first call on a device does a one-time set-up with that device
  * current (it looks up the array's device address and sets kernel
