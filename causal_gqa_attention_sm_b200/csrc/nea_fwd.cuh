@@ -22,12 +22,12 @@
 //              for float32 storage); the running max m moves only when it
 //              grows by more than 2^8 (O rescaled in TMEM then); the epilogue
 //              writes O / l and LSE.
-//   8          MMA issuer (one thread): S_X = Q_X K_j^T, O_X += P_X V_j for X
-//              in {A, B}, ping-ponging so one tile's softmax overlaps the
-//              other tile's MMAs.
-//   9          TMA: query tiles, then K and V tiles into two rings (K stages
+//   8, 9       MMA issuers, one thread each: warp 8 for tile A, warp 9 for tile B;
+//              S_X = Q_X K_j^T, O_X += P_X V_j, each waiting only on its own
+//              tile, so one tile's softmax overlaps the other tile's MMAs.
+//   10         TMA: query tiles, then K and V tiles into two rings (K stages
 //              free as soon as S is computed, V stages after PV).
-//   10-13      (bf16 only) converter: in-place RoPE of the Q and K tiles.
+//   11-14      (bf16 only) converter: in-place RoPE of the Q and K tiles.
 // TMEM per tile X: S [256X, 256X+128), O [256X+128, +D), P lo [256X+192, +64).
 // Causal tiles above the diagonal are never visited; only the diagonal tile
 // and a ragged last tile are masked.
@@ -102,13 +102,13 @@ struct FwdSmem {
   static constexpr uint32_t kVStage = kTile;
   static constexpr uint32_t kBars = kV0 + kNV * kVStage;
   // qtma, qready, K tma/full/empty, V tma/empty, s[2], p[2], o[2], fin
-  static constexpr int kNumBars = 2 + 3 * kNK + 2 * kNV + 6 + 1;
+  static constexpr int kNumBars = 2 + 3 * kNK + 2 * kNV + 6 + 2;
   static constexpr uint32_t kMisc = kBars + 8 * kNumBars;
   static constexpr uint32_t kUsed = kMisc + 16;
   // +1024 for manual alignment; at least 116 KB so two CTAs never share an SM
   // (each takes all 512 TMEM columns)
   static constexpr uint32_t kAlloc = kUsed + 1024 > 116u * 1024u ? kUsed + 1024 : 116u * 1024u;
-  static constexpr int kThreads = kConv ? 448 : 320;
+  static constexpr int kThreads = kConv ? 480 : 352;
   static_assert(kK0 % 1024 == 0 && kKStage % 1024 == 0 && kV0 % 1024 == 0 && kVStage % 1024 == 0,
                 "operand tiles need 1024-byte alignment");
   static_assert(2 * kBase <= 1024, "query base rows");
@@ -137,7 +137,7 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
   uint64_t* bar_s = bars + 2 + 3 * NK + 2 * NV;         // [2] S_X landed
   uint64_t* bar_p = bar_s + 2;                          // [2] P_X written (count 128)
   uint64_t* bar_o = bar_s + 4;                          // [2] PV_X done
-  uint64_t* bar_fin = bar_s + 6;
+  uint64_t* bar_fin = bar_s + 6;                        // [2] per issuer
   // what the MMA issuer waits for: converted tiles (bf16) or landed planes (fp32)
   uint64_t* bar_qready = L::kConv ? bar_qconv : bar_qtma;
   uint64_t* bar_kready = L::kConv ? bar_kconv : bar_ktma;
@@ -166,18 +166,19 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
     for (int s = 0; s < NK; ++s) {
       mbar_init(&bar_ktma[s], 1);
       mbar_init(&bar_kconv[s], 128);
-      mbar_init(&bar_kempty[s], 1);
+      mbar_init(&bar_kempty[s], has_b ? 2 : 1);  // one commit per tile using the stage
     }
     for (int s = 0; s < NV; ++s) {
       mbar_init(&bar_vtma[s], 1);
-      mbar_init(&bar_vempty[s], 1);
+      mbar_init(&bar_vempty[s], has_b ? 2 : 1);
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&bar_s[x], 1);
       mbar_init(&bar_p[x], 128);
       mbar_init(&bar_o[x], 1);
     }
-    mbar_init(bar_fin, 1);
+    mbar_init(&bar_fin[0], 1);
+    mbar_init(&bar_fin[1], 1);
     mbar_init_fence();
   }
   if (warp == 0) tmem_alloc(tmem_holder, 512);
@@ -187,7 +188,7 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
   const uint32_t tbase = *tmem_holder;
   NEA_TRACE_STAMP(p, 1, tid == 0);
 
-  if (warp == 9) {
+  if (warp == 10) {
     // ------------------------------------------------------------ TMA
     if ((tid & 31) == 0) {
       prefetch_tmap(&p.tm_q);
@@ -241,9 +242,9 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (L::kConv && warp >= 10) {
+  } else if (L::kConv && warp >= 11) {
     // ------------------------------------------------------------ converter (bf16: in-place RoPE)
-    const int pt = tid - 320;
+    const int pt = tid - 352;
     uint32_t conv_count = 0;  // unused: bf16 tiles need no rendezvous
     const float2* qbase = p.rope ? reinterpret_cast<const float2*>(smem + L::kQBase) : nullptr;
     bool ok = wait_warp(bar_qtma, 0, wc, kErrWaitProducer);
@@ -267,13 +268,20 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
       mbar_arrive(&bar_kconv[sk]);
       NEA_TRACE_STAMP(p, 36 + min(j, 7), pt == 0);
     }
-  } else if (warp == 8) {
-    // ------------------------------------------------------------ MMA issuer
-    if ((tid & 31) == 0) {
+  } else if (warp == 8 || warp == 9) {
+    // ------------------------------------------------------------ MMA issuers
+    // Issuer X runs tile X on its own: S_X(0); then per key tile j: wait for
+    // P_X(j), O_X += P_X(j) V_j; wait for that to finish reading P_X(j) (which
+    // S_X(j+1) overwrites), S_X(j+1).  Stage releases count one commit per
+    // tile; the last key tile of a causal pair is used by B alone, but its
+    // stages are never refilled, so no one waits for that release.
+    const int x = warp - 8;
+    if ((tid & 31) == 0 && (x == 0 || has_b)) {
       constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
       constexpr uint32_t idO = idesc_bf16(128, D, 0, 1);
-      const uint32_t sQ[2] = {smem_u32(smem + L::kQA), smem_u32(smem + L::kQB)};
-      auto issue_s = [&](int x, int j) {
+      const uint32_t sQ = smem_u32(smem + (x ? L::kQB : L::kQA));
+      const int my_nkv = x ? nkv_b : nkv_a;
+      auto issue_s = [&](int j) {
         const uint32_t sK = smem_u32(smem + L::kK0 + (j % NK) * L::kKStage);
         const uint32_t dS = tbase + 256 * x;
 #pragma unroll
@@ -281,7 +289,7 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
 #pragma unroll
           for (int term = 0; term < kTerms; ++term) {
             // float32 storage: hi*hi + hi*lo + lo*hi
-            const uint32_t qa = sQ[x] + (term == 2 ? OPB : 0) + kk * 32;
+            const uint32_t qa = sQ + (term == 2 ? OPB : 0) + kk * 32;
             const uint32_t kb = sK + (term == 1 ? OPB : 0) + kk * 32;
             mma_ss(dS, smem_desc(qa, RB, 16), smem_desc(kb, RB, 16), idS, (kk | term) != 0);
           }
@@ -292,50 +300,43 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
                 wait_thread(&bar_kready[0], 0, wc, kErrWaitProducer);
       if (ok) {
         tc_fence_after();
-        issue_s(0, 0);
-        if (has_b) issue_s(1, 0);
+        issue_s(0);
         tc_commit(&bar_kempty[0]);
       }
-      for (int j = 0; ok && j < n_kv; ++j) {
+      for (int j = 0; ok && j < my_nkv; ++j) {
         const int sv = j % NV;
-        if (!wait_thread(&bar_vtma[sv], (j / NV) & 1, wc, kErrWaitProducer)) break;
+        if (!wait_thread(&bar_p[x], j & 1, wc, kErrWaitSoftmax) ||
+            !wait_thread(&bar_vtma[sv], (j / NV) & 1, wc, kErrWaitProducer))
+          break;
+        tc_fence_after();
         const uint32_t sV = smem_u32(smem + L::kV0 + sv * L::kVStage);
-        bool next_k = false;
-        for (int x = 0; ok && x < 2; ++x) {
-          if (!active(x, j)) continue;
-          if (!wait_thread(&bar_p[x], j & 1, wc, kErrWaitSoftmax)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t phi = tbase + 256 * x, plo = tbase + 256 * x + 192, dO = tbase + 256 * x + 128;
+        const uint32_t phi = tbase + 256 * x, plo = tbase + 256 * x + 192, dO = tbase + 256 * x + 128;
 #pragma unroll
-          for (int kk = 0; kk < kTileRows / 16; ++kk) {
+        for (int kk = 0; kk < kTileRows / 16; ++kk) {
 #pragma unroll
-            for (int term = 0; term < kTerms; ++term) {
-              // float32 storage: Phi*Vhi + Phi*Vlo + Plo*Vhi
-              const uint32_t pa = (term == 2 ? plo : phi) + kk * 8;
-              const uint32_t vb = sV + (term == 1 ? OPB : 0) + kk * 16 * RB;
-              mma_ts(dO, pa, smem_desc(vb, RB, kTileRows * RB), idO, (j | kk | term) != 0);
-            }
-          }
-          tc_commit(&bar_o[x]);
-          NEA_TRACE_STAMP(p, 68 + min(j, 7), x == 0);
-          if (active(x, j + 1)) {
-            if (!next_k) {
-              const int sk = (j + 1) % NK;
-              if (!wait_thread(&bar_kready[sk], ((j + 1) / NK) & 1, wc, kErrWaitProducer)) { ok = false; break; }
-              next_k = true;
-            }
-            // S_X(j+1) overwrites P_X(j): wait until PV_X(j) has read it
-            if (!wait_thread(&bar_o[x], j & 1, wc, kErrWaitMma)) { ok = false; break; }
-            tc_fence_after();
-            issue_s(x, j + 1);
+          for (int term = 0; term < kTerms; ++term) {
+            // float32 storage: Phi*Vhi + Phi*Vlo + Plo*Vhi
+            const uint32_t pa = (term == 2 ? plo : phi) + kk * 8;
+            const uint32_t vb = sV + (term == 1 ? OPB : 0) + kk * 16 * RB;
+            mma_ts(dO, pa, smem_desc(vb, RB, kTileRows * RB), idO, (j | kk | term) != 0);
           }
         }
-        if (!ok) break;
+        tc_commit(&bar_o[x]);
         tc_commit(&bar_vempty[sv]);
-        if (next_k) tc_commit(&bar_kempty[(j + 1) % NK]);
+        NEA_TRACE_STAMP(p, 68 + min(j, 7), x == 0);
+        if (j + 1 < my_nkv) {
+          // S_X(j+1) overwrites P_X(j): wait until PV_X(j) has read it
+          const int sk = (j + 1) % NK;
+          if (!wait_thread(&bar_o[x], j & 1, wc, kErrWaitMma) ||
+              !wait_thread(&bar_kready[sk], ((j + 1) / NK) & 1, wc, kErrWaitProducer))
+            break;
+          tc_fence_after();
+          issue_s(j + 1);
+          tc_commit(&bar_kempty[sk]);
+        }
       }
-      tc_commit(bar_fin);
-      drain_wait(bar_fin, 0, wc);
+      tc_commit(&bar_fin[x]);
+      drain_wait(&bar_fin[x], 0, wc);
     }
     __syncwarp();
   } else if (warp < 8) {
