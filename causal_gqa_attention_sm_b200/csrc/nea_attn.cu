@@ -135,13 +135,8 @@ int device_state(DeviceState** out) {
   return NEA_OK;
 }
 
-// Rows of the rotary table: T positions, then two block-start rows per tile.
-size_t rope_rows(int T) { return size_t(T) + 2 * ((size_t(T) + nea::kTileRows - 1) / nea::kTileRows); }
-
-// Rotary table [T][D/2] of (cos, sin) of t * base^(-2i/D), computed in double,
-// followed by, per 128-row tile j, the rows of its two 64-row block starts
-// (j*128 and j*128+64, clamped to T-1), contiguous so a kernel can bulk-copy
-// a tile's bases in one piece.
+// Rotary table [T][D/2] of (cos, sin) of t * base^(-2i/D), angles computed
+// in double and rounded to float once.
 int rope_table(DeviceState& st, int T, int D, float base, cudaStream_t stream, const float2** out) {
   if (!(base > 0.f)) {
     *out = nullptr;
@@ -155,16 +150,12 @@ int rope_table(DeviceState& st, int T, int D, float base, cudaStream_t stream, c
     *out = it->second;
     return NEA_OK;
   }
-  std::vector<float2> h(rope_rows(T) * (D / 2));
+  std::vector<float2> h(size_t(T) * (D / 2));
   for (int t = 0; t < T; ++t)
     for (int i = 0; i < D / 2; ++i) {
       const double a = double(t) * std::pow(double(base), -2.0 * i / double(D));
       h[size_t(t) * (D / 2) + i] = make_float2(float(std::cos(a)), float(std::sin(a)));
     }
-  for (size_t r = 0; r + T < rope_rows(T); ++r) {
-    const int t = std::min(int(r) * nea::kRopeRows, T - 1);
-    std::memcpy(&h[(T + r) * (D / 2)], &h[size_t(t) * (D / 2)], sizeof(float2) * (D / 2));
-  }
   float2* d = nullptr;
   cudaError_t e = cudaMalloc(&d, h.size() * sizeof(float2));
   if (e != cudaSuccess) return cuda_fail(e);
@@ -231,42 +222,60 @@ int dispatch(int D, int dtype, F&& f) {
              : f(std::integral_constant<int, 32>{}, std::false_type{});
 }
 
-// ----------------------------------------------------------------- fp32 operand planes
-// Byte layout of the planes of `n` tensors of `elems[i]` elements: hi, then
-// lo, each 256-byte aligned.
-size_t planes_bytes(const size_t* elems, int n) {
+// ----------------------------------------------------------------- operand prologue
+// Workspace bytes the prologue writes for `n` tensors of `elems[i]` elements:
+// float32 storage, hi and lo planes of every tensor; bfloat16 storage, a
+// rotated copy of each tensor with rot[i] set (none when the rotation is off).
+// Every plane starts 256-byte aligned.
+size_t prep_bytes(const size_t* elems, const int* rot, int n, bool f32, bool rope_on) {
   size_t b = 0;
-  for (int i = 0; i < n; ++i) b += 2 * round_up(elems[i] * 2, 256);
+  for (int i = 0; i < n; ++i) {
+    if (f32) b += 2 * round_up(elems[i] * 2, 256);
+    else if (rot[i] && rope_on) b += round_up(elems[i] * 2, 256);
+  }
   return b;
 }
 
-// Carves the planes out of `base` and runs the operand prologue over the
-// tensors (rotating those with rope[i] set).
-int run_prep(uint8_t* base, const float* const* src, const size_t* elems, const int* H, const int* rope, int n,
-             int T, int D, const float2* table, nea::PrepJob* jobs_out, cudaStream_t stream) {
+// Carves the prologue's outputs out of `base` (prep_bytes() bytes) and runs
+// it.  jobs_out[i].hi (and .lo for float32 storage) are the operand tensors
+// the attention kernels read: for bfloat16 storage the rotated copy or, for
+// tensors left as they are, the input itself.
+int run_prep(uint8_t* base, const void* const* src, const size_t* elems, const int* H, const int* rot, int n,
+             int T, int D, bool f32, const float2* table, nea::PrepJob* jobs_out, cudaStream_t stream) {
   nea::PrepParams pp{};
   size_t off = 0;
-  pp.n_jobs = n;
   pp.T = T;
   pp.rope = table;
   for (int i = 0; i < n; ++i) {
-    nea::PrepJob& j = pp.job[i];
+    nea::PrepJob j{};
     j.src = src[i];
+    j.H = H[i];
+    j.rope = rot[i] && table != nullptr;
+    if (!f32 && !j.rope) {  // read in place
+      j.hi = static_cast<__nv_bfloat16*>(const_cast<void*>(src[i]));
+      jobs_out[i] = j;
+      continue;
+    }
     j.hi = reinterpret_cast<__nv_bfloat16*>(base + off);
     off += round_up(elems[i] * 2, 256);
-    j.lo = reinterpret_cast<__nv_bfloat16*>(base + off);
-    off += round_up(elems[i] * 2, 256);
-    j.chunks = static_cast<long long>(elems[i] / 4);
-    j.H = H[i];
-    j.rope = rope[i] && table != nullptr;
+    if (f32) {
+      j.lo = reinterpret_cast<__nv_bfloat16*>(base + off);
+      off += round_up(elems[i] * 2, 256);
+    }
+    j.chunks = static_cast<long long>(elems[i] / (f32 ? 4 : 8));
+    pp.job[pp.n_jobs++] = j;
     pp.total += j.chunks;
     jobs_out[i] = j;
   }
+  if (pp.n_jobs == 0) return NEA_OK;
   const long long blocks = std::min<long long>((pp.total + 255) / 256, 148LL * 16);
+  const unsigned g = unsigned(blocks);
   if (D == 64)
-    nea::attn_prep_split_kernel<64><<<unsigned(blocks), 256, 0, stream>>>(pp);
+    f32 ? nea::attn_prep_kernel<64, true><<<g, 256, 0, stream>>>(pp)
+        : nea::attn_prep_kernel<64, false><<<g, 256, 0, stream>>>(pp);
   else
-    nea::attn_prep_split_kernel<32><<<unsigned(blocks), 256, 0, stream>>>(pp);
+    f32 ? nea::attn_prep_kernel<32, true><<<g, 256, 0, stream>>>(pp)
+        : nea::attn_prep_kernel<32, false><<<g, 256, 0, stream>>>(pp);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? NEA_OK : cuda_fail(e);
 }
@@ -328,15 +337,16 @@ int check_bwd_args(const void* Q, const void* K, const void* V, const void* O, c
   return NEA_OK;
 }
 
-// Bytes of backward workspace: the padded row terms, then (fp32) the planes
-// of Q, K, V, dO.
-size_t bwd_ws_bytes(int B, int T, int Hq, int Hkv, int D, bool f32, size_t* rowterm_bytes) {
+// Bytes of backward workspace: the padded row terms, then the operand
+// prologue's output (fp32: planes of Q, K, V, dO; bf16 with the rotation on:
+// rotated Q and K).
+size_t bwd_ws_bytes(int B, int T, int Hq, int Hkv, int D, bool f32, bool rope_on, size_t* rowterm_bytes) {
   const size_t Tp = round_up(size_t(T), nea::kTileRows);
   *rowterm_bytes = round_up(size_t(B) * Hq * 2 * Tp * sizeof(float), 256);
-  if (!f32) return *rowterm_bytes;
   const size_t nq = size_t(B) * T * Hq * D, nk = size_t(B) * T * Hkv * D;
   const size_t elems[4] = {nq, nk, nk, nq};
-  return *rowterm_bytes + planes_bytes(elems, 4);
+  const int rot[4] = {1, 1, 0, 0};
+  return *rowterm_bytes + prep_bytes(elems, rot, 4, f32, rope_on);
 }
 
 // The backward after argument checks, given a workspace of bwd_ws_bytes()
@@ -346,32 +356,30 @@ int run_bwd(uint32_t& attr_done, uint8_t* ws, const float2* rope, int* status, c
             int T, int Hq, int Hkv, int D, int dtype, int causal, cudaStream_t stream, bool ev) {
   const bool f32 = dtype == NEA_F32;
   size_t rowterm_bytes = 0;
-  (void)bwd_ws_bytes(B, T, Hq, Hkv, D, f32, &rowterm_bytes);
+  (void)bwd_ws_bytes(B, T, Hq, Hkv, D, f32, rope != nullptr, &rowterm_bytes);
   nea::BwdParams p{};
   p.Tp = int(round_up(size_t(T), nea::kTileRows));
   p.ws = reinterpret_cast<const float*>(ws);
   int rc;
   if (ev) prof_record(2, stream);
-  if (f32) {
+  {
+    // operand prologue: rotated Q and K (float32 storage: hi/lo planes of
+    // rotated Q, K and of V, dO)
     const size_t nq = size_t(B) * T * Hq * D, nk = size_t(B) * T * Hkv * D;
-    const float* src[4] = {static_cast<const float*>(Q), static_cast<const float*>(K),
-                           static_cast<const float*>(V), static_cast<const float*>(dO)};
+    const void* src[4] = {Q, K, V, dO};
     const size_t elems[4] = {nq, nk, nk, nq};
     const int H[4] = {Hq, Hkv, Hkv, Hq}, rot[4] = {1, 1, 0, 0};
     nea::PrepJob jobs[4];
-    if ((rc = run_prep(ws + rowterm_bytes, src, elems, H, rot, 4, T, D, rope, jobs, stream))) return rc;
+    if ((rc = run_prep(ws + rowterm_bytes, src, elems, H, rot, 4, T, D, f32, rope, jobs, stream))) return rc;
     if ((rc = make_tile_map(&p.tm_q, jobs[0].hi, B, T, Hq, D)) ||
-        (rc = make_tile_map(&p.tm_q_lo, jobs[0].lo, B, T, Hq, D)) ||
         (rc = make_tile_map(&p.tm_k, jobs[1].hi, B, T, Hkv, D)) ||
-        (rc = make_tile_map(&p.tm_k_lo, jobs[1].lo, B, T, Hkv, D)) ||
         (rc = make_tile_map(&p.tm_v, jobs[2].hi, B, T, Hkv, D)) ||
-        (rc = make_tile_map(&p.tm_v_lo, jobs[2].lo, B, T, Hkv, D)) ||
-        (rc = make_tile_map(&p.tm_do, jobs[3].hi, B, T, Hq, D)) ||
-        (rc = make_tile_map(&p.tm_do_lo, jobs[3].lo, B, T, Hq, D)))
+        (rc = make_tile_map(&p.tm_do, jobs[3].hi, B, T, Hq, D)))
       return rc;
-  } else {
-    if ((rc = make_tile_map(&p.tm_q, Q, B, T, Hq, D)) || (rc = make_tile_map(&p.tm_k, K, B, T, Hkv, D)) ||
-        (rc = make_tile_map(&p.tm_v, V, B, T, Hkv, D)) || (rc = make_tile_map(&p.tm_do, dO, B, T, Hq, D)))
+    if (f32 && ((rc = make_tile_map(&p.tm_q_lo, jobs[0].lo, B, T, Hq, D)) ||
+                (rc = make_tile_map(&p.tm_k_lo, jobs[1].lo, B, T, Hkv, D)) ||
+                (rc = make_tile_map(&p.tm_v_lo, jobs[2].lo, B, T, Hkv, D)) ||
+                (rc = make_tile_map(&p.tm_do_lo, jobs[3].lo, B, T, Hq, D))))
       return rc;
   }
   if ((rc = make_rowterm_map(&p.tm_ws, p.ws, B * Hq, p.Tp))) return rc;
@@ -415,28 +423,26 @@ int nea_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
   DeviceState* st = nullptr;
   if ((rc = device_state(&st))) return rc;
   nea::FwdParams p{};
-  if ((rc = rope_table(*st, T, D, rope_base, stream, &p.rope))) return rc;
+  const float2* rope = nullptr;
+  if ((rc = rope_table(*st, T, D, rope_base, stream, &rope))) return rc;
   prof_record(0, stream);
-  if (f32) {
-    // operand prologue: rotated, split Q and K; split V
+  {
+    // operand prologue: rotated Q and K (float32 storage: hi/lo planes of
+    // rotated Q, K and of V)
     const size_t nq = size_t(B) * T * Hq * D, nk = size_t(B) * T * Hkv * D;
-    const float* src[3] = {static_cast<const float*>(Q), static_cast<const float*>(K),
-                           static_cast<const float*>(V)};
+    const void* src[3] = {Q, K, V};
     const size_t elems[3] = {nq, nk, nk};
     const int H[3] = {Hq, Hkv, Hkv}, rot[3] = {1, 1, 0};
-    if ((rc = ensure_ws(*st, planes_bytes(elems, 3)))) return rc;
+    if ((rc = ensure_ws(*st, prep_bytes(elems, rot, 3, f32, rope != nullptr)))) return rc;
     nea::PrepJob jobs[3];
-    if ((rc = run_prep(st->ws, src, elems, H, rot, 3, T, D, p.rope, jobs, stream))) return rc;
+    if ((rc = run_prep(st->ws, src, elems, H, rot, 3, T, D, f32, rope, jobs, stream))) return rc;
     if ((rc = make_tile_map(&p.tm_q, jobs[0].hi, B, T, Hq, D)) ||
-        (rc = make_tile_map(&p.tm_q_lo, jobs[0].lo, B, T, Hq, D)) ||
         (rc = make_tile_map(&p.tm_k, jobs[1].hi, B, T, Hkv, D)) ||
-        (rc = make_tile_map(&p.tm_k_lo, jobs[1].lo, B, T, Hkv, D)) ||
-        (rc = make_tile_map(&p.tm_v, jobs[2].hi, B, T, Hkv, D)) ||
-        (rc = make_tile_map(&p.tm_v_lo, jobs[2].lo, B, T, Hkv, D)))
+        (rc = make_tile_map(&p.tm_v, jobs[2].hi, B, T, Hkv, D)))
       return rc;
-  } else {
-    if ((rc = make_tile_map(&p.tm_q, Q, B, T, Hq, D)) || (rc = make_tile_map(&p.tm_k, K, B, T, Hkv, D)) ||
-        (rc = make_tile_map(&p.tm_v, V, B, T, Hkv, D)))
+    if (f32 && ((rc = make_tile_map(&p.tm_q_lo, jobs[0].lo, B, T, Hq, D)) ||
+                (rc = make_tile_map(&p.tm_k_lo, jobs[1].lo, B, T, Hkv, D)) ||
+                (rc = make_tile_map(&p.tm_v_lo, jobs[2].lo, B, T, Hkv, D))))
       return rc;
   }
   p.O = O;
@@ -478,7 +484,8 @@ int nea_attn_bwd(const void* Q, const void* K, const void* V, const void* O, con
   const float2* rope = nullptr;
   if ((rc = rope_table(*st, T, D, rope_base, stream, &rope))) return rc;
   size_t rowterm_bytes = 0;
-  if ((rc = ensure_ws(*st, bwd_ws_bytes(B, T, Hq, Hkv, D, dtype == NEA_F32, &rowterm_bytes)))) return rc;
+  if ((rc = ensure_ws(*st, bwd_ws_bytes(B, T, Hq, Hkv, D, dtype == NEA_F32, rope != nullptr, &rowterm_bytes))))
+    return rc;
   return run_bwd(st->attr_done, st->ws, rope, st->err, Q, K, V, O, LSE, dO, dQ, dK, dV, B, T, Hq, Hkv, D, dtype,
                  causal, stream, true);
 }
@@ -556,16 +563,13 @@ struct NoAllocDevice {
 NoAllocDevice g_noalloc_dev[kNoAllocMaxDevices];
 std::mutex g_noalloc_mu;
 
-// Rotary table [T][D/2] of (cos, sin) of t * base^(-2i/D), angles in double;
-// rows T .. rope_rows(T)-1 repeat the rows of the 64-row block starts
-// (row r -> position min(64 (r - T), T - 1)), as in the regular table.
+// Rotary table [T][D/2] of (cos, sin) of t * base^(-2i/D), angles in double,
+// as in the regular table.
 __global__ void noalloc_rope_table_kernel(float2* out, int T, int D, double base) {
   const long idx = long(blockIdx.x) * blockDim.x + threadIdx.x;
   const int half = D / 2;
-  const int rows = T + 2 * ((T + nea::kTileRows - 1) / nea::kTileRows);
-  if (idx >= long(rows) * half) return;
-  const int row = int(idx / half), i = int(idx % half);
-  const int t = row < T ? row : min((row - T) * nea::kRopeRows, T - 1);
+  if (idx >= long(T) * half) return;
+  const int t = int(idx / half), i = int(idx % half);
   const double a = double(t) * pow(base, -2.0 * double(i) / double(D));
   double sn, cs;
   sincos(a, &sn, &cs);
@@ -581,8 +585,9 @@ extern "C" int nea_attn_bwd_noalloc(const void* Q, const void* K, const void* V,
   int rc = check_bwd_args(Q, K, V, O, LSE, dO, dQ, dK, dV, B, T, Hq, Hkv, D, dtype, rope_base, causal, &empty);
   if (rc || empty) return rc;
   size_t rowterm_bytes = 0;
-  const size_t ws_bytes = bwd_ws_bytes(B, T, Hq, Hkv, D, dtype == NEA_F32, &rowterm_bytes);
-  const size_t rope_bytes = (rope_base > 0.f) ? round_up(rope_rows(T) * D * sizeof(float), 256) : 0;
+  const bool rope_on = rope_base > 0.f;
+  const size_t ws_bytes = bwd_ws_bytes(B, T, Hq, Hkv, D, dtype == NEA_F32, rope_on, &rowterm_bytes);
+  const size_t rope_bytes = rope_on ? round_up(size_t(T) * D * sizeof(float), 256) : 0;
   if (kNoAllocStatusBytes + ws_bytes + rope_bytes > kNoAllocScratchFloats * sizeof(float))
     return NEA_ERR_SCRATCH_LIMIT;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
@@ -618,7 +623,7 @@ extern "C" int nea_attn_bwd_noalloc(const void* Q, const void* K, const void* V,
   // fully rewritten by their kernels, so they need no clearing
   if ((e = cudaMemsetAsync(status, 0, sizeof(int), stream)) != cudaSuccess) return cuda_fail(e);
   if (rope) {
-    const long n = long(rope_rows(T)) * (D / 2);
+    const long n = long(T) * (D / 2);
     noalloc_rope_table_kernel<<<unsigned((n + 255) / 256), 256, 0, stream>>>(rope, T, D, double(rope_base));
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
   }

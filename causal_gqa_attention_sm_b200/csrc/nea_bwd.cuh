@@ -17,17 +17,20 @@
 //         over the GQA group needs no extra pass or atomics.
 //   DQ    row = query tile i of head h (Q'_i, dO_i), columns = key tiles
 //         j <= i (K'_j, V_j).
-// Operands arrive by TMA: bf16 storage lands tiles in the swizzled operand
-// layout and the converter warps rotate queries/keys in place (RoPE fused into
-// the tile load); float32 storage reads the pre-rotated bf16 hi/lo planes of
-// the operand prologue (nea_prep.cuh) and forms S and dP from three bf16
-// products, the gradient products from the hi parts.
-// Warps: 0-3 own the 128 rows (TMEM lanes), 4 issues the MMAs, 5 issues TMA
-// (resident tiles, then column tiles and, for DKDV, the LSE/Dv slices into a
-// ring), 6-9 (bf16 only) rotate tiles.
+// Operands arrive by TMA in the swizzled operand layout, already rotated by
+// the operand prologue (nea_prep.cuh): bf16 storage reads rotated copies of Q
+// and K and the inputs V, dO; float32 storage reads the bf16 hi/lo planes and
+// forms S and dP from three bf16 products, the gradient products from the hi
+// parts.
+// Warps: 0-7 elementwise work, warp w on TMEM lanes 32 (w % 4) .. + 31 (its
+// rows) and columns 64 (w / 4) .. + 63 of the tile; 8 issues the MMAs; 9
+// issues TMA (resident tiles, then column tiles and, for DKDV, the LSE/Dv
+// slices into a ring).
 //   S_rc  = R1 C1^T      (R1 = K' or Q', C1 = Q' or K')   -> TMEM [0,128)
 //   dP_rc = R2 C2^T      (R2 = V or dO,  C2 = dO or V)    -> TMEM [128,256)
-//   P (bf16 hi, lo) is kept in TMEM [384,512); dS overwrites dP in place
+//   P is kept in fp32 registers for dS and, for DKDV, as bf16 in TMEM
+//   [384,448) for the dV product; each warp writes its bf16 dS over the first
+//   half of its own dP columns
 //   DKDV: acc1 += P  C2   (dV), acc2 += dS C1 (dK)   (C1, C2 as MN-major B)
 //   DQ:   acc1 += dS C1   (dQ)
 // S of item k+1 is issued as soon as the rows have read S of item k, so it
@@ -43,9 +46,9 @@ namespace nea {
 // ---------------------------------------------------------------- row term
 // Per-row terms of the backward, in a workspace ws[B*Hq][2][Tp] (Tp = T
 // rounded up to whole 128-row tiles, so a tile of it is one TMA box):
-//   ws[bh][0][t] = LSE[b][h][t] * log2(e)          (+inf for t >= T)
+//   ws[bh][0][t] = -LSE[b][h][t] * log2(e)          (-inf for t >= T)
 //   ws[bh][1][t] = Dv = sum_d dO[b][t][h][d] O[b][t][h][d]   (0 for t >= T)
-// The padding makes P = exp2(s*c - lse2) vanish for queries past T.  One group
+// The padding makes P = exp2(s*c + ws0) vanish for queries past T.  One group
 // of D/ELEMS lanes per (b, t, h) row, t over [0, Tp).
 template <int D, bool F32IO>
 __global__ void __launch_bounds__(256) attn_bwd_rowterm_kernel(const void* __restrict__ O,
@@ -66,7 +69,7 @@ __global__ void __launch_bounds__(256) attn_bwd_rowterm_kernel(const void* __res
   float* out = ws + (b * Hq + h) * 2 * long(Tp) + t;
   if (t >= T) {
     if (c == 0) {
-      out[0] = INFINITY;
+      out[0] = -INFINITY;
       out[Tp] = 0.f;
     }
     return;
@@ -91,14 +94,15 @@ __global__ void __launch_bounds__(256) attn_bwd_rowterm_kernel(const void* __res
 #pragma unroll
   for (int off = kLanes / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(group, acc, off);
   if (c == 0) {
-    out[0] = __ldg(LSE + (b * Hq + h) * long(T) + t) * 1.4426950408889634f;
+    out[0] = __ldg(LSE + (b * Hq + h) * long(T) + t) * -1.4426950408889634f;
     out[Tp] = acc;
   }
 }
 
 // ---------------------------------------------------------------- main kernel
 struct BwdParams {
-  // bf16 storage: the inputs.  float32 storage: the hi planes.
+  // bf16 storage: rotated Q, K (the inputs when the rotation is off), V, dO.
+  // float32 storage: the hi planes.
   CUtensorMap tm_q;    // [B][T][Hq][D]
   CUtensorMap tm_k;    // [B][T][Hkv][D]
   CUtensorMap tm_v;
@@ -114,9 +118,7 @@ struct BwdParams {
   void* dQ;
   void* dK;
   void* dV;
-  // rotary table [T][D/2] (+ block-start rows): in-place rotation of bf16
-  // tiles and the inverse rotation of dQ, dK
-  const float2* rope;
+  const float2* rope;  // rotary table [T][D/2] for the inverse rotation of dQ, dK; nullptr: off
   int B, T, Hq, Hkv, G;
   int n_tiles;
   int causal;
@@ -128,29 +130,61 @@ struct BwdParams {
 
 template <int D, bool F32IO, bool DKDV>
 struct BwdSmem {
-  static constexpr bool kConv = !F32IO;  // converter warps (in-place RoPE)
   static constexpr int kStages = F32IO ? 2 : 3;
   static constexpr uint32_t kTile = Stage<D, F32IO>::kBytes;
-  static constexpr uint32_t kBase = RopeBaseRows<D>::kBytes;
-  static constexpr uint32_t kSide = kConv ? 1024 : 0;
   static constexpr uint32_t kR1 = 0;
   static constexpr uint32_t kR2 = kR1 + kTile;
-  static constexpr uint32_t kR1Base = kR2 + kTile;  // rotary base rows of the row tile
-  static constexpr uint32_t kRope = kR1Base + kSide;
-  static constexpr uint32_t kStage0 = kRope + (kConv ? TileGeom<D>::kRopeBytes : 0);
-  static constexpr uint32_t kCBase = 2 * kTile;              // rotary base rows of C1
-  static constexpr uint32_t kColVec = kCBase + kSide;        // per-column LSE and Dv (DKDV)
+  static constexpr uint32_t kStage0 = kR2 + kTile;
+  static constexpr uint32_t kColVec = 2 * kTile;             // per-column -LSE*log2e and Dv (DKDV)
   static constexpr uint32_t kStageBytes = kColVec + (DKDV ? 1024 : 0);
   static constexpr uint32_t kBars = kStage0 + kStages * kStageBytes;
-  // res_tma, res, tma[S], full[S], empty[S], s, dp, p, ds, dk, fin
-  static constexpr int kNumBars = 2 + 3 * kStages + 6;
+  // rtma, tma[S], empty[S], s, dp, p, ds, dk, fin
+  static constexpr int kNumBars = 1 + 2 * kStages + 6;
   static constexpr uint32_t kMisc = kBars + 8 * kNumBars;
   static constexpr uint32_t kUsed = kMisc + 16;
   static constexpr uint32_t kAlloc = kUsed + 1024 > 116u * 1024u ? kUsed + 1024 : 116u * 1024u;
-  static constexpr int kThreads = kConv ? 320 : 192;
+  static constexpr int kThreads = 320;
   static_assert(kStage0 % 1024 == 0 && kStageBytes % 1024 == 0, "operand tiles need 1024-byte alignment");
   static_assert(kAlloc <= 232448, "shared memory");
 };
+
+// Writes N consecutive elements of a row held in registers (float) at
+// element offset `off` of a tensor in the storage type (16-byte aligned).
+template <int N, bool F32IO>
+__device__ __forceinline__ void store_span(void* dst, size_t off, const float* v) {
+  if constexpr (F32IO) {
+    float4* q = reinterpret_cast<float4*>(static_cast<float*>(dst) + off);
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i) q[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  } else {
+    uint4* q = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dst) + off);
+#pragma unroll
+    for (int i = 0; i < N / 8; ++i)
+      q[i] = make_uint4(pack_bf16(v[8 * i], v[8 * i + 1]), pack_bf16(v[8 * i + 2], v[8 * i + 3]),
+                        pack_bf16(v[8 * i + 4], v[8 * i + 5]), pack_bf16(v[8 * i + 6], v[8 * i + 7]));
+  }
+}
+
+// N consecutive TMEM columns of this thread's lane (N = 16, 32 or 64).
+template <int N>
+__device__ __forceinline__ void tmem_ld_n(uint32_t taddr, float* v) {
+  if constexpr (N == 64) {
+    uint32_t r[64];
+    tmem_ld64(taddr, r);
+#pragma unroll
+    for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+  } else if constexpr (N == 32) {
+    uint32_t r[32];
+    tmem_ld32(taddr, r);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  } else {
+    uint32_t r[16];
+    tmem_ld16(taddr, r);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+  }
+}
 
 template <int D, bool F32IO, bool DKDV>
 __global__ void __launch_bounds__(BwdSmem<D, F32IO, DKDV>::kThreads, 1)
@@ -164,22 +198,17 @@ __global__ void __launch_bounds__(BwdSmem<D, F32IO, DKDV>::kThreads, 1)
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
-  uint64_t* bar_rtma = bars + 0;             // resident tiles (+ rotary rows) landed
-  uint64_t* bar_rconv = bars + 1;            // resident tiles rotated (count 128)
-  uint64_t* bar_tma = bars + 2;              // [NS] column tiles landed
-  uint64_t* bar_conv = bars + 2 + NS;        // [NS] column tiles rotated (count 128)
-  uint64_t* bar_empty = bars + 2 + 2 * NS;   // [NS] MMAs done with the stage
-  uint64_t* bar_s = bars + 2 + 3 * NS;       // S landed
+  uint64_t* bar_rtma = bars + 0;             // resident tiles landed
+  uint64_t* bar_tma = bars + 1;              // [NS] column tiles landed
+  uint64_t* bar_empty = bars + 1 + NS;       // [NS] MMAs done with the stage
+  uint64_t* bar_s = bars + 1 + 2 * NS;       // S landed
   uint64_t* bar_dp = bar_s + 1;              // dP landed
-  uint64_t* bar_p = bar_s + 2;               // rows read S, wrote P (count 128)
-  uint64_t* bar_ds = bar_s + 3;              // rows wrote dS (count 128)
+  uint64_t* bar_p = bar_s + 2;               // rows read S, wrote P (count 256)
+  uint64_t* bar_ds = bar_s + 3;              // rows wrote dS (count 256)
   uint64_t* bar_dk = bar_s + 4;              // dS MMA of an item done
   uint64_t* bar_fin = bar_s + 5;
-  uint64_t* bar_res = L::kConv ? bar_rconv : bar_rtma;  // resident operands ready
-  uint64_t* bar_full = L::kConv ? bar_conv : bar_tma;   // column operands ready
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
-  const float2* rope_off = reinterpret_cast<const float2*>(smem + L::kRope);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -214,16 +243,14 @@ __global__ void __launch_bounds__(BwdSmem<D, F32IO, DKDV>::kThreads, 1)
   if (tid == 0) {
     *abort_flag = 0;
     mbar_init(bar_rtma, 1);
-    mbar_init(bar_rconv, 128);
     for (int s = 0; s < NS; ++s) {
       mbar_init(&bar_tma[s], 1);
-      mbar_init(&bar_conv[s], 128);
       mbar_init(&bar_empty[s], 1);
     }
     mbar_init(bar_s, 1);
     mbar_init(bar_dp, 1);
-    mbar_init(bar_p, 128);
-    mbar_init(bar_ds, 128);
+    mbar_init(bar_p, 256);
+    mbar_init(bar_ds, 256);
     mbar_init(bar_dk, 1);
     mbar_init(bar_fin, 1);
     mbar_init_fence();
@@ -233,9 +260,9 @@ __global__ void __launch_bounds__(BwdSmem<D, F32IO, DKDV>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_holder;
-  constexpr uint32_t kColS = 0, kColDP = 128, kColAcc1 = 256, kColAcc2 = 256 + D, kColP = 384, kColPlo = 448;
+  constexpr uint32_t kColS = 0, kColDP = 128, kColAcc1 = 256, kColAcc2 = 256 + D, kColP = 384;
 
-  if (warp == 5) {
+  if (warp == 9) {
     // ------------------------------------------------------------ TMA
     if ((tid & 31) == 0) {
       const CUtensorMap* m_r1 = DKDV ? &p.tm_k : &p.tm_q;
@@ -250,33 +277,24 @@ __global__ void __launch_bounds__(BwdSmem<D, F32IO, DKDV>::kThreads, 1)
       prefetch_tmap(m_r2);
       prefetch_tmap(m_c1);
       prefetch_tmap(m_c2);
-      const bool rot = L::kConv && p.rope != nullptr;
-      const uint32_t rope_bytes = rot ? uint32_t(min(p.T, kRopeRows)) * (D / 2) * 8 : 0;
-      const uint32_t base_bytes = rot ? L::kBase : 0;
-      const float2* base_table = rot ? p.rope + size_t(p.T) * (D / 2) : nullptr;
       auto load_tile = [&](uint8_t* dst, const CUtensorMap* hi, const CUtensorMap* lo, int head, int row0,
                            uint64_t* bar) {
         tma_load_4d(dst, hi, 0, head, row0, b, bar);
         if (F32IO) tma_load_4d(dst + OPB, lo, 0, head, row0, b, bar);
       };
-      mbar_arrive_expect_tx(bar_rtma, 2 * L::kTile + rope_bytes + base_bytes);
+      mbar_arrive_expect_tx(bar_rtma, 2 * L::kTile);
       load_tile(smem + L::kR1, m_r1, m_r1l, head_r, rt * kTileRows, bar_rtma);
       load_tile(smem + L::kR2, m_r2, m_r2l, head_r, rt * kTileRows, bar_rtma);
-      if (rot) {
-        bulk_load(smem + L::kRope, p.rope, rope_bytes, bar_rtma);
-        bulk_load(smem + L::kR1Base, base_table + size_t(2 * rt) * (D / 2), base_bytes, bar_rtma);
-      }
       int armed = 0;
       for (int k = 0; k < n_items; ++k) {
         const int s = k % NS;
         if (k >= NS && !wait_thread(&bar_empty[s], ((k / NS) - 1) & 1, wc, kErrWaitEmpty)) break;
         uint8_t* st = smem + L::kStage0 + s * L::kStageBytes;
         const int ch = item_head(k), ct = item_tile(k);
-        mbar_arrive_expect_tx(&bar_tma[s], 2 * L::kTile + base_bytes + (DKDV ? 1024 : 0));
+        mbar_arrive_expect_tx(&bar_tma[s], 2 * L::kTile + (DKDV ? 1024 : 0));
         load_tile(st, m_c1, m_c1l, ch, ct * kTileRows, &bar_tma[s]);
         load_tile(st + L::kTile, m_c2, m_c2l, ch, ct * kTileRows, &bar_tma[s]);
-        if (rot) bulk_load(st + L::kCBase, base_table + size_t(2 * ct) * (D / 2), base_bytes, &bar_tma[s]);
-        if (DKDV)  // LSE*log2e then Dv of the 128 queries of this column tile
+        if (DKDV)  // -LSE*log2e then Dv of the 128 queries of this column tile
           tma_load_3d(st + L::kColVec, &p.tm_ws, ct * kTileRows, 0, b * p.Hq + ch, &bar_tma[s]);
         armed = k + 1;
       }
@@ -286,29 +304,7 @@ __global__ void __launch_bounds__(BwdSmem<D, F32IO, DKDV>::kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (L::kConv && warp >= 6) {
-    // ------------------------------------------------------------ converter (bf16: in-place RoPE)
-    const int pt = tid - 192;
-    uint32_t conv_count = 0;  // unused: bf16 tiles need no rendezvous
-    const float2* r1base = p.rope ? reinterpret_cast<const float2*>(smem + L::kR1Base) : nullptr;
-    bool ok = wait_warp(bar_rtma, 0, wc, kErrWaitProducer);
-    if (ok) {
-      prepare_tile<D, false, true>(smem + L::kR1, rope_off, r1base, rt * kTileRows, p.T, nullptr, conv_count, wc,
-                                   pt);
-      fence_async_smem();
-      mbar_arrive(bar_rconv);
-    }
-    for (int k = 0; ok && k < n_items; ++k) {
-      const int s = k % NS;
-      if (!wait_warp(&bar_tma[s], (k / NS) & 1, wc, kErrWaitProducer)) break;
-      uint8_t* st = smem + L::kStage0 + s * L::kStageBytes;
-      const float2* cbase = p.rope ? reinterpret_cast<const float2*>(st + L::kCBase) : nullptr;
-      prepare_tile<D, false, true>(st, rope_off, cbase, item_tile(k) * kTileRows, p.T, nullptr, conv_count, wc,
-                                   pt);
-      fence_async_smem();
-      mbar_arrive(&bar_conv[s]);
-    }
-  } else if (warp == 4) {
+  } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issuer
     if ((tid & 31) == 0) {
       constexpr uint32_t idSS = idesc_bf16(128, 128, 0, 0);
@@ -316,23 +312,24 @@ __global__ void __launch_bounds__(BwdSmem<D, F32IO, DKDV>::kThreads, 1)
       const uint32_t sR1 = smem_u32(smem + L::kR1), sR2 = smem_u32(smem + L::kR2);
       constexpr uint32_t accG = DKDV ? kColAcc2 : kColAcc1;  // accumulator of dS C1
       auto stage_c1 = [&](int k) { return smem_u32(smem + L::kStage0 + (k % NS) * L::kStageBytes); };
-      // acc += dS_k C1_k, then release the stage of item k
+      // acc += dS_k C1_k, then release the stage of item k.  dS of columns
+      // [64h, 64h+64) sits in TMEM columns kColDP + 64h .. + 31.
       auto issue_ds = [&](int k) -> bool {
         if (!wait_thread(bar_ds, k & 1, wc, kErrWaitSoftmax)) return false;
         tc_fence_after();
         const uint32_t sC1 = stage_c1(k);
 #pragma unroll
         for (int kk = 0; kk < kTileRows / 16; ++kk)
-          mma_ts(tbase + accG, tbase + kColDP + kk * 8, smem_desc(sC1 + kk * 16 * RB, RB, kTileRows * RB), idAcc,
-                 (k | kk) != 0);
+          mma_ts(tbase + accG, tbase + kColDP + (kk >> 2) * 64 + (kk & 3) * 8,
+                 smem_desc(sC1 + kk * 16 * RB, RB, kTileRows * RB), idAcc, (k | kk) != 0);
         tc_commit(&bar_empty[k % NS]);
         tc_commit(bar_dk);
         return true;
       };
-      bool ok = wait_thread(bar_res, 0, wc, kErrWaitProducer);
+      bool ok = wait_thread(bar_rtma, 0, wc, kErrWaitProducer);
       for (int k = 0; ok && k < n_items; ++k) {
         const int s = k % NS;
-        if (!wait_thread(&bar_full[s], (k / NS) & 1, wc, kErrWaitProducer)) { ok = false; break; }
+        if (!wait_thread(&bar_tma[s], (k / NS) & 1, wc, kErrWaitProducer)) { ok = false; break; }
         // S_k overwrites S_{k-1}: the rows must have read it
         if (k > 0 && !wait_thread(bar_p, (k - 1) & 1, wc, kErrWaitSoftmax)) { ok = false; break; }
         tc_fence_after();
@@ -369,86 +366,98 @@ __global__ void __launch_bounds__(BwdSmem<D, F32IO, DKDV>::kThreads, 1)
       drain_wait(bar_fin, 0, wc);
     }
     __syncwarp();
-  } else if (warp < 4) {
-    // ------------------------------------------------------------ rows
-    const int r = tid;
+  } else {
+    // ------------------------------------------------------------ elementwise (warps 0-7)
+    const int hf = warp >> 2;            // column half
+    const int r = (warp & 3) * 32 + (tid & 31);
     const int row = rt * kTileRows + r;  // key position (DKDV) or query position (DQ)
-    const uint32_t lane_base = tmem_addr(tbase, uint32_t(warp) * 32, 0);
-    float row_lse2 = 0.f, row_dv = 0.f;
-    if (!DKDV) {  // padded rows read +inf / 0, so their P and dS vanish
+    const int cb = 64 * hf;              // first column of this warp
+    const uint32_t lane_base = tmem_addr(tbase, uint32_t(warp & 3) * 32, 0);
+    const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
+    uint64_t nl2_row = 0, dv_row = 0;
+    if (!DKDV) {  // padded rows read -inf / 0, so their P and dS vanish
       const float* w = p.ws + (size_t(b) * p.Hq + head_r) * 2 * p.Tp + row;
-      row_lse2 = __ldg(w);
-      row_dv = __ldg(w + p.Tp);
+      const float nl2 = __ldg(w), dv = __ldg(w + p.Tp);
+      nl2_row = f2_pack(nl2, nl2);
+      dv_row = f2_pack(dv, dv);
     }
     bool ok = true;
     for (int k = 0; k < n_items; ++k) {
       const int s = k % NS;
-      const float* colvec = reinterpret_cast<const float*>(smem + L::kStage0 + s * L::kStageBytes + L::kColVec);
+      const float4* colvec =
+          reinterpret_cast<const float4*>(smem + L::kStage0 + s * L::kStageBytes + L::kColVec) + cb / 4;
       const int ct = item_tile(k);
-      // DKDV reads the per-column LSE/Dv the TMA landed in the stage
+      // DKDV reads the per-column -LSE*log2e / Dv the TMA landed in the stage
       if (DKDV && !wait_warp(&bar_tma[s], (k / NS) & 1, wc, kErrWaitProducer)) { ok = false; break; }
       if (!wait_warp(bar_s, k & 1, wc, kErrWaitMma)) { ok = false; break; }
       tc_fence_after();
-      const int col0 = ct * kTileRows;
-      const bool diag = p.causal && ct == rt;
-      const bool tail = col0 + kTileRows > p.T;
-      // ---- P phase: P = exp2(s * scale_log2 - LSE*log2e), masked, kept in TMEM
+      const int col0 = ct * kTileRows + cb;  // position of this warp's first column
+      // ---- P phase: P = exp2(s * scale_log2 - LSE*log2e), masked
+      uint32_t sv[64];
+      tmem_ld64(lane_base + kColS + cb, sv);
+      if ((p.causal && ct == rt) || ct * kTileRows + kTileRows > p.T) {  // same for the whole tile
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(lane_base + kColS + 32 * c, rr);
-        uint32_t hi[16], lo[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float pv[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int cc = 32 * c + 2 * i + e;
-            const float l2 = DKDV ? colvec[cc] : row_lse2;  // +inf past T: P = 0
-            float v = ex2(fmaf(__uint_as_float(rr[2 * i + e]), p.scale_log2, -l2));
-            if (DKDV) {
-              if (diag && row > col0 + cc) v = 0.f;  // key after query
-            } else {
-              if ((diag && col0 + cc > row) || (tail && col0 + cc >= p.T)) v = 0.f;
-            }
-            pv[e] = v;
-          }
-          if (F32IO) {
-            split_bf16(pv[0], pv[1], hi[i], lo[i]);
-          } else {
-            hi[i] = pack_bf16(pv[0], pv[1]);
-          }
+        for (int i = 0; i < 64; ++i) {
+          // DKDV: key (row) after query (column); DQ: key (column) after query
+          // (row) or past T.  Queries past T have -inf row terms already.
+          const bool masked = DKDV ? (p.causal && row > col0 + i) : ((p.causal && col0 + i > row) || col0 + i >= p.T);
+          sv[i] = masked ? 0xff800000u : sv[i];
         }
-        tmem_st16(lane_base + kColP + 16 * c, hi);
-        if (F32IO) tmem_st16(lane_base + kColPlo + 16 * c, lo);
       }
-      tmem_st_wait();
+      float pv[64];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {  // four columns per step
+        uint64_t nl2a = nl2_row, nl2b = nl2_row;
+        if (DKDV) {
+          const float4 c = colvec[i];
+          nl2a = f2_pack(c.x, c.y);
+          nl2b = f2_pack(c.z, c.w);
+        }
+        float t0, t1, t2, t3;
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[4 * i]), __uint_as_float(sv[4 * i + 1])), sc2, nl2a), t0, t1);
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[4 * i + 2]), __uint_as_float(sv[4 * i + 3])), sc2, nl2b), t2, t3);
+        pv[4 * i] = ex2(t0);
+        pv[4 * i + 1] = ex2(t1);
+        pv[4 * i + 2] = ex2(t2);
+        pv[4 * i + 3] = ex2(t3);
+      }
+      if (DKDV) {  // bf16 P for the dV product
+        uint32_t ph[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ph[i] = pack_bf16(pv[2 * i], pv[2 * i + 1]);
+        tmem_st32(lane_base + kColP + 32 * hf, ph);
+        tmem_st_wait();
+      }
       tc_fence_before();
       mbar_arrive(bar_p);
       // ---- dS phase: dS = P (dP - Dv), bf16, over dP in TMEM
       if (!wait_warp(bar_dp, k & 1, wc, kErrWaitMma)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t rr[32], ph[16], pl[16];
-        tmem_ld32(lane_base + kColDP + 32 * c, rr);
-        tmem_ld16(lane_base + kColP + 16 * c, ph);
-        if (F32IO) tmem_ld16(lane_base + kColPlo + 16 * c, pl);
-        uint32_t pk[16];
+      for (int c = 0; c < 2; ++c) {
+        uint32_t rr[32], pk[16];
+        tmem_ld32(lane_base + kColDP + cb + 32 * c, rr);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int cc = 32 * c + 2 * i;
-          float p0 = bf16_lo_f(ph[i]), p1 = bf16_hi_f(ph[i]);
-          if (F32IO) {
-            p0 += bf16_lo_f(pl[i]);
-            p1 += bf16_hi_f(pl[i]);
+        for (int i = 0; i < 8; ++i) {  // four columns per step
+          const int e = 32 * c + 4 * i;
+          uint64_t dva = dv_row, dvb = dv_row;
+          if (DKDV) {
+            const float4 d = colvec[32 + e / 4];
+            dva = f2_pack(d.x, d.y);
+            dvb = f2_pack(d.z, d.w);
           }
-          const float d0 = DKDV ? colvec[128 + cc] : row_dv;
-          const float d1 = DKDV ? colvec[128 + cc + 1] : row_dv;
-          pk[i] = pack_bf16(p0 * (__uint_as_float(rr[2 * i]) - d0), p1 * (__uint_as_float(rr[2 * i + 1]) - d1));
+          float a0, a1, a2, a3;
+          f2_unpack(f2_mul(f2_pack(pv[e], pv[e + 1]),
+                           f2_sub(f2_pack(__uint_as_float(rr[4 * i]), __uint_as_float(rr[4 * i + 1])), dva)),
+                    a0, a1);
+          f2_unpack(f2_mul(f2_pack(pv[e + 2], pv[e + 3]),
+                           f2_sub(f2_pack(__uint_as_float(rr[4 * i + 2]), __uint_as_float(rr[4 * i + 3])), dvb)),
+                    a2, a3);
+          pk[2 * i] = pack_bf16(a0, a1);
+          pk[2 * i + 1] = pack_bf16(a2, a3);
         }
-        // columns [16c, 16c+16) of dP were read in chunk c/2 <= c already
-        tmem_st16(lane_base + kColDP + 16 * c, pk);
+        // packed columns [16c, 16c+16) of this warp's dP were read in chunk 0
+        tmem_st16(lane_base + kColDP + cb + 16 * c, pk);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -457,39 +466,48 @@ __global__ void __launch_bounds__(BwdSmem<D, F32IO, DKDV>::kThreads, 1)
     if (ok && wait_warp(bar_fin, 0, wc, kErrWaitMma)) {
       tc_fence_after();
       // TMEM loads are warp-collective: every lane loads, only valid rows store
-      float acc[D];
+      constexpr int DH = D / 2;
       if (DKDV) {
+        // half 0 writes the row of dV, half 1 the row of dK
+        float acc[D];
+        tmem_ld_n<D>(lane_base + (hf ? kColAcc2 : kColAcc1), acc);
+        if (hf) {
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t rr[32];
-          tmem_ld32(lane_base + kColAcc1 + 32 * c, rr);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) acc[32 * c + i] = __uint_as_float(rr[i]);
+          for (int i = 0; i < D; ++i) acc[i] *= p.scale;
         }
-        if (row < p.T) store_row<D, F32IO>(p.dV, b, row, head_r, p.T, p.Hkv, acc);
-      }
+        if (row < p.T) {
+          if (hf && p.rope) {
+            // gradient w.r.t. the un-rotated input: apply R_t^T
+            const float4* tp = reinterpret_cast<const float4*>(p.rope + size_t(row) * (D / 2));
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(lane_base + (DKDV ? kColAcc2 : kColAcc1) + 32 * c, rr);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) acc[32 * c + i] = __uint_as_float(rr[i]) * p.scale;
-      }
-      if (row < p.T) {
-        if (p.rope) {
-          // gradient w.r.t. the un-rotated input: apply R_t^T
-          const float4* tp = reinterpret_cast<const float4*>(p.rope + size_t(row) * (D / 2));
-#pragma unroll
-          for (int i = 0; i < D / 4; ++i) {
-            const float4 cs = __ldg(tp + i);
-            rot2(acc[4 * i], acc[4 * i + 1], cs.x, -cs.y);
-            rot2(acc[4 * i + 2], acc[4 * i + 3], cs.z, -cs.w);
+            for (int i = 0; i < D / 4; ++i) {
+              const float4 cs = __ldg(tp + i);
+              rot2(acc[4 * i], acc[4 * i + 1], cs.x, -cs.y);
+              rot2(acc[4 * i + 2], acc[4 * i + 3], cs.z, -cs.w);
+            }
           }
+          const size_t off = ((size_t(b) * p.T + row) * p.Hkv + head_r) * D;
+          store_span<D, F32IO>(hf ? p.dK : p.dV, off, acc);
         }
-        if (DKDV)
-          store_row<D, F32IO>(p.dK, b, row, head_r, p.T, p.Hkv, acc);
-        else
-          store_row<D, F32IO>(p.dQ, b, row, head_r, p.T, p.Hq, acc);
+      } else {
+        // half h writes columns [h D/2, h D/2 + D/2) of the row of dQ
+        float acc[DH];
+        tmem_ld_n<DH>(lane_base + kColAcc1 + DH * hf, acc);
+#pragma unroll
+        for (int i = 0; i < DH; ++i) acc[i] *= p.scale;
+        if (row < p.T) {
+          if (p.rope) {
+            const float4* tp = reinterpret_cast<const float4*>(p.rope + size_t(row) * (D / 2) + DH / 2 * hf);
+#pragma unroll
+            for (int i = 0; i < DH / 4; ++i) {
+              const float4 cs = __ldg(tp + i);
+              rot2(acc[4 * i], acc[4 * i + 1], cs.x, -cs.y);
+              rot2(acc[4 * i + 2], acc[4 * i + 3], cs.z, -cs.w);
+            }
+          }
+          const size_t off = ((size_t(b) * p.T + row) * p.Hq + head_r) * D + DH * hf;
+          store_span<DH, F32IO>(p.dQ, off, acc);
+        }
       }
     }
   }

@@ -8,26 +8,26 @@
 // one (batch, query head); both read the same key/value tiles, so every K/V
 // tile is loaded (and rotated) once per pair.
 //
-// Operands.  bf16 storage: TMA lands each tile already in the swizzled
-// tensor-core layout and the converter warps rotate queries and keys in place
-// (RoPE fused into the tile load).  float32 storage: the tiles come from the
-// bf16 hi/lo planes written by the operand prologue (nea_prep.cuh, queries and
-// keys already rotated); TMA lands the hi and lo halves of each tile and every
-// product is formed from three bf16 products (hi*hi + hi*lo + lo*hi).
+// Operands.  An operand prologue (nea_prep.cuh) applies the rotary embedding
+// to Q and K once, before this kernel: bf16 storage gets rotated bf16 copies
+// (V is read in place), float32 storage gets bf16 hi/lo planes of Q, K, V.
+// TMA lands every tile already in the swizzled tensor-core layout; for
+// float32 storage it lands the hi and lo halves of each tile and every product
+// is formed from three bf16 products (hi*hi + hi*lo + lo*hi).
 //
 // Warps:
 //   0-3, 4-7   softmax of tile A, of tile B: thread r owns row r (TMEM lane
-//              r); pass 1 over S finds the row max, pass 2 writes
-//              P = exp(s - m) back as bf16 (hi over S, lo in its own columns
-//              for float32 storage); the running max m moves only when it
-//              grows by more than 2^8 (O rescaled in TMEM then); the epilogue
-//              writes O / l and LSE.
+//              r) and loads its whole 128-column score row with one TMEM
+//              load; the row max comes from a three-input max tree, then
+//              P = exp(s - m) is written back as bf16 (hi over S, lo in its
+//              own columns for float32 storage), with paired fp32 arithmetic;
+//              the running max m moves only when it grows by more than 2^8
+//              (O rescaled in TMEM then); the epilogue writes O / l and LSE.
 //   8, 9       MMA issuers, one thread each: warp 8 for tile A, warp 9 for tile B;
 //              S_X = Q_X K_j^T, O_X += P_X V_j, each waiting only on its own
 //              tile, so one tile's softmax overlaps the other tile's MMAs.
 //   10         TMA: query tiles, then K and V tiles into two rings (K stages
 //              free as soon as S is computed, V stages after PV).
-//   11-14      (bf16 only) converter: in-place RoPE of the Q and K tiles.
 // TMEM per tile X: S [256X, 256X+128), O [256X+128, +D), P lo [256X+192, +64).
 // Causal tiles above the diagonal are never visited; only the diagonal tile
 // and a ragged last tile are masked.
@@ -60,7 +60,8 @@
 namespace nea {
 
 struct FwdParams {
-  // bf16 storage: the inputs.  float32 storage: the hi planes.
+  // bf16 storage: rotated Q, K (or the inputs when the rotation is off) and
+  // V.  float32 storage: the hi planes.
   CUtensorMap tm_q;  // [B][T][Hq][D], box {D, 1, 128, 1}
   CUtensorMap tm_k;  // [B][T][Hkv][D]
   CUtensorMap tm_v;
@@ -70,9 +71,6 @@ struct FwdParams {
   CUtensorMap tm_v_lo;
   void* O;
   float* LSE;
-  // [T][D/2] (cos, sin), then [2*n_tiles][D/2] block-start rows; nullptr
-  // when the rotation is off (bf16 storage only; fp32 planes are pre-rotated)
-  const float2* rope;
   int B, T, Hq, Hkv, G;
   int n_tiles;         // ceil(T / 128)
   int n_pairs;         // ceil(n_tiles / 2)
@@ -86,32 +84,27 @@ struct FwdParams {
 
 template <int D, bool F32IO>
 struct FwdSmem {
-  static constexpr bool kConv = !F32IO;        // converter warps (in-place RoPE)
   static constexpr int kNK = F32IO ? 3 : 4;    // K ring stages
   static constexpr int kNV = F32IO ? 2 : 3;    // V ring stages
   static constexpr uint32_t kTile = Stage<D, F32IO>::kBytes;  // one tile: hi (+ lo)
-  static constexpr uint32_t kBase = RopeBaseRows<D>::kBytes;
-  static constexpr uint32_t kSide = kConv ? 1024 : 0;          // per-tile rotary base rows
   static constexpr uint32_t kQA = 0;
   static constexpr uint32_t kQB = kTile;
-  static constexpr uint32_t kQBase = 2 * kTile;  // base rows of A then B
-  static constexpr uint32_t kRope = kQBase + kSide;
-  static constexpr uint32_t kK0 = kRope + (kConv ? TileGeom<D>::kRopeBytes : 0);
-  static constexpr uint32_t kKStage = kTile + kSide;  // tile, then its base rows
+  static constexpr uint32_t kK0 = 2 * kTile;
+  static constexpr uint32_t kKStage = kTile;
   static constexpr uint32_t kV0 = kK0 + kNK * kKStage;
   static constexpr uint32_t kVStage = kTile;
   static constexpr uint32_t kBars = kV0 + kNV * kVStage;
-  // qtma, qready, K tma/full/empty, V tma/empty, s[2], p[2], o[2], fin
-  static constexpr int kNumBars = 2 + 3 * kNK + 2 * kNV + 6 + 2;
+  // qtma, K tma/empty, V tma/empty, s[2], p[2], o[2], fin[2], turn[2]
+  static constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 10;
   static constexpr uint32_t kMisc = kBars + 8 * kNumBars;
   static constexpr uint32_t kUsed = kMisc + 16;
   // +1024 for manual alignment; at least 116 KB so two CTAs never share an SM
   // (each takes all 512 TMEM columns)
   static constexpr uint32_t kAlloc = kUsed + 1024 > 116u * 1024u ? kUsed + 1024 : 116u * 1024u;
-  static constexpr int kThreads = kConv ? 480 : 352;
+  // 11 warps: up to 184 registers per thread, room for a whole score row
+  static constexpr int kThreads = 352;
   static_assert(kK0 % 1024 == 0 && kKStage % 1024 == 0 && kV0 % 1024 == 0 && kVStage % 1024 == 0,
                 "operand tiles need 1024-byte alignment");
-  static_assert(2 * kBase <= 1024, "query base rows");
   static_assert(kAlloc <= 232448, "shared memory");
 };
 
@@ -128,22 +121,17 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
   uint64_t* bar_qtma = bars + 0;
-  uint64_t* bar_qconv = bars + 1;                       // Q tiles rotated (count 128)
-  uint64_t* bar_ktma = bars + 2;                        // [NK]
-  uint64_t* bar_kconv = bars + 2 + NK;                  // [NK] (count 128)
-  uint64_t* bar_kempty = bars + 2 + 2 * NK;             // [NK]
-  uint64_t* bar_vtma = bars + 2 + 3 * NK;               // [NV]
-  uint64_t* bar_vempty = bars + 2 + 3 * NK + NV;        // [NV]
-  uint64_t* bar_s = bars + 2 + 3 * NK + 2 * NV;         // [2] S_X landed
+  uint64_t* bar_ktma = bars + 1;                        // [NK]
+  uint64_t* bar_kempty = bars + 1 + NK;                 // [NK]
+  uint64_t* bar_vtma = bars + 1 + 2 * NK;               // [NV]
+  uint64_t* bar_vempty = bars + 1 + 2 * NK + NV;        // [NV]
+  uint64_t* bar_s = bars + 1 + 2 * NK + 2 * NV;         // [2] S_X landed
   uint64_t* bar_p = bar_s + 2;                          // [2] P_X written (count 128)
   uint64_t* bar_o = bar_s + 4;                          // [2] PV_X done
   uint64_t* bar_fin = bar_s + 6;                        // [2] per issuer
-  // what the MMA issuer waits for: converted tiles (bf16) or landed planes (fp32)
-  uint64_t* bar_qready = L::kConv ? bar_qconv : bar_qtma;
-  uint64_t* bar_kready = L::kConv ? bar_kconv : bar_ktma;
+  uint64_t* bar_turn = bar_s + 8;                       // [2] exponentials of X done (count 128)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
-  const float2* rope_off = reinterpret_cast<const float2*>(smem + L::kRope);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -155,17 +143,14 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
   const bool has_b = qt_b < p.n_tiles;
   const int nkv_a = p.causal ? qt_a + 1 : p.n_tiles, nkv_b = has_b ? (p.causal ? qt_b + 1 : p.n_tiles) : 0;
   const int n_kv = has_b ? nkv_b : nkv_a;
-  auto active = [&](int x, int j) { return j < (x ? nkv_b : nkv_a); };
   const WaitCtl wc{p.err, p.wait_limit, abort_flag};
   NEA_TRACE_STAMP(p, 0, tid == 0);
 
   if (tid == 0) {
     *abort_flag = 0;
     mbar_init(bar_qtma, 1);
-    mbar_init(bar_qconv, 128);
     for (int s = 0; s < NK; ++s) {
       mbar_init(&bar_ktma[s], 1);
-      mbar_init(&bar_kconv[s], 128);
       mbar_init(&bar_kempty[s], has_b ? 2 : 1);  // one commit per tile using the stage
     }
     for (int s = 0; s < NV; ++s) {
@@ -176,6 +161,7 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
       mbar_init(&bar_s[x], 1);
       mbar_init(&bar_p[x], 128);
       mbar_init(&bar_o[x], 1);
+      mbar_init(&bar_turn[x], 128);
     }
     mbar_init(&bar_fin[0], 1);
     mbar_init(&bar_fin[1], 1);
@@ -188,158 +174,7 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
   const uint32_t tbase = *tmem_holder;
   NEA_TRACE_STAMP(p, 1, tid == 0);
 
-  if (warp == 10) {
-    // ------------------------------------------------------------ TMA
-    if ((tid & 31) == 0) {
-      prefetch_tmap(&p.tm_q);
-      prefetch_tmap(&p.tm_k);
-      prefetch_tmap(&p.tm_v);
-      const int nq = has_b ? 2 : 1;
-      const bool rot = L::kConv && p.rope != nullptr;
-      const uint32_t rope_bytes = rot ? uint32_t(min(p.T, kRopeRows)) * (D / 2) * 8 : 0;
-      const uint32_t qbase_bytes = rot ? nq * L::kBase : 0;
-      const float2* base_table = rot ? p.rope + size_t(p.T) * (D / 2) : nullptr;
-      // a load of `row0` of tensor X: the tile (bf16) or its hi and lo planes
-      auto load_tile = [&](uint8_t* dst, const CUtensorMap* hi, const CUtensorMap* lo, int head, int row0,
-                           uint64_t* bar) {
-        tma_load_4d(dst, hi, 0, head, row0, b, bar);
-        if (F32IO) tma_load_4d(dst + OPB, lo, 0, head, row0, b, bar);
-      };
-      // fault-injection hook: withhold the query tiles so every wait on them
-      // runs into its limit
-      const bool q_armed = !(p.debug & 1);
-      if (q_armed) {
-        mbar_arrive_expect_tx(bar_qtma, nq * L::kTile + rope_bytes + qbase_bytes);
-        load_tile(smem + L::kQA, &p.tm_q, &p.tm_q_lo, h, qt_a * kTileRows, bar_qtma);
-        if (has_b) load_tile(smem + L::kQB, &p.tm_q, &p.tm_q_lo, h, qt_b * kTileRows, bar_qtma);
-        if (rot) {
-          bulk_load(smem + L::kRope, p.rope, rope_bytes, bar_qtma);
-          bulk_load(smem + L::kQBase, base_table + size_t(2 * qt_a) * (D / 2), qbase_bytes, bar_qtma);
-        }
-      }
-      int armed_k = 0, armed_v = 0;
-      for (int j = 0; j < n_kv; ++j) {
-        const int sk = j % NK, sv = j % NV;
-        if (j >= NK && !wait_thread(&bar_kempty[sk], ((j / NK) - 1) & 1, wc, kErrWaitEmpty)) break;
-        uint8_t* kst = smem + L::kK0 + sk * L::kKStage;
-        mbar_arrive_expect_tx(&bar_ktma[sk], L::kTile + (rot ? L::kBase : 0));
-        load_tile(kst, &p.tm_k, &p.tm_k_lo, g, j * kTileRows, &bar_ktma[sk]);
-        if (rot) bulk_load(kst + L::kTile, base_table + size_t(2 * j) * (D / 2), L::kBase, &bar_ktma[sk]);
-        NEA_TRACE_STAMP(p, 52 + min(j, 7), true);
-        armed_k = j + 1;
-        if (j >= NV && !wait_thread(&bar_vempty[sv], ((j / NV) - 1) & 1, wc, kErrWaitEmpty)) break;
-        mbar_arrive_expect_tx(&bar_vtma[sv], L::kTile);
-        load_tile(smem + L::kV0 + sv * L::kVStage, &p.tm_v, &p.tm_v_lo, g, j * kTileRows, &bar_vtma[sv]);
-        NEA_TRACE_STAMP(p, 60 + min(j, 7), true);
-        armed_v = j + 1;
-      }
-      // never leave copies in flight: on an abort, wait (bounded) for every
-      // load still outstanding before the CTA exits
-      if (*abort_flag) {
-        for (int j = max(0, armed_k - NK); j < armed_k; ++j) drain_wait(&bar_ktma[j % NK], (j / NK) & 1, wc);
-        for (int j = max(0, armed_v - NV); j < armed_v; ++j) drain_wait(&bar_vtma[j % NV], (j / NV) & 1, wc);
-        if (q_armed) drain_wait(bar_qtma, 0, wc);
-      }
-    }
-    __syncwarp();
-  } else if (L::kConv && warp >= 11) {
-    // ------------------------------------------------------------ converter (bf16: in-place RoPE)
-    const int pt = tid - 352;
-    uint32_t conv_count = 0;  // unused: bf16 tiles need no rendezvous
-    const float2* qbase = p.rope ? reinterpret_cast<const float2*>(smem + L::kQBase) : nullptr;
-    bool ok = wait_warp(bar_qtma, 0, wc, kErrWaitProducer);
-    if (ok) {
-      prepare_tile<D, false, true>(smem + L::kQA, rope_off, qbase, qt_a * kTileRows, p.T, nullptr, conv_count,
-                                   wc, pt);
-      if (has_b)
-        prepare_tile<D, false, true>(smem + L::kQB, rope_off, qbase ? qbase + 2 * (D / 2) : nullptr,
-                                     qt_b * kTileRows, p.T, nullptr, conv_count, wc, pt);
-      fence_async_smem();
-      mbar_arrive(bar_qconv);
-      NEA_TRACE_STAMP(p, 2, pt == 0);
-    }
-    for (int j = 0; ok && j < n_kv; ++j) {
-      const int sk = j % NK;
-      if (!wait_warp(&bar_ktma[sk], (j / NK) & 1, wc, kErrWaitProducer)) break;
-      uint8_t* kst = smem + L::kK0 + sk * L::kKStage;
-      const float2* kbase = p.rope ? reinterpret_cast<const float2*>(kst + L::kTile) : nullptr;
-      prepare_tile<D, false, true>(kst, rope_off, kbase, j * kTileRows, p.T, nullptr, conv_count, wc, pt);
-      fence_async_smem();
-      mbar_arrive(&bar_kconv[sk]);
-      NEA_TRACE_STAMP(p, 36 + min(j, 7), pt == 0);
-    }
-  } else if (warp == 8 || warp == 9) {
-    // ------------------------------------------------------------ MMA issuers
-    // Issuer X runs tile X on its own: S_X(0); then per key tile j: wait for
-    // P_X(j), O_X += P_X(j) V_j; wait for that to finish reading P_X(j) (which
-    // S_X(j+1) overwrites), S_X(j+1).  Stage releases count one commit per
-    // tile; the last key tile of a causal pair is used by B alone, but its
-    // stages are never refilled, so no one waits for that release.
-    const int x = warp - 8;
-    if ((tid & 31) == 0 && (x == 0 || has_b)) {
-      constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
-      constexpr uint32_t idO = idesc_bf16(128, D, 0, 1);
-      const uint32_t sQ = smem_u32(smem + (x ? L::kQB : L::kQA));
-      const int my_nkv = x ? nkv_b : nkv_a;
-      auto issue_s = [&](int j) {
-        const uint32_t sK = smem_u32(smem + L::kK0 + (j % NK) * L::kKStage);
-        const uint32_t dS = tbase + 256 * x;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-#pragma unroll
-          for (int term = 0; term < kTerms; ++term) {
-            // float32 storage: hi*hi + hi*lo + lo*hi
-            const uint32_t qa = sQ + (term == 2 ? OPB : 0) + kk * 32;
-            const uint32_t kb = sK + (term == 1 ? OPB : 0) + kk * 32;
-            mma_ss(dS, smem_desc(qa, RB, 16), smem_desc(kb, RB, 16), idS, (kk | term) != 0);
-          }
-        }
-        tc_commit(&bar_s[x]);
-      };
-      bool ok = wait_thread(bar_qready, 0, wc, kErrWaitProducer) &&
-                wait_thread(&bar_kready[0], 0, wc, kErrWaitProducer);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0);
-        tc_commit(&bar_kempty[0]);
-      }
-      for (int j = 0; ok && j < my_nkv; ++j) {
-        const int sv = j % NV;
-        if (!wait_thread(&bar_p[x], j & 1, wc, kErrWaitSoftmax) ||
-            !wait_thread(&bar_vtma[sv], (j / NV) & 1, wc, kErrWaitProducer))
-          break;
-        tc_fence_after();
-        const uint32_t sV = smem_u32(smem + L::kV0 + sv * L::kVStage);
-        const uint32_t phi = tbase + 256 * x, plo = tbase + 256 * x + 192, dO = tbase + 256 * x + 128;
-#pragma unroll
-        for (int kk = 0; kk < kTileRows / 16; ++kk) {
-#pragma unroll
-          for (int term = 0; term < kTerms; ++term) {
-            // float32 storage: Phi*Vhi + Phi*Vlo + Plo*Vhi
-            const uint32_t pa = (term == 2 ? plo : phi) + kk * 8;
-            const uint32_t vb = sV + (term == 1 ? OPB : 0) + kk * 16 * RB;
-            mma_ts(dO, pa, smem_desc(vb, RB, kTileRows * RB), idO, (j | kk | term) != 0);
-          }
-        }
-        tc_commit(&bar_o[x]);
-        tc_commit(&bar_vempty[sv]);
-        NEA_TRACE_STAMP(p, 68 + min(j, 7), x == 0);
-        if (j + 1 < my_nkv) {
-          // S_X(j+1) overwrites P_X(j): wait until PV_X(j) has read it
-          const int sk = (j + 1) % NK;
-          if (!wait_thread(&bar_o[x], j & 1, wc, kErrWaitMma) ||
-              !wait_thread(&bar_kready[sk], ((j + 1) / NK) & 1, wc, kErrWaitProducer))
-            break;
-          tc_fence_after();
-          issue_s(j + 1);
-          tc_commit(&bar_kempty[sk]);
-        }
-      }
-      tc_commit(&bar_fin[x]);
-      drain_wait(&bar_fin[x], 0, wc);
-    }
-    __syncwarp();
-  } else if (warp < 8) {
+  if (warp < 8) {
     // ------------------------------------------------------------ softmax (warps 0-7)
     const int x = warp >> 2;   // query tile A or B
     const int r = tid & 127;   // row inside the tile, TMEM lane
@@ -347,62 +182,64 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
     const int q = my_qt * kTileRows + r;
     const uint32_t lane_base = tmem_addr(tbase, uint32_t(warp & 3) * 32, 0);
     const uint32_t scol = lane_base + 256 * x, ocol = scol + 128, plocol = scol + 192;
-    float m_run = -INFINITY, l0 = 0.f, l1 = 0.f;
+    float m_run = -INFINITY;
+    uint64_t l01 = 0, l23 = 0;  // partial row sums, two packed pairs
+    const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
     bool ok = x == 0 || has_b;
     for (int j = 0; ok && j < my_nkv; ++j) {
       if (!wait_warp(&bar_s[x], j & 1, wc, kErrWaitMma)) { ok = false; break; }
       NEA_TRACE_STAMP(p, 4 + 16 * x + 2 * min(j, 7), r == 0);
       tc_fence_after();
+      uint32_t sv[128];
+      tmem_ld128(scol, sv);
       const int kv0 = j * kTileRows;
-      const bool need_mask = (p.causal && j == my_qt) || kv0 + kTileRows > p.T;
-      const int lim = (p.causal ? min(q, p.T - 1) : p.T - 1) - kv0;  // last visible column
-      // pass 1: row maximum
-      float mx = -INFINITY;
+      if ((p.causal && j == my_qt) || kv0 + kTileRows > p.T) {  // same for the whole tile
+        const int lim = (p.causal ? min(q, p.T - 1) : p.T - 1) - kv0;  // last visible column
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t rr[64];
-        tmem_ld64(scol + 64 * c, rr);
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float v = __uint_as_float(rr[i]);
-          mx = fmaxf(mx, (need_mask && 64 * c + i > lim) ? -INFINITY : v);
-        }
+        for (int i = 0; i < 128; ++i) sv[i] = i > lim ? 0xff800000u : sv[i];  // -inf: P = 0
       }
-      const float m_tile = mx * p.scale_log2;
+      const float m_tile = row_max128(sv) * p.scale_log2;
       float alpha = 1.f;
       if (m_tile > m_run + 8.f) {  // keep a stale max unless it grew by > 2^8
         alpha = ex2(m_run - m_tile);
         m_run = m_tile;
       }
-      l0 *= alpha;
-      l1 *= alpha;
-      // pass 2: P = exp2(s * scale_log2 - m) -> bf16 (hi over S, lo apart)
+      const uint64_t a2 = f2_pack(alpha, alpha);
+      l01 = f2_mul(l01, a2);
+      l23 = f2_mul(l23, a2);
+      const uint64_t nm2 = f2_pack(-m_run, -m_run);
+      // The two tiles take turns on the exponential unit, A(j) after B(j-1)
+      // and B(j) after A(j), so that each tile's MMAs run under the other
+      // tile's exponentials instead of both tiles waiting on the MMAs at once.
+      if (has_b && ((x == 0 && j > 0) || (x == 1 && j < nkv_a)) &&
+          !wait_warp(&bar_turn[x ^ 1], (x == 0 ? j - 1 : j) & 1, wc, kErrWaitSoftmax)) {
+        ok = false;
+        break;
+      }
+      // P = exp2(s * scale_log2 - m) -> bf16 (hi over S, lo apart)
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(scol + 32 * c, rr);
         uint32_t hi[16], lo[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const int c0 = 32 * c + 2 * i;
-          float p0 = ex2(fmaf(__uint_as_float(rr[2 * i]), p.scale_log2, -m_run));
-          float p1 = ex2(fmaf(__uint_as_float(rr[2 * i + 1]), p.scale_log2, -m_run));
-          if (need_mask) {
-            p0 = (c0 > lim) ? 0.f : p0;
-            p1 = (c0 + 1 > lim) ? 0.f : p1;
-          }
-          l0 += p0;
-          l1 += p1;
+          const int e = 32 * c + 2 * i;
+          float t0, t1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sc2, nm2), t0, t1);
+          const float p0 = ex2(t0), p1 = ex2(t1);
+          const uint64_t pp = f2_pack(p0, p1);
+          if (i & 1) l23 = f2_add(l23, pp); else l01 = f2_add(l01, pp);
+          hi[i] = pack_bf16(p0, p1);
           if (F32IO) {
-            split_bf16(p0, p1, hi[i], lo[i]);
-          } else {
-            hi[i] = pack_bf16(p0, p1);
+            float r0, r1;
+            f2_unpack(f2_sub(pp, f2_pack(bf16_lo_f(hi[i]), bf16_hi_f(hi[i]))), r0, r1);
+            lo[i] = pack_bf16(r0, r1);
           }
         }
-        // columns [16c, 16c+16) of S were read in chunk c/2 <= c already
+        // every column of S is in registers already
         tmem_st16(scol + 16 * c, hi);
         if (F32IO) tmem_st16(plocol + 16 * c, lo);
       }
+      mbar_arrive(&bar_turn[x]);
       if (__any_sync(kFullMask, alpha != 1.f && j > 0)) {
         // O holds the sum over tiles < j: PV_X(j-1) has landed (S_X(j) was
         // issued after it); rescale
@@ -433,7 +270,10 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
         for (int i = 0; i < 32; ++i) o[32 * c + i] = __uint_as_float(rr[i]);
       }
       if (q < p.T) {
-        const float l_run = l0 + l1;
+        float la, lb, lc, ld;
+        f2_unpack(l01, la, lb);
+        f2_unpack(l23, lc, ld);
+        const float l_run = (la + lb) + (lc + ld);
         const float inv = 1.f / l_run;
 #pragma unroll
         for (int i = 0; i < D; ++i) o[i] *= inv;
@@ -442,6 +282,126 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
         p.LSE[(size_t(b) * p.Hq + h) * p.T + q] = (m_run + log2f(l_run)) * 0.69314718055994531f;
       }
       NEA_TRACE_STAMP(p, 76 + x, r == 0);
+    }
+  } else {
+    if (warp == 10) {
+      // ------------------------------------------------------------ TMA
+      if ((tid & 31) == 0) {
+        prefetch_tmap(&p.tm_q);
+        prefetch_tmap(&p.tm_k);
+        prefetch_tmap(&p.tm_v);
+        const int nq = has_b ? 2 : 1;
+        // a load of `row0` of tensor X: the tile (bf16) or its hi and lo planes
+        auto load_tile = [&](uint8_t* dst, const CUtensorMap* hi, const CUtensorMap* lo, int head, int row0,
+                             uint64_t* bar) {
+          tma_load_4d(dst, hi, 0, head, row0, b, bar);
+          if (F32IO) tma_load_4d(dst + OPB, lo, 0, head, row0, b, bar);
+        };
+        // fault-injection hook: withhold the query tiles so every wait on them
+        // runs into its limit
+        const bool q_armed = !(p.debug & 1);
+        if (q_armed) {
+          mbar_arrive_expect_tx(bar_qtma, nq * L::kTile);
+          load_tile(smem + L::kQA, &p.tm_q, &p.tm_q_lo, h, qt_a * kTileRows, bar_qtma);
+          if (has_b) load_tile(smem + L::kQB, &p.tm_q, &p.tm_q_lo, h, qt_b * kTileRows, bar_qtma);
+        }
+        int armed_k = 0, armed_v = 0;
+        for (int j = 0; j < n_kv; ++j) {
+          const int sk = j % NK, sv = j % NV;
+          if (j >= NK && !wait_thread(&bar_kempty[sk], ((j / NK) - 1) & 1, wc, kErrWaitEmpty)) break;
+          uint8_t* kst = smem + L::kK0 + sk * L::kKStage;
+          mbar_arrive_expect_tx(&bar_ktma[sk], L::kTile);
+          load_tile(kst, &p.tm_k, &p.tm_k_lo, g, j * kTileRows, &bar_ktma[sk]);
+          NEA_TRACE_STAMP(p, 52 + min(j, 7), true);
+          armed_k = j + 1;
+          if (j >= NV && !wait_thread(&bar_vempty[sv], ((j / NV) - 1) & 1, wc, kErrWaitEmpty)) break;
+          mbar_arrive_expect_tx(&bar_vtma[sv], L::kTile);
+          load_tile(smem + L::kV0 + sv * L::kVStage, &p.tm_v, &p.tm_v_lo, g, j * kTileRows, &bar_vtma[sv]);
+          NEA_TRACE_STAMP(p, 60 + min(j, 7), true);
+          armed_v = j + 1;
+        }
+        // never leave copies in flight: on an abort, wait (bounded) for every
+        // load still outstanding before the CTA exits
+        if (*abort_flag) {
+          for (int j = max(0, armed_k - NK); j < armed_k; ++j) drain_wait(&bar_ktma[j % NK], (j / NK) & 1, wc);
+          for (int j = max(0, armed_v - NV); j < armed_v; ++j) drain_wait(&bar_vtma[j % NV], (j / NV) & 1, wc);
+          if (q_armed) drain_wait(bar_qtma, 0, wc);
+        }
+      }
+      __syncwarp();
+    } else if (warp < 10) {
+      // ------------------------------------------------------------ MMA issuers
+      // Issuer X runs tile X on its own: S_X(0); then per key tile j: wait for
+      // P_X(j), O_X += P_X(j) V_j; wait for that to finish reading P_X(j) (which
+      // S_X(j+1) overwrites), S_X(j+1).  Stage releases count one commit per
+      // tile; the last key tile of a causal pair is used by B alone, but its
+      // stages are never refilled, so no one waits for that release.
+      const int x = warp - 8;
+      if ((tid & 31) == 0 && (x == 0 || has_b)) {
+        constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
+        constexpr uint32_t idO = idesc_bf16(128, D, 0, 1);
+        const uint32_t sQ = smem_u32(smem + (x ? L::kQB : L::kQA));
+        const int my_nkv = x ? nkv_b : nkv_a;
+        auto issue_s = [&](int j) {
+          const uint32_t sK = smem_u32(smem + L::kK0 + (j % NK) * L::kKStage);
+          const uint32_t dS = tbase + 256 * x;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+#pragma unroll
+            for (int term = 0; term < kTerms; ++term) {
+              // float32 storage: hi*hi + hi*lo + lo*hi
+              const uint32_t qa = sQ + (term == 2 ? OPB : 0) + kk * 32;
+              const uint32_t kb = sK + (term == 1 ? OPB : 0) + kk * 32;
+              mma_ss(dS, smem_desc(qa, RB, 16), smem_desc(kb, RB, 16), idS, (kk | term) != 0);
+            }
+          }
+          tc_commit(&bar_s[x]);
+        };
+        bool ok = wait_thread(bar_qtma, 0, wc, kErrWaitProducer) &&
+                  wait_thread(&bar_ktma[0], 0, wc, kErrWaitProducer);
+        if (ok) {
+          tc_fence_after();
+          issue_s(0);
+          tc_commit(&bar_kempty[0]);
+        }
+        for (int j = 0; ok && j < my_nkv; ++j) {
+          const int sv = j % NV;
+          if (!wait_thread(&bar_p[x], j & 1, wc, kErrWaitSoftmax) ||
+              !wait_thread(&bar_vtma[sv], (j / NV) & 1, wc, kErrWaitProducer))
+            break;
+          NEA_TRACE_STAMP(p, 36 + min(j, 7), x == 0);
+          tc_fence_after();
+          const uint32_t sV = smem_u32(smem + L::kV0 + sv * L::kVStage);
+          const uint32_t phi = tbase + 256 * x, plo = tbase + 256 * x + 192, dO = tbase + 256 * x + 128;
+#pragma unroll
+          for (int kk = 0; kk < kTileRows / 16; ++kk) {
+#pragma unroll
+            for (int term = 0; term < kTerms; ++term) {
+              // float32 storage: Phi*Vhi + Phi*Vlo + Plo*Vhi
+              const uint32_t pa = (term == 2 ? plo : phi) + kk * 8;
+              const uint32_t vb = sV + (term == 1 ? OPB : 0) + kk * 16 * RB;
+              mma_ts(dO, pa, smem_desc(vb, RB, kTileRows * RB), idO, (j | kk | term) != 0);
+            }
+          }
+          tc_commit(&bar_o[x]);
+          tc_commit(&bar_vempty[sv]);
+          NEA_TRACE_STAMP(p, 68 + min(j, 7), x == 0);
+          if (j + 1 < my_nkv) {
+            // S_X(j+1) overwrites P_X(j): wait until PV_X(j) has read it
+            const int sk = (j + 1) % NK;
+            if (!wait_thread(&bar_o[x], j & 1, wc, kErrWaitMma) ||
+                !wait_thread(&bar_ktma[sk], ((j + 1) / NK) & 1, wc, kErrWaitProducer))
+              break;
+            NEA_TRACE_STAMP(p, 44 + min(j, 7), x == 0);
+            tc_fence_after();
+            issue_s(j + 1);
+            tc_commit(&bar_kempty[sk]);
+          }
+        }
+        tc_commit(&bar_fin[x]);
+        drain_wait(&bar_fin[x], 0, wc);
+      }
+      __syncwarp();
     }
   }
   tc_fence_before();

@@ -1,12 +1,14 @@
-// Operand prologue of the float32-storage path: one pass over Q, K, V (and
-// dO in the backward) that applies the rotary embedding to queries and keys
-// ("NanoEuler" write-up, aimsg.uk, section 2 "Model components": RoPE on
-// queries and keys) and writes every element as two bf16 planes, hi = bf16(x)
-// and lo = bf16(x - hi), in the same [B][T][H][D] layout.  The attention
-// kernels then stage those planes with TMA directly in the tensor-core
-// operand layout and form each product from three bf16 products
-// (hi*hi + hi*lo + lo*hi).  The pass reads each fp32 element once and writes
-// 4 bytes for it, so it is bound by HBM bandwidth.
+// Operand prologue: one pass over the inputs that applies the rotary
+// embedding to queries and keys ("NanoEuler" write-up, aimsg.uk, section 2
+// "Model components": RoPE on queries and keys) before the attention kernels
+// stage them with TMA directly in the tensor-core operand layout.
+//   - float32 storage: every element of Q, K, V (and dO in the backward) is
+//     written as two bf16 planes, hi = bf16(x) and lo = bf16(x - hi), in the
+//     same [B][T][H][D] layout; the kernels form each product from three bf16
+//     products (hi*hi + hi*lo + lo*hi).  Reads 4 bytes and writes 4 per element.
+//   - bfloat16 storage: Q and K are rotated into bf16 copies (V and dO are
+//     read in place).  Reads 2 bytes and writes 2 per element.
+// Both are bound by HBM bandwidth.
 #pragma once
 
 #include "nea_device.cuh"
@@ -14,10 +16,10 @@
 namespace nea {
 
 struct PrepJob {
-  const float* src;       // [B][T][H][D] fp32
-  __nv_bfloat16* hi;      // same layout, bf16(x)
-  __nv_bfloat16* lo;      // same layout, bf16(x - hi)
-  long long chunks;       // B*T*H*D / 4 (16-byte chunks of four floats)
+  const void* src;        // [B][T][H][D], fp32 or bf16
+  __nv_bfloat16* hi;      // same layout: bf16(x) (fp32), the rotated copy (bf16)
+  __nv_bfloat16* lo;      // same layout: bf16(x - hi) (fp32 only)
+  long long chunks;       // 16-byte chunks: B*T*H*D / 4 (fp32), / 8 (bf16)
   int H;                  // heads of this tensor
   int rope;               // 1: rotate (queries, keys)
 };
@@ -30,8 +32,10 @@ struct PrepParams {
   long long total;        // sum of chunks
 };
 
-template <int D>
-__global__ void __launch_bounds__(256) attn_prep_split_kernel(const __grid_constant__ PrepParams p) {
+template <int D, bool F32IO>
+__global__ void __launch_bounds__(256) attn_prep_kernel(const __grid_constant__ PrepParams p) {
+  constexpr int kPerChunk = F32IO ? 4 : 8;  // elements per 16-byte chunk
+  constexpr int kCpr = D / kPerChunk;       // chunks per head vector
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < p.total; i += stride) {
     int j = 0;
@@ -41,22 +45,40 @@ __global__ void __launch_bounds__(256) attn_prep_split_kernel(const __grid_const
       ++j;
     }
     const PrepJob& job = p.job[j];
-    float4 x = __ldg(reinterpret_cast<const float4*>(job.src) + ci);
-    if (job.rope && p.rope != nullptr) {
-      constexpr int kCpr = D / 4;           // chunks per head vector
-      const long long row = ci / kCpr;      // (b, t, h) row index
-      const int c = int(ci % kCpr);         // pairs 2c, 2c+1
-      const int t = int((row / job.H) % p.T);
-      const float4 cs = __ldg(reinterpret_cast<const float4*>(p.rope + size_t(t) * (D / 2) + 2 * c));
-      const float y0 = x.x * cs.x - x.y * cs.y, y1 = x.x * cs.y + x.y * cs.x;
-      const float y2 = x.z * cs.z - x.w * cs.w, y3 = x.z * cs.w + x.w * cs.z;
-      x = make_float4(y0, y1, y2, y3);
+    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(job.src) + ci);
+    float x[kPerChunk];
+    if constexpr (F32IO) {
+      x[0] = __uint_as_float(raw.x), x[1] = __uint_as_float(raw.y);
+      x[2] = __uint_as_float(raw.z), x[3] = __uint_as_float(raw.w);
+    } else {
+      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) x[2 * k] = bf16_lo_f(w[k]), x[2 * k + 1] = bf16_hi_f(w[k]);
     }
-    uint2 hi, lo;
-    split_bf16(x.x, x.y, hi.x, lo.x);
-    split_bf16(x.z, x.w, hi.y, lo.y);
-    reinterpret_cast<uint2*>(job.hi)[ci] = hi;
-    reinterpret_cast<uint2*>(job.lo)[ci] = lo;
+    if (job.rope && p.rope != nullptr) {
+      const long long row = ci / kCpr;      // (b, t, h) row index
+      const int c = int(ci % kCpr);         // pairs kPerChunk/2 * c ...
+      const int t = int((row / job.H) % p.T);
+      const float4* cs = reinterpret_cast<const float4*>(p.rope + size_t(t) * (D / 2) + (kPerChunk / 2) * c);
+#pragma unroll
+      for (int k = 0; k < kPerChunk / 4; ++k) {
+        const float4 r = __ldg(cs + k);  // (cos, sin) of two pairs
+        float* y = x + 4 * k;
+        const float y0 = y[0] * r.x - y[1] * r.y, y1 = y[0] * r.y + y[1] * r.x;
+        const float y2 = y[2] * r.z - y[3] * r.w, y3 = y[2] * r.w + y[3] * r.z;
+        y[0] = y0, y[1] = y1, y[2] = y2, y[3] = y3;
+      }
+    }
+    if constexpr (F32IO) {
+      uint2 hi, lo;
+      split_bf16(x[0], x[1], hi.x, lo.x);
+      split_bf16(x[2], x[3], hi.y, lo.y);
+      reinterpret_cast<uint2*>(job.hi)[ci] = hi;
+      reinterpret_cast<uint2*>(job.lo)[ci] = lo;
+    } else {
+      reinterpret_cast<uint4*>(job.hi)[ci] =
+          make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
+    }
   }
 }
 

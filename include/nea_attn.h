@@ -26,7 +26,7 @@
  * Ownership: every pointer is a device pointer owned by the caller; the
  * library never frees or retains them.  The library keeps, per device, a
  * cached workspace (the rotary cos/sin tables, the backward's per-row terms
- * and, for NEA_F32, the bf16 hi/lo operand planes), allocated on first use and
+ * and the operand prologue's output), allocated on first use and
  * grown only when a call needs more; steady-state calls allocate nothing.
  *
  * Streams: work is enqueued on `stream` (a cudaStream_t, NULL for the legacy
@@ -77,12 +77,12 @@ enum {
  *   causal      1: key j visible to query i iff j <= i; 0: all keys visible
  *   stream      cudaStream_t to enqueue on
  *
- * NEA_BF16: plain bf16 tensor-core products, fp32 accumulation; the rotation
- * is applied to each Q/K tile as it is staged in shared memory.
- * NEA_F32: an operand prologue kernel first rotates Q and K and writes Q, K,
- * V as bf16 high and low planes in the workspace; each score and output
- * contraction is then formed from them as hi*hi + hi*lo + lo*hi (fp32
- * accumulation), about 2^-16 relative per product.
+ * An operand prologue kernel first applies the rotation to Q and K, once per
+ * element, into the workspace.  NEA_BF16: the rotated copies (rounded to
+ * bf16) feed plain bf16 tensor-core products with fp32 accumulation.
+ * NEA_F32: the prologue writes Q, K, V as bf16 high and low planes; each
+ * score and output contraction is formed from them as hi*hi + hi*lo + lo*hi
+ * (fp32 accumulation), about 2^-16 relative per product.
  */
 int nea_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int T, int Hq,
                  int Hkv, int D, int dtype, float rope_base, int causal, void* stream);
@@ -95,10 +95,12 @@ int nea_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
  * dV the shape of K.  O and LSE must be the forward's results for the same
  * Q, K, V, rope_base and causal.
  *
- * Runs on `stream`: (NEA_F32) the operand prologue over Q, K, V, dO; the row
- * terms LSE*log2(e) and D_i = sum_d dO_id O_id; the dK/dV kernel (one CTA per
- * key tile and kv head, looping over the query heads of the group); the dQ
- * kernel (one CTA per query tile and head); both recompute P from LSE.
+ * Runs on `stream`: the operand prologue (NEA_F32: bf16 hi/lo planes of the
+ * rotated Q and K and of V, dO; NEA_BF16: rotated copies of Q and K, none
+ * when the rotation is off); the row terms -LSE*log2(e) and
+ * D_i = sum_d dO_id O_id; the dK/dV kernel (one CTA per key tile and kv head,
+ * looping over the query heads of the group); the dQ kernel (one CTA per
+ * query tile and head); both recompute P from LSE.
  *
  * NEA_F32: the score product and dO V^T use split bf16 (as in the forward);
  * the three gradient products use the bf16 high parts with fp32
@@ -156,14 +158,17 @@ void nea_set_profile_events(void* const* events, int n);
  *
  * Same arguments, layouts and results as nea_attn_bwd.  The caller passes all
  * inputs and outputs; everything else the backward needs (the per-row terms
- * LSE*log2(e) and D_i = sum_d dO_id O_id, the rotary cos/sin table, computed
- * on the device in double precision, a device status word and, for NEA_F32,
- * the bf16 hi/lo planes of Q, K, V, dO) lives in one fixed array of 4 MiB
- * compiled into the library: every GPU that loads the library keeps it until
- * the process exits.  With Tp = 128*ceil(T/128), a call needs about
- * 256 + 8*B*Hq*Tp + 4*(T + 2*ceil(T/128))*D bytes of it, plus
- * 8*B*T*(Hq + Hkv)*D bytes for NEA_F32 (each part rounded up to 256 bytes);
- * larger problems return NEA_ERR_SCRATCH_LIMIT before anything is launched.
+ * -LSE*log2(e) and D_i = sum_d dO_id O_id, the rotary cos/sin table, computed
+ * on the device in double precision, a device status word and the operand
+ * prologue's output: for NEA_F32 the bf16 hi/lo planes of Q, K, V, dO, for
+ * NEA_BF16 with the rotation on the rotated copies of Q and K) lives in one
+ * fixed array of 4 MiB compiled into the library: every GPU that loads the
+ * library keeps it until the process exits.  With Tp = 128*ceil(T/128), a
+ * call needs about 256 + 8*B*Hq*Tp bytes of it, plus 4*T*D bytes with the
+ * rotation on, plus 8*B*T*(Hq + Hkv)*D bytes for NEA_F32 or, with the
+ * rotation on, 2*B*T*(Hq + Hkv)*D bytes for NEA_BF16 (each part rounded up to
+ * 256 bytes); larger problems return NEA_ERR_SCRATCH_LIMIT before anything
+ * is launched.
  *
  * The first call on a device does a one-time set-up with that device
  * current (it looks up the array's device address and sets kernel
