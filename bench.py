@@ -11,8 +11,10 @@ configuration of the NanoEuler GPU model shape.
 
 Prints one JSON line (rank 0).  value = algorithmic TFLOP/s of the whole job
 (7 * B * Hq * T^2 * D per causal step and layer, summed over ranks, divided by
-the slowest rank's device time of the K timed steps).  L2 is flushed (a 256 MiB
-write) before every timed step, outside the step's events.
+the slowest rank's device time of the K timed steps).  L2 is flushed before
+every timed step, outside the step's events: a 256 MiB write, then a 256 MiB
+read of another buffer, which evicts the written lines so that their
+write-back is not charged to the first kernel of the step.
 """
 from __future__ import annotations
 
@@ -29,7 +31,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "causal GQA attention fwd+bwd TFLOP/s (% of tensor-core peak) and tokens/s"
-KERNELS = ("attn_fwd", "attn_bwd_rowterm", "attn_bwd_dkdv", "attn_bwd_dq")
+KERNELS = ("attn_fwd_prologue", "attn_fwd", "attn_bwd_prologue", "attn_bwd_dkdv", "attn_bwd_dq")
 # Algorithmic work per kernel in units of B*Hq*T^2*D (causal): the forward's
 # two products; the dK/dV kernel's S, dP, dV, dK products; the dQ kernel's S,
 # dP, dQ products (S and dP are recomputed there, so the two backward kernels
@@ -37,6 +39,23 @@ KERNELS = ("attn_fwd", "attn_bwd_rowterm", "attn_bwd_dkdv", "attn_bwd_dq")
 # their distinct outputs: dK/dV gets dP, dV, dK; dQ gets S and dQ).
 UNITS = {"attn_fwd": 2.0, "attn_bwd_dkdv": 3.0, "attn_bwd_dq": 2.0}
 L2_FLUSH_BYTES = 256 << 20
+
+
+def prologue_bytes(w, kernel):
+    """Algorithmic HBM bytes of one operand-prologue launch: every input
+    element read once and every output element written once."""
+    nq, nk = w.B * w.T * w.Hq * w.D, w.B * w.T * w.Hkv * w.D
+    rope = w.rope_base > 0
+    if w.dtype == "f32":  # fp32 in, bf16 hi + lo out
+        conv = (nq + 2 * nk) if kernel == "attn_fwd_prologue" else (2 * nq + 2 * nk)
+        b = conv * (4 + 4)
+    else:  # rotated bf16 copies of Q, K
+        b = (nq + nk) * (2 + 2) if rope else 0
+    if kernel == "attn_bwd_prologue":  # row terms: read O, dO, LSE; write ws[B*Hq][2][Tp]
+        e = 4 if w.dtype == "f32" else 2
+        tp = -(-w.T // 128) * 128
+        b += 2 * nq * e + 4 * w.B * w.Hq * w.T + 8 * w.B * w.Hq * tp
+    return b
 
 
 def parse():
@@ -269,6 +288,12 @@ def main():
         outs.append({"o": o, "lse": lse, "dq": torch.empty_like(L["q"]), "dk": torch.empty_like(L["k"]),
                      "dv": torch.empty_like(L["v"])})
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    drain = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    drain_sum = torch.empty((), dtype=torch.float32, device=dev)
+
+    def flush_l2(i):
+        flush.fill_(float(i))
+        torch.sum(drain, dim=0, out=drain_sum)
 
     def step():
         for L, O in zip(layers, outs):
@@ -277,7 +302,7 @@ def main():
                              dq=O["dq"], dk=O["dk"], dv=O["dv"])
 
     for _ in range(a.warmup):
-        flush.fill_(1.0)
+        flush_l2(1)
         step()
     torch.cuda.synchronize(dev)
     status = nea.nea_device_status()
@@ -286,8 +311,8 @@ def main():
 
     K = a.steps
     ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    # per-layer kernel-boundary events of every step (6 per layer)
-    ev_k = [[[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(w.layers)] for _ in range(K)]
+    # per-layer kernel-boundary events of every step (7 per layer)
+    ev_k = [[[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(w.layers)] for _ in range(K)]
     for evs in ev_k:
         for row in evs:
             for e in row:
@@ -300,7 +325,7 @@ def main():
     with clocks:
         wall0 = time.perf_counter()
         for i in range(K):
-            flush.fill_(float(i))
+            flush_l2(i)
             ev_step[i][0].record(stream)
             for li, (L, O) in enumerate(zip(layers, outs)):
                 nea.nea_set_profile_events(ev_k[i][li])
@@ -322,8 +347,9 @@ def main():
     for i in range(K):
         for li in range(w.layers):
             ev = ev_k[i][li]
-            kern_ms["attn_fwd"] += ev[0].elapsed_time(ev[1])
-            kern_ms["attn_bwd_rowterm"] += ev[2].elapsed_time(ev[3])
+            kern_ms["attn_fwd_prologue"] += ev[0].elapsed_time(ev[6])
+            kern_ms["attn_fwd"] += ev[6].elapsed_time(ev[1])
+            kern_ms["attn_bwd_prologue"] += ev[2].elapsed_time(ev[3])
             kern_ms["attn_bwd_dkdv"] += ev[3].elapsed_time(ev[4])
             kern_ms["attn_bwd_dq"] += ev[4].elapsed_time(ev[5])
     launches_per_kernel = K * w.layers
@@ -343,8 +369,7 @@ def main():
                 "frac": achieved / pk["bf16_tflops"], "traffic": ncu_traffic(dominant, w.name),
                 "kernel": dominant, "peak_kind": f"bf16 dense burst ({pk['source']})"}
     else:
-        e = 2 if w.dtype == "bf16" else 4
-        byts = 2 * w.B * w.T * w.Hq * w.D * e + 4 * w.B * w.Hq * w.T
+        byts = prologue_bytes(w, dominant)
         achieved = byts / (per_launch_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / pk["hbm_gbs"], "traffic": ncu_traffic(dominant, w.name), "kernel": dominant}
@@ -401,7 +426,7 @@ def main():
             "dtype": "bf16x3" if w.dtype == "f32" else "bf16", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
                        "storage": storage, "causal": w.causal, "rope_base": w.rope_base, "layers": w.layers,
-                       "qk_std": w.qk_std, "l2": "flushed (256 MiB write) before every timed step",
+                       "qk_std": w.qk_std, "l2": "flushed before every timed step (256 MiB write, then 256 MiB read of another buffer)",
                        "parallelism": f"dp{world} (independent batches per GPU)"},
             "tokens_per_s": tokens_s,
             "frac_of_bf16_peak": value / pk["bf16_tflops"],

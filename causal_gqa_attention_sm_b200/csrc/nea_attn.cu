@@ -34,6 +34,7 @@ thread_local int t_prof_n = 0;
 // Performance-analysis builds only: destination of the forward kernel's phase
 // stamps (80 per CTA), set through nea_debug_set_trace.
 thread_local unsigned long long* t_trace = nullptr;
+thread_local unsigned long long* t_trace_bwd = nullptr;
 #endif
 
 void prof_record(int i, cudaStream_t stream) {
@@ -241,15 +242,25 @@ size_t prep_bytes(const size_t* elems, const int* rot, int n, bool f32, bool rop
 // the attention kernels read: for bfloat16 storage the rotated copy or, for
 // tensors left as they are, the input itself.
 int run_prep(uint8_t* base, const void* const* src, const size_t* elems, const int* H, const int* rot, int n,
-             int T, int D, bool f32, const float2* table, nea::PrepJob* jobs_out, cudaStream_t stream) {
+             int T, int D, bool f32, const float2* table, nea::PrepJob* jobs_out, cudaStream_t stream,
+             const nea::PrepParams* rowterm = nullptr) {
   nea::PrepParams pp{};
+  if (rowterm) pp = *rowterm;  // row-term fields of the backward
+  pp.n_jobs = 0;
+  pp.total = 0;
   size_t off = 0;
   pp.T = T;
   pp.rope = table;
+  pp.divT = nea::make_fastdiv(uint32_t(T));
+  if (pp.rt_threads) {
+    pp.divTp = nea::make_fastdiv(uint32_t(pp.Tp));
+    pp.divHq = nea::make_fastdiv(uint32_t(pp.Hq));
+  }
   for (int i = 0; i < n; ++i) {
     nea::PrepJob j{};
     j.src = src[i];
     j.H = H[i];
+    j.divH = nea::make_fastdiv(uint32_t(H[i]));
     j.rope = rot[i] && table != nullptr;
     if (!f32 && !j.rope) {  // read in place
       j.hi = static_cast<__nv_bfloat16*>(const_cast<void*>(src[i]));
@@ -267,8 +278,10 @@ int run_prep(uint8_t* base, const void* const* src, const size_t* elems, const i
     pp.total += j.chunks;
     jobs_out[i] = j;
   }
-  if (pp.n_jobs == 0) return NEA_OK;
-  const long long blocks = std::min<long long>((pp.total + 255) / 256, 148LL * 16);
+  const long long per_block = 256LL * nea::kPrepUnroll;
+  pp.prep_blocks = int((pp.total + per_block - 1) / per_block);
+  const long long blocks = pp.prep_blocks + (pp.rt_threads + 255) / 256;
+  if (blocks == 0) return NEA_OK;
   const unsigned g = unsigned(blocks);
   if (D == 64)
     f32 ? nea::attn_prep_kernel<64, true><<<g, 256, 0, stream>>>(pp)
@@ -293,24 +306,20 @@ int launch_fwd(uint32_t& attr_done, const nea::FwdParams& p, cudaStream_t stream
 }
 
 // ----------------------------------------------------------------- backward
-// Row terms, dK/dV kernel, dQ kernel.  `ev` selects profiling events (the
+// dK/dV kernel, dQ kernel.  `ev` selects profiling events (the
 // regular backward records them, the allocation-free one does not).
 template <int D, bool F32IO>
-int launch_bwd(uint32_t& attr_done, const nea::BwdParams& p, const void* O, const void* dO, const float* LSE,
-               cudaStream_t stream, bool ev) {
-  constexpr int kLanes = D / (F32IO ? 4 : 8);
-  const long long threads = static_cast<long long>(p.B) * p.Tp * p.Hq * kLanes;
-  nea::attn_bwd_rowterm_kernel<D, F32IO><<<unsigned((threads + 255) / 256), 256, 0, stream>>>(
-      O, dO, LSE, const_cast<float*>(p.ws), p.B, p.T, p.Tp, p.Hq);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e);
-  if (ev) prof_record(3, stream);
-
+int launch_bwd(uint32_t& attr_done, const nea::BwdParams& p, cudaStream_t stream, bool ev) {
+  cudaError_t e;
   using LK = nea::BwdSmem<D, F32IO, true>;
   auto kk = nea::attn_bwd_kernel<D, F32IO, true>;
   int rc = set_smem(attr_done, 4 + (D == 64) * 2 + F32IO, kk, LK::kAlloc);
   if (rc) return rc;
   kk<<<p.B * p.Hkv * p.n_tiles, LK::kThreads, LK::kAlloc, stream>>>(p);
+  nea::BwdParams pq = p;
+#ifdef NEA_TRACE
+  if (pq.trace) pq.trace += size_t(p.B) * p.Hkv * p.n_tiles * 80;  // dQ stamps follow the dK/dV ones
+#endif
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
   if (ev) prof_record(4, stream);
 
@@ -318,7 +327,7 @@ int launch_bwd(uint32_t& attr_done, const nea::BwdParams& p, const void* O, cons
   auto kq = nea::attn_bwd_kernel<D, F32IO, false>;
   rc = set_smem(attr_done, 8 + (D == 64) * 2 + F32IO, kq, LQ::kAlloc);
   if (rc) return rc;
-  kq<<<p.B * p.Hq * p.n_tiles, LQ::kThreads, LQ::kAlloc, stream>>>(p);
+  kq<<<p.B * p.Hq * p.n_tiles, LQ::kThreads, LQ::kAlloc, stream>>>(pq);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
   if (ev) prof_record(5, stream);
   return NEA_OK;
@@ -370,7 +379,17 @@ int run_bwd(uint32_t& attr_done, uint8_t* ws, const float2* rope, int* status, c
     const size_t elems[4] = {nq, nk, nk, nq};
     const int H[4] = {Hq, Hkv, Hkv, Hq}, rot[4] = {1, 1, 0, 0};
     nea::PrepJob jobs[4];
-    if ((rc = run_prep(ws + rowterm_bytes, src, elems, H, rot, 4, T, D, f32, rope, jobs, stream))) return rc;
+    nea::PrepParams rt{};  // the row terms ride in the same launch
+    rt.O = O;
+    rt.dO = dO;
+    rt.LSE = LSE;
+    rt.ws = reinterpret_cast<float*>(ws);
+    rt.B = B;
+    rt.Tp = p.Tp;
+    rt.Hq = Hq;
+    rt.rt_threads = static_cast<long long>(B) * p.Tp * Hq * (D / (f32 ? 4 : 8));
+    if ((rc = run_prep(ws + rowterm_bytes, src, elems, H, rot, 4, T, D, f32, rope, jobs, stream, &rt))) return rc;
+    if (ev) prof_record(3, stream);
     if ((rc = make_tile_map(&p.tm_q, jobs[0].hi, B, T, Hq, D)) ||
         (rc = make_tile_map(&p.tm_k, jobs[1].hi, B, T, Hkv, D)) ||
         (rc = make_tile_map(&p.tm_v, jobs[2].hi, B, T, Hkv, D)) ||
@@ -398,8 +417,11 @@ int run_bwd(uint32_t& attr_done, uint8_t* ws, const float2* rope, int* status, c
   p.scale_log2 = float(1.4426950408889634 / std::sqrt(double(D)));
   p.err = status;
   p.wait_limit = static_cast<unsigned long long>(t_wait_limit_ns);
+#ifdef NEA_TRACE
+  p.trace = t_trace_bwd;
+#endif
   return dispatch(D, dtype, [&](auto d, auto f) {
-    return launch_bwd<decltype(d)::value, decltype(f)::value>(attr_done, p, O, dO, LSE, stream, ev);
+    return launch_bwd<decltype(d)::value, decltype(f)::value>(attr_done, p, stream, ev);
   });
 }
 
@@ -436,6 +458,7 @@ int nea_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
     if ((rc = ensure_ws(*st, prep_bytes(elems, rot, 3, f32, rope != nullptr)))) return rc;
     nea::PrepJob jobs[3];
     if ((rc = run_prep(st->ws, src, elems, H, rot, 3, T, D, f32, rope, jobs, stream))) return rc;
+    prof_record(6, stream);
     if ((rc = make_tile_map(&p.tm_q, jobs[0].hi, B, T, Hq, D)) ||
         (rc = make_tile_map(&p.tm_k, jobs[1].hi, B, T, Hkv, D)) ||
         (rc = make_tile_map(&p.tm_v, jobs[2].hi, B, T, Hkv, D)))
@@ -514,6 +537,7 @@ void nea_debug_inject(int flags) { t_debug_flags = flags; }
 
 #ifdef NEA_TRACE
 void nea_debug_set_trace(void* buffer) { t_trace = static_cast<unsigned long long*>(buffer); }
+void nea_debug_set_trace_bwd(void* buffer) { t_trace_bwd = static_cast<unsigned long long*>(buffer); }
 #endif
 
 void nea_set_profile_events(void* const* events, int n) {

@@ -3,7 +3,7 @@
 // 3-4; agentlenshq.com summary, "Validation and stability"); the design here
 // is the recompute-from-LSE backward of tiled attention:
 //
-//   row term     Dv_i = sum_d dO_id O_id                 (attn_bwd_rowterm)
+//   row term     Dv_i = sum_d dO_id O_id                 (operand prologue, nea_prep.cuh)
 //   per tile     S = Q' K'^T, P = exp(scale S - LSE), dP = dO V^T,
 //                dS = P o (dP - Dv),
 //                dV += P^T dO, dK' += dS^T Q', dQ' += dS K'  (x scale)
@@ -29,75 +29,21 @@
 //   S_rc  = R1 C1^T      (R1 = K' or Q', C1 = Q' or K')   -> TMEM [0,128)
 //   dP_rc = R2 C2^T      (R2 = V or dO,  C2 = dO or V)    -> TMEM [128,256)
 //   P is kept in fp32 registers for dS and, for DKDV, as bf16 in TMEM
-//   [384,448) for the dV product; each warp writes its bf16 dS over the first
-//   half of its own dP columns
+//   [384,448) for the dV product; bf16 dS goes to TMEM [448,512)
 //   DKDV: acc1 += P  C2   (dV), acc2 += dS C1 (dK)   (C1, C2 as MN-major B)
 //   DQ:   acc1 += dS C1   (dQ)
-// S of item k+1 is issued as soon as the rows have read S of item k, so it
-// overlaps the dS phase; dP of item k+1 waits for the dS MMA of item k.
+// Issue order per item k: dP(k); S(k+1) as soon as the rows hold S(k) in
+// registers; dV(k) once P(k) is written; dK/dQ(k) once dS(k) is written.  The
+// rows overwrite P and dS of item k-1 only after the commit that follows
+// dK/dQ(k-1) (which covers every earlier MMA).
 #pragma once
 
 #include <cuda.h>
 
+#include "nea_prep.cuh"
 #include "nea_tiles.cuh"
 
 namespace nea {
-
-// ---------------------------------------------------------------- row term
-// Per-row terms of the backward, in a workspace ws[B*Hq][2][Tp] (Tp = T
-// rounded up to whole 128-row tiles, so a tile of it is one TMA box):
-//   ws[bh][0][t] = -LSE[b][h][t] * log2(e)          (-inf for t >= T)
-//   ws[bh][1][t] = Dv = sum_d dO[b][t][h][d] O[b][t][h][d]   (0 for t >= T)
-// The padding makes P = exp2(s*c + ws0) vanish for queries past T.  One group
-// of D/ELEMS lanes per (b, t, h) row, t over [0, Tp).
-template <int D, bool F32IO>
-__global__ void __launch_bounds__(256) attn_bwd_rowterm_kernel(const void* __restrict__ O,
-                                                               const void* __restrict__ dO,
-                                                               const float* __restrict__ LSE,
-                                                               float* __restrict__ ws, int B, int T, int Tp,
-                                                               int Hq) {
-  constexpr int kElems = F32IO ? 4 : 8;    // elements per 16-byte chunk
-  constexpr int kLanes = D / kElems;       // lanes per row: 4, 8 or 16
-  const long gtid = long(blockIdx.x) * blockDim.x + threadIdx.x;
-  const long prow = gtid / kLanes;         // (b, t, h) over t in [0, Tp)
-  const int c = int(gtid % kLanes);
-  const int h = int(prow % Hq);
-  const long bt = prow / Hq;
-  const int t = int(bt % Tp);
-  const long b = bt / Tp;
-  if (b >= B) return;  // whole groups of lanes leave together
-  float* out = ws + (b * Hq + h) * 2 * long(Tp) + t;
-  if (t >= T) {
-    if (c == 0) {
-      out[0] = -INFINITY;
-      out[Tp] = 0.f;
-    }
-    return;
-  }
-  const long row = (b * T + t) * Hq + h;
-  float acc = 0.f;
-  {
-    if constexpr (F32IO) {
-      const float4 a = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(O) + row * D) + c);
-      const float4 z = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(dO) + row * D) + c);
-      acc = a.x * z.x + a.y * z.y + a.z * z.z + a.w * z.w;
-    } else {
-      const uint4 a = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(O) + row * D) + c);
-      const uint4 z = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(dO) + row * D) + c);
-      acc = bf16_lo_f(a.x) * bf16_lo_f(z.x) + bf16_hi_f(a.x) * bf16_hi_f(z.x) + bf16_lo_f(a.y) * bf16_lo_f(z.y) +
-            bf16_hi_f(a.y) * bf16_hi_f(z.y) + bf16_lo_f(a.z) * bf16_lo_f(z.z) + bf16_hi_f(a.z) * bf16_hi_f(z.z) +
-            bf16_lo_f(a.w) * bf16_lo_f(z.w) + bf16_hi_f(a.w) * bf16_hi_f(z.w);
-    }
-  }
-  // the kLanes lanes of a row are consecutive and leave or stay together
-  const unsigned group = (kLanes == 32 ? kFullMask : ((1u << kLanes) - 1u) << (threadIdx.x & 31 & ~(kLanes - 1)));
-#pragma unroll
-  for (int off = kLanes / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(group, acc, off);
-  if (c == 0) {
-    out[0] = __ldg(LSE + (b * Hq + h) * long(T) + t) * -1.4426950408889634f;
-    out[Tp] = acc;
-  }
-}
 
 // ---------------------------------------------------------------- main kernel
 struct BwdParams {
@@ -113,7 +59,7 @@ struct BwdParams {
   CUtensorMap tm_v_lo;
   CUtensorMap tm_do_lo;
   CUtensorMap tm_ws;   // row terms ws[B*Hq][2][Tp] fp32, box {128, 2, 1}
-  const float* ws;     // see attn_bwd_rowterm_kernel
+  const float* ws;     // row terms, see nea_prep.cuh
   int Tp;              // T rounded up to a multiple of 128
   void* dQ;
   void* dK;
@@ -126,6 +72,7 @@ struct BwdParams {
   float scale;        // 1 / sqrt(D)
   int* err;
   unsigned long long wait_limit;
+  unsigned long long* trace;  // per-CTA phase stamps (NEA_TRACE builds only)
 };
 
 template <int D, bool F32IO, bool DKDV>
@@ -138,8 +85,8 @@ struct BwdSmem {
   static constexpr uint32_t kColVec = 2 * kTile;             // per-column -LSE*log2e and Dv (DKDV)
   static constexpr uint32_t kStageBytes = kColVec + (DKDV ? 1024 : 0);
   static constexpr uint32_t kBars = kStage0 + kStages * kStageBytes;
-  // rtma, tma[S], empty[S], s, dp, p, ds, dk, fin
-  static constexpr int kNumBars = 1 + 2 * kStages + 6;
+  // rtma, tma[S], empty[S], s, dp, p, ds, dk, fin, sread
+  static constexpr int kNumBars = 1 + 2 * kStages + 7;
   static constexpr uint32_t kMisc = kBars + 8 * kNumBars;
   static constexpr uint32_t kUsed = kMisc + 16;
   static constexpr uint32_t kAlloc = kUsed + 1024 > 116u * 1024u ? kUsed + 1024 : 116u * 1024u;
@@ -147,23 +94,6 @@ struct BwdSmem {
   static_assert(kStage0 % 1024 == 0 && kStageBytes % 1024 == 0, "operand tiles need 1024-byte alignment");
   static_assert(kAlloc <= 232448, "shared memory");
 };
-
-// Writes N consecutive elements of a row held in registers (float) at
-// element offset `off` of a tensor in the storage type (16-byte aligned).
-template <int N, bool F32IO>
-__device__ __forceinline__ void store_span(void* dst, size_t off, const float* v) {
-  if constexpr (F32IO) {
-    float4* q = reinterpret_cast<float4*>(static_cast<float*>(dst) + off);
-#pragma unroll
-    for (int i = 0; i < N / 4; ++i) q[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-  } else {
-    uint4* q = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dst) + off);
-#pragma unroll
-    for (int i = 0; i < N / 8; ++i)
-      q[i] = make_uint4(pack_bf16(v[8 * i], v[8 * i + 1]), pack_bf16(v[8 * i + 2], v[8 * i + 3]),
-                        pack_bf16(v[8 * i + 4], v[8 * i + 5]), pack_bf16(v[8 * i + 6], v[8 * i + 7]));
-  }
-}
 
 // N consecutive TMEM columns of this thread's lane (N = 16, 32 or 64).
 template <int N>
@@ -207,12 +137,14 @@ __global__ void __launch_bounds__(BwdSmem<D, F32IO, DKDV>::kThreads, 1)
   uint64_t* bar_ds = bar_s + 3;              // rows wrote dS (count 256)
   uint64_t* bar_dk = bar_s + 4;              // dS MMA of an item done
   uint64_t* bar_fin = bar_s + 5;
+  uint64_t* bar_sread = bar_s + 6;           // rows hold S in registers (count 256)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const WaitCtl wc{p.err, p.wait_limit, abort_flag};
+  NEA_TRACE_STAMP(p, 0, tid == 0);
 
   // ---- work decomposition
   // DKDV: blockIdx -> (key tile ascending = most causal work first, b, g)
@@ -253,6 +185,7 @@ __global__ void __launch_bounds__(BwdSmem<D, F32IO, DKDV>::kThreads, 1)
     mbar_init(bar_ds, 256);
     mbar_init(bar_dk, 1);
     mbar_init(bar_fin, 1);
+    mbar_init(bar_sread, 256);
     mbar_init_fence();
   }
   if (warp == 0) tmem_alloc(tmem_holder, 512);
@@ -260,7 +193,7 @@ __global__ void __launch_bounds__(BwdSmem<D, F32IO, DKDV>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_holder;
-  constexpr uint32_t kColS = 0, kColDP = 128, kColAcc1 = 256, kColAcc2 = 256 + D, kColP = 384;
+  constexpr uint32_t kColS = 0, kColDP = 128, kColAcc1 = 256, kColAcc2 = 256 + D, kColP = 384, kColDS = 448;
 
   if (warp == 9) {
     // ------------------------------------------------------------ TMA
@@ -312,28 +245,8 @@ __global__ void __launch_bounds__(BwdSmem<D, F32IO, DKDV>::kThreads, 1)
       const uint32_t sR1 = smem_u32(smem + L::kR1), sR2 = smem_u32(smem + L::kR2);
       constexpr uint32_t accG = DKDV ? kColAcc2 : kColAcc1;  // accumulator of dS C1
       auto stage_c1 = [&](int k) { return smem_u32(smem + L::kStage0 + (k % NS) * L::kStageBytes); };
-      // acc += dS_k C1_k, then release the stage of item k.  dS of columns
-      // [64h, 64h+64) sits in TMEM columns kColDP + 64h .. + 31.
-      auto issue_ds = [&](int k) -> bool {
-        if (!wait_thread(bar_ds, k & 1, wc, kErrWaitSoftmax)) return false;
-        tc_fence_after();
+      auto issue_s = [&](int k) {
         const uint32_t sC1 = stage_c1(k);
-#pragma unroll
-        for (int kk = 0; kk < kTileRows / 16; ++kk)
-          mma_ts(tbase + accG, tbase + kColDP + (kk >> 2) * 64 + (kk & 3) * 8,
-                 smem_desc(sC1 + kk * 16 * RB, RB, kTileRows * RB), idAcc, (k | kk) != 0);
-        tc_commit(&bar_empty[k % NS]);
-        tc_commit(bar_dk);
-        return true;
-      };
-      bool ok = wait_thread(bar_rtma, 0, wc, kErrWaitProducer);
-      for (int k = 0; ok && k < n_items; ++k) {
-        const int s = k % NS;
-        if (!wait_thread(&bar_tma[s], (k / NS) & 1, wc, kErrWaitProducer)) { ok = false; break; }
-        // S_k overwrites S_{k-1}: the rows must have read it
-        if (k > 0 && !wait_thread(bar_p, (k - 1) & 1, wc, kErrWaitSoftmax)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t sC1 = stage_c1(k), sC2 = sC1 + L::kTile;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
 #pragma unroll
@@ -341,10 +254,16 @@ __global__ void __launch_bounds__(BwdSmem<D, F32IO, DKDV>::kThreads, 1)
             mma_ss(tbase + kColS, smem_desc(sR1 + (term == 2 ? OPB : 0) + kk * 32, RB, 16),
                    smem_desc(sC1 + (term == 1 ? OPB : 0) + kk * 32, RB, 16), idSS, (kk | term) != 0);
         tc_commit(bar_s);
-        if (k > 0) {
-          // dP_k overwrites dS_{k-1}: issue its MMA and wait until it has run
-          if (!issue_ds(k - 1) || !wait_thread(bar_dk, (k - 1) & 1, wc, kErrWaitMma)) { ok = false; break; }
-        }
+      };
+      bool ok = wait_thread(bar_rtma, 0, wc, kErrWaitProducer) &&
+                (n_items == 0 || wait_thread(&bar_tma[0], 0, wc, kErrWaitProducer));
+      if (ok && n_items > 0) {
+        tc_fence_after();
+        issue_s(0);
+      }
+      for (int k = 0; ok && k < n_items; ++k) {
+        const uint32_t sC1 = stage_c1(k), sC2 = sC1 + L::kTile;
+        // dP(k) overwrites dP(k-1), which the rows read before dS(k-1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
 #pragma unroll
@@ -352,6 +271,18 @@ __global__ void __launch_bounds__(BwdSmem<D, F32IO, DKDV>::kThreads, 1)
             mma_ss(tbase + kColDP, smem_desc(sR2 + (term == 2 ? OPB : 0) + kk * 32, RB, 16),
                    smem_desc(sC2 + (term == 1 ? OPB : 0) + kk * 32, RB, 16), idSS, (kk | term) != 0);
         tc_commit(bar_dp);
+        NEA_TRACE_STAMP(p, 36 + min(k, 7), true);
+        if (k + 1 < n_items) {
+          // S(k+1) overwrites S(k): the rows must hold it in registers
+          if (!wait_thread(bar_sread, k & 1, wc, kErrWaitSoftmax) ||
+              !wait_thread(&bar_tma[(k + 1) % NS], ((k + 1) / NS) & 1, wc, kErrWaitProducer)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_s(k + 1);
+          NEA_TRACE_STAMP(p, 44 + min(k, 7), true);
+        }
         if (DKDV) {
           if (!wait_thread(bar_p, k & 1, wc, kErrWaitSoftmax)) { ok = false; break; }
           tc_fence_after();
@@ -359,9 +290,19 @@ __global__ void __launch_bounds__(BwdSmem<D, F32IO, DKDV>::kThreads, 1)
           for (int kk = 0; kk < kTileRows / 16; ++kk)
             mma_ts(tbase + kColAcc1, tbase + kColP + kk * 8, smem_desc(sC2 + kk * 16 * RB, RB, kTileRows * RB),
                    idAcc, (k | kk) != 0);
+          NEA_TRACE_STAMP(p, 52 + min(k, 7), true);
         }
+        // acc += dS(k) C1(k), then release the stage of item k
+        if (!wait_thread(bar_ds, k & 1, wc, kErrWaitSoftmax)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kTileRows / 16; ++kk)
+          mma_ts(tbase + accG, tbase + kColDS + kk * 8, smem_desc(sC1 + kk * 16 * RB, RB, kTileRows * RB), idAcc,
+                 (k | kk) != 0);
+        tc_commit(&bar_empty[k % NS]);
+        tc_commit(bar_dk);
+        NEA_TRACE_STAMP(p, 60 + min(k, 7), true);
       }
-      if (ok && n_items > 0) issue_ds(n_items - 1);
       tc_commit(bar_fin);
       drain_wait(bar_fin, 0, wc);
     }
@@ -390,11 +331,14 @@ __global__ void __launch_bounds__(BwdSmem<D, F32IO, DKDV>::kThreads, 1)
       // DKDV reads the per-column -LSE*log2e / Dv the TMA landed in the stage
       if (DKDV && !wait_warp(&bar_tma[s], (k / NS) & 1, wc, kErrWaitProducer)) { ok = false; break; }
       if (!wait_warp(bar_s, k & 1, wc, kErrWaitMma)) { ok = false; break; }
+      NEA_TRACE_STAMP(p, 4 + min(k, 7), tid == 0);
       tc_fence_after();
       const int col0 = ct * kTileRows + cb;  // position of this warp's first column
       // ---- P phase: P = exp2(s * scale_log2 - LSE*log2e), masked
       uint32_t sv[64];
       tmem_ld64(lane_base + kColS + cb, sv);
+      tc_fence_before();
+      mbar_arrive(bar_sread);  // S(k+1) may overwrite S(k) now
       if ((p.causal && ct == rt) || ct * kTileRows + kTileRows > p.T) {  // same for the whole tile
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
@@ -421,17 +365,22 @@ __global__ void __launch_bounds__(BwdSmem<D, F32IO, DKDV>::kThreads, 1)
         pv[4 * i + 2] = ex2(t2);
         pv[4 * i + 3] = ex2(t3);
       }
+      // P(k-1) and dS(k-1) stay in TMEM until dV/dK/dQ(k-1) have read them
+      if (k > 0 && !wait_warp(bar_dk, (k - 1) & 1, wc, kErrWaitMma)) { ok = false; break; }
       if (DKDV) {  // bf16 P for the dV product
+        tc_fence_after();
         uint32_t ph[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) ph[i] = pack_bf16(pv[2 * i], pv[2 * i + 1]);
         tmem_st32(lane_base + kColP + 32 * hf, ph);
         tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar_p);
       }
-      tc_fence_before();
-      mbar_arrive(bar_p);
-      // ---- dS phase: dS = P (dP - Dv), bf16, over dP in TMEM
+      NEA_TRACE_STAMP(p, 12 + min(k, 7), tid == 0);
+      // ---- dS phase: dS = P (dP - Dv), bf16, into its own TMEM columns
       if (!wait_warp(bar_dp, k & 1, wc, kErrWaitMma)) { ok = false; break; }
+      NEA_TRACE_STAMP(p, 20 + min(k, 7), tid == 0);
       tc_fence_after();
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
@@ -456,12 +405,12 @@ __global__ void __launch_bounds__(BwdSmem<D, F32IO, DKDV>::kThreads, 1)
           pk[2 * i] = pack_bf16(a0, a1);
           pk[2 * i + 1] = pack_bf16(a2, a3);
         }
-        // packed columns [16c, 16c+16) of this warp's dP were read in chunk 0
-        tmem_st16(lane_base + kColDP + cb + 16 * c, pk);
+        tmem_st16(lane_base + kColDS + 32 * hf + 16 * c, pk);
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar_ds);
+      NEA_TRACE_STAMP(p, 28 + min(k, 7), tid == 0);
     }
     if (ok && wait_warp(bar_fin, 0, wc, kErrWaitMma)) {
       tc_fence_after();
@@ -517,6 +466,7 @@ __global__ void __launch_bounds__(BwdSmem<D, F32IO, DKDV>::kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tbase, 512);
   }
+  NEA_TRACE_STAMP(p, 78, tid == 0);
 }
 
 }  // namespace nea

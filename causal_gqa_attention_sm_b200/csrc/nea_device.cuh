@@ -15,6 +15,26 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+// Phase stamps for performance analysis: compiled only with -DNEA_TRACE, when
+// `p.trace` receives per CTA 80 %globaltimer values (slot 79: SM id).
+#ifdef NEA_TRACE
+#define NEA_TRACE_STAMP(p, slot, cond)                                                  \
+  do {                                                                                  \
+    if ((p).trace && (cond)) {                                                          \
+      (p).trace[size_t(blockIdx.x) * 80 + (slot)] = nea::global_timer_ns();             \
+      if ((slot) == 0) {                                                                \
+        unsigned smid_;                                                                 \
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid_));                              \
+        (p).trace[size_t(blockIdx.x) * 80 + 79] = smid_;                                \
+      }                                                                                 \
+    }                                                                                   \
+  } while (0)
+#else
+#define NEA_TRACE_STAMP(p, slot, cond) \
+  do {                                 \
+  } while (0)
+#endif
+
 namespace nea {
 
 constexpr uint32_t kFullMask = 0xffffffffu;
@@ -81,8 +101,7 @@ __device__ __forceinline__ void raise_error(const WaitCtl& c, int code) {
 // Wait of a single thread for the phase of `bar` with the given parity to
 // complete.  Returns false, after recording `code`, once the CTA aborted or
 // the wait exceeded its limit.
-__device__ __noinline__ bool wait_thread(uint64_t* bar, uint32_t parity, const WaitCtl& c, int code) {
-  if (mbar_try_wait(bar, parity)) return true;
+__device__ __noinline__ bool wait_thread_slow(uint64_t* bar, uint32_t parity, const WaitCtl& c, int code) {
   const uint64_t t0 = global_timer_ns();
   for (;;) {
 #pragma unroll 1
@@ -99,9 +118,8 @@ __device__ __noinline__ bool wait_thread(uint64_t* bar, uint32_t parity, const W
 // Same wait, taken by all 32 lanes of a warp with a warp-uniform outcome, so
 // that warp-collective tcgen05 loads/stores after it stay converged.  Every
 // lane performs its own successful try_wait (acquire) before proceeding.
-__device__ __noinline__ bool wait_warp(uint64_t* bar, uint32_t parity, const WaitCtl& c, int code) {
-  bool done = mbar_try_wait(bar, parity);
-  if (__all_sync(kFullMask, done)) return true;
+__device__ __noinline__ bool wait_warp_slow(uint64_t* bar, uint32_t parity, const WaitCtl& c, int code) {
+  bool done = false;
   const uint64_t t0 = global_timer_ns();
   for (;;) {
     done = done || mbar_try_wait(bar, parity);
@@ -113,6 +131,15 @@ __device__ __noinline__ bool wait_warp(uint64_t* bar, uint32_t parity, const Wai
       return false;
     }
   }
+}
+
+// The waits proper: a first test inline (no call, so nothing is saved around
+// it when the phase is already complete), the bounded loop out of line.
+__device__ __forceinline__ bool wait_thread(uint64_t* bar, uint32_t parity, const WaitCtl& c, int code) {
+  return mbar_try_wait(bar, parity) || wait_thread_slow(bar, parity, c, code);
+}
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, const WaitCtl& c, int code) {
+  return __all_sync(kFullMask, mbar_try_wait(bar, parity)) || wait_warp_slow(bar, parity, c, code);
 }
 
 // Wait that ignores the CTA's abort flag (still bounded by the limit, records
@@ -252,6 +279,27 @@ __device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[128]) {
       : "memory");
 }
 
+// Two runs of 64 columns (at taddr0 into r[0..63], at taddr1 into
+// r[64..127]) with one wait.
+__device__ __forceinline__ void tmem_ld64x2(uint32_t taddr0, uint32_t taddr1, uint32_t (&r)[128]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%128];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,"
+      "%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,"
+      "%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,"
+      "%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%129];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : NEA_R8(0), NEA_R8(8), NEA_R8(16), NEA_R8(24), NEA_R8(32), NEA_R8(40), NEA_R8(48), NEA_R8(56),
+        NEA_R8(64), NEA_R8(72), NEA_R8(80), NEA_R8(88), NEA_R8(96), NEA_R8(104), NEA_R8(112), NEA_R8(120)
+      : "r"(taddr0), "r"(taddr1)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
@@ -345,6 +393,27 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// ------------------------------------------------------- integer division
+// Division of 32-bit unsigned n by an invariant divisor d >= 1 with one
+// multiply-high, an add and two shifts (Granlund and Montgomery, "Division by
+// invariant integers using multiplication", PLDI 1994: with l = ceil(log2 d),
+// m = floor(2^32 (2^l - d) / d) + 1, n / d = (t + ((n - t) >> 1)) >> (l - 1)
+// where t = mulhi(m, n), for every n < 2^32).
+struct FastDiv {
+  uint32_t d, m, l;
+};
+__host__ __device__ inline FastDiv make_fastdiv(uint32_t d) {
+  uint32_t l = 0;
+  while (l < 32 && (uint64_t(1) << l) < d) ++l;
+  const uint32_t m = uint32_t(((uint64_t(1) << 32) * ((uint64_t(1) << l) - d)) / d + 1);
+  return FastDiv{d, m, l};
+}
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
+  if (f.l == 0) return n;  // d == 1
+  const uint32_t t = __umulhi(f.m, n);
+  return (t + ((n - t) >> 1)) >> (f.l - 1);
 }
 
 // ------------------------------------------------------- packed fp32 pairs

@@ -19,16 +19,20 @@
 //   0-3, 4-7   softmax of tile A, of tile B: thread r owns row r (TMEM lane
 //              r) and loads its whole 128-column score row with one TMEM
 //              load; the row max comes from a three-input max tree, then
-//              P = exp(s - m) is written back as bf16 (hi over S, lo in its
-//              own columns for float32 storage), with paired fp32 arithmetic;
-//              the running max m moves only when it grows by more than 2^8
-//              (O rescaled in TMEM then); the epilogue writes O / l and LSE.
+//              P = exp(s - m) is written as bf16, with paired fp32
+//              arithmetic; the running max m moves only when it grows by more
+//              than 2^8 (O rescaled in TMEM then); the epilogue writes O / l
+//              and LSE.
 //   8, 9       MMA issuers, one thread each: warp 8 for tile A, warp 9 for tile B;
 //              S_X = Q_X K_j^T, O_X += P_X V_j, each waiting only on its own
 //              tile, so one tile's softmax overlaps the other tile's MMAs.
 //   10         TMA: query tiles, then K and V tiles into two rings (K stages
 //              free as soon as S is computed, V stages after PV).
-// TMEM per tile X: S [256X, 256X+128), O [256X+128, +D), P lo [256X+192, +64).
+// TMEM per tile X: S [256X, 256X+128), O [256X+128, +D), and
+//   bf16 storage: P [256X+192, +64) in its own columns, so S_X(j+1) is issued
+//     as soon as the softmax has loaded S_X(j) and runs under its exponentials;
+//   float32 storage: P hi over S [256X, +64), P lo [256X+192, +64) (hi and lo
+//     need the room), so S_X(j+1) waits until PV_X(j) has read P.
 // Causal tiles above the diagonal are never visited; only the diagonal tile
 // and a ragged last tile are masked.
 #pragma once
@@ -36,26 +40,6 @@
 #include <cuda.h>
 
 #include "nea_tiles.cuh"
-
-// Phase stamps for performance analysis: compiled only with -DNEA_TRACE, when
-// `p.trace` receives per CTA 80 %globaltimer values (slot 79: SM id).
-#ifdef NEA_TRACE
-#define NEA_TRACE_STAMP(p, slot, cond)                                                  \
-  do {                                                                                  \
-    if ((p).trace && (cond)) {                                                          \
-      (p).trace[size_t(blockIdx.x) * 80 + (slot)] = nea::global_timer_ns();             \
-      if ((slot) == 0) {                                                                \
-        unsigned smid_;                                                                 \
-        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid_));                              \
-        (p).trace[size_t(blockIdx.x) * 80 + 79] = smid_;                                \
-      }                                                                                 \
-    }                                                                                   \
-  } while (0)
-#else
-#define NEA_TRACE_STAMP(p, slot, cond) \
-  do {                                 \
-  } while (0)
-#endif
 
 namespace nea {
 
@@ -94,7 +78,7 @@ struct FwdSmem {
   static constexpr uint32_t kV0 = kK0 + kNK * kKStage;
   static constexpr uint32_t kVStage = kTile;
   static constexpr uint32_t kBars = kV0 + kNV * kVStage;
-  // qtma, K tma/empty, V tma/empty, s[2], p[2], o[2], fin[2], turn[2]
+  // qtma, K tma/empty, V tma/empty, s[2], p[2], o[2], fin[2], sread[2]
   static constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 10;
   static constexpr uint32_t kMisc = kBars + 8 * kNumBars;
   static constexpr uint32_t kUsed = kMisc + 16;
@@ -116,6 +100,7 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
   constexpr uint32_t OPB = TileGeom<D>::kOpBytes;
   constexpr int NK = L::kNK, NV = L::kNV;
   constexpr int kTerms = F32IO ? 3 : 1;
+  constexpr bool kSepP = !F32IO;  // P in its own TMEM columns
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
@@ -129,7 +114,7 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
   uint64_t* bar_p = bar_s + 2;                          // [2] P_X written (count 128)
   uint64_t* bar_o = bar_s + 4;                          // [2] PV_X done
   uint64_t* bar_fin = bar_s + 6;                        // [2] per issuer
-  uint64_t* bar_turn = bar_s + 8;                       // [2] exponentials of X done (count 128)
+  uint64_t* bar_sread = bar_s + 8;                      // [2] S_X loaded by the softmax (count 128)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
 
@@ -161,7 +146,7 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
       mbar_init(&bar_s[x], 1);
       mbar_init(&bar_p[x], 128);
       mbar_init(&bar_o[x], 1);
-      mbar_init(&bar_turn[x], 128);
+      mbar_init(&bar_sread[x], 128);
     }
     mbar_init(&bar_fin[0], 1);
     mbar_init(&bar_fin[1], 1);
@@ -181,7 +166,8 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
     const int my_qt = x ? qt_b : qt_a, my_nkv = x ? nkv_b : nkv_a;
     const int q = my_qt * kTileRows + r;
     const uint32_t lane_base = tmem_addr(tbase, uint32_t(warp & 3) * 32, 0);
-    const uint32_t scol = lane_base + 256 * x, ocol = scol + 128, plocol = scol + 192;
+    // pcol: P (bf16 storage) or P lo (float32 storage)
+    const uint32_t scol = lane_base + 256 * x, ocol = scol + 128, pcol = scol + 192;
     float m_run = -INFINITY;
     uint64_t l01 = 0, l23 = 0;  // partial row sums, two packed pairs
     const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
@@ -192,6 +178,10 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
       tc_fence_after();
       uint32_t sv[128];
       tmem_ld128(scol, sv);
+      if (kSepP) {  // S_X(j) is in registers: the next S may overwrite it
+        tc_fence_before();
+        mbar_arrive(&bar_sread[x]);
+      }
       const int kv0 = j * kTileRows;
       if ((p.causal && j == my_qt) || kv0 + kTileRows > p.T) {  // same for the whole tile
         const int lim = (p.causal ? min(q, p.T - 1) : p.T - 1) - kv0;  // last visible column
@@ -208,43 +198,9 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
       l01 = f2_mul(l01, a2);
       l23 = f2_mul(l23, a2);
       const uint64_t nm2 = f2_pack(-m_run, -m_run);
-      // The two tiles take turns on the exponential unit, A(j) after B(j-1)
-      // and B(j) after A(j), so that each tile's MMAs run under the other
-      // tile's exponentials instead of both tiles waiting on the MMAs at once.
-      if (has_b && ((x == 0 && j > 0) || (x == 1 && j < nkv_a)) &&
-          !wait_warp(&bar_turn[x ^ 1], (x == 0 ? j - 1 : j) & 1, wc, kErrWaitSoftmax)) {
-        ok = false;
-        break;
-      }
-      // P = exp2(s * scale_log2 - m) -> bf16 (hi over S, lo apart)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t hi[16], lo[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int e = 32 * c + 2 * i;
-          float t0, t1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sc2, nm2), t0, t1);
-          const float p0 = ex2(t0), p1 = ex2(t1);
-          const uint64_t pp = f2_pack(p0, p1);
-          if (i & 1) l23 = f2_add(l23, pp); else l01 = f2_add(l01, pp);
-          hi[i] = pack_bf16(p0, p1);
-          if (F32IO) {
-            float r0, r1;
-            f2_unpack(f2_sub(pp, f2_pack(bf16_lo_f(hi[i]), bf16_hi_f(hi[i]))), r0, r1);
-            lo[i] = pack_bf16(r0, r1);
-          }
-        }
-        // every column of S is in registers already
-        tmem_st16(scol + 16 * c, hi);
-        if (F32IO) tmem_st16(plocol + 16 * c, lo);
-      }
-      mbar_arrive(&bar_turn[x]);
-      if (__any_sync(kFullMask, alpha != 1.f && j > 0)) {
-        // O holds the sum over tiles < j: PV_X(j-1) has landed (S_X(j) was
-        // issued after it); rescale
-        if (!wait_warp(&bar_o[x], (j - 1) & 1, wc, kErrWaitMma)) { ok = false; break; }
-        tc_fence_after();
+      // O rescale by alpha: O holds the sum over key tiles < j once PV_X(j-1)
+      // has completed
+      auto rescale_o = [&]() {
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t rr[32];
@@ -252,6 +208,57 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
           tmem_st32(ocol + 32 * c, rr);
+        }
+      };
+      if constexpr (kSepP) {
+        // P = exp2(s * scale_log2 - m) -> bf16, all 128 columns in registers
+        uint32_t pk[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          float t0, t1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), sc2, nm2), t0, t1);
+          const float p0 = ex2(t0), p1 = ex2(t1);
+          if (i & 1) l23 = f2_add(l23, f2_pack(p0, p1)); else l01 = f2_add(l01, f2_pack(p0, p1));
+          pk[i] = pack_bf16(p0, p1);
+        }
+        // PV_X(j-1) has read P_X(j-1) and updated O before both are touched
+        if (j > 0 && !wait_warp(&bar_o[x], (j - 1) & 1, wc, kErrWaitMma)) { ok = false; break; }
+        tc_fence_after();
+        if (__any_sync(kFullMask, alpha != 1.f && j > 0)) rescale_o();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t part[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) part[i] = pk[16 * c + i];
+          tmem_st16(pcol + 16 * c, part);
+        }
+      } else {
+        // P = exp2(s * scale_log2 - m) -> bf16 hi over S, lo apart
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t hi[16], lo[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int e = 32 * c + 2 * i;
+            float t0, t1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sc2, nm2), t0, t1);
+            const float p0 = ex2(t0), p1 = ex2(t1);
+            const uint64_t pp = f2_pack(p0, p1);
+            if (i & 1) l23 = f2_add(l23, pp); else l01 = f2_add(l01, pp);
+            hi[i] = pack_bf16(p0, p1);
+            float r0, r1;
+            f2_unpack(f2_sub(pp, f2_pack(bf16_lo_f(hi[i]), bf16_hi_f(hi[i]))), r0, r1);
+            lo[i] = pack_bf16(r0, r1);
+          }
+          // every column of S is in registers already
+          tmem_st16(scol + 16 * c, hi);
+          tmem_st16(pcol + 16 * c, lo);
+        }
+        if (__any_sync(kFullMask, alpha != 1.f && j > 0)) {
+          // PV_X(j-1) has landed (S_X(j) was issued after it)
+          if (!wait_warp(&bar_o[x], (j - 1) & 1, wc, kErrWaitMma)) { ok = false; break; }
+          tc_fence_after();
+          rescale_o();
         }
       }
       tmem_st_wait();
@@ -277,7 +284,7 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
         const float inv = 1.f / l_run;
 #pragma unroll
         for (int i = 0; i < D; ++i) o[i] *= inv;
-        store_row<D, F32IO>(p.O, b, q, h, p.T, p.Hq, o);
+        store_span<D, F32IO>(p.O, ((size_t(b) * p.T + q) * p.Hq + h) * D, o);
         // LSE = ln(2^m * l) with m in log2 units of the scaled scores
         p.LSE[(size_t(b) * p.Hq + h) * p.T + q] = (m_run + log2f(l_run)) * 0.69314718055994531f;
       }
@@ -366,9 +373,21 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
         }
         for (int j = 0; ok && j < my_nkv; ++j) {
           const int sv = j % NV;
+          if (kSepP && j + 1 < my_nkv) {
+            // S_X(j+1) as soon as the softmax holds S_X(j) in registers
+            const int sk = (j + 1) % NK;
+            if (!wait_thread(&bar_sread[x], j & 1, wc, kErrWaitSoftmax) ||
+                !wait_thread(&bar_ktma[sk], ((j + 1) / NK) & 1, wc, kErrWaitProducer))
+              break;
+            NEA_TRACE_STAMP(p, 44 + min(j, 7), x == 0);
+            tc_fence_after();
+            issue_s(j + 1);
+            tc_commit(&bar_kempty[sk]);
+          }
           if (!wait_thread(&bar_p[x], j & 1, wc, kErrWaitSoftmax) ||
               !wait_thread(&bar_vtma[sv], (j / NV) & 1, wc, kErrWaitProducer))
             break;
+          NEA_TRACE_STAMP(p, 36 + min(j, 7), x == 0);
           NEA_TRACE_STAMP(p, 36 + min(j, 7), x == 0);
           tc_fence_after();
           const uint32_t sV = smem_u32(smem + L::kV0 + sv * L::kVStage);
@@ -378,7 +397,7 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
 #pragma unroll
             for (int term = 0; term < kTerms; ++term) {
               // float32 storage: Phi*Vhi + Phi*Vlo + Plo*Vhi
-              const uint32_t pa = (term == 2 ? plo : phi) + kk * 8;
+              const uint32_t pa = (kSepP ? plo : (term == 2 ? plo : phi)) + kk * 8;
               const uint32_t vb = sV + (term == 1 ? OPB : 0) + kk * 16 * RB;
               mma_ts(dO, pa, smem_desc(vb, RB, kTileRows * RB), idO, (j | kk | term) != 0);
             }
@@ -386,7 +405,7 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
           tc_commit(&bar_o[x]);
           tc_commit(&bar_vempty[sv]);
           NEA_TRACE_STAMP(p, 68 + min(j, 7), x == 0);
-          if (j + 1 < my_nkv) {
+          if (!kSepP && j + 1 < my_nkv) {
             // S_X(j+1) overwrites P_X(j): wait until PV_X(j) has read it
             const int sk = (j + 1) % NK;
             if (!wait_thread(&bar_o[x], j & 1, wc, kErrWaitMma) ||

@@ -8,7 +8,8 @@
 //     products (hi*hi + hi*lo + lo*hi).  Reads 4 bytes and writes 4 per element.
 //   - bfloat16 storage: Q and K are rotated into bf16 copies (V and dO are
 //     read in place).  Reads 2 bytes and writes 2 per element.
-// Both are bound by HBM bandwidth.
+// In the backward the same launch also writes the per-row terms of every
+// query row (below).  Everything here is bound by HBM bandwidth.
 #pragma once
 
 #include "nea_device.cuh"
@@ -22,6 +23,7 @@ struct PrepJob {
   long long chunks;       // 16-byte chunks: B*T*H*D / 4 (fp32), / 8 (bf16)
   int H;                  // heads of this tensor
   int rope;               // 1: rotate (queries, keys)
+  FastDiv divH;           // division by H
 };
 
 struct PrepParams {
@@ -30,56 +32,136 @@ struct PrepParams {
   int T;
   const float2* rope;     // [T][D/2] (cos, sin) or nullptr
   long long total;        // sum of chunks
+  int prep_blocks;        // blocks [0, prep_blocks) rotate/split, kPrepUnroll chunks per thread
+  // backward row terms (rt_threads == 0: none), blocks from prep_blocks on
+  const void* O;
+  const void* dO;
+  const float* LSE;
+  float* ws;
+  int B, Tp, Hq;
+  long long rt_threads;
+  FastDiv divT, divTp, divHq;
 };
+
+constexpr int kPrepUnroll = 4;  // 16-byte chunks in flight per thread
+
+// ---------------------------------------------------------------- row term
+// Per-row terms of the backward, in a workspace ws[B*Hq][2][Tp] (Tp = T
+// rounded up to whole 128-row tiles, so a tile of it is one TMA box):
+//   ws[bh][0][t] = -LSE[b][h][t] * log2(e)          (-inf for t >= T)
+//   ws[bh][1][t] = Dv = sum_d dO[b][t][h][d] O[b][t][h][d]   (0 for t >= T)
+// The padding makes P = exp2(s*c + ws0) vanish for queries past T.  One group
+// of D/ELEMS lanes per (b, t, h) row, t over [0, Tp).
+template <int D, bool F32IO>
+__device__ __forceinline__ void rowterm_lane(const PrepParams& p, long long gtid) {
+  constexpr int kElems = F32IO ? 4 : 8;    // elements per 16-byte chunk
+  constexpr int kLanes = D / kElems;       // lanes per row: 4, 8 or 16
+  if (gtid >= p.rt_threads) return;        // whole groups of lanes leave together
+  const uint32_t prow = uint32_t(gtid / kLanes);  // (b, t, h) over t in [0, Tp)
+  const int c = int(gtid % kLanes);
+  const uint32_t bt = fdiv(prow, p.divHq);
+  const int h = int(prow - bt * uint32_t(p.Hq));
+  const uint32_t bq = fdiv(bt, p.divTp);
+  const int t = int(bt - bq * uint32_t(p.Tp));
+  const long long b = bq;
+  float* out = p.ws + (b * p.Hq + h) * 2 * (long long)p.Tp + t;
+  if (t >= p.T) {
+    if (c == 0) {
+      out[0] = -INFINITY;
+      out[p.Tp] = 0.f;
+    }
+    return;
+  }
+  const long long row = (b * p.T + t) * p.Hq + h;
+  const uint4 a = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.O) + row * D * (F32IO ? 4 : 2)) + c);
+  const uint4 z = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.dO) + row * D * (F32IO ? 4 : 2)) + c);
+  float acc;
+  if constexpr (F32IO) {
+    acc = __uint_as_float(a.x) * __uint_as_float(z.x) + __uint_as_float(a.y) * __uint_as_float(z.y) +
+          __uint_as_float(a.z) * __uint_as_float(z.z) + __uint_as_float(a.w) * __uint_as_float(z.w);
+  } else {
+    acc = bf16_lo_f(a.x) * bf16_lo_f(z.x) + bf16_hi_f(a.x) * bf16_hi_f(z.x) + bf16_lo_f(a.y) * bf16_lo_f(z.y) +
+          bf16_hi_f(a.y) * bf16_hi_f(z.y) + bf16_lo_f(a.z) * bf16_lo_f(z.z) + bf16_hi_f(a.z) * bf16_hi_f(z.z) +
+          bf16_lo_f(a.w) * bf16_lo_f(z.w) + bf16_hi_f(a.w) * bf16_hi_f(z.w);
+  }
+  // the kLanes lanes of a row are consecutive and leave or stay together
+  const unsigned group = (kLanes == 32 ? kFullMask : ((1u << kLanes) - 1u) << (threadIdx.x & 31 & ~(kLanes - 1)));
+#pragma unroll
+  for (int off = kLanes / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(group, acc, off);
+  if (c == 0) {
+    out[0] = __ldg(p.LSE + (b * p.Hq + h) * (long long)p.T + t) * -1.4426950408889634f;
+    out[p.Tp] = acc;
+  }
+}
+
+// One 16-byte chunk of job tensor data: rotate (queries, keys) and convert.
+template <int D, bool F32IO>
+__device__ __forceinline__ void prep_chunk(const PrepParams& p, const PrepJob& job, long long ci, uint4 raw) {
+  constexpr int kPerChunk = F32IO ? 4 : 8;  // elements per 16-byte chunk
+  constexpr int kCpr = D / kPerChunk;       // chunks per head vector
+  float x[kPerChunk];
+  if constexpr (F32IO) {
+    x[0] = __uint_as_float(raw.x), x[1] = __uint_as_float(raw.y);
+    x[2] = __uint_as_float(raw.z), x[3] = __uint_as_float(raw.w);
+  } else {
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) x[2 * k] = bf16_lo_f(w[k]), x[2 * k + 1] = bf16_hi_f(w[k]);
+  }
+  if (job.rope && p.rope != nullptr) {
+    const uint32_t row = uint32_t(ci / kCpr);  // (b, t, h) row index
+    const int c = int(ci % kCpr);              // pairs kPerChunk/2 * c ...
+    const uint32_t bt = fdiv(row, job.divH);
+    const int t = int(bt - fdiv(bt, p.divT) * uint32_t(p.T));
+    const float4* cs = reinterpret_cast<const float4*>(p.rope + size_t(t) * (D / 2) + (kPerChunk / 2) * c);
+#pragma unroll
+    for (int k = 0; k < kPerChunk / 4; ++k) {
+      const float4 r = __ldg(cs + k);  // (cos, sin) of two pairs
+      float* y = x + 4 * k;
+      const float y0 = y[0] * r.x - y[1] * r.y, y1 = y[0] * r.y + y[1] * r.x;
+      const float y2 = y[2] * r.z - y[3] * r.w, y3 = y[2] * r.w + y[3] * r.z;
+      y[0] = y0, y[1] = y1, y[2] = y2, y[3] = y3;
+    }
+  }
+  if constexpr (F32IO) {
+    uint2 hi, lo;
+    split_bf16(x[0], x[1], hi.x, lo.x);
+    split_bf16(x[2], x[3], hi.y, lo.y);
+    reinterpret_cast<uint2*>(job.hi)[ci] = hi;
+    reinterpret_cast<uint2*>(job.lo)[ci] = lo;
+  } else {
+    reinterpret_cast<uint4*>(job.hi)[ci] =
+        make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
+  }
+}
 
 template <int D, bool F32IO>
 __global__ void __launch_bounds__(256) attn_prep_kernel(const __grid_constant__ PrepParams p) {
-  constexpr int kPerChunk = F32IO ? 4 : 8;  // elements per 16-byte chunk
-  constexpr int kCpr = D / kPerChunk;       // chunks per head vector
-  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < p.total; i += stride) {
+  if (int(blockIdx.x) >= p.prep_blocks) {
+    rowterm_lane<D, F32IO>(p, (long long)(blockIdx.x - p.prep_blocks) * blockDim.x + threadIdx.x);
+    return;
+  }
+  // kPrepUnroll chunks per thread, each step of them coalesced across the block
+  const long long base = (long long)blockIdx.x * blockDim.x * kPrepUnroll + threadIdx.x;
+  uint4 raw[kPrepUnroll];
+  int jj[kPrepUnroll];
+  long long cc[kPrepUnroll];
+#pragma unroll
+  for (int u = 0; u < kPrepUnroll; ++u) {
+    const long long i = base + (long long)u * blockDim.x;
     int j = 0;
     long long ci = i;
     while (j + 1 < p.n_jobs && ci >= p.job[j].chunks) {
       ci -= p.job[j].chunks;
       ++j;
     }
-    const PrepJob& job = p.job[j];
-    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(job.src) + ci);
-    float x[kPerChunk];
-    if constexpr (F32IO) {
-      x[0] = __uint_as_float(raw.x), x[1] = __uint_as_float(raw.y);
-      x[2] = __uint_as_float(raw.z), x[3] = __uint_as_float(raw.w);
-    } else {
-      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) x[2 * k] = bf16_lo_f(w[k]), x[2 * k + 1] = bf16_hi_f(w[k]);
-    }
-    if (job.rope && p.rope != nullptr) {
-      const long long row = ci / kCpr;      // (b, t, h) row index
-      const int c = int(ci % kCpr);         // pairs kPerChunk/2 * c ...
-      const int t = int((row / job.H) % p.T);
-      const float4* cs = reinterpret_cast<const float4*>(p.rope + size_t(t) * (D / 2) + (kPerChunk / 2) * c);
-#pragma unroll
-      for (int k = 0; k < kPerChunk / 4; ++k) {
-        const float4 r = __ldg(cs + k);  // (cos, sin) of two pairs
-        float* y = x + 4 * k;
-        const float y0 = y[0] * r.x - y[1] * r.y, y1 = y[0] * r.y + y[1] * r.x;
-        const float y2 = y[2] * r.z - y[3] * r.w, y3 = y[2] * r.w + y[3] * r.z;
-        y[0] = y0, y[1] = y1, y[2] = y2, y[3] = y3;
-      }
-    }
-    if constexpr (F32IO) {
-      uint2 hi, lo;
-      split_bf16(x[0], x[1], hi.x, lo.x);
-      split_bf16(x[2], x[3], hi.y, lo.y);
-      reinterpret_cast<uint2*>(job.hi)[ci] = hi;
-      reinterpret_cast<uint2*>(job.lo)[ci] = lo;
-    } else {
-      reinterpret_cast<uint4*>(job.hi)[ci] =
-          make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
-    }
+    jj[u] = j;
+    cc[u] = ci;
+    if (i < p.total) raw[u] = __ldg(reinterpret_cast<const uint4*>(p.job[j].src) + ci);
   }
+#pragma unroll
+  for (int u = 0; u < kPrepUnroll; ++u)
+    if (base + (long long)u * blockDim.x < p.total) prep_chunk<D, F32IO>(p, p.job[jj[u]], cc[u], raw[u]);
 }
 
 }  // namespace nea

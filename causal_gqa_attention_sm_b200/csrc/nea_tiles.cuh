@@ -37,19 +37,19 @@ __device__ __forceinline__ void rot2(float& x0, float& x1, float c, float s) {
   x1 = y1;
 }
 
-// Writes one D-wide output row held in registers (float) to a [B][T][H][D]
-// tensor in the storage type.
-template <int D, bool F32IO>
-__device__ __forceinline__ void store_row(void* dst, int b, int t, int head, int T, int H, const float* v) {
+// Writes N consecutive elements of a row held in registers (float) at
+// element offset `off` of a tensor in the storage type (16-byte aligned).
+template <int N, bool F32IO>
+__device__ __forceinline__ void store_span(void* dst, size_t off, const float* v) {
   if constexpr (F32IO) {
-    float4* p = reinterpret_cast<float4*>(static_cast<float*>(dst) + ((size_t(b) * T + t) * H + head) * D);
+    float4* q = reinterpret_cast<float4*>(static_cast<float*>(dst) + off);
 #pragma unroll
-    for (int i = 0; i < D / 4; ++i) p[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    for (int i = 0; i < N / 4; ++i) q[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
   } else {
-    uint4* p = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dst) + ((size_t(b) * T + t) * H + head) * D);
+    uint4* q = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dst) + off);
 #pragma unroll
-    for (int i = 0; i < D / 8; ++i)
-      p[i] = make_uint4(pack_bf16(v[8 * i], v[8 * i + 1]), pack_bf16(v[8 * i + 2], v[8 * i + 3]),
+    for (int i = 0; i < N / 8; ++i)
+      q[i] = make_uint4(pack_bf16(v[8 * i], v[8 * i + 1]), pack_bf16(v[8 * i + 2], v[8 * i + 3]),
                         pack_bf16(v[8 * i + 4], v[8 * i + 5]), pack_bf16(v[8 * i + 6], v[8 * i + 7]));
   }
 }

@@ -97,8 +97,8 @@ int nea_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
  *
  * Runs on `stream`: the operand prologue (NEA_F32: bf16 hi/lo planes of the
  * rotated Q and K and of V, dO; NEA_BF16: rotated copies of Q and K, none
- * when the rotation is off); the row terms -LSE*log2(e) and
- * D_i = sum_d dO_id O_id; the dK/dV kernel (one CTA per key tile and kv head,
+ * when the rotation is off), which in the same launch writes the row terms
+ * -LSE*log2(e) and D_i = sum_d dO_id O_id; the dK/dV kernel (one CTA per key tile and kv head,
  * looping over the query heads of the group); the dQ kernel (one CTA per
  * query tile and head); both recompute P from LSE.
  *
@@ -137,13 +137,12 @@ void nea_debug_inject(int flags);
  * Profiling hook.  `events` points at `n` cudaEvent_t handles owned by the
  * caller (NULL / 0 disables).  While set, later calls on this host thread
  * record them on their stream at kernel boundaries:
- *   nea_attn_fwd: events[0] before the first kernel (the NEA_F32 operand
- *                 prologue, else the forward kernel), events[1] after the
- *                 forward kernel;
- *   nea_attn_bwd: events[2] before the first kernel (NEA_F32 operand
- *                 prologue, else the row-term kernel), events[3] after the
- *                 row-term kernel, events[4] after the dK/dV kernel,
- *                 events[5] after the dQ kernel.
+ *   nea_attn_fwd: events[0] before the operand prologue, events[6] after it
+ *                 (before the forward kernel), events[1] after the forward
+ *                 kernel;
+ *   nea_attn_bwd: events[2] before the operand prologue (which also writes
+ *                 the row terms), events[3] after it, events[4] after the
+ *                 dK/dV kernel, events[5] after the dQ kernel.
  * Indices >= n are skipped.  The array must stay valid while set.
  */
 void nea_set_profile_events(void* const* events, int n);
