@@ -198,11 +198,12 @@ def ncu_traffic(kernel, workload):
 
 
 # ---------------------------------------------------------------- CPU baseline (oracle)
-def run_oracle_sample(w, max_units=None):
+def run_oracle_sample(w, max_units=None, min_seconds=0.0):
     """Times the fp64 oracle on (batch, kv-group) slices of the workload (each
     slice: one batch element, the G query heads of one kv head), all slices in
-    one call so OpenMP spreads them over the host cores.  Returns (seconds,
-    flops, threads, description)."""
+    one call so OpenMP spreads them over the host cores, repeated until at
+    least `min_seconds` have passed.  Returns (seconds, flops, threads,
+    description)."""
     import numpy as np
 
     import oracle
@@ -221,12 +222,16 @@ def run_oracle_sample(w, max_units=None):
     vs = np.concatenate([arr["v"][b:b + 1, :, g:g + 1] for b, g in pairs])
     threads = min(cores, n)
     oracle.set_threads(threads)
-    t0 = time.perf_counter()
-    oracle.attn_fwd(qs, ks, vs, w.rope_base, w.causal)
-    oracle.attn_bwd(qs, ks, vs, dos, w.rope_base, w.causal)
-    dt = time.perf_counter() - t0
-    flops = w.flops() / w.layers * n / units
-    desc = f"{n} of {units} (batch, kv-group) slices of one layer, fwd+bwd, fp64, {threads} threads"
+    reps, dt = 0, 0.0
+    while reps == 0 or dt < min_seconds:
+        t0 = time.perf_counter()
+        oracle.attn_fwd(qs, ks, vs, w.rope_base, w.causal)
+        oracle.attn_bwd(qs, ks, vs, dos, w.rope_base, w.causal)
+        dt += time.perf_counter() - t0
+        reps += 1
+    flops = w.flops() / w.layers * n / units * reps
+    desc = (f"{n} of {units} (batch, kv-group) slices of one layer, fwd+bwd, fp64, {threads} threads"
+            + (f", {reps} repetitions" if reps > 1 else ""))
     return dt, flops, threads, desc
 
 
@@ -414,7 +419,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        dt, fl, threads, desc = run_oracle_sample(w)
+        dt, fl, threads, desc = run_oracle_sample(w, min_seconds=10.0)
         cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc,
                "seconds": dt}
 
