@@ -31,13 +31,11 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "causal GQA attention fwd+bwd TFLOP/s (% of tensor-core peak) and tokens/s"
-KERNELS = ("attn_fwd_prologue", "attn_fwd", "attn_bwd_prologue", "attn_bwd_dkdv", "attn_bwd_dq")
+KERNELS = ("attn_fwd_prologue", "attn_fwd", "attn_bwd_prologue", "attn_bwd")
 # Algorithmic work per kernel in units of B*Hq*T^2*D (causal): the forward's
-# two products; the dK/dV kernel's S, dP, dV, dK products; the dQ kernel's S,
-# dP, dQ products (S and dP are recomputed there, so the two backward kernels
-# together are credited 5 units, the conventional backward count, split 3:2 by
-# their distinct outputs: dK/dV gets dP, dV, dK; dQ gets S and dQ).
-UNITS = {"attn_fwd": 2.0, "attn_bwd_dkdv": 3.0, "attn_bwd_dq": 2.0}
+# two products; the gradient kernel's five (S, dP, dV, dK, dQ: its dQ units
+# recompute S and dP, which are not credited again).
+UNITS = {"attn_fwd": 2.0, "attn_bwd": 5.0}
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -355,8 +353,7 @@ def main():
             kern_ms["attn_fwd_prologue"] += ev[0].elapsed_time(ev[6])
             kern_ms["attn_fwd"] += ev[6].elapsed_time(ev[1])
             kern_ms["attn_bwd_prologue"] += ev[2].elapsed_time(ev[3])
-            kern_ms["attn_bwd_dkdv"] += ev[3].elapsed_time(ev[4])
-            kern_ms["attn_bwd_dq"] += ev[4].elapsed_time(ev[5])
+            kern_ms["attn_bwd"] += ev[3].elapsed_time(ev[4])
     launches_per_kernel = K * w.layers
 
     flops_step = w.flops()

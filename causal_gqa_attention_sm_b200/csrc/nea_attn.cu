@@ -306,29 +306,18 @@ int launch_fwd(uint32_t& attr_done, const nea::FwdParams& p, cudaStream_t stream
 }
 
 // ----------------------------------------------------------------- backward
-// dK/dV kernel, dQ kernel.  `ev` selects profiling events (the
+// The gradient kernel (dK/dV and dQ units in one launch).  `ev` selects profiling events (the
 // regular backward records them, the allocation-free one does not).
 template <int D, bool F32IO>
 int launch_bwd(uint32_t& attr_done, const nea::BwdParams& p, cudaStream_t stream, bool ev) {
   cudaError_t e;
-  using LK = nea::BwdSmem<D, F32IO, true>;
-  auto kk = nea::attn_bwd_kernel<D, F32IO, true>;
-  int rc = set_smem(attr_done, 4 + (D == 64) * 2 + F32IO, kk, LK::kAlloc);
+  using L = nea::BwdSmem<D, F32IO>;
+  auto kern = nea::attn_bwd_kernel<D, F32IO>;
+  int rc = set_smem(attr_done, 4 + (D == 64) * 2 + F32IO, kern, L::kAlloc);
   if (rc) return rc;
-  kk<<<p.B * p.Hkv * p.n_tiles, LK::kThreads, LK::kAlloc, stream>>>(p);
-  nea::BwdParams pq = p;
-#ifdef NEA_TRACE
-  if (pq.trace) pq.trace += size_t(p.B) * p.Hkv * p.n_tiles * 80;  // dQ stamps follow the dK/dV ones
-#endif
+  kern<<<p.n_dkdv + p.B * p.Hq * p.n_tiles, L::kThreads, L::kAlloc, stream>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
   if (ev) prof_record(4, stream);
-
-  using LQ = nea::BwdSmem<D, F32IO, false>;
-  auto kq = nea::attn_bwd_kernel<D, F32IO, false>;
-  rc = set_smem(attr_done, 8 + (D == 64) * 2 + F32IO, kq, LQ::kAlloc);
-  if (rc) return rc;
-  kq<<<p.B * p.Hq * p.n_tiles, LQ::kThreads, LQ::kAlloc, stream>>>(pq);
-  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
   if (ev) prof_record(5, stream);
   return NEA_OK;
 }
@@ -412,6 +401,7 @@ int run_bwd(uint32_t& attr_done, uint8_t* ws, const float2* rope, int* status, c
   p.Hkv = Hkv;
   p.G = Hq / Hkv;
   p.n_tiles = (T + 127) / 128;
+  p.n_dkdv = B * Hkv * p.n_tiles;
   p.causal = causal;
   p.scale = float(1.0 / std::sqrt(double(D)));
   p.scale_log2 = float(1.4426950408889634 / std::sqrt(double(D)));

@@ -9,8 +9,10 @@
 //                dV += P^T dO, dK' += dS^T Q', dQ' += dS K'  (x scale)
 //   epilogue     dQ = R^T dQ', dK = R^T dK'   (inverse rotation per position)
 //
-// One kernel template serves both gradient passes, the "row" tile being
-// resident in shared memory and the "column" tiles streamed past it:
+// One kernel serves both gradient passes in one launch (the dK/dV units
+// first, the longest first; the dQ units after them, longest first, so they
+// fill the SMs the dK/dV units leave free), the "row" tile being resident in
+// shared memory and the "column" tiles streamed past it:
 //   DKDV  row = key tile j of kv head g (K'_j, V_j), columns = query tiles
 //         i >= j of every query head of the group (Q'_i, dO_i, LSE, Dv); the
 //         group's dK/dV sums stay in TMEM for the whole CTA, so the reduction
@@ -72,10 +74,12 @@ struct BwdParams {
   float scale;        // 1 / sqrt(D)
   int* err;
   unsigned long long wait_limit;
+  int n_dkdv;                 // units [0, n_dkdv) are dK/dV units, the rest dQ units
+  int unit0;                  // unit of blockIdx.x == 0
   unsigned long long* trace;  // per-CTA phase stamps (NEA_TRACE builds only)
 };
 
-template <int D, bool F32IO, bool DKDV>
+template <int D, bool F32IO>
 struct BwdSmem {
   static constexpr int kStages = F32IO ? 2 : 3;
   static constexpr uint32_t kTile = Stage<D, F32IO>::kBytes;
@@ -83,7 +87,7 @@ struct BwdSmem {
   static constexpr uint32_t kR2 = kR1 + kTile;
   static constexpr uint32_t kStage0 = kR2 + kTile;
   static constexpr uint32_t kColVec = 2 * kTile;             // per-column -LSE*log2e and Dv (DKDV)
-  static constexpr uint32_t kStageBytes = kColVec + (DKDV ? 1024 : 0);
+  static constexpr uint32_t kStageBytes = kColVec + 1024;
   static constexpr uint32_t kBars = kStage0 + kStages * kStageBytes;
   // rtma, tma[S], empty[S], s, dp, p, ds, dk, fin, sread
   static constexpr int kNumBars = 1 + 2 * kStages + 7;
@@ -116,10 +120,12 @@ __device__ __forceinline__ void tmem_ld_n(uint32_t taddr, float* v) {
   }
 }
 
+// One unit (a dK/dV unit when DKDV, else a dQ unit; `bid` its index among
+// units of its kind), specialised per pass so that neither pays for the
+// other's branches.
 template <int D, bool F32IO, bool DKDV>
-__global__ void __launch_bounds__(BwdSmem<D, F32IO, DKDV>::kThreads, 1)
-    attn_bwd_kernel(const __grid_constant__ BwdParams p) {
-  using L = BwdSmem<D, F32IO, DKDV>;
+__device__ __forceinline__ void attn_bwd_unit(const BwdParams& p, int bid) {
+  using L = BwdSmem<D, F32IO>;
   constexpr uint32_t RB = TileGeom<D>::kRowBytes;
   constexpr uint32_t OPB = TileGeom<D>::kOpBytes;
   constexpr int NS = L::kStages;
@@ -152,16 +158,16 @@ __global__ void __launch_bounds__(BwdSmem<D, F32IO, DKDV>::kThreads, 1)
   int b, rt, head_r, n_items, c0;
   if (DKDV) {
     const int n_bg = p.B * p.Hkv;
-    rt = int(blockIdx.x) / n_bg;
-    const int bg = int(blockIdx.x) % n_bg;
+    rt = bid / n_bg;
+    const int bg = bid % n_bg;
     b = bg / p.Hkv;
     head_r = bg % p.Hkv;
     c0 = p.causal ? rt : 0;                       // first query tile
     n_items = p.G * (p.n_tiles - c0);
   } else {
     const int n_bh = p.B * p.Hq;
-    rt = p.n_tiles - 1 - int(blockIdx.x) / n_bh;
-    const int bh = int(blockIdx.x) % n_bh;
+    rt = p.n_tiles - 1 - bid / n_bh;
+    const int bh = bid % n_bh;
     b = bh / p.Hq;
     head_r = bh % p.Hq;
     c0 = 0;
@@ -467,6 +473,16 @@ __global__ void __launch_bounds__(BwdSmem<D, F32IO, DKDV>::kThreads, 1)
     tmem_dealloc(tbase, 512);
   }
   NEA_TRACE_STAMP(p, 78, tid == 0);
+}
+
+template <int D, bool F32IO>
+__global__ void __launch_bounds__(BwdSmem<D, F32IO>::kThreads, 1)
+    attn_bwd_kernel(const __grid_constant__ BwdParams p) {
+  const int unit = p.unit0 + int(blockIdx.x);
+  if (unit < p.n_dkdv)
+    attn_bwd_unit<D, F32IO, true>(p, unit);
+  else
+    attn_bwd_unit<D, F32IO, false>(p, unit - p.n_dkdv);
 }
 
 }  // namespace nea

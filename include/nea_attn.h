@@ -98,9 +98,10 @@ int nea_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
  * Runs on `stream`: the operand prologue (NEA_F32: bf16 hi/lo planes of the
  * rotated Q and K and of V, dO; NEA_BF16: rotated copies of Q and K, none
  * when the rotation is off), which in the same launch writes the row terms
- * -LSE*log2(e) and D_i = sum_d dO_id O_id; the dK/dV kernel (one CTA per key tile and kv head,
- * looping over the query heads of the group); the dQ kernel (one CTA per
- * query tile and head); both recompute P from LSE.
+ * -LSE*log2(e) and D_i = sum_d dO_id O_id; one gradient kernel whose CTAs
+ * run dK/dV units (one per key tile and kv head, looping over the query heads
+ * of the group) and dQ units (one per query tile and head); both recompute P
+ * from LSE.
  *
  * NEA_F32: the score product and dO V^T use split bf16 (as in the forward);
  * the three gradient products use the bf16 high parts with fp32
@@ -141,8 +142,8 @@ void nea_debug_inject(int flags);
  *                 (before the forward kernel), events[1] after the forward
  *                 kernel;
  *   nea_attn_bwd: events[2] before the operand prologue (which also writes
- *                 the row terms), events[3] after it, events[4] after the
- *                 dK/dV kernel, events[5] after the dQ kernel.
+ *                 the row terms), events[3] after it, events[4] and events[5]
+ *                 after the gradient kernel.
  * Indices >= n are skipped.  The array must stay valid while set.
  */
 void nea_set_profile_events(void* const* events, int n);
