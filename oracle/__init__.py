@@ -53,9 +53,12 @@ def _load():
                                         i, i, i, i, i, d, i]
         lib.oracle_attn_probs.argtypes = [_dp, _dp, _dp, i, i, i, i, i, d, i, i, i]
         lib.oracle_rope.argtypes = [_dp, _dp, i, i, i, i, d]
+        lib.oracle_attn_decode.argtypes = [_dp, _dp, _dp, ctypes.POINTER(ctypes.c_int), _dp, _dp,
+                                           i, i, i, i, i, d]
         lib.oracle_set_threads.argtypes = [i]
         lib.oracle_get_threads.restype = i
-        for f in (lib.oracle_attn_fwd, lib.oracle_attn_bwd, lib.oracle_attn_probs, lib.oracle_rope):
+        for f in (lib.oracle_attn_fwd, lib.oracle_attn_bwd, lib.oracle_attn_probs, lib.oracle_rope,
+                  lib.oracle_attn_decode):
             f.restype = i
         _lib = lib
     return _lib
@@ -137,3 +140,22 @@ def attn_probs(q, k, b: int, h: int, rope_base: float = 10000.0, causal: bool = 
     _check(_load().oracle_attn_probs(_ptr(q), _ptr(k), _ptr(p), B, T, Hq, Hkv, D,
                                      float(rope_base), int(bool(causal)), int(b), int(h)))
     return p
+
+
+def attn_decode(q, kc, vc, lens, rope_base: float = 10000.0):
+    """Decode attention of one query per sequence over a key/value cache.
+
+    ``q [B, Hq, D]`` un-rotated query of the token at position ``lens[b]-1``;
+    ``kc, vc [B, Tc, Hkv, D]`` the cache (keys already rotated at their
+    positions); ``lens [B]`` valid lengths.  Returns ``(O [B, Hq, D],
+    LSE [B, Hq])``; an empty cache gives O = 0 and LSE = -inf.
+    """
+    q, kc, vc = _c(q), _c(kc), _c(vc)
+    B, Hq, D = q.shape
+    _, Tc, Hkv, _ = kc.shape
+    ln = np.ascontiguousarray(lens, dtype=np.int32)
+    o = np.zeros_like(q)
+    lse = np.zeros((B, Hq), dtype=np.float64)
+    _check(_load().oracle_attn_decode(_ptr(q), _ptr(kc), _ptr(vc), ln.ctypes.data_as(ctypes.POINTER(ctypes.c_int)),
+                                      _ptr(o), _ptr(lse), B, Tc, Hq, Hkv, D, float(rope_base)))
+    return o, lse

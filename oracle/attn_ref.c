@@ -325,3 +325,69 @@ int oracle_attn_bwd(const double* Q, const double* K, const double* V, const dou
     }
     return err ? ORACLE_ERR_NOMEM : ORACLE_OK;
 }
+
+/*
+ * Decode attention over a key/value cache: one new query per sequence
+ * attends to the cached positions 0 .. len_b - 1, the last of which is its
+ * own (the generation path of the same causal attention: "NanoEuler"
+ * write-up, aimsg.uk, section 1, head-0 generation; the scores, softmax and
+ * GQA head map as in oracle_attn_fwd).
+ *
+ *   Q   [B][Hq][D]     un-rotated query of the token at position len_b - 1
+ *   Kc  [B][Tc][Hkv][D] cached keys, already rotated at their positions
+ *   Vc  [B][Tc][Hkv][D] cached values
+ *   lens[B]            valid cache length, 0 <= len_b <= Tc
+ *   O   [B][Hq][D], LSE [B][Hq]
+ *
+ * q' = R_{len_b - 1} q; s_j = q' . k_j / sqrt(D) for j < len_b;
+ * LSE = ln sum_j exp(s_j); O = sum_j exp(s_j - LSE) v_j.  An empty cache
+ * (len_b = 0) gives O = 0 and LSE = -inf.
+ */
+int oracle_attn_decode(const double* Q, const double* Kc, const double* Vc, const int* lens, double* O,
+                       double* LSE, int B, int Tc, int Hq, int Hkv, int D, double rope_base) {
+    if (!check_shape(B, Tc, Hq, Hkv, D)) return ORACLE_ERR_ARG;
+    for (int b = 0; b < B; ++b)
+        if (lens[b] < 0 || lens[b] > Tc) return ORACLE_ERR_ARG;
+    const int G = Hq / Hkv;
+    const double scale = 1.0 / sqrt((double)D);
+    int err = 0;
+#pragma omp parallel for schedule(dynamic) reduction(| : err)
+    for (long bh = 0; bh < (long)B * Hq; ++bh) {
+        const int b = (int)(bh / Hq), h = (int)(bh % Hq), g = h / G, len = lens[b];
+        double* o = O + bh * D;
+        double* qr = (double*)malloc(sizeof(double) * D);
+        double* s = (double*)malloc(sizeof(double) * (len > 0 ? len : 1));
+        if (!qr || !s) {
+            err |= 1;
+            free(qr);
+            free(s);
+            continue;
+        }
+        for (int d = 0; d < D; ++d) o[d] = 0.0;
+        if (len == 0) {
+            LSE[bh] = -INFINITY;
+        } else {
+            rope_rotate(Q + bh * D, qr, len - 1, D, rope_base);
+            double m = -INFINITY;
+            for (int j = 0; j < len; ++j) {
+                const double* k = Kc + (((long)b * Tc + j) * Hkv + g) * D;
+                double acc = 0.0;
+                for (int d = 0; d < D; ++d) acc += qr[d] * k[d];
+                s[j] = scale * acc;
+                if (s[j] > m) m = s[j];
+            }
+            double l = 0.0;
+            for (int j = 0; j < len; ++j) l += exp(s[j] - m);
+            const double lse = m + log(l);
+            for (int j = 0; j < len; ++j) {
+                const double p = exp(s[j] - lse);
+                const double* v = Vc + (((long)b * Tc + j) * Hkv + g) * D;
+                for (int d = 0; d < D; ++d) o[d] += p * v[d];
+            }
+            LSE[bh] = lse;
+        }
+        free(qr);
+        free(s);
+    }
+    return err ? ORACLE_ERR_NOMEM : ORACLE_OK;
+}

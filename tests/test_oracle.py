@@ -250,3 +250,65 @@ def test_empty_inputs():
 def test_rejects_bad_head_grouping():
     with pytest.raises(ValueError):
         oracle.attn_fwd(np.zeros((1, 2, 5, 8)), np.zeros((1, 2, 2, 8)), np.zeros((1, 2, 2, 8)))
+
+
+# ----------------------------------------------------------------- decode over a key/value cache
+BASE = 10000.0
+def _decode_case(B=3, T=11, Hq=6, Hkv=2, D=8, seed=7):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, T, Hq, D))
+    k = rng.standard_normal((B, T, Hkv, D))
+    v = rng.standard_normal((B, T, Hkv, D))
+    return q, k, v
+
+
+def test_decode_is_last_row_of_causal_attention():
+    """Decoding the token at position L-1 over a cache holding the rotated
+    keys 0..L-1 reproduces row L-1 of the full causal attention, per batch
+    element with ragged lengths."""
+    q, k, v = _decode_case()
+    o, lse = oracle.attn_fwd(q, k, v, BASE, True)
+    kc = oracle.rope(k, BASE)
+    lens = np.array([1, 6, 11])
+    qd = np.stack([q[b, lens[b] - 1] for b in range(3)])
+    od, ld = oracle.attn_decode(qd, kc, v, lens, BASE)
+    for b in range(3):
+        np.testing.assert_allclose(od[b], o[b, lens[b] - 1], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(ld[b], lse[b, :, lens[b] - 1], rtol=0, atol=1e-13)
+
+
+def test_decode_single_position_closed_form():
+    """len = 1: the only key is the query's own position 0 (no rotation):
+    O = v_0 and LSE = q . k_0 / sqrt(D)."""
+    q, k, v = _decode_case(B=1, T=4, Hq=2, Hkv=1, D=6)
+    od, ld = oracle.attn_decode(q[:, 0], k, v, np.array([1]), BASE)
+    for h in range(2):
+        np.testing.assert_allclose(od[0, h], v[0, 0, 0], rtol=0, atol=1e-14)
+        assert abs(ld[0, h] - float(q[0, 0, h] @ k[0, 0, 0]) / math.sqrt(6)) < 1e-13
+
+
+def test_decode_equal_scores_give_mean_and_log_length():
+    """Zero keys make every score 0: O is the mean of the cached values and
+    LSE = ln(len)."""
+    q, _, v = _decode_case(B=2, T=9, Hq=3, Hkv=1, D=4)
+    kc = np.zeros((2, 9, 1, 4))
+    lens = np.array([4, 9])
+    od, ld = oracle.attn_decode(q[:, 0], kc, v, lens, BASE)
+    for b in range(2):
+        np.testing.assert_allclose(od[b], np.broadcast_to(v[b, :lens[b], 0].mean(axis=0), (3, 4)), atol=1e-14)
+        np.testing.assert_allclose(ld[b], math.log(lens[b]), atol=1e-14)
+
+
+def test_decode_gqa_equals_mha_and_empty_cache():
+    """Query heads of one group read the same cached head (GQA = MHA with the
+    cache repeated per group); an empty cache gives O = 0, LSE = -inf."""
+    q, k, v = _decode_case(B=2, T=5, Hq=4, Hkv=2, D=8)
+    kc = oracle.rope(k, BASE)
+    lens = np.array([5, 0])
+    od, ld = oracle.attn_decode(q[:, 4], kc, v, lens, BASE)
+    om, lm = oracle.attn_decode(q[:, 4], np.repeat(kc, 2, axis=2), np.repeat(v, 2, axis=2), lens, BASE)
+    np.testing.assert_allclose(od, om, atol=1e-14)
+    np.testing.assert_allclose(ld[0], lm[0], atol=1e-14)
+    assert np.all(od[1] == 0.0) and np.all(np.isneginf(ld[1]))
+    with pytest.raises(Exception):
+        oracle.attn_decode(q[:, 4], kc, v, np.array([6, 1]), BASE)
