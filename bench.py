@@ -260,6 +260,150 @@ def reference_arm(a, w):
     return 0
 
 
+# ---------------------------------------------------------------- decode workloads
+DECODE_METRIC = "GQA decode attention over a key/value cache: cache GB/s (HBM) and tokens/s"
+
+
+def run_oracle_decode(w, min_seconds=0.0):
+    """Times the fp64 oracle's decode on the whole workload, repeated until at
+    least `min_seconds` have passed.  Returns (seconds, cache bytes, threads,
+    description)."""
+    import oracle
+    from causal_gqa_attention_sm_b200.workloads import make_decode_inputs
+
+    inp = make_decode_inputs(w)
+    arr = {k: v.float().double().numpy() if k != "lens" else v.numpy() for k, v in inp.items()}
+    threads = min(len(os.sched_getaffinity(0)), w.B * w.Hq)
+    oracle.set_threads(threads)
+    reps, dt = 0, 0.0
+    while reps == 0 or dt < min_seconds:
+        t0 = time.perf_counter()
+        oracle.attn_decode(arr["q"], arr["kc"], arr["vc"], arr["lens"], w.rope_base)
+        dt += time.perf_counter() - t0
+        reps += 1
+    desc = f"whole decode step ({w.B} sequences x {w.T} cached positions), fp64, {threads} threads, {reps} repetitions"
+    return dt, w.cache_bytes() * reps, threads, desc
+
+
+def decode_main(a, w, rank, world, local):
+    import torch
+
+    import causal_gqa_attention_sm_b200 as nea
+    from causal_gqa_attention_sm_b200.workloads import make_decode_inputs
+
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    inp = {n: t.to(dev) for n, t in make_decode_inputs(w).items()}
+    o = torch.empty_like(inp["q"])
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    drain = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    drain_sum = torch.empty((), dtype=torch.float32, device=dev)
+
+    def step():
+        nea.nea_attn_decode(inp["q"], inp["kc"], inp["vc"], inp["lens"], w.rope_base, o=o, lse=lse)
+
+    for i in range(a.warmup):
+        flush.fill_(float(i))
+        torch.sum(drain, dim=0, out=drain_sum)
+        step()
+    torch.cuda.synchronize(dev)
+    if nea.nea_device_status() != nea.NEA_OK:
+        raise SystemExit("device status after warm-up")
+    K = a.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    clocks = ClockSampler(local)
+    barrier(world)
+    with clocks:
+        for i in range(K):
+            flush.fill_(float(i))
+            torch.sum(drain, dim=0, out=drain_sum)
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    if nea.nea_device_status() != nea.NEA_OK:
+        raise SystemExit("device status after timing")
+    total_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in ev), world)
+    byts = w.cache_bytes()
+    value = byts * K * world / (total_ms * 1e-3) / 1e9
+    pk = peaks()
+    roof = {"bound": "hbm", "achieved": value / world, "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": value / world / pk["hbm_gbs"], "traffic": ncu_traffic("attn_decode", w.name),
+            "kernel": "attn_decode (split + combine)"}
+    e2e = None
+    if not a.no_e2e:
+        host = {n: t.cpu().pin_memory() for n, t in inp.items()}
+        ho, hl = torch.empty(o.shape, dtype=o.dtype, pin_memory=True), torch.empty(lse.shape, pin_memory=True)
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+
+        def e2e_step():
+            for n in inp:
+                inp[n].copy_(host[n], non_blocking=True)
+            step()
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+
+        for _ in range(a.warmup):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(K):
+            e2e_step()
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(s0.elapsed_time(s1), world)
+        e2e = {"value": byts * K * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "tokens_per_s": w.B * K * world / (e2e_ms * 1e-3)}
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        dt, cb, threads, desc = run_oracle_decode(w, min_seconds=10.0)
+        cpu = {"value": cb / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc,
+               "seconds": dt}
+    if rank == 0:
+        line = {
+            "metric": DECODE_METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
+            "warmup": a.warmup, "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "Tc": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+                       "storage": {"f32": "float32", "bf16": "bfloat16"}[w.dtype], "rope_base": w.rope_base,
+                       "lens": "all Tc",
+                       "l2": "flushed before every timed step (256 MiB write, then 256 MiB read of another buffer)",
+                       "parallelism": f"dp{world} (independent sequences per GPU)"},
+            "tokens_per_s": w.B * K * world / (total_ms * 1e-3),
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks.summary(),
+            "gpu_launches": 2 * K,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def reference_decode(a, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    secs, byts, threads, desc = 0.0, 0, None, None
+    for _ in range(a.steps):
+        dt, cb, threads, desc = run_oracle_decode(w)
+        secs += dt
+        byts += cb
+    value = byts / secs / 1e9
+    line = {
+        "impl": "reference", "metric": DECODE_METRIC, "value": value, "unit": "GB/s", "n_gpus": a.gpus,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": secs / a.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Tc": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+                   "storage": w.dtype, "rope_base": w.rope_base, "lens": "all Tc"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 # ---------------------------------------------------------------- GPU arm
 def main():
     a = parse()
@@ -267,7 +411,7 @@ def main():
 
     w = WORKLOADS[a.workload]
     if a.impl == "reference":
-        return reference_arm(a, w)
+        return reference_decode(a, w) if w.decode else reference_arm(a, w)
 
     import torch
 
@@ -276,6 +420,13 @@ def main():
 
     rank, world, local = dist_init(a.gpus)
     torch.cuda.set_device(local)
+    if w.decode:
+        rc = decode_main(a, w, rank, world, local)
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+        return rc
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
 

@@ -18,7 +18,7 @@ __all__ = [
     "nea_attn_fwd", "nea_attn_bwd", "nea_device_status", "nea_set_wait_limit_ns", "nea_debug_inject",
     "nea_status_string", "nea_version", "nea_set_profile_events", "NeaError", "LIB_PATH", "NEA_OK", "NEA_ERR_ARG", "NEA_ERR_CUDA",
     "NEA_ERR_TIMEOUT", "NEA_ERR_UNSUPPORTED", "NEA_ERR_NOMEM", "NEA_ERR_SCRATCH_LIMIT", "NEA_F32", "NEA_BF16",
-    "nea_attn_bwd_noalloc",
+    "nea_attn_bwd_noalloc", "nea_attn_decode",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnea.so")
@@ -47,6 +47,8 @@ _lib.nea_set_profile_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), _i]
 _lib.nea_set_profile_events.restype = None
 _lib.nea_attn_bwd_noalloc.argtypes = list(_lib.nea_attn_bwd.argtypes)
 _lib.nea_attn_bwd_noalloc.restype = _i
+_lib.nea_attn_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp]
+_lib.nea_attn_decode.restype = _i
 _lib.nea_version.argtypes = []
 _lib.nea_version.restype = _i
 
@@ -207,3 +209,34 @@ def nea_set_profile_events(events) -> None:
     arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
     _prof_keep = (arr, list(events))
     _lib.nea_set_profile_events(arr, len(events))
+
+
+def nea_attn_decode(q, kc, vc, lens, rope_base: float = 10000.0, o=None, lse=None, stream=None):
+    """Decode attention of one query per sequence over a key/value cache:
+    ``q [B, Hq, D]`` (un-rotated, the token at position ``lens[b]-1``),
+    ``kc, vc [B, Tc, Hkv, D]`` (keys already rotated at their positions),
+    ``lens`` int32 ``[B]`` on the same device.  Returns ``(o [B, Hq, D],
+    lse [B, Hq])``."""
+    import torch
+
+    if q.dim() != 3 or kc.dim() != 4:
+        raise ValueError("q must be [B, Hq, D] and kc, vc [B, Tc, Hkv, D]")
+    B, Hq, D = q.shape
+    Tc, Hkv = kc.shape[1], kc.shape[2]
+    dev, dt = q.device, q.dtype
+    code = _dtype_code(q)
+    _check(kc, "kc", (B, Tc, Hkv, D), dt, dev)
+    _check(vc, "vc", (B, Tc, Hkv, D), dt, dev)
+    _check(lens, "lens", (B,), torch.int32, dev)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    _check(o, "o", (B, Hq, D), dt, dev)
+    _check(lse, "lse", (B, Hq), torch.float32, dev)
+    rc = _lib.nea_attn_decode(_ptr(q), _ptr(kc), _ptr(vc), _ptr(lens), _ptr(o), _ptr(lse), B, Tc, Hq, Hkv, D, code,
+                              float(rope_base), _stream(stream))
+    if rc != NEA_OK:
+        raise NeaError(rc, "nea_attn_decode")
+    return o, lse
+

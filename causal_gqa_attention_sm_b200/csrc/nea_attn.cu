@@ -18,6 +18,7 @@
 
 #include "nea_attn.h"
 #include "nea_bwd.cuh"
+#include "nea_decode.cuh"
 #include "nea_fwd.cuh"
 #include "nea_prep.cuh"
 
@@ -52,6 +53,7 @@ struct DeviceState {
   // runs, so in-flight kernels on any stream keep valid pointers
   std::map<std::tuple<int, int, uint32_t>, float2*> rope;
   uint32_t attr_done = 0;      // bitmask of kernels whose smem attribute is set
+  uint64_t attr_dec = 0;       // the same for the decode split kernels
 };
 
 std::mutex g_mu;
@@ -94,6 +96,24 @@ int make_tile_map(CUtensorMap* m, const void* base, int B, int T, int H, int D) 
   const CUtensorMapSwizzle sw = D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? NEA_OK : NEA_ERR_CUDA;
+}
+
+// Descriptor of a decode cache [B][Tc][Hkv][D] (fp32 or bf16), box
+// {D, 1, 128, 1}: 128 consecutive positions of one kv head, rows contiguous
+// in shared memory (no swizzle), positions past Tc read as zero.
+int make_cache_map(CUtensorMap* m, const void* base, int B, int Tc, int Hkv, int D, bool f32) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return NEA_ERR_CUDA;
+  const cuuint64_t e = f32 ? 4 : 2;
+  const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(Hkv), cuuint64_t(Tc), cuuint64_t(B)};
+  const cuuint64_t strides[3] = {D * e, cuuint64_t(Hkv) * D * e, cuuint64_t(Tc) * Hkv * D * e};
+  const cuuint32_t box[4] = {cuuint32_t(D), 1, cuuint32_t(nea::kDecChunk), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                         const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? NEA_OK : NEA_ERR_CUDA;
 }
@@ -514,7 +534,88 @@ int nea_device_status(void* stream_) {
   int v = 0;
   if ((e = cudaMemcpy(&v, st->err, sizeof v, cudaMemcpyDeviceToHost)) != cudaSuccess) return cuda_fail(e);
   if (v != 0 && (e = cudaMemset(st->err, 0, sizeof(int))) != cudaSuccess) return cuda_fail(e);
+  if (v == nea::kErrBadLength) return NEA_ERR_ARG;
   return v ? NEA_ERR_TIMEOUT : NEA_OK;
+}
+
+int nea_attn_decode(const void* Q, const void* Kc, const void* Vc, const int* lens, void* O, float* LSE, int B,
+                    int Tc, int Hq, int Hkv, int D, int dtype, float rope_base, void* stream_) {
+  if (B < 0 || Tc < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return NEA_ERR_ARG;
+  if (D != 32 && D != 64) return NEA_ERR_ARG;
+  if (dtype != NEA_F32 && dtype != NEA_BF16) return NEA_ERR_ARG;
+  if (Hq / Hkv > nea::kDecMaxG || Hkv > 65535 || B > 65535) return NEA_ERR_ARG;
+  if (!std::isfinite(rope_base)) return NEA_ERR_ARG;
+  if (B == 0) return NEA_OK;
+  if (Tc < 1 || Tc > (1 << 24)) return NEA_ERR_ARG;
+  if (!Q || !Kc || !Vc || !lens || !O || !LSE) return NEA_ERR_ARG;
+  if (!aligned16(Q) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(O) || !aligned16(LSE) ||
+      (reinterpret_cast<uintptr_t>(lens) & 3u))
+    return NEA_ERR_ARG;
+  const int n_split = (Tc + nea::kDecChunk - 1) / nea::kDecChunk;
+  const size_t part_bytes = round_up(size_t(B) * Hq * n_split * (D + 2) * sizeof(float), 256);
+  const size_t count_bytes = size_t(B) * Hkv * sizeof(int);
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc) return rc;
+  nea::DecodeParams p{};
+  if ((rc = rope_table(*st, Tc, D, rope_base, stream, &p.rope))) return rc;
+  if ((rc = ensure_ws(*st, part_bytes + count_bytes))) return rc;
+  p.Q = Q;
+  p.lens = lens;
+  p.O = O;
+  p.LSE = LSE;
+  p.part = reinterpret_cast<float*>(st->ws);
+  p.count = reinterpret_cast<int*>(st->ws + part_bytes);
+  cudaError_t em = cudaMemsetAsync(p.count, 0, count_bytes, stream);
+  if (em != cudaSuccess) return cuda_fail(em);
+  p.B = B;
+  p.Tc = Tc;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.n_split = n_split;
+  p.scale_log2 = float(1.4426950408889634 / std::sqrt(double(D)));
+  p.err = st->err;
+  p.wait_limit = static_cast<unsigned long long>(t_wait_limit_ns);
+  if ((rc = make_cache_map(&p.tm_k, Kc, B, Tc, Hkv, D, dtype == NEA_F32)) ||
+      (rc = make_cache_map(&p.tm_v, Vc, B, Tc, Hkv, D, dtype == NEA_F32)))
+    return rc;
+  const dim3 grid(static_cast<unsigned>(n_split), static_cast<unsigned>(Hkv), static_cast<unsigned>(B));
+  rc = dispatch(D, dtype, [&](auto d, auto f) {
+    constexpr int DD = decltype(d)::value;
+    constexpr bool FF = decltype(f)::value;
+    using S = nea::DecSmem<DD, FF>;
+    auto launch = [&](auto gtag) -> int {
+      constexpr int GG = decltype(gtag)::value;
+      auto kern = nea::attn_decode_split_kernel<DD, FF, GG>;
+      const int bit = ((DD == 64) * 2 + FF) * 8 + (GG - 1);
+      if (!(st->attr_dec >> bit & 1)) {
+        const cudaError_t ea = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(S::kBytes));
+        if (ea != cudaSuccess) return cuda_fail(ea);
+        st->attr_dec |= uint64_t(1) << bit;
+      }
+      kern<<<grid, 128, S::kBytes, stream>>>(p);
+      return NEA_OK;
+    };
+    int r2;
+    switch (p.G) {
+      case 1: r2 = launch(std::integral_constant<int, 1>{}); break;
+      case 2: r2 = launch(std::integral_constant<int, 2>{}); break;
+      case 3: r2 = launch(std::integral_constant<int, 3>{}); break;
+      case 4: r2 = launch(std::integral_constant<int, 4>{}); break;
+      case 5: r2 = launch(std::integral_constant<int, 5>{}); break;
+      case 6: r2 = launch(std::integral_constant<int, 6>{}); break;
+      case 7: r2 = launch(std::integral_constant<int, 7>{}); break;
+      default: r2 = launch(std::integral_constant<int, 8>{}); break;
+    }
+    return r2;
+  });
+  if (rc) return rc;
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? NEA_OK : cuda_fail(e);
 }
 
 long long nea_set_wait_limit_ns(long long ns) {

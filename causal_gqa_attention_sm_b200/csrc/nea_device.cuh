@@ -48,6 +48,7 @@ enum : int {
   kErrWaitMma = 0x200,       // a consumer gave up waiting for an MMA commit
   kErrWaitSoftmax = 0x300,   // the MMA issuer gave up waiting for P / dS
   kErrWaitEmpty = 0x400,     // the producer gave up waiting for a free stage
+  kErrBadLength = 0x800,     // a decode cache length outside [0, Tc] (clamped)
 };
 
 struct WaitCtl {

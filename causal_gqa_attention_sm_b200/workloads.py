@@ -32,6 +32,7 @@ class Workload:
     rope_base: float = 10000.0
     layers: int = 1     # independent attention layers per step
     seed: int = 0
+    decode: bool = False  # one query per sequence over a cache of T positions
 
     @property
     def torch_dtype(self):
@@ -50,7 +51,11 @@ class Workload:
         return f * self.layers
 
     def tokens(self) -> int:
-        return self.B * self.T * self.layers
+        return self.B * (1 if self.decode else self.T) * self.layers
+
+    def cache_bytes(self) -> int:
+        """Bytes of the key and value cache a full-length decode step reads."""
+        return 2 * self.B * self.T * self.Hkv * self.D * (4 if self.dtype == "f32" else 2)
 
 
 WORKLOADS = {
@@ -67,6 +72,9 @@ WORKLOADS = {
     "sweep1024": Workload("sweep1024", 16, 1024, 12, 4, 64, "bf16", seed=5001),
     "sweep2048": Workload("sweep2048", 8, 2048, 12, 4, 64, "bf16", seed=5002),
     "sweep4096": Workload("sweep4096", 4, 4096, 12, 4, 64, "bf16", seed=5003),
+    # generation over a key/value cache: 16 sequences, one new token each
+    "decode1024": Workload("decode1024", 16, 1024, 12, 4, 64, "f32", seed=6000, decode=True),
+    "decode4096": Workload("decode4096", 16, 4096, 12, 4, 64, "bf16", seed=6001, decode=True),
 }
 
 
@@ -83,6 +91,20 @@ def make_inputs(w: Workload, layer: int = 0, device="cpu"):
     do = torch.randn(shp_q, generator=g, dtype=torch.float32) * w.do_std
     out = {"q": q, "k": k, "v": v, "do": do}
     return {n: t.to(w.torch_dtype).to(device).contiguous() for n, t in out.items()}
+
+
+def make_decode_inputs(w: Workload, device="cpu"):
+    """Returns ``dict(q, kc, vc, lens)`` for a decode workload: the new tokens'
+    queries ``[B, Hq, D]``, a full cache ``[B, T, Hkv, D]`` of keys (standing
+    for keys already rotated at their positions) and values, and the lengths
+    (all ``T``), drawn like ``make_inputs``."""
+    g = torch.Generator(device="cpu").manual_seed(int(w.seed))
+    q = torch.randn((w.B, w.Hq, w.D), generator=g, dtype=torch.float32) * w.qk_std
+    kc = torch.randn((w.B, w.T, w.Hkv, w.D), generator=g, dtype=torch.float32) * w.qk_std
+    vc = torch.randn((w.B, w.T, w.Hkv, w.D), generator=g, dtype=torch.float32) * w.v_std
+    out = {n: t.to(w.torch_dtype).to(device).contiguous() for n, t in {"q": q, "kc": kc, "vc": vc}.items()}
+    out["lens"] = torch.full((w.B,), w.T, dtype=torch.int32, device=device)
+    return out
 
 
 def custom(name="custom", **kw) -> Workload:

@@ -114,7 +114,8 @@ int nea_attn_bwd(const void* Q, const void* K, const void* V, const void* O, con
 /*
  * Synchronises `stream`, then reads and clears the device error word of the
  * current device.  Returns NEA_OK, NEA_ERR_TIMEOUT when a kernel since the
- * last call abandoned a bounded wait (its outputs are then undefined), or
+ * last call abandoned a bounded wait (its outputs are then undefined),
+ * NEA_ERR_ARG when a decode call met a cache length outside [0, Tc], or
  * NEA_ERR_CUDA when the synchronisation itself failed.
  */
 int nea_device_status(void* stream);
@@ -183,6 +184,39 @@ void nea_set_profile_events(void* const* events, int n);
 int nea_attn_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O, const float* LSE,
                          const void* dO, void* dQ, void* dK, void* dV, int B, int T, int Hq, int Hkv, int D,
                          int dtype, float rope_base, int causal, void* stream);
+
+/*
+ * Decode: attention of one new query per sequence over a key/value cache,
+ * the generation path of the same causal attention ("NanoEuler" write-up,
+ * aimsg.uk, section 1, head-0 generation; RoPE on the query at its position,
+ * section 2 "Model components").
+ *
+ *   Q      [B][Hq][D] un-rotated query of the token at position lens[b] - 1
+ *   Kc     [B][Tc][Hkv][D] cached keys, already rotated at their positions
+ *          (R_t k_t, the same rotation the training path applies)
+ *   Vc     [B][Tc][Hkv][D] cached values
+ *   lens   device int32 [B]: valid cache length of each sequence,
+ *          0 <= lens[b] <= Tc; position lens[b] - 1 is the query's own
+ *   O      output [B][Hq][D], same dtype as Q
+ *   LSE    output float32 [B][Hq], natural-log log-sum-exp of the scores
+ *   Tc     cache capacity (positions), 1 <= Tc <= 2^24
+ *   Hq / Hkv <= 8; D 32 or 64; dtype NEA_F32 or NEA_BF16 (all arithmetic in
+ *   fp32); rope_base <= 0 disables the rotation of the query.
+ *
+ *   q' = R_{lens[b]-1} q, s_j = q' . k_j / sqrt(D) for j < lens[b],
+ *   LSE = ln sum_j exp(s_j), O = sum_j exp(s_j - LSE) v_j;
+ *   lens[b] = 0 gives O = 0 and LSE = -inf.
+ *
+ * Runs one kernel over 128-position pieces of the cache (the last piece of
+ * each sequence and kv head to finish merges them); uses the per-device
+ * workspace (B*Hq*ceil(Tc/128)*(D+2) floats and B*Hkv counters, cleared by
+ * the call).
+ * The lengths are read on the device: a value outside [0, Tc] is clamped and
+ * reported by the next nea_device_status() as NEA_ERR_ARG.  B == 0 is a
+ * no-op; argument errors return NEA_ERR_ARG with nothing launched.
+ */
+int nea_attn_decode(const void* Q, const void* Kc, const void* Vc, const int* lens, void* O, float* LSE, int B,
+                    int Tc, int Hq, int Hkv, int D, int dtype, float rope_base, void* stream);
 
 /* Human-readable name of a status code (static storage). */
 const char* nea_status_string(int status);
