@@ -268,6 +268,7 @@ int run_prep(uint8_t* base, const void* const* src, const size_t* elems, const i
   if (rowterm) pp = *rowterm;  // row-term fields of the backward
   pp.n_jobs = 0;
   pp.total = 0;
+  pp.prep_blocks = 0;
   size_t off = 0;
   pp.T = T;
   pp.rope = table;
@@ -294,12 +295,14 @@ int run_prep(uint8_t* base, const void* const* src, const size_t* elems, const i
       off += round_up(elems[i] * 2, 256);
     }
     j.chunks = static_cast<long long>(elems[i] / (f32 ? 4 : 8));
+    j.rows = static_cast<int>(elems[i] / D);
+    const int rows_per_block = 256 / (D * (f32 ? 4 : 2) / 16) * nea::kPrepUnroll;
+    j.block0 = pp.prep_blocks;
+    pp.prep_blocks += (j.rows + rows_per_block - 1) / rows_per_block;
     pp.job[pp.n_jobs++] = j;
     pp.total += j.chunks;
     jobs_out[i] = j;
   }
-  const long long per_block = 256LL * nea::kPrepUnroll;
-  pp.prep_blocks = int((pp.total + per_block - 1) / per_block);
   const long long blocks = pp.prep_blocks + (pp.rt_threads + 255) / 256;
   if (blocks == 0) return NEA_OK;
   const unsigned g = unsigned(blocks);

@@ -21,6 +21,8 @@ struct PrepJob {
   __nv_bfloat16* hi;      // same layout: bf16(x) (fp32), the rotated copy (bf16)
   __nv_bfloat16* lo;      // same layout: bf16(x - hi) (fp32 only)
   long long chunks;       // 16-byte chunks: B*T*H*D / 4 (fp32), / 8 (bf16)
+  int rows;               // B*T*H head vectors
+  int block0;             // first block of this job
   int H;                  // heads of this tensor
   int rope;               // 1: rotate (queries, keys)
   FastDiv divH;           // division by H
@@ -32,7 +34,7 @@ struct PrepParams {
   int T;
   const float2* rope;     // [T][D/2] (cos, sin) or nullptr
   long long total;        // sum of chunks
-  int prep_blocks;        // blocks [0, prep_blocks) rotate/split, kPrepUnroll chunks per thread
+  int prep_blocks;        // blocks [0, prep_blocks) rotate/split, kPrepUnroll rows' chunks per thread
   // backward row terms (rt_threads == 0: none), blocks from prep_blocks on
   const void* O;
   const void* dO;
@@ -94,11 +96,12 @@ __device__ __forceinline__ void rowterm_lane(const PrepParams& p, long long gtid
   }
 }
 
-// One 16-byte chunk of job tensor data: rotate (queries, keys) and convert.
+// One 16-byte chunk (chunk c of a head vector at position t) of job tensor
+// data: rotate (queries, keys) and convert.
 template <int D, bool F32IO>
-__device__ __forceinline__ void prep_chunk(const PrepParams& p, const PrepJob& job, long long ci, uint4 raw) {
+__device__ __forceinline__ void prep_chunk(const PrepParams& p, const PrepJob& job, size_t ci, int c, int t,
+                                           uint4 raw) {
   constexpr int kPerChunk = F32IO ? 4 : 8;  // elements per 16-byte chunk
-  constexpr int kCpr = D / kPerChunk;       // chunks per head vector
   float x[kPerChunk];
   if constexpr (F32IO) {
     x[0] = __uint_as_float(raw.x), x[1] = __uint_as_float(raw.y);
@@ -108,11 +111,7 @@ __device__ __forceinline__ void prep_chunk(const PrepParams& p, const PrepJob& j
 #pragma unroll
     for (int k = 0; k < 4; ++k) x[2 * k] = bf16_lo_f(w[k]), x[2 * k + 1] = bf16_hi_f(w[k]);
   }
-  if (job.rope && p.rope != nullptr) {
-    const uint32_t row = uint32_t(ci / kCpr);  // (b, t, h) row index
-    const int c = int(ci % kCpr);              // pairs kPerChunk/2 * c ...
-    const uint32_t bt = fdiv(row, job.divH);
-    const int t = int(bt - fdiv(bt, p.divT) * uint32_t(p.T));
+  if (job.rope) {
     const float4* cs = reinterpret_cast<const float4*>(p.rope + size_t(t) * (D / 2) + (kPerChunk / 2) * c);
 #pragma unroll
     for (int k = 0; k < kPerChunk / 4; ++k) {
@@ -135,33 +134,39 @@ __device__ __forceinline__ void prep_chunk(const PrepParams& p, const PrepJob& j
   }
 }
 
+// Blocks [0, prep_blocks) cover the jobs' head vectors in memory order, the
+// job chosen once per block: thread t takes chunk t % CPR of kPrepUnroll rows
+// (CPR chunks per row), so a warp reads and writes contiguous 512-byte runs
+// and the position of each row is found once per row, not per element.  The
+// remaining blocks write the row terms.
 template <int D, bool F32IO>
 __global__ void __launch_bounds__(256) attn_prep_kernel(const __grid_constant__ PrepParams p) {
   if (int(blockIdx.x) >= p.prep_blocks) {
-    rowterm_lane<D, F32IO>(p, (long long)(blockIdx.x - p.prep_blocks) * blockDim.x + threadIdx.x);
+    const long long g = (long long)(blockIdx.x - p.prep_blocks) * blockDim.x + threadIdx.x;
+    if (g < p.rt_threads) rowterm_lane<D, F32IO>(p, g);
     return;
   }
-  // kPrepUnroll chunks per thread, each step of them coalesced across the block
-  const long long base = (long long)blockIdx.x * blockDim.x * kPrepUnroll + threadIdx.x;
+  constexpr int CPR = D * (F32IO ? 4 : 2) / 16;   // 16-byte chunks per head vector
+  constexpr int kSlots = 256 / CPR;               // rows per block step
+  int j = 0;
+  while (j + 1 < p.n_jobs && int(blockIdx.x) >= p.job[j + 1].block0) ++j;
+  const PrepJob& job = p.job[j];
+  const int c = threadIdx.x % CPR;
+  const int row0 = (int(blockIdx.x) - job.block0) * kSlots * kPrepUnroll + threadIdx.x / CPR;
   uint4 raw[kPrepUnroll];
-  int jj[kPrepUnroll];
-  long long cc[kPrepUnroll];
 #pragma unroll
   for (int u = 0; u < kPrepUnroll; ++u) {
-    const long long i = base + (long long)u * blockDim.x;
-    int j = 0;
-    long long ci = i;
-    while (j + 1 < p.n_jobs && ci >= p.job[j].chunks) {
-      ci -= p.job[j].chunks;
-      ++j;
-    }
-    jj[u] = j;
-    cc[u] = ci;
-    if (i < p.total) raw[u] = __ldg(reinterpret_cast<const uint4*>(p.job[j].src) + ci);
+    const int ri = row0 + u * kSlots;
+    if (ri < job.rows) raw[u] = __ldg(reinterpret_cast<const uint4*>(job.src) + size_t(ri) * CPR + c);
   }
 #pragma unroll
-  for (int u = 0; u < kPrepUnroll; ++u)
-    if (base + (long long)u * blockDim.x < p.total) prep_chunk<D, F32IO>(p, p.job[jj[u]], cc[u], raw[u]);
+  for (int u = 0; u < kPrepUnroll; ++u) {
+    const int ri = row0 + u * kSlots;
+    if (ri >= job.rows) break;
+    const uint32_t bt = fdiv(uint32_t(ri), job.divH);  // (b, t) of the row
+    const int t = int(bt - fdiv(bt, p.divT) * uint32_t(p.T));
+    prep_chunk<D, F32IO>(p, job, size_t(ri) * CPR + c, c, t, raw[u]);
+  }
 }
 
 }  // namespace nea
