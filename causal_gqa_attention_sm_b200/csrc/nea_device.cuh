@@ -450,6 +450,32 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   return r;
 }
 
+// 2^x for a pair of floats on the FMA pipe, leaving the exponential unit
+// free: x = j + f with j the nearest integer (adding and subtracting
+// 1.5 * 2^23 rounds to it), 2^f from the degree-3 polynomial that
+// exp2_poly_fit.py derives (relative error below 7.5e-5 for f in
+// [-1/2, 1/2]), and 2^j added to the exponent field.  Inputs below -125
+// (-inf included) are clamped: their result is 2^-125 (about 2.4e-38).
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  const uint64_t xc = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t magic = f2_pack(12582912.f, 12582912.f);
+  const uint64_t y = f2_add(xc, magic);
+  const uint64_t f = f2_sub(xc, f2_sub(y, magic));
+  uint64_t p = f2_fma(f, f2_pack(0.05517132207751274f, 0.05517132207751274f),
+                      f2_pack(0.24261054396629333f, 0.24261054396629333f));
+  p = f2_fma(p, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+  p = f2_fma(p, f, f2_pack(0.9999281167984009f, 0.9999281167984009f));
+  float y0, y1, p0, p1;
+  f2_unpack(y, y0, y1);
+  f2_unpack(p, p0, p1);
+  // the low bits of y hold j; shifted into the exponent field (the bits of
+  // 1.5 * 2^23 shift out of the word)
+  return f2_pack(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(y0) << 23)),
+                 __uint_as_float(__float_as_uint(p1) + (__float_as_uint(y1) << 23)));
+}
+
 // Maximum of three floats in one instruction (sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;

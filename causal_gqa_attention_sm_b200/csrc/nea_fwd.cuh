@@ -211,13 +211,21 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
         }
       };
       if constexpr (kSepP) {
-        // P = exp2(s * scale_log2 - m) -> bf16, all 128 columns in registers
+        // P = exp2(s * scale_log2 - m) -> bf16, all 128 columns in registers;
+        // one pair in four on the FMA pipe, the rest on the exponential unit
         uint32_t pk[64];
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
-          float t0, t1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), sc2, nm2), t0, t1);
-          const float p0 = ex2(t0), p1 = ex2(t1);
+          const uint64_t t2 = f2_fma(f2_pack(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), sc2, nm2);
+          float p0, p1;
+          if ((i & 3) == 3) {
+            f2_unpack(exp2_poly2(t2), p0, p1);
+          } else {
+            float t0, t1;
+            f2_unpack(t2, t0, t1);
+            p0 = ex2(t0);
+            p1 = ex2(t1);
+          }
           if (i & 1) l23 = f2_add(l23, f2_pack(p0, p1)); else l01 = f2_add(l01, f2_pack(p0, p1));
           pk[i] = pack_bf16(p0, p1);
         }
