@@ -375,7 +375,7 @@ def decode_main(a, w, rank, world, local):
                        "parallelism": f"dp{world} (independent sequences per GPU)"},
             "tokens_per_s": w.B * K * world / (total_ms * 1e-3),
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks.summary(),
-            "gpu_launches": 2 * K,
+            "gpu_launches": K,
         }
         print(json.dumps(line), flush=True)
     return 0
