@@ -173,10 +173,17 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- ncu traffic records
-def kernel_source_hash():
+# The sources that make up each kernel: its own header plus the shared device
+# helpers, tile geometry and the host code that sets up its launch.
+KERNEL_SOURCES = {"attn_fwd_prologue": "nea_prep.cuh", "attn_bwd_prologue": "nea_prep.cuh",
+                  "attn_fwd": "nea_fwd.cuh", "attn_bwd": "nea_bwd.cuh", "attn_decode": "nea_decode.cuh"}
+SHARED_SOURCES = ("nea_attn.cu", "nea_device.cuh", "nea_tiles.cuh")
+
+
+def kernel_source_hash(kernel):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "causal_gqa_attention_sm_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(SHARED_SOURCES + (KERNEL_SOURCES[kernel],)):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -184,13 +191,13 @@ def kernel_source_hash():
 
 def ncu_traffic(kernel, workload):
     """DRAM bytes per launch from a committed ncu summary, or None when absent
-    or when the kernel sources changed since it was captured."""
+    or when the kernel's sources changed since it was captured."""
     path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         rec = json.load(f)
-    if rec.get("source_hash") != kernel_source_hash():
+    if rec.get("source_hash") != kernel_source_hash(kernel):
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -465,7 +472,10 @@ def main():
 
     K = a.steps
     ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    # per-layer kernel-boundary events of every step (7 per layer)
+    # per-layer kernel-boundary events (7 per layer) of the profiling steps that
+    # follow the timed ones: an event between two kernels would stop the next
+    # kernel from starting while the previous one drains, so the timed steps
+    # carry none
     ev_k = [[[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(w.layers)] for _ in range(K)]
     for evs in ev_k:
         for row in evs:
@@ -481,16 +491,21 @@ def main():
         for i in range(K):
             flush_l2(i)
             ev_step[i][0].record(stream)
-            for li, (L, O) in enumerate(zip(layers, outs)):
-                nea.nea_set_profile_events(ev_k[i][li])
-                nea.nea_attn_fwd(L["q"], L["k"], L["v"], w.rope_base, w.causal, o=O["o"], lse=O["lse"])
-                nea.nea_attn_bwd(L["q"], L["k"], L["v"], O["o"], O["lse"], L["do"], w.rope_base, w.causal,
-                                 dq=O["dq"], dk=O["dk"], dv=O["dv"])
-            nea.nea_set_profile_events(None)
+            step()
             ev_step[i][1].record(stream)
         torch.cuda.synchronize(dev)
         wall = time.perf_counter() - wall0
     barrier(world)
+    # per-kernel durations: the same steps again with events between the kernels
+    for i in range(K):
+        flush_l2(i)
+        for li, (L, O) in enumerate(zip(layers, outs)):
+            nea.nea_set_profile_events(ev_k[i][li])
+            nea.nea_attn_fwd(L["q"], L["k"], L["v"], w.rope_base, w.causal, o=O["o"], lse=O["lse"])
+            nea.nea_attn_bwd(L["q"], L["k"], L["v"], O["o"], O["lse"], L["do"], w.rope_base, w.causal,
+                             dq=O["dq"], dk=O["dk"], dv=O["dv"])
+        nea.nea_set_profile_events(None)
+    torch.cuda.synchronize(dev)
     status = nea.nea_device_status()
     if status != nea.NEA_OK:
         raise SystemExit(f"device status after timing: {nea.nea_status_string(status)}")

@@ -14,6 +14,7 @@
 #include <mutex>
 #include <tuple>
 #include <type_traits>
+#include <utility>
 #include <vector>
 
 #include "nea_attn.h"
@@ -223,6 +224,26 @@ int check_shape(int B, int T, int Hq, int Hkv, int D, int dtype, int causal, boo
   return NEA_OK;
 }
 
+// Launches a kernel with programmatic stream serialization: its blocks may
+// start (barrier set-up, TMEM allocation) while the previous kernel in the
+// stream drains; each kernel launched this way calls grid_dep_wait() before
+// its first global access, so stream order still holds for memory.
+template <typename... P, typename... A>
+cudaError_t launch_dependent(void (*kern)(P...), unsigned grid, unsigned block, size_t smem, cudaStream_t stream,
+                             A&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
+}
+
 template <typename Kern>
 int set_smem(uint32_t& attr_done, int bit, Kern kern, uint32_t bytes) {
   if (attr_done & (1u << bit)) return NEA_OK;
@@ -306,13 +327,9 @@ int run_prep(uint8_t* base, const void* const* src, const size_t* elems, const i
   const long long blocks = pp.prep_blocks + (pp.rt_threads + 255) / 256;
   if (blocks == 0) return NEA_OK;
   const unsigned g = unsigned(blocks);
-  if (D == 64)
-    f32 ? nea::attn_prep_kernel<64, true><<<g, 256, 0, stream>>>(pp)
-        : nea::attn_prep_kernel<64, false><<<g, 256, 0, stream>>>(pp);
-  else
-    f32 ? nea::attn_prep_kernel<32, true><<<g, 256, 0, stream>>>(pp)
-        : nea::attn_prep_kernel<32, false><<<g, 256, 0, stream>>>(pp);
-  const cudaError_t e = cudaGetLastError();
+  auto kern = D == 64 ? (f32 ? nea::attn_prep_kernel<64, true> : nea::attn_prep_kernel<64, false>)
+                      : (f32 ? nea::attn_prep_kernel<32, true> : nea::attn_prep_kernel<32, false>);
+  const cudaError_t e = launch_dependent(kern, g, 256, 0, stream, pp);
   return e == cudaSuccess ? NEA_OK : cuda_fail(e);
 }
 
@@ -323,8 +340,7 @@ int launch_fwd(uint32_t& attr_done, const nea::FwdParams& p, cudaStream_t stream
   auto kern = nea::attn_fwd_kernel<D, F32IO>;
   int rc = set_smem(attr_done, (D == 64) * 2 + F32IO, kern, L::kAlloc);
   if (rc) return rc;
-  kern<<<p.B * p.Hq * p.n_pairs, L::kThreads, L::kAlloc, stream>>>(p);
-  cudaError_t e = cudaGetLastError();
+  const cudaError_t e = launch_dependent(kern, unsigned(p.B * p.Hq * p.n_pairs), L::kThreads, L::kAlloc, stream, p);
   return e == cudaSuccess ? NEA_OK : cuda_fail(e);
 }
 
@@ -338,8 +354,8 @@ int launch_bwd(uint32_t& attr_done, const nea::BwdParams& p, cudaStream_t stream
   auto kern = nea::attn_bwd_kernel<D, F32IO>;
   int rc = set_smem(attr_done, 4 + (D == 64) * 2 + F32IO, kern, L::kAlloc);
   if (rc) return rc;
-  kern<<<p.n_dkdv + p.B * p.Hq * p.n_tiles, L::kThreads, L::kAlloc, stream>>>(p);
-  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+  e = launch_dependent(kern, unsigned(p.n_dkdv + p.B * p.Hq * p.n_tiles), L::kThreads, L::kAlloc, stream, p);
+  if (e != cudaSuccess) return cuda_fail(e);
   if (ev) prof_record(4, stream);
   if (ev) prof_record(5, stream);
   return NEA_OK;

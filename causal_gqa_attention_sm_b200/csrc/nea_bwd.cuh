@@ -199,6 +199,8 @@ __device__ __forceinline__ void attn_bwd_unit(const BwdParams& p, int bid) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_holder;
+  grid_dep_wait();  // operand planes and row terms come from the prologue grid
+  grid_dep_launch();
   constexpr uint32_t kColS = 0, kColDP = 128, kColAcc1 = 256, kColAcc2 = 256 + D, kColP = 384, kColDS = 448;
 
   if (warp == 9) {

@@ -191,6 +191,16 @@ __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// A grid launched with programmatic stream serialization may start while the
+// previous grid in its stream still runs.  grid_dep_wait() returns once every
+// grid it depends on has completed and its memory writes are visible (at once
+// for an ordinary launch); every block calls it before its first global
+// access.  grid_dep_launch() lets the next such grid start its launch once
+// every block of this one has called it or exited.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ proxies
 // Generic-proxy shared-memory writes -> visible to tcgen05.mma operand reads.
 __device__ __forceinline__ void fence_async_smem() {

@@ -157,6 +157,8 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_holder;
+  grid_dep_wait();  // the operand planes come from the prologue grid
+  grid_dep_launch();
   NEA_TRACE_STAMP(p, 1, tid == 0);
 
   if (warp < 8) {

@@ -141,6 +141,8 @@ __device__ __forceinline__ void prep_chunk(const PrepParams& p, const PrepJob& j
 // remaining blocks write the row terms.
 template <int D, bool F32IO>
 __global__ void __launch_bounds__(256) attn_prep_kernel(const __grid_constant__ PrepParams p) {
+  grid_dep_wait();
+  grid_dep_launch();
   if (int(blockIdx.x) >= p.prep_blocks) {
     const long long g = (long long)(blockIdx.x - p.prep_blocks) * blockDim.x + threadIdx.x;
     if (g < p.rt_threads) rowterm_lane<D, F32IO>(p, g);

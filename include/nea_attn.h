@@ -33,7 +33,11 @@
  * default stream) and the call returns without synchronising.  Calls on one
  * device share its workspace, so calls on different streams must not overlap
  * in time.  Device-side wait limits are reported asynchronously: see
- * nea_device_status().
+ * nea_device_status().  The training-path kernels are launched with
+ * programmatic stream serialization: a kernel may begin its set-up while the
+ * kernel before it in the stream drains, but it touches no global memory
+ * until that kernel has completed, so stream order holds for every buffer
+ * (the caller's kernels included).
  *
  * Errors: a call returns NEA_OK or one of the codes below; on NEA_ERR_ARG
  * nothing is launched and no output is touched.  Kernels never trap.
@@ -145,7 +149,9 @@ void nea_debug_inject(int flags);
  *   nea_attn_bwd: events[2] before the operand prologue (which also writes
  *                 the row terms), events[3] after it, events[4] and events[5]
  *                 after the gradient kernel.
- * Indices >= n are skipped.  The array must stay valid while set.
+ * Indices >= n are skipped.  The array must stay valid while set.  An event
+ * between two kernels stops the second from starting early, so profiled
+ * calls run their kernels strictly one after the other.
  */
 void nea_set_profile_events(void* const* events, int n);
 
