@@ -68,6 +68,20 @@ __device__ __forceinline__ void smem_chunk(const uint8_t* row, int c, float* x) 
   }
 }
 
+// The same chunk as packed float pairs (elements 2k, 2k + 1 in pair k).
+template <bool F32IO>
+__device__ __forceinline__ void smem_chunk2(const uint8_t* row, int c, uint64_t* x) {
+  const uint4 u = reinterpret_cast<const uint4*>(row)[c];
+  if constexpr (F32IO) {
+    x[0] = f2_pack(__uint_as_float(u.x), __uint_as_float(u.y));
+    x[1] = f2_pack(__uint_as_float(u.z), __uint_as_float(u.w));
+  } else {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) x[k] = f2_pack(bf16_lo_f(w[k]), bf16_hi_f(w[k]));
+  }
+}
+
 template <bool F32IO>
 __device__ __forceinline__ float load_elem(const void* base, size_t elem_off) {
   if constexpr (F32IO) return __ldg(static_cast<const float*>(base) + elem_off);
@@ -118,7 +132,6 @@ __global__ void __launch_bounds__(128) attn_decode_split_kernel(const __grid_con
   if (j0 >= len) return;  // no cached position of this split
   const int n = min(kDecChunk, len - j0);
   const int r = tid / L, c = tid % L;  // row slot, chunk of the row
-  const unsigned grp = (L == 32 ? kFullMask : ((1u << L) - 1u) << (lane & ~(L - 1)));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + S::kBar + 8);
   const WaitCtl wc{p.err, p.wait_limit, abort_flag};
 
@@ -147,29 +160,48 @@ __global__ void __launch_bounds__(128) attn_decode_split_kernel(const __grid_con
   __syncthreads();  // also publishes the barrier's initialisation
   const bool ok = wait_warp(bar, 0, wc, kErrWaitProducer);
 
-  // ---- scores: the lanes of row slot r take positions r, r + R, ...
-  float qr[G][EPC];  // this lane's chunk of every query
-#pragma unroll
-  for (int gi = 0; gi < G; ++gi)
-#pragma unroll
-    for (int e = 0; e < EPC; ++e) qr[gi][e] = qs[gi][c * EPC + e];
+  // ---- scores: lane (r, c) forms the partial dot products of its chunk c
+  // with every head for the rows r, r + R, ... of its slot (NR == L rows; the
+  // rows past n hold cache data or the copy's zero fill and are masked by the
+  // softmax), then the L lanes of the slot trade halves of their partials,
+  // log2 L times, so that lane c ends with the complete scores of row r + c R:
+  // G (L - 1) shuffles per lane instead of G L log2 L.
+  static_assert(NR == L, "one complete row per lane after the exchange");
   if (ok) {
+    uint64_t q2[G][EPC / 2];  // this lane's chunk of every query, in pairs
+#pragma unroll
+    for (int gi = 0; gi < G; ++gi)
+#pragma unroll
+      for (int e = 0; e < EPC / 2; ++e) q2[gi][e] = f2_pack(qs[gi][c * EPC + 2 * e], qs[gi][c * EPC + 2 * e + 1]);
+    float part[NR][G];
 #pragma unroll
     for (int i = 0; i < NR; ++i) {
-      const int t = r + i * R;
-      if (t >= n) break;
-      float k[EPC];
-      smem_chunk<F32IO>(sm + S::kK + t * S::kRow, c, k);
+      uint64_t k2[EPC / 2];
+      smem_chunk2<F32IO>(sm + S::kK + (r + i * R) * S::kRow, c, k2);
 #pragma unroll
       for (int gi = 0; gi < G; ++gi) {
-        float acc = 0.f;
+        uint64_t acc = f2_mul(q2[gi][0], k2[0]);
 #pragma unroll
-        for (int e = 0; e < EPC; ++e) acc = fmaf(qr[gi][e], k[e], acc);
-#pragma unroll
-        for (int off = L / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(grp, acc, off);
-        if (c == 0) sc[gi][t] = acc;
+        for (int e = 1; e < EPC / 2; ++e) acc = f2_fma(q2[gi][e], k2[e], acc);
+        float a0, a1;
+        f2_unpack(acc, a0, a1);
+        part[i][gi] = a0 + a1;
       }
     }
+#pragma unroll
+    for (int h = L / 2; h >= 1; h /= 2) {
+      const bool up = (c & h) != 0;
+#pragma unroll
+      for (int j = 0; j < h; ++j)
+#pragma unroll
+        for (int gi = 0; gi < G; ++gi) {
+          const float keep = up ? part[j + h][gi] : part[j][gi];
+          const float send = up ? part[j][gi] : part[j + h][gi];
+          part[j][gi] = keep + __shfl_xor_sync(kFullMask, send, h);
+        }
+    }
+#pragma unroll
+    for (int gi = 0; gi < G; ++gi) sc[gi][r + c * R] = part[0][gi];
   }
   __syncthreads();
 
@@ -203,23 +235,24 @@ __global__ void __launch_bounds__(128) attn_decode_split_kernel(const __grid_con
 
   // ---- o = P V: lane (r, c) sums rows r, r + R, ... of its chunk's columns,
   // then the row slots of a warp are folded by shuffles, the warps in smem
-  float o[G][EPC];
+  uint64_t o2[G][EPC / 2];  // packed pairs of this lane's chunk columns
 #pragma unroll
   for (int gi = 0; gi < G; ++gi)
 #pragma unroll
-    for (int e = 0; e < EPC; ++e) o[gi][e] = 0.f;
+    for (int e = 0; e < EPC / 2; ++e) o2[gi][e] = 0;  // the bit pattern of (+0, +0)
   if (ok) {
 #pragma unroll
     for (int i = 0; i < NR; ++i) {
       const int t = r + i * R;
-      if (t >= n) break;
-      float v[EPC];
-      smem_chunk<F32IO>(sm + S::kV + t * S::kRow, c, v);
+      if (t >= n) break;  // never touch values past the cache length
+      uint64_t v2[EPC / 2];
+      smem_chunk2<F32IO>(sm + S::kV + t * S::kRow, c, v2);
 #pragma unroll
       for (int gi = 0; gi < G; ++gi) {
         const float pw = sc[gi][t];
+        const uint64_t pw2 = f2_pack(pw, pw);
 #pragma unroll
-        for (int e = 0; e < EPC; ++e) o[gi][e] = fmaf(pw, v[e], o[gi][e]);
+        for (int e = 0; e < EPC / 2; ++e) o2[gi][e] = f2_fma(pw2, v2[e], o2[gi][e]);
       }
     }
   }
@@ -228,12 +261,20 @@ __global__ void __launch_bounds__(128) attn_decode_split_kernel(const __grid_con
 #pragma unroll
     for (int gi = 0; gi < G; ++gi)
 #pragma unroll
-      for (int e = 0; e < EPC; ++e) o[gi][e] += __shfl_xor_sync(kFullMask, o[gi][e], off);
+      for (int e = 0; e < EPC / 2; ++e) {
+        float lo, hi;
+        f2_unpack(o2[gi][e], lo, hi);
+        o2[gi][e] = f2_add(o2[gi][e], f2_pack(__shfl_xor_sync(kFullMask, lo, off), __shfl_xor_sync(kFullMask, hi, off)));
+      }
   if (lane < L)
 #pragma unroll
     for (int gi = 0; gi < G; ++gi)
 #pragma unroll
-      for (int e = 0; e < EPC; ++e) red[(warp * kDecMaxG + gi) * D + c * EPC + e] = o[gi][e];
+      for (int e = 0; e < EPC / 2; ++e) {
+        float lo, hi;
+        f2_unpack(o2[gi][e], lo, hi);
+        *reinterpret_cast<float2*>(&red[(warp * kDecMaxG + gi) * D + c * EPC + 2 * e]) = make_float2(lo, hi);
+      }
   __syncthreads();
   for (int e = tid; ok && e < G * D; e += blockDim.x) {
     const int gi = e / D, d = e % D;
