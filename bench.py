@@ -1,7 +1,9 @@
 """Throughput of causal GQA attention forward+backward on B200.
 
-One step = nea_attn_fwd + nea_attn_bwd (four kernels: forward, row term,
-dK/dV, dQ) over one batch of synthetic inputs already resident in HBM.
+One step = nea_attn_fwd + nea_attn_bwd (four kernels: the forward operand
+prologue, the forward, the backward prologue with the row terms, and the
+gradient kernel with its dK/dV and dQ units) over one batch of synthetic
+inputs already resident in HBM.
 Default workload: B=4, T=1024, Hq=12, Hkv=4, D=64, float32 storage, causal,
 RoPE base 10000, Q,K ~ N(0, 9), V, dO ~ N(0, 1) -- the longer-context
 configuration of the NanoEuler GPU model shape.
