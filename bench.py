@@ -27,6 +27,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -67,6 +68,7 @@ def parse():
     ap.add_argument("--impl", default="nea", choices=["nea", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--clocks-csv", default=None, help="keep the raw nvidia-smi clock samples in this file")
     a = ap.parse_args()
     a.warmup = max(a.warmup, 3)
     return a
@@ -129,14 +131,16 @@ class ClockSampler:
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index):
+    def __init__(self, gpu_index, path=None):
         self.idx = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        # the raw samples: a file of the caller's choosing, else a temporary one
+        self.path = path or os.path.join(tempfile.gettempdir(), f"nea_clocks_{os.getpid()}_{gpu_index}.csv")
 
     def __enter__(self):
+        self.f = None
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            os.makedirs(os.path.dirname(os.path.abspath(self.path)), exist_ok=True)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
                                           "--format=csv,noheader,nounits", "-lms", "200"],
@@ -144,6 +148,8 @@ class ClockSampler:
             time.sleep(0.3)
         except OSError:
             self.proc = None
+            if self.f is not None:
+                self.f.close()
         return self
 
     def __exit__(self, *a):
@@ -321,7 +327,7 @@ def decode_main(a, w, rank, world, local):
         raise SystemExit("device status after warm-up")
     K = a.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(local, a.clocks_csv)
     barrier(world)
     with clocks:
         for i in range(K):
@@ -485,7 +491,7 @@ def main():
                 e.record(stream)  # materialise the CUDA events
     torch.cuda.synchronize(dev)
 
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(local, a.clocks_csv)
     barrier(world)
     torch.cuda.synchronize(dev)
     with clocks:

@@ -87,3 +87,13 @@ def test_reference_arm_prints_the_contract_line(workload):
     assert line["config"]["workload"] == workload
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_clock_sampler_without_nvidia_smi_reports_it(tmp_path, monkeypatch):
+    monkeypatch.setenv("PATH", str(tmp_path))  # no nvidia-smi on the path
+    c = bench.ClockSampler(0, str(tmp_path / "clocks.csv"))
+    with c:
+        pass
+    assert c.summary()["reasons"] == ["nvidia-smi unavailable"]
+    assert c.f.closed
+    assert not bench.ClockSampler(3).path.startswith(ROOT)  # raw samples go to a temporary file by default
