@@ -9,6 +9,11 @@ Every function takes and returns float64 arrays in the library's layout:
 Q, O, dO, dQ ``[B, T, Hq, D]``; K, V, dK, dV ``[B, T, Hkv, D]``;
 LSE and the row term ``Dvec`` ``[B, Hq, T]``.
 
+``block_ref`` (numpy, float64) holds the steps on either side of the
+attention in a decoder block: the RMSNorm pre-norm with the Q/K/V
+projections, and the output projection with the residual add; its pins are
+in ``tests/test_block_oracle.py``.
+
 Parity pins: every function here is checked in ``tests/test_oracle.py``
 against closed forms, invariants, central finite differences and a library
 cross-check; see the header of ``attn_ref.c`` for the passages each step
