@@ -59,6 +59,38 @@ def prologue_bytes(w, kernel):
     return b
 
 
+def load_workloads():
+    """The workload table and input generator, loaded by file path: importing
+    it through the package would run the package's ``__init__``, which loads
+    the CUDA library, and the reference arm must not load it."""
+    import importlib.util
+
+    name = "_nea_workloads"
+    if name in sys.modules:
+        return sys.modules[name]
+    spec = importlib.util.spec_from_file_location(
+        name, os.path.join(ROOT, "causal_gqa_attention_sm_b200", "workloads.py"))
+    mod = importlib.util.module_from_spec(spec)
+    sys.modules[name] = mod
+    spec.loader.exec_module(mod)
+    return mod
+
+
+L2_NOTE = "flushed before every timed step (256 MiB write, then 256 MiB read of another buffer)"
+
+
+def config_of(w, world):
+    """The `config` object of a bench line; both arms print the same one."""
+    storage = {"f32": "float32", "bf16": "bfloat16"}[w.dtype]
+    if w.decode:
+        return {"workload": w.name, "B": w.B, "Tc": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "storage": storage,
+                "rope_base": w.rope_base, "lens": "all Tc", "l2": L2_NOTE,
+                "parallelism": f"dp{world} (independent sequences per GPU)"}
+    return {"workload": w.name, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "storage": storage,
+            "causal": w.causal, "rope_base": w.rope_base, "layers": w.layers, "qk_std": w.qk_std, "l2": L2_NOTE,
+            "parallelism": f"dp{world} (independent batches per GPU)"}
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -170,14 +202,77 @@ class ClockSampler:
                     rows.append(parts)
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
-        load = [s for s in sm if s > 0.5 * mx] or sm
+        num = lambda v: v.replace(".", "", 1).isdigit()  # noqa: E731  ("[N/A]" and the like are skipped)
+        sm = [float(r[1]) for r in rows if num(r[1])]
+        mx = max((float(r[2]) for r in rows if num(r[2])), default=None)
+        load = ([s for s in sm if s > 0.5 * mx] if mx else []) or sm
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(load), "sm_max_mhz": mx, "reasons": reasons,
-                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows
-                                                         if r[3].replace(".", "").isdigit())}
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows),
+                "power_w_max": max((float(r[3]) for r in rows if num(r[3])), default=None)}
+
+
+def clock_window(step, flush_l2, stream, dev, seconds):
+    """Runs identical steps (each after an L2 flush) for at least `seconds`
+    and returns their count and mean device time per step."""
+    import torch
+
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n, t0 = 0, time.perf_counter()
+    s0.record(stream)
+    while True:
+        for _ in range(20):
+            flush_l2(n)
+            step()
+            n += 1
+        torch.cuda.synchronize(dev)
+        if time.perf_counter() - t0 >= seconds:
+            break
+    s1.record(stream)
+    torch.cuda.synchronize(dev)
+    return {"steps": n, "seconds": time.perf_counter() - t0,
+            "ms_per_step_incl_flush": s0.elapsed_time(s1) / n,
+            "note": "steps run under the clock sampler before the timed ones; not part of `value`"}
+
+
+def measure_tf32_peak(dev, sustain_s=4.0):
+    """Dense TF32 tensor-core throughput of this GPU, measured the way the
+    bf16 peak is: a float32 8192^3 torch.matmul with TF32 allowed (a cuBLAS
+    call, used only as a yardstick), as a burst of 10 and as a loop of about
+    `sustain_s` seconds."""
+    import torch
+
+    prev = torch.backends.cuda.matmul.allow_tf32
+    torch.backends.cuda.matmul.allow_tf32 = True
+    try:
+        n = 8192
+        g = torch.Generator(device=dev).manual_seed(0)
+        a = torch.randn((n, n), device=dev, generator=g)
+        b = torch.randn((n, n), device=dev, generator=g)
+        c = torch.empty((n, n), device=dev)
+        for _ in range(3):
+            torch.matmul(a, b, out=c)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record()
+        for _ in range(10):
+            torch.matmul(a, b, out=c)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        burst = 2.0 * n ** 3 * 10 / (e0.elapsed_time(e1) * 1e-3) / 1e12
+        reps = max(10, int(sustain_s * burst * 1e12 / (2.0 * n ** 3)))
+        e0.record()
+        for _ in range(reps):
+            torch.matmul(a, b, out=c)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        sustained = 2.0 * n ** 3 * reps / (e0.elapsed_time(e1) * 1e-3) / 1e12
+        del a, b, c
+        return {"tf32_tflops": burst, "tf32_tflops_sustained": sustained,
+                "how": "torch.matmul float32 8192^3 with TF32 allowed (cuBLAS), burst of 10 and a ~4 s loop"}
+    finally:
+        torch.backends.cuda.matmul.allow_tf32 = prev
 
 
 # ---------------------------------------------------------------- ncu traffic records
@@ -220,8 +315,8 @@ def run_oracle_sample(w, max_units=None, min_seconds=0.0):
     import numpy as np
 
     import oracle
-    from causal_gqa_attention_sm_b200.workloads import make_inputs
 
+    make_inputs = load_workloads().make_inputs
     cores = len(os.sched_getaffinity(0))
     units = w.B * w.Hkv
     n = min(units, max_units or units)
@@ -252,11 +347,11 @@ def reference_arm(a, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    for _ in range(a.warmup):
-        pass  # the oracle has no state to warm; each step is a full independent run
+    per_step_units = max(1, min(w.B * w.Hkv, len(os.sched_getaffinity(0))))
+    for _ in range(a.warmup):  # untimed steps of the same sample (page in, spin up the thread pool)
+        run_oracle_sample(w, per_step_units)
     secs, flops = 0.0, 0.0
     threads = desc = None
-    per_step_units = max(1, min(w.B * w.Hkv, len(os.sched_getaffinity(0))))
     for _ in range(a.steps):
         dt, fl, threads, desc = run_oracle_sample(w, per_step_units)
         secs += dt
@@ -266,8 +361,7 @@ def reference_arm(a, w):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": a.gpus,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": secs / a.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
-                   "storage": w.dtype, "causal": w.causal, "rope_base": w.rope_base, "layers": w.layers},
+        "config": config_of(w, a.gpus),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -284,9 +378,8 @@ def run_oracle_decode(w, min_seconds=0.0):
     least `min_seconds` have passed.  Returns (seconds, cache bytes, threads,
     description)."""
     import oracle
-    from causal_gqa_attention_sm_b200.workloads import make_decode_inputs
 
-    inp = make_decode_inputs(w)
+    inp = load_workloads().make_decode_inputs(w)
     arr = {k: v.float().double().numpy() if k != "lens" else v.numpy() for k, v in inp.items()}
     threads = min(len(os.sched_getaffinity(0)), w.B * w.Hq)
     oracle.set_threads(threads)
@@ -330,6 +423,8 @@ def decode_main(a, w, rank, world, local):
     clocks = ClockSampler(local, a.clocks_csv)
     barrier(world)
     with clocks:
+        window = clock_window(step, lambda i: (flush.fill_(float(i)), torch.sum(drain, dim=0, out=drain_sum)),
+                              stream, dev, 1.2)
         for i in range(K):
             flush.fill_(float(i))
             torch.sum(drain, dim=0, out=drain_sum)
@@ -383,14 +478,10 @@ def decode_main(a, w, rank, world, local):
             "metric": DECODE_METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
             "warmup": a.warmup, "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "Tc": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
-                       "storage": {"f32": "float32", "bf16": "bfloat16"}[w.dtype], "rope_base": w.rope_base,
-                       "lens": "all Tc",
-                       "l2": "flushed before every timed step (256 MiB write, then 256 MiB read of another buffer)",
-                       "parallelism": f"dp{world} (independent sequences per GPU)"},
+            "config": config_of(w, world),
             "tokens_per_s": w.B * K * world / (total_ms * 1e-3),
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks.summary(),
-            "gpu_launches": K,
+            "clock_window": window, "gpu_launches": K,
         }
         print(json.dumps(line), flush=True)
     return 0
@@ -410,8 +501,7 @@ def reference_decode(a, w):
         "impl": "reference", "metric": DECODE_METRIC, "value": value, "unit": "GB/s", "n_gpus": a.gpus,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": secs / a.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "Tc": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
-                   "storage": w.dtype, "rope_base": w.rope_base, "lens": "all Tc"},
+        "config": config_of(w, a.gpus),
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -422,9 +512,7 @@ def reference_decode(a, w):
 # ---------------------------------------------------------------- GPU arm
 def main():
     a = parse()
-    from causal_gqa_attention_sm_b200.workloads import WORKLOADS
-
-    w = WORKLOADS[a.workload]
+    w = load_workloads().WORKLOADS[a.workload]
     if a.impl == "reference":
         return reference_decode(a, w) if w.decode else reference_arm(a, w)
 
@@ -495,6 +583,11 @@ def main():
     barrier(world)
     torch.cuda.synchronize(dev)
     with clocks:
+        # the sampler polls every 200 ms, far longer than the timed steps: a
+        # block of identical steps of at least 1.2 s runs under it first, so
+        # that the clock record spans kernel execution (reported apart as
+        # `clock_window`; the value comes from the K steps after it only)
+        window = clock_window(step, flush_l2, stream, dev, 1.2)
         wall0 = time.perf_counter()
         for i in range(K):
             flush_l2(i)
@@ -622,20 +715,20 @@ def main():
         cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc,
                "seconds": dt}
 
+    tf32 = measure_tf32_peak(dev) if w.dtype == "f32" else None
     if rank == 0:
-        storage = {"f32": "float32", "bf16": "bfloat16"}[w.dtype]
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": a.warmup,
             "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16x3" if w.dtype == "f32" else "bf16", "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
-                       "storage": storage, "causal": w.causal, "rope_base": w.rope_base, "layers": w.layers,
-                       "qk_std": w.qk_std, "l2": "flushed before every timed step (256 MiB write, then 256 MiB read of another buffer)",
-                       "parallelism": f"dp{world} (independent batches per GPU)"},
+            "config": config_of(w, world),
             "tokens_per_s": tokens_s,
             "frac_of_bf16_peak": value / pk["bf16_tflops"],
+            "tf32_peak": tf32,
+            "frac_of_tf32_peak": (value / world / tf32["tf32_tflops"]) if tf32 else None,
             "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
-            "clocks": clocks.summary(), "gpu_launches": 4 * K * w.layers, "wall_s_timed": wall,
+            "clocks": clocks.summary(), "clock_window": window, "gpu_launches": 4 * K * w.layers,
+            "wall_s_timed": wall,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -157,8 +157,28 @@ int device_state(DeviceState** out) {
   return NEA_OK;
 }
 
-// Rotary table [T][D/2] of (cos, sin) of t * base^(-2i/D), angles computed
-// in double and rounded to float once.
+// Rotary table [T][D/2] of (cos, sin) of t * base^(-2i/D): angle, cosine and
+// sine in double precision, each rounded to float once.  Both the cached
+// tables of the regular entry points and the allocation-free backward's table
+// come from this kernel, so the two are bit-identical.
+__global__ void rope_table_kernel(float2* out, int T, int D, double base) {
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int half = D / 2;
+  if (idx >= (long long)T * half) return;
+  const int t = int(idx / half), i = int(idx % half);
+  const double a = double(t) * pow(base, -2.0 * double(i) / double(D));
+  double sn, cs;
+  sincos(a, &sn, &cs);
+  out[idx] = make_float2(float(cs), float(sn));
+}
+
+cudaError_t launch_rope_table(float2* out, int T, int D, float base, cudaStream_t stream) {
+  const long long n = (long long)T * (D / 2);
+  rope_table_kernel<<<unsigned((n + 255) / 256), 256, 0, stream>>>(out, T, D, double(base));
+  return cudaGetLastError();
+}
+
+// The cached table for (T, D, base), built on first use.
 int rope_table(DeviceState& st, int T, int D, float base, cudaStream_t stream, const float2** out) {
   if (!(base > 0.f)) {
     *out = nullptr;
@@ -172,17 +192,12 @@ int rope_table(DeviceState& st, int T, int D, float base, cudaStream_t stream, c
     *out = it->second;
     return NEA_OK;
   }
-  std::vector<float2> h(size_t(T) * (D / 2));
-  for (int t = 0; t < T; ++t)
-    for (int i = 0; i < D / 2; ++i) {
-      const double a = double(t) * std::pow(double(base), -2.0 * i / double(D));
-      h[size_t(t) * (D / 2) + i] = make_float2(float(std::cos(a)), float(std::sin(a)));
-    }
   float2* d = nullptr;
-  cudaError_t e = cudaMalloc(&d, h.size() * sizeof(float2));
+  cudaError_t e = cudaMalloc(&d, size_t(T) * (D / 2) * sizeof(float2));
   if (e != cudaSuccess) return cuda_fail(e);
-  e = cudaMemcpyAsync(d, h.data(), h.size() * sizeof(float2), cudaMemcpyHostToDevice, stream);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);  // host buffer dies below
+  e = launch_rope_table(d, T, D, base, stream);
+  // later calls may use the table from another stream: finish it now
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
   if (e != cudaSuccess) {
     cudaFree(d);
     return cuda_fail(e);
@@ -446,6 +461,8 @@ int run_bwd(uint32_t& attr_done, uint8_t* ws, const float2* rope, int* status, c
   p.scale_log2 = float(1.4426950408889634 / std::sqrt(double(D)));
   p.err = status;
   p.wait_limit = static_cast<unsigned long long>(t_wait_limit_ns);
+  p.debug = t_debug_flags & 2;  // bit 1 arms the next backward launch
+  t_debug_flags &= ~2;
 #ifdef NEA_TRACE
   p.trace = t_trace_bwd;
 #endif
@@ -510,8 +527,8 @@ int nea_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
   p.scale_log2 = float(1.4426950408889634 / std::sqrt(double(D)));
   p.err = st->err;
   p.wait_limit = static_cast<unsigned long long>(t_wait_limit_ns);
-  p.debug = t_debug_flags;
-  t_debug_flags = 0;
+  p.debug = t_debug_flags & 1;  // bit 0 arms the next forward launch
+  t_debug_flags &= ~1;
 #ifdef NEA_TRACE
   p.trace = t_trace;
 #endif
@@ -540,21 +557,6 @@ int nea_attn_bwd(const void* Q, const void* K, const void* V, const void* O, con
     return rc;
   return run_bwd(st->attr_done, st->ws, rope, st->err, Q, K, V, O, LSE, dO, dQ, dK, dV, B, T, Hq, Hkv, D, dtype,
                  causal, stream, true);
-}
-
-int nea_device_status(void* stream_) {
-  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-  cudaError_t e = cudaStreamSynchronize(stream);
-  if (e != cudaSuccess) return cuda_fail(e);
-  std::lock_guard<std::mutex> lock(g_mu);
-  DeviceState* st = nullptr;
-  int rc = device_state(&st);
-  if (rc) return rc;
-  int v = 0;
-  if ((e = cudaMemcpy(&v, st->err, sizeof v, cudaMemcpyDeviceToHost)) != cudaSuccess) return cuda_fail(e);
-  if (v != 0 && (e = cudaMemset(st->err, 0, sizeof(int))) != cudaSuccess) return cuda_fail(e);
-  if (v == nea::kErrBadLength) return NEA_ERR_ARG;
-  return v ? NEA_ERR_TIMEOUT : NEA_OK;
 }
 
 int nea_attn_decode(const void* Q, const void* Kc, const void* Vc, const int* lens, void* O, float* LSE, int B,
@@ -697,19 +699,6 @@ struct NoAllocDevice {
 NoAllocDevice g_noalloc_dev[kNoAllocMaxDevices];
 std::mutex g_noalloc_mu;
 
-// Rotary table [T][D/2] of (cos, sin) of t * base^(-2i/D), angles in double,
-// as in the regular table.
-__global__ void noalloc_rope_table_kernel(float2* out, int T, int D, double base) {
-  const long idx = long(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int half = D / 2;
-  if (idx >= long(T) * half) return;
-  const int t = int(idx / half), i = int(idx % half);
-  const double a = double(t) * pow(base, -2.0 * double(i) / double(D));
-  double sn, cs;
-  sincos(a, &sn, &cs);
-  out[idx] = make_float2(float(cs), float(sn));
-}
-
 }  // namespace
 
 extern "C" int nea_attn_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O, const float* LSE,
@@ -749,18 +738,59 @@ extern "C" int nea_attn_bwd_noalloc(const void* Q, const void* K, const void* V,
   }
   if (!st.sm100) return NEA_ERR_UNSUPPORTED;
 
-  // scratch: status word | row terms (+ fp32 operand planes) | rotary table
+  // scratch: status word | row terms (+ fp32 operand planes) | rotary table.
+  // The status word starts at zero (static storage) and is read and cleared
+  // by nea_device_status; the row terms, planes and table are rewritten in
+  // full by their kernels, so nothing else needs clearing.
   int* status = reinterpret_cast<int*>(st.scratch);
   uint8_t* ws = st.scratch + kNoAllocStatusBytes;
   float2* rope = rope_bytes ? reinterpret_cast<float2*>(ws + ws_bytes) : nullptr;
-  // the status word must start at zero; the row terms, planes and table are
-  // fully rewritten by their kernels, so they need no clearing
-  if ((e = cudaMemsetAsync(status, 0, sizeof(int), stream)) != cudaSuccess) return cuda_fail(e);
-  if (rope) {
-    const long n = long(T) * (D / 2);
-    noalloc_rope_table_kernel<<<unsigned((n + 255) / 256), 256, 0, stream>>>(rope, T, D, double(rope_base));
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
-  }
+  if (rope && (e = launch_rope_table(rope, T, D, rope_base, stream)) != cudaSuccess) return cuda_fail(e);
   return run_bwd(st.attr_done, ws, rope, status, Q, K, V, O, LSE, dO, dQ, dK, dV, B, T, Hq, Hkv, D, dtype, causal,
                  stream, false);
+}
+
+// ===================================================================== device status
+namespace {
+
+// Reads and clears one device status word (a synchronous copy and a memset;
+// neither allocates).  Returns the CUDA error, or success with *v set.
+cudaError_t take_status(int* word, int* v) {
+  int x = 0;
+  cudaError_t e = cudaMemcpy(&x, word, sizeof x, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && x != 0) e = cudaMemset(word, 0, sizeof(int));
+  *v = x;
+  return e;
+}
+
+}  // namespace
+
+// Reads the status words of the current device -- the regular entry points'
+// and the allocation-free backward's -- without setting either up, so that a
+// caller of nea_attn_bwd_noalloc alone never causes an allocation here.
+extern "C" int nea_device_status(void* stream_) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  int dev = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return cuda_fail(e);
+  int v = 0;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    auto it = g_dev.find(dev);
+    if (it != g_dev.end() && it->second.probed && it->second.err) {
+      if ((e = take_status(it->second.err, &v)) != cudaSuccess) return cuda_fail(e);
+    }
+  }
+  if (dev >= 0 && dev < kNoAllocMaxDevices) {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    const NoAllocDevice& na = g_noalloc_dev[dev];
+    int w = 0;
+    if (na.ready && na.scratch) {
+      if ((e = take_status(reinterpret_cast<int*>(na.scratch), &w)) != cudaSuccess) return cuda_fail(e);
+    }
+    if (v == 0) v = w;
+  }
+  if (v == nea::kErrBadLength) return NEA_ERR_ARG;
+  return v ? NEA_ERR_TIMEOUT : NEA_OK;
 }

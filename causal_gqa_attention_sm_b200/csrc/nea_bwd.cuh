@@ -76,6 +76,7 @@ struct BwdParams {
   unsigned long long wait_limit;
   int n_dkdv;                 // units [0, n_dkdv) are dK/dV units, the rest dQ units
   int unit0;                  // unit of blockIdx.x == 0
+  int debug;                  // bit 1: withhold the resident tiles (fault-injection hook)
   unsigned long long* trace;  // per-CTA phase stamps (NEA_TRACE builds only)
 };
 
@@ -223,9 +224,14 @@ __device__ __forceinline__ void attn_bwd_unit(const BwdParams& p, int bid) {
         tma_load_4d(dst, hi, 0, head, row0, b, bar);
         if (F32IO) tma_load_4d(dst + OPB, lo, 0, head, row0, b, bar);
       };
-      mbar_arrive_expect_tx(bar_rtma, 2 * L::kTile);
-      load_tile(smem + L::kR1, m_r1, m_r1l, head_r, rt * kTileRows, bar_rtma);
-      load_tile(smem + L::kR2, m_r2, m_r2l, head_r, rt * kTileRows, bar_rtma);
+      // fault-injection hook: withhold the resident tiles so every wait on
+      // them runs into its limit
+      const bool r_armed = !(p.debug & 2);
+      if (r_armed) {
+        mbar_arrive_expect_tx(bar_rtma, 2 * L::kTile);
+        load_tile(smem + L::kR1, m_r1, m_r1l, head_r, rt * kTileRows, bar_rtma);
+        load_tile(smem + L::kR2, m_r2, m_r2l, head_r, rt * kTileRows, bar_rtma);
+      }
       int armed = 0;
       for (int k = 0; k < n_items; ++k) {
         const int s = k % NS;
@@ -241,7 +247,7 @@ __device__ __forceinline__ void attn_bwd_unit(const BwdParams& p, int bid) {
       }
       if (*abort_flag) {
         for (int k = max(0, armed - NS); k < armed; ++k) drain_wait(&bar_tma[k % NS], (k / NS) & 1, wc);
-        drain_wait(bar_rtma, 0, wc);
+        if (r_armed) drain_wait(bar_rtma, 0, wc);
       }
     }
     __syncwarp();

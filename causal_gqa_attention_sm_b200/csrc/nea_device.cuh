@@ -465,7 +465,8 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
 // 1.5 * 2^23 rounds to it), 2^f from the degree-3 polynomial that
 // exp2_poly_fit.py derives (relative error below 7.5e-5 for f in
 // [-1/2, 1/2]), and 2^j added to the exponent field.  Inputs below -125
-// (-inf included) are clamped: their result is 2^-125 (about 2.4e-38).
+// (-inf included) give 0, as the exponential unit's flush-to-zero form does;
+// a NaN input gives NaN.
 __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
   float x0, x1;
   f2_unpack(x, x0, x1);
@@ -482,8 +483,10 @@ __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
   f2_unpack(p, p0, p1);
   // the low bits of y hold j; shifted into the exponent field (the bits of
   // 1.5 * 2^23 shift out of the word)
-  return f2_pack(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(y0) << 23)),
-                 __uint_as_float(__float_as_uint(p1) + (__float_as_uint(y1) << 23)));
+  const float r0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(y0) << 23));
+  const float r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(y1) << 23));
+  // below the clamp: 0; NaN (every comparison false): the input itself
+  return f2_pack(x0 >= -125.f ? r0 : (x0 < -125.f ? 0.f : x0), x1 >= -125.f ? r1 : (x1 < -125.f ? 0.f : x1));
 }
 
 // Maximum of three floats in one instruction (sm_100).

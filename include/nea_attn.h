@@ -116,11 +116,14 @@ int nea_attn_bwd(const void* Q, const void* K, const void* V, const void* O, con
                  int causal, void* stream);
 
 /*
- * Synchronises `stream`, then reads and clears the device error word of the
- * current device.  Returns NEA_OK, NEA_ERR_TIMEOUT when a kernel since the
- * last call abandoned a bounded wait (its outputs are then undefined),
- * NEA_ERR_ARG when a decode call met a cache length outside [0, Tc], or
- * NEA_ERR_CUDA when the synchronisation itself failed.
+ * Synchronises `stream`, then reads and clears the device status words of the
+ * current device: the one the regular entry points write and the one inside
+ * the fixed scratch of nea_attn_bwd_noalloc.  Returns NEA_OK, NEA_ERR_TIMEOUT
+ * when a kernel since the last call abandoned a bounded wait (its outputs
+ * are then undefined), NEA_ERR_ARG when a decode call met a cache length
+ * outside [0, Tc], or NEA_ERR_CUDA when the synchronisation or the read
+ * failed.  It sets up neither word (a word that was never set up reads as
+ * clear), so it never allocates device memory.
  */
 int nea_device_status(void* stream);
 
@@ -132,10 +135,15 @@ int nea_device_status(void* stream);
 long long nea_set_wait_limit_ns(long long ns);
 
 /*
- * Fault-injection hook for tests: when `flags` & 1, the next forward launch
- * on this host thread withholds the query-tile arrival its MMA issuer waits
- * for, so every dependent wait runs into its limit and the kernel returns
- * with NEA_ERR_TIMEOUT pending.  Cleared after one launch.
+ * Fault-injection hook for tests, for later launches on this host thread:
+ *   flags & 1: the next forward launch withholds the query-tile arrival its
+ *              MMA issuers wait for;
+ *   flags & 2: the next backward launch (nea_attn_bwd or
+ *              nea_attn_bwd_noalloc) withholds the resident-tile arrival of
+ *              its gradient kernel.
+ * Every dependent wait then runs into its limit, the kernel returns, and
+ * NEA_ERR_TIMEOUT is pending for nea_device_status().  Each bit is cleared
+ * by the launch it arms.
  */
 void nea_debug_inject(int flags);
 
@@ -165,27 +173,28 @@ void nea_set_profile_events(void* const* events, int n);
  *
  * Same arguments, layouts and results as nea_attn_bwd.  The caller passes all
  * inputs and outputs; everything else the backward needs (the per-row terms
- * -LSE*log2(e) and D_i = sum_d dO_id O_id, the rotary cos/sin table, computed
- * on the device in double precision, a device status word and the operand
- * prologue's output: for NEA_F32 the bf16 hi/lo planes of Q, K, V, dO, for
- * NEA_BF16 with the rotation on the rotated copies of Q and K) lives in one
- * fixed array of 4 MiB compiled into the library: every GPU that loads the
- * library keeps it until the process exits.  With Tp = 128*ceil(T/128), a
- * call needs about 256 + 8*B*Hq*Tp bytes of it, plus 4*T*D bytes with the
- * rotation on, plus 8*B*T*(Hq + Hkv)*D bytes for NEA_F32 or, with the
- * rotation on, 2*B*T*(Hq + Hkv)*D bytes for NEA_BF16 (each part rounded up to
- * 256 bytes); larger problems return NEA_ERR_SCRATCH_LIMIT before anything
- * is launched.
+ * -LSE*log2(e) and D_i = sum_d dO_id O_id, the rotary cos/sin table -- built
+ * by the same device kernel as the regular entry points' table, so the two
+ * are bit-identical -- a device status word and the operand prologue's
+ * output: for NEA_F32 the bf16 hi/lo planes of Q, K, V, dO, for NEA_BF16 with
+ * the rotation on the rotated copies of Q and K) lives in one fixed array of
+ * 4 MiB compiled into the library: every GPU that loads the library keeps it
+ * until the process exits.  With Tp = 128*ceil(T/128), a call needs about
+ * 256 + 8*B*Hq*Tp bytes of it, plus 4*T*D bytes with the rotation on, plus
+ * 8*B*T*(Hq + Hkv)*D bytes for NEA_F32 or, with the rotation on,
+ * 2*B*T*(Hq + Hkv)*D bytes for NEA_BF16 (each part rounded up to 256
+ * bytes); larger problems return NEA_ERR_SCRATCH_LIMIT before anything is
+ * launched.
  *
  * The first call on a device does a one-time set-up with that device
  * current (it looks up the array's device address and sets kernel
  * attributes); make that first call before any stream capture.  All calls
  * share the one array and it keeps the last call's contents, so calls whose
  * work may overlap on the GPU (different streams without ordering, or
- * several host threads) race and must be serialised by the caller.  Each
- * call clears the status word it uses; a device-side wait that runs into its
- * limit is recorded only there (outputs are then undefined) and is not
- * reported by nea_device_status.
+ * several host threads) race and must be serialised by the caller.  A
+ * device-side wait that runs into its limit sets the array's status word
+ * (outputs are then undefined); nea_device_status() reports it as
+ * NEA_ERR_TIMEOUT and clears it, allocating nothing.
  */
 int nea_attn_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O, const float* LSE,
                          const void* dO, void* dQ, void* dK, void* dV, int B, int T, int Hq, int Hkv, int D,

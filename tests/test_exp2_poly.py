@@ -34,10 +34,11 @@ def test_coefficients_match_the_fit():
 def _replay(x):
     """The device steps in float32: clamp, round to the nearest integer with
     the 1.5 * 2^23 trick, polynomial on the remainder, integer add of j << 23
-    to the polynomial's bits."""
+    to the polynomial's bits; then 0 below the clamp and NaN through."""
     c0, c1, c2, c3 = _coefficients_in_source()
     f32 = np.float32
-    x = np.maximum(x.astype(f32), f32(-125.0))
+    x_in = x.astype(f32)
+    x = np.maximum(x_in, f32(-125.0))
     magic = f32(12582912.0)
     y = (x + magic).astype(f32)
     f = (x - (y - magic).astype(f32)).astype(f32)
@@ -45,7 +46,9 @@ def _replay(x):
     p = (p * f + c1).astype(f32)
     p = (p * f + c0).astype(f32)
     bits = (p.view(np.uint32).astype(np.uint64) + (y.view(np.uint32).astype(np.uint64) << 23)) & 0xFFFFFFFF
-    return bits.astype(np.uint32).view(np.float32)
+    r = bits.astype(np.uint32).view(np.float32)
+    with np.errstate(invalid="ignore"):
+        return np.where(x_in >= f32(-125.0), r, np.where(x_in < f32(-125.0), f32(0.0), x_in))
 
 
 def test_replayed_algorithm_relative_error():
@@ -57,7 +60,10 @@ def test_replayed_algorithm_relative_error():
     assert rel.max() < 8e-5, rel.max()
 
 
-def test_clamped_inputs_give_a_negligible_positive_value():
-    x = np.array([-np.inf, -1e30, -200.0, -126.0], dtype=np.float32)
-    got = _replay(x).astype(np.float64)
-    assert np.all(got > 0) and np.all(np.abs(got / 2.0 ** -125 - 1) < 8e-5)
+def test_below_the_range_gives_zero_and_nan_passes_through():
+    """Masked scores (-inf) must contribute exactly nothing, like the
+    exponential unit's flush-to-zero 2^x, and a NaN score must stay NaN."""
+    x = np.array([-np.inf, -1e30, -200.0, -126.0, np.nan], dtype=np.float32)
+    got = _replay(x)
+    assert np.all(got[:4] == 0.0)
+    assert np.isnan(got[4])

@@ -270,3 +270,22 @@ def test_repeated_calls_are_deterministic(cuda_lib):
     b = run_gpu(cuda_lib, w, inp)
     for n in a:
         assert np.array_equal(a[n], b[n]), n
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_nan_key_reaches_every_later_output_row(cuda_lib, dtype):
+    """A NaN in one key makes every output row that sees that key NaN and
+    leaves earlier rows finite.  Key 7 sits in a column pair whose bf16
+    exponentials are taken by the polynomial on the FMA pipe, so this also
+    checks that the polynomial lets NaN through."""
+    import torch
+
+    w = custom("nan_key", B=1, T=160, Hq=2, Hkv=1, D=64, dtype=dtype, seed=5)
+    inp = {n: t.cuda() for n, t in make_inputs(w).items()}
+    inp["k"][0, 7, 0, 3] = float("nan")
+    o, lse = cuda_lib.nea_attn_fwd(inp["q"], inp["k"], inp["v"], w.rope_base, True)
+    torch.cuda.synchronize()
+    assert cuda_lib.nea_device_status() == cuda_lib.NEA_OK
+    o = o.float().cpu()
+    assert torch.isfinite(o[0, :7]).all()
+    assert torch.isnan(o[0, 7:]).all()
