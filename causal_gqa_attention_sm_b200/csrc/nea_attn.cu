@@ -19,6 +19,7 @@
 
 #include "nea_attn.h"
 #include "nea_bwd.cuh"
+#include "nea_bwd_f32.cuh"
 #include "nea_decode.cuh"
 #include "nea_fwd.cuh"
 #include "nea_prep.cuh"
@@ -362,11 +363,13 @@ int launch_fwd(uint32_t& attr_done, const nea::FwdParams& p, cudaStream_t stream
 // ----------------------------------------------------------------- backward
 // The gradient kernel (dK/dV and dQ units in one launch).  `ev` selects profiling events (the
 // regular backward records them, the allocation-free one does not).
+// Float32 storage runs the split-bf16 gradient kernel (nea_bwd_f32.cuh),
+// bfloat16 storage the bf16 one (nea_bwd.cuh).
 template <int D, bool F32IO>
 int launch_bwd(uint32_t& attr_done, const nea::BwdParams& p, cudaStream_t stream, bool ev) {
   cudaError_t e;
-  using L = nea::BwdSmem<D, F32IO>;
-  auto kern = nea::attn_bwd_kernel<D, F32IO>;
+  using L = std::conditional_t<F32IO, nea::Bwd32Smem<D>, nea::BwdSmem<D, false>>;
+  auto kern = F32IO ? nea::attn_bwd_f32_kernel<D> : nea::attn_bwd_kernel<D, false>;
   int rc = set_smem(attr_done, 4 + (D == 64) * 2 + F32IO, kern, L::kAlloc);
   if (rc) return rc;
   e = launch_dependent(kern, unsigned(p.n_dkdv + p.B * p.Hq * p.n_tiles), L::kThreads, L::kAlloc, stream, p);

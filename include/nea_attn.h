@@ -51,7 +51,7 @@ extern "C" {
 
 /* Element type of Q, K, V, O, dO, dQ, dK, dV. */
 typedef enum {
-  NEA_F32 = 0,  /* float32 storage; contractions in split bf16 (see below) */
+  NEA_F32 = 0,  /* float32 storage; every contraction in split bf16 (see below) */
   NEA_BF16 = 1  /* bfloat16 storage; bf16 tensor-core operands, fp32 accumulation */
 } nea_dtype;
 
@@ -107,9 +107,11 @@ int nea_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
  * of the group) and dQ units (one per query tile and head); both recompute P
  * from LSE.
  *
- * NEA_F32: the score product and dO V^T use split bf16 (as in the forward);
- * the three gradient products use the bf16 high parts with fp32
- * accumulation.
+ * NEA_F32: all five products (S, dP = dO V^T, dV, dK, dQ) use split bf16 as
+ * in the forward -- each operand as bf16 high and low parts, each product as
+ * hi*hi + hi*lo + lo*hi with fp32 accumulation (about 2^-16 relative per
+ * product, finer than TF32); P and dS are split by the kernel before their
+ * products.
  */
 int nea_attn_bwd(const void* Q, const void* K, const void* V, const void* O, const float* LSE, const void* dO,
                  void* dQ, void* dK, void* dV, int B, int T, int Hq, int Hkv, int D, int dtype, float rope_base,
