@@ -101,7 +101,12 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--clocks-csv", default=None, help="keep the raw nvidia-smi clock samples in this file")
+    ap.add_argument("--profile", action="store_true",
+                    help="for runs under ncu: only warm-up, timed and per-kernel steps (no CPU baseline, no e2e, "
+                         "no TF32 peak, no clock window); its numbers are not bench values")
     a = ap.parse_args()
+    if a.profile:
+        a.no_cpu_baseline = a.no_e2e = True
     a.warmup = max(a.warmup, 3)
     return a
 
@@ -423,8 +428,8 @@ def decode_main(a, w, rank, world, local):
     clocks = ClockSampler(local, a.clocks_csv)
     barrier(world)
     with clocks:
-        window = clock_window(step, lambda i: (flush.fill_(float(i)), torch.sum(drain, dim=0, out=drain_sum)),
-                              stream, dev, 1.2)
+        window = None if a.profile else clock_window(
+            step, lambda i: (flush.fill_(float(i)), torch.sum(drain, dim=0, out=drain_sum)), stream, dev, 1.2)
         for i in range(K):
             flush.fill_(float(i))
             torch.sum(drain, dim=0, out=drain_sum)
@@ -587,7 +592,7 @@ def main():
         # block of identical steps of at least 1.2 s runs under it first, so
         # that the clock record spans kernel execution (reported apart as
         # `clock_window`; the value comes from the K steps after it only)
-        window = clock_window(step, flush_l2, stream, dev, 1.2)
+        window = None if a.profile else clock_window(step, flush_l2, stream, dev, 1.2)
         wall0 = time.perf_counter()
         for i in range(K):
             flush_l2(i)
@@ -632,7 +637,7 @@ def main():
     dominant = max(kern_ms, key=kern_ms.get)
     per_launch_ms = kern_ms[dominant] / launches_per_kernel
     unit_flops = w.B * w.Hq * w.T * w.T * w.D * (1.0 if w.causal else 2.0)
-    tf32 = measure_tf32_peak(dev) if w.dtype == "f32" else None
+    tf32 = measure_tf32_peak(dev) if (w.dtype == "f32" and not a.profile) else None
     if dominant in UNITS:
         achieved = UNITS[dominant] * unit_flops / (per_launch_ms * 1e-3) / 1e12
         if tf32:

@@ -56,6 +56,7 @@ struct DeviceState {
   std::map<std::tuple<int, int, uint32_t>, float2*> rope;
   uint32_t attr_done = 0;      // bitmask of kernels whose smem attribute is set
   uint64_t attr_dec = 0;       // the same for the decode split kernels
+  int n_sm = 148;              // streaming multiprocessors
 };
 
 std::mutex g_mu;
@@ -147,6 +148,8 @@ int device_state(DeviceState** out) {
         (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
       return cuda_fail(e);
     st.sm100 = (major == 10 && minor == 0);
+    if ((e = cudaDeviceGetAttribute(&st.n_sm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(e);
     if (st.sm100) {
       if ((e = cudaMalloc(&st.err, sizeof(int))) != cudaSuccess) return cuda_fail(e);
       if ((e = cudaMemset(st.err, 0, sizeof(int))) != cudaSuccess) return cuda_fail(e);

@@ -100,7 +100,7 @@ struct BwdSmem {
   static_assert(kAlloc <= 232448, "shared memory");
 };
 
-// N consecutive TMEM columns of this thread's lane (N = 16, 32 or 64).
+// N consecutive TMEM columns of this thread's lane (N = 8, 16, 32 or 64).
 template <int N>
 __device__ __forceinline__ void tmem_ld_n(uint32_t taddr, float* v) {
   if constexpr (N == 64) {
@@ -113,11 +113,17 @@ __device__ __forceinline__ void tmem_ld_n(uint32_t taddr, float* v) {
     tmem_ld32(taddr, r);
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-  } else {
+  } else if constexpr (N == 16) {
     uint32_t r[16];
     tmem_ld16(taddr, r);
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+  } else {
+    static_assert(N == 8, "8, 16, 32 or 64 columns");
+    uint32_t r[8];
+    tmem_ld8(taddr, r);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
   }
 }
 

@@ -22,26 +22,28 @@
 // dQ unit keeps query tile i of head h resident (Q'_i, dO_i) and streams the
 // key tiles j <= i.
 //
-// Gradient products.  The hi and lo planes of a streamed tile sit side by side
-// in shared memory, so one MN-major B operand of N = 2D spans [C_hi | C_lo]:
-//   [X | Y] += A_hi [C_hi | C_lo]   (one N = 2D product, full tensor rate)
-//        Y  += A_lo  C_hi            (N = D)
-// and the gradient is X + Y, summed in the epilogue.
+// Gradient products: three bf16 products of N = D per 16-row step
+// (A_hi C_hi, A_hi C_lo, A_lo C_hi) into one accumulator of D columns.
 //
-// TMEM (D = 64): S [0,128) -- P_hi / P_lo written over it; dP [128,256) --
-// dS_hi / dS_lo over it; accumulator A [256, 256+2D) (dV or dQ, as [X | Y]),
-// accumulator B [256+2D, 256+4D) (dK).  Warp half h rewrites only its own
-// columns [64h, 64h+64) of S and dP: hi parts in the first 32, lo parts in
-// the next 32 (two bf16 per column), so no warp overwrites scores another
-// still has to read.
+// TMEM (D = 64): S in two buffers [0,128) and [128,256) (item k uses buffer
+// k % 2; P_hi / P_lo are written over it); dP [256,384) (dS_hi / dS_lo
+// over it); accumulator A [384, 384+D) (dV or dQ), accumulator B
+// [384+D, 384+2D) (dK).  Column quarter q of the elementwise warps rewrites
+// only its own columns [32q, 32q+32) of S and dP: hi parts in the first 16,
+// lo parts in the next 16 (two bf16 per column), so no warp overwrites
+// scores another still has to read.
 // Issue order of the MMA thread, per item k (the streamed tiles one stage
-// ahead):   dP(k) | dV(k) | dK(k) or dQ(k) | S(k+1) | dP(k+1) | ...
-// dV(k) waits for P(k), dK/dQ(k) for dS(k) (the rows form it while dV(k)
-// runs), S(k+1) for dV(k) to have read P(k), dP(k+1) for dK/dQ(k) to have
-// read dS(k) -- each of these last two waits overlaps the product issued
-// just before it.
-// Warps: 0-7 elementwise (warp w: TMEM lanes 32 (w % 4) .. + 31, columns
-// 64 (w / 4) .. + 63 of each 128-column tile), 8 MMA issue, 9 TMA.
+// ahead):
+//   dK/dV units:  dV(k) | S(k+1) | dK(k) | dP(k+1) | dV(k+1) | S(k+2) | ...
+//   dQ units:     S(k+1) | dQ(k) | dP(k+1) | S(k+2) | ...
+// S(k+1) goes to the other S buffer as soon as its tiles have landed, so the
+// rows form P(k+1) while dK/dQ(k) and dP(k+1) run; dV(k) waits for P(k),
+// dK/dQ(k) for dS(k) (formed while dV(k) and S(k+1) run), dP(k+1) for
+// dK/dQ(k) to have read dS(k) (the wait overlaps S(k+1) or dK(k)).
+// Warps: 0-15 elementwise (warp w: TMEM lanes 32 (w % 4) .. + 31, columns
+// 32 (w / 4) .. + 31 of each 128-column tile; four warps per SM
+// sub-partition, so that one warp's TMEM loads overlap the others' work),
+// 16 MMA issue, 17 TMA.
 #pragma once
 
 #include <cuda.h>
@@ -61,12 +63,14 @@ struct Bwd32Smem {
   static constexpr uint32_t kColVec = 2 * kTile;  // per-column -LSE*log2e and Dv (dK/dV units)
   static constexpr uint32_t kStageBytes = kColVec + 1024;
   static constexpr uint32_t kBars = kStage0 + kStages * kStageBytes;
-  // rtma, tma[S], empty[S], s, dp, p, ds, pv, dk, fin
+  // rtma, tma[S], empty[S], s[2], dp, p, ds, dk, fin
   static constexpr int kNumBars = 1 + 2 * kStages + 7;
   static constexpr uint32_t kMisc = kBars + 8 * kNumBars;
   static constexpr uint32_t kUsed = kMisc + 16;
   static constexpr uint32_t kAlloc = kUsed + 1024 > 116u * 1024u ? kUsed + 1024 : 116u * 1024u;
-  static constexpr int kThreads = 320;
+  static constexpr int kRowWarps = 16;  // elementwise warps
+  static constexpr int kRowThreads = 32 * kRowWarps;
+  static constexpr int kThreads = kRowThreads + 64;
   static_assert(kStage0 % 1024 == 0 && kStageBytes % 1024 == 0, "operand tiles need 1024-byte alignment");
   static_assert(kAlloc <= 232448, "shared memory");
 };
@@ -84,11 +88,10 @@ __device__ __forceinline__ void attn_bwd_f32_unit(const BwdParams& p, int bid) {
   uint64_t* bar_rtma = bars + 0;        // resident tiles landed
   uint64_t* bar_tma = bars + 1;         // [NS] streamed tiles landed
   uint64_t* bar_empty = bars + 1 + NS;  // [NS] products done with the stage
-  uint64_t* bar_s = bars + 1 + 2 * NS;  // S landed
-  uint64_t* bar_dp = bar_s + 1;         // dP landed
-  uint64_t* bar_p = bar_s + 2;          // rows wrote P over S (count 256; dK/dV units)
-  uint64_t* bar_ds = bar_s + 3;         // rows wrote dS over dP (count 256)
-  uint64_t* bar_pv = bar_s + 4;         // dV product of an item done
+  uint64_t* bar_s = bars + 1 + 2 * NS;  // [2] S landed in buffer 0 / 1
+  uint64_t* bar_dp = bar_s + 2;         // dP landed
+  uint64_t* bar_p = bar_s + 3;          // rows wrote P over S (all row threads; dK/dV units)
+  uint64_t* bar_ds = bar_s + 4;         // rows wrote dS over dP (all row threads)
   uint64_t* bar_dk = bar_s + 5;         // all products of an item done
   uint64_t* bar_fin = bar_s + 6;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
@@ -97,6 +100,7 @@ __device__ __forceinline__ void attn_bwd_f32_unit(const BwdParams& p, int bid) {
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const WaitCtl wc{p.err, p.wait_limit, abort_flag};
+  NEA_TRACE_STAMP(p, 0, tid == 0);
 
   // ---- work decomposition (as in the bf16 kernel)
   int b, rt, head_r, n_items, c0;
@@ -128,11 +132,11 @@ __device__ __forceinline__ void attn_bwd_f32_unit(const BwdParams& p, int bid) {
       mbar_init(&bar_tma[s], 1);
       mbar_init(&bar_empty[s], 1);
     }
-    mbar_init(bar_s, 1);
+    mbar_init(&bar_s[0], 1);
+    mbar_init(&bar_s[1], 1);
     mbar_init(bar_dp, 1);
-    mbar_init(bar_p, 256);
-    mbar_init(bar_ds, 256);
-    mbar_init(bar_pv, 1);
+    mbar_init(bar_p, L::kRowThreads);
+    mbar_init(bar_ds, L::kRowThreads);
     mbar_init(bar_dk, 1);
     mbar_init(bar_fin, 1);
     mbar_init_fence();
@@ -144,9 +148,11 @@ __device__ __forceinline__ void attn_bwd_f32_unit(const BwdParams& p, int bid) {
   const uint32_t tbase = *tmem_holder;
   grid_dep_wait();  // operand planes and row terms come from the prologue grid
   grid_dep_launch();
-  constexpr uint32_t kColS = 0, kColDP = 128, kColAccA = 256, kColAccB = 256 + 2 * D;
+  NEA_TRACE_STAMP(p, 1, tid == 0);
+  constexpr uint32_t kColS = 0, kColDP = 256, kColAccA = 384, kColAccB = 384 + D;
 
-  if (warp == 9) {
+  constexpr int kWarpMma = L::kRowWarps, kWarpTma = L::kRowWarps + 1;
+  if (warp == kWarpTma) {
     // ------------------------------------------------------------ TMA
     if ((tid & 31) == 0) {
       const CUtensorMap* m_r1 = DKDV ? &p.tm_k : &p.tm_q;
@@ -174,6 +180,7 @@ __device__ __forceinline__ void attn_bwd_f32_unit(const BwdParams& p, int bid) {
         load_tile(smem + L::kR1, m_r1, m_r1l, head_r, rt * kTileRows, bar_rtma);
         load_tile(smem + L::kR2, m_r2, m_r2l, head_r, rt * kTileRows, bar_rtma);
       }
+      NEA_TRACE_STAMP(p, 73, true);
       int armed = 0;
       for (int k = 0; k < n_items; ++k) {
         const int s = k % NS;
@@ -193,12 +200,11 @@ __device__ __forceinline__ void attn_bwd_f32_unit(const BwdParams& p, int bid) {
       }
     }
     __syncwarp();
-  } else if (warp == 8) {
+  } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if ((tid & 31) == 0) {
       constexpr uint32_t idSS = idesc_bf16(128, 128, 0, 0);
-      constexpr uint32_t idG2 = idesc_bf16(128, 2 * D, 0, 1);  // A_hi [C_hi | C_lo]
-      constexpr uint32_t idG1 = idesc_bf16(128, D, 0, 1);      // A_lo C_hi
+      constexpr uint32_t idG = idesc_bf16(128, D, 0, 1);
       const uint32_t sR1 = smem_u32(smem + L::kR1), sR2 = smem_u32(smem + L::kR2);
       auto stage_c1 = [&](int k) { return smem_u32(smem + L::kStage0 + (k % NS) * L::kStageBytes); };
       // dst (+)= R C^T from the three split products, contraction over D
@@ -210,57 +216,66 @@ __device__ __forceinline__ void attn_bwd_f32_unit(const BwdParams& p, int bid) {
             mma_ss(tbase + dst, smem_desc(sR + (term == 2 ? OPB : 0) + kk * 32, RB, 16),
                    smem_desc(sC + (term == 1 ? OPB : 0) + kk * 32, RB, 16), idSS, (kk | term) != 0);
       };
-      // [X | Y] (+)= A_hi [C_hi | C_lo],  Y += A_lo C_hi; contraction over the
-      // 128 rows of the streamed tile.  A (P or dS) sits at a_col: warp half h
-      // wrote its 64 columns' hi parts at a_col + 64 h and lo parts 32 after.
+      auto issue_s = [&](int k) {
+        issue_sc(kColS + 128 * (k & 1), sR1, stage_c1(k));
+        tc_commit(&bar_s[k & 1]);
+      };
+      auto issue_dp = [&](int k) {
+        issue_sc(kColDP, sR2, stage_c1(k) + L::kTile);
+        tc_commit(bar_dp);
+      };
+      // acc (+)= A C, contraction over the 128 rows of the streamed tile, as
+      // A_hi C_hi + A_hi C_lo + A_lo C_hi.  A (P or dS) sits at a_col: column
+      // quarter q wrote its 32 columns' hi parts at a_col + 32 q and lo parts
+      // 16 after; K-step kk (16 columns) is half kk % 2 of quarter kk / 2.
       auto issue_grad = [&](uint32_t acc, uint32_t a_col, uint32_t sC, bool first) {
 #pragma unroll
         for (int kk = 0; kk < kTileRows / 16; ++kk) {
-          const uint32_t a_hi = tbase + a_col + 64 * (kk >> 2) + 8 * (kk & 3);
-          const uint64_t bd = smem_desc(sC + kk * 16 * RB, RB, OPB);
-          mma_ts(tbase + acc, a_hi, bd, idG2, (first && kk == 0) ? 0u : 1u);
-          mma_ts(tbase + acc + D, a_hi + 32, bd, idG1, 1u);
+          const uint32_t a_hi = tbase + a_col + 32 * (kk >> 1) + 8 * (kk & 1);
+          const uint32_t c = sC + kk * 16 * RB;
+          mma_ts(tbase + acc, a_hi, smem_desc(c, RB, OPB), idG, (first && kk == 0) ? 0u : 1u);
+          mma_ts(tbase + acc, a_hi, smem_desc(c + OPB, RB, OPB), idG, 1u);
+          mma_ts(tbase + acc, a_hi + 16, smem_desc(c, RB, OPB), idG, 1u);
         }
       };
       bool ok = wait_thread(bar_rtma, 0, wc, kErrWaitProducer) &&
                 (n_items == 0 || wait_thread(&bar_tma[0], 0, wc, kErrWaitProducer));
       if (ok && n_items > 0) {
+        NEA_TRACE_STAMP(p, 72, true);
         tc_fence_after();
-        issue_sc(kColS, sR1, stage_c1(0));
-        tc_commit(bar_s);
-        issue_sc(kColDP, sR2, stage_c1(0) + L::kTile);
-        tc_commit(bar_dp);
+        issue_s(0);
+        issue_dp(0);
       }
       for (int k = 0; ok && k < n_items; ++k) {
         const uint32_t sC1 = stage_c1(k), sC2 = sC1 + L::kTile;
         if (DKDV) {  // dV += P(k) C2(k), once the rows have written P(k) over S(k)
           if (!wait_thread(bar_p, k & 1, wc, kErrWaitSoftmax)) { ok = false; break; }
+          NEA_TRACE_STAMP(p, 8 + min(k, 7), true);
           tc_fence_after();
-          issue_grad(kColAccA, kColS, sC2, k == 0);
-          tc_commit(bar_pv);
+          issue_grad(kColAccA, kColS + 128 * (k & 1), sC2, k == 0);
+        }
+        if (k + 1 < n_items) {
+          // S(k+1) into the other buffer: its P(k-1) (or, in dQ units, S(k-1))
+          // was consumed before item k-1's products completed, waited for
+          // before dP(k)
+          if (!wait_thread(&bar_tma[(k + 1) % NS], ((k + 1) / NS) & 1, wc, kErrWaitProducer)) { ok = false; break; }
+          NEA_TRACE_STAMP(p, 24 + min(k, 7), true);
+          tc_fence_after();
+          issue_s(k + 1);
         }
         // dK (dK/dV units) or dQ (dQ units) += dS(k) C1(k), then release the stage
         if (!wait_thread(bar_ds, k & 1, wc, kErrWaitSoftmax)) { ok = false; break; }
+        NEA_TRACE_STAMP(p, 16 + min(k, 7), true);
         tc_fence_after();
         issue_grad(DKDV ? kColAccB : kColAccA, kColDP, sC1, k == 0);
         tc_commit(&bar_empty[k % NS]);
         tc_commit(bar_dk);
         if (k + 1 < n_items) {
-          // S(k+1) overwrites P(k): dV(k) must have read it (dQ units: the
-          // rows read S(k) before they wrote dS(k))
-          if (!wait_thread(&bar_tma[(k + 1) % NS], ((k + 1) / NS) & 1, wc, kErrWaitProducer) ||
-              (DKDV && !wait_thread(bar_pv, k & 1, wc, kErrWaitMma))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          issue_sc(kColS, sR1, stage_c1(k + 1));
-          tc_commit(bar_s);
-          // dP(k+1) overwrites dS(k): wait for item k's last product
+          // dP(k+1) overwrites dS(k): wait for item k's products
           if (!wait_thread(bar_dk, k & 1, wc, kErrWaitMma)) { ok = false; break; }
+          NEA_TRACE_STAMP(p, 32 + min(k, 7), true);
           tc_fence_after();
-          issue_sc(kColDP, sR2, stage_c1(k + 1) + L::kTile);
-          tc_commit(bar_dp);
+          issue_dp(k + 1);
         }
       }
       tc_commit(bar_fin);
@@ -268,11 +283,11 @@ __device__ __forceinline__ void attn_bwd_f32_unit(const BwdParams& p, int bid) {
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ elementwise (warps 0-7)
-    const int hf = warp >> 2;            // column half
+    // ------------------------------------------------------------ elementwise (warps 0-15)
+    const int q = warp >> 2;             // column quarter
     const int r = (warp & 3) * 32 + (tid & 31);
     const int row = rt * kTileRows + r;  // key position (dK/dV) or query position (dQ)
-    const int cb = 64 * hf;              // first column of this warp
+    const int cb = 32 * q;               // first column of this warp
     const uint32_t lane_base = tmem_addr(tbase, uint32_t(warp & 3) * 32, 0);
     const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
     uint64_t nl2_row = 0, dv_row = 0;
@@ -282,16 +297,13 @@ __device__ __forceinline__ void attn_bwd_f32_unit(const BwdParams& p, int bid) {
       nl2_row = f2_pack(nl2, nl2);
       dv_row = f2_pack(dv, dv);
     }
-    // writes 64 values as bf16 hi parts at col, lo parts at col + 32
+    // writes 32 values as bf16 hi parts at col, lo parts at col + 16
     auto store_split = [&](uint32_t col, const float* v) {
+      uint32_t hi[16], lo[16];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t hi[16], lo[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) split_bf16(v[32 * c + 2 * i], v[32 * c + 2 * i + 1], hi[i], lo[i]);
-        tmem_st16(col + 16 * c, hi);
-        tmem_st16(col + 32 + 16 * c, lo);
-      }
+      for (int i = 0; i < 16; ++i) split_bf16(v[2 * i], v[2 * i + 1], hi[i], lo[i]);
+      tmem_st16(col, hi);
+      tmem_st16(col + 16, lo);
     };
     bool ok = true;
     for (int k = 0; k < n_items; ++k) {
@@ -300,22 +312,24 @@ __device__ __forceinline__ void attn_bwd_f32_unit(const BwdParams& p, int bid) {
           reinterpret_cast<const float4*>(smem + L::kStage0 + s * L::kStageBytes + L::kColVec) + cb / 4;
       const int ct = item_tile(k);
       if (DKDV && !wait_warp(&bar_tma[s], (k / NS) & 1, wc, kErrWaitProducer)) { ok = false; break; }
-      if (!wait_warp(bar_s, k & 1, wc, kErrWaitMma)) { ok = false; break; }
+      if (!wait_warp(&bar_s[k & 1], (k >> 1) & 1, wc, kErrWaitMma)) { ok = false; break; }
+      NEA_TRACE_STAMP(p, 40 + min(k, 7), tid == 0);
       tc_fence_after();
       const int col0 = ct * kTileRows + cb;  // position of this warp's first column
       // ---- P = exp2(s * scale_log2 - LSE*log2e), masked
-      uint32_t sv[64];
-      tmem_ld64(lane_base + kColS + cb, sv);
+      uint32_t sv[32];
+      const uint32_t scol = lane_base + kColS + 128 * (k & 1) + cb;
+      tmem_ld32(scol, sv);
       if ((p.causal && ct == rt) || ct * kTileRows + kTileRows > p.T) {  // same for the whole tile
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
+        for (int i = 0; i < 32; ++i) {
           const bool masked = DKDV ? (p.causal && row > col0 + i) : ((p.causal && col0 + i > row) || col0 + i >= p.T);
           sv[i] = masked ? 0xff800000u : sv[i];
         }
       }
-      float pv[64];
+      float pv[32];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {  // four columns per step
+      for (int i = 0; i < 8; ++i) {  // four columns per step
         uint64_t nl2a = nl2_row, nl2b = nl2_row;
         if (DKDV) {
           const float4 c = colvec[i];
@@ -331,33 +345,34 @@ __device__ __forceinline__ void attn_bwd_f32_unit(const BwdParams& p, int bid) {
         pv[4 * i + 3] = ex2(t3);
       }
       if (DKDV) {  // P hi / lo over this warp's S columns: the A operand of dV(k)
-        store_split(lane_base + kColS + cb, pv);
+        store_split(scol, pv);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(bar_p);
+        NEA_TRACE_STAMP(p, 48 + min(k, 7), tid == 0);
       }
       // ---- dS = P (dP - Dv), hi / lo over this warp's dP columns
       if (!wait_warp(bar_dp, k & 1, wc, kErrWaitMma)) { ok = false; break; }
+      NEA_TRACE_STAMP(p, 56 + min(k, 7), tid == 0);
       tc_fence_after();
-      float ds[64];
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      float ds[32];
+      {
         uint32_t rr[32];
-        tmem_ld32(lane_base + kColDP + cb + 32 * c, rr);
+        tmem_ld32(lane_base + kColDP + cb, rr);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {  // four columns per step
-          const int e = 32 * c + 4 * i;
+          const int e = 4 * i;
           uint64_t dva = dv_row, dvb = dv_row;
           if (DKDV) {
-            const float4 d = colvec[32 + e / 4];
+            const float4 d = colvec[32 + i];
             dva = f2_pack(d.x, d.y);
             dvb = f2_pack(d.z, d.w);
           }
           f2_unpack(f2_mul(f2_pack(pv[e], pv[e + 1]),
-                           f2_sub(f2_pack(__uint_as_float(rr[4 * i]), __uint_as_float(rr[4 * i + 1])), dva)),
+                           f2_sub(f2_pack(__uint_as_float(rr[e]), __uint_as_float(rr[e + 1])), dva)),
                     ds[e], ds[e + 1]);
           f2_unpack(f2_mul(f2_pack(pv[e + 2], pv[e + 3]),
-                           f2_sub(f2_pack(__uint_as_float(rr[4 * i + 2]), __uint_as_float(rr[4 * i + 3])), dvb)),
+                           f2_sub(f2_pack(__uint_as_float(rr[e + 2]), __uint_as_float(rr[e + 3])), dvb)),
                     ds[e + 2], ds[e + 3]);
         }
       }
@@ -365,42 +380,24 @@ __device__ __forceinline__ void attn_bwd_f32_unit(const BwdParams& p, int bid) {
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar_ds);
+      NEA_TRACE_STAMP(p, 64 + min(k, 7), tid == 0);
     }
-    if (ok && wait_warp(bar_fin, 0, wc, kErrWaitMma)) {
-      tc_fence_after();
+    // warp-uniform: every lane of a warp saw the same waits
+    const bool epi = ok && wait_warp(bar_fin, 0, wc, kErrWaitMma);
+    NEA_TRACE_STAMP(p, 76, tid == 0);
+    if (epi) tc_fence_after();
+    if (DKDV) {
+      // quarter q: tensor q / 2 (dV, dK), columns [(q % 2) D/2, +D/2)
       constexpr int DH = D / 2;
-      if (DKDV) {
-        // half 0 writes the row of dV, half 1 the row of dK: X + Y
-        float acc[D], y[D];
-        const uint32_t a = lane_base + (hf ? kColAccB : kColAccA);
-        tmem_ld_n<D>(a, acc);
-        tmem_ld_n<D>(a + D, y);
+      const int tensor = q >> 1, c0h = (q & 1) * DH;
+      float acc[DH];
+      if (epi) tmem_ld_n<DH>(lane_base + (tensor ? kColAccB : kColAccA) + c0h, acc);
+      if (epi && row < p.T) {
+        if (tensor) {
 #pragma unroll
-        for (int i = 0; i < D; ++i) acc[i] = hf ? (acc[i] + y[i]) * p.scale : acc[i] + y[i];
-        if (row < p.T) {
-          if (hf && p.rope) {
-            // gradient w.r.t. the un-rotated input: apply R_t^T
-            const float4* tp = reinterpret_cast<const float4*>(p.rope + size_t(row) * (D / 2));
-#pragma unroll
-            for (int i = 0; i < D / 4; ++i) {
-              const float4 cs = __ldg(tp + i);
-              rot2(acc[4 * i], acc[4 * i + 1], cs.x, -cs.y);
-              rot2(acc[4 * i + 2], acc[4 * i + 3], cs.z, -cs.w);
-            }
-          }
-          const size_t off = ((size_t(b) * p.T + row) * p.Hkv + head_r) * D;
-          store_span<D, true>(hf ? p.dK : p.dV, off, acc);
-        }
-      } else {
-        // half h writes columns [h D/2, h D/2 + D/2) of the row of dQ
-        float acc[DH], y[DH];
-        tmem_ld_n<DH>(lane_base + kColAccA + DH * hf, acc);
-        tmem_ld_n<DH>(lane_base + kColAccA + D + DH * hf, y);
-#pragma unroll
-        for (int i = 0; i < DH; ++i) acc[i] = (acc[i] + y[i]) * p.scale;
-        if (row < p.T) {
-          if (p.rope) {
-            const float4* tp = reinterpret_cast<const float4*>(p.rope + size_t(row) * (D / 2) + DH / 2 * hf);
+          for (int i = 0; i < DH; ++i) acc[i] *= p.scale;
+          if (p.rope) {  // gradient w.r.t. the un-rotated input: apply R_t^T
+            const float4* tp = reinterpret_cast<const float4*>(p.rope + size_t(row) * (D / 2) + c0h / 2);
 #pragma unroll
             for (int i = 0; i < DH / 4; ++i) {
               const float4 cs = __ldg(tp + i);
@@ -408,18 +405,41 @@ __device__ __forceinline__ void attn_bwd_f32_unit(const BwdParams& p, int bid) {
               rot2(acc[4 * i + 2], acc[4 * i + 3], cs.z, -cs.w);
             }
           }
-          const size_t off = ((size_t(b) * p.T + row) * p.Hq + head_r) * D + DH * hf;
-          store_span<DH, true>(p.dQ, off, acc);
         }
+        const size_t off = ((size_t(b) * p.T + row) * p.Hkv + head_r) * D + c0h;
+        store_span<DH, true>(tensor ? p.dK : p.dV, off, acc);
+      }
+    } else if (epi) {
+      // quarter q writes columns [q D/4, q D/4 + D/4) of the row of dQ
+      constexpr int DQQ = D / 4;
+      const int c0q = q * DQQ;
+      float acc[DQQ];
+      tmem_ld_n<DQQ>(lane_base + kColAccA + c0q, acc);
+#pragma unroll
+      for (int i = 0; i < DQQ; ++i) acc[i] *= p.scale;
+      if (row < p.T) {
+        if (p.rope) {
+          const float4* tp = reinterpret_cast<const float4*>(p.rope + size_t(row) * (D / 2) + c0q / 2);
+#pragma unroll
+          for (int i = 0; i < DQQ / 4; ++i) {
+            const float4 cs = __ldg(tp + i);
+            rot2(acc[4 * i], acc[4 * i + 1], cs.x, -cs.y);
+            rot2(acc[4 * i + 2], acc[4 * i + 3], cs.z, -cs.w);
+          }
+        }
+        const size_t off = ((size_t(b) * p.T + row) * p.Hq + head_r) * D + c0q;
+        store_span<DQQ, true>(p.dQ, off, acc);
       }
     }
   }
+  NEA_TRACE_STAMP(p, 77, tid == 0);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tbase, 512);
   }
+  NEA_TRACE_STAMP(p, 78, tid == 0);
 }
 
 template <int D>

@@ -23,9 +23,16 @@
 //              arithmetic; the running max m moves only when it grows by more
 //              than 2^8 (O rescaled in TMEM then); the epilogue writes O / l
 //              and LSE.
-//   8, 9       MMA issuers, one thread each: warp 8 for tile A, warp 9 for tile B;
-//              S_X = Q_X K_j^T, O_X += P_X V_j, each waiting only on its own
-//              tile, so one tile's softmax overlaps the other tile's MMAs.
+//   8, 9       MMA issuers.  bfloat16 storage: warp 8 for tile A, warp 9 for
+//              tile B, each issuing S_X(j+1) as soon as its softmax holds
+//              S_X(j) in registers, so S_X(j+1) runs under the exponentials
+//              of step j.  float32 storage (S_X(j+1) must wait for PV_X(j),
+//              which reads P over S): warp 8 alone, for both tiles, in a
+//              fixed ping-pong order -- S_A(0); PV_A(0), S_B(0); then per key
+//              tile j S_A(j+1), PV_B(j), S_B(j+1), PV_A(j+1) -- so that tile
+//              B runs half a step behind tile A and each tile's softmax
+//              overlaps the other tile's products (issued per tile, the two
+//              tiles fall into step and share the exponential unit).
 //   10         TMA: query tiles, then K and V tiles into two rings (K stages
 //              free as soon as S is computed, V stages after PV).
 // TMEM per tile X: S [256X, 256X+128), O [256X+128, +D), and
@@ -113,7 +120,7 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
   uint64_t* bar_s = bars + 1 + 2 * NK + 2 * NV;         // [2] S_X landed
   uint64_t* bar_p = bar_s + 2;                          // [2] P_X written (count 128)
   uint64_t* bar_o = bar_s + 4;                          // [2] PV_X done
-  uint64_t* bar_fin = bar_s + 6;                        // [2] per issuer
+  uint64_t* bar_fin = bar_s + 6;                        // [2] each issuer's last products
   uint64_t* bar_sread = bar_s + 8;                      // [2] S_X loaded by the softmax (count 128)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
@@ -347,19 +354,20 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
       }
       __syncwarp();
     } else if (warp < 10) {
-      // ------------------------------------------------------------ MMA issuers
-      // Issuer X runs tile X on its own: S_X(0); then per key tile j: wait for
-      // P_X(j), O_X += P_X(j) V_j; wait for that to finish reading P_X(j) (which
-      // S_X(j+1) overwrites), S_X(j+1).  Stage releases count one commit per
+      // ------------------------------------------------------------ MMA issuers (warps 8, 9)
+      // Fixed ping-pong order over the two tiles (see the header).  S_X(j+1)
+      // may overwrite S_X(j) once the softmax holds S_X(j) in registers
+      // (bf16 storage: P in its own columns) or once PV_X(j) has read P_X(j)
+      // (float32 storage: P hi over S).  Stage releases count one commit per
       // tile; the last key tile of a causal pair is used by B alone, but its
       // stages are never refilled, so no one waits for that release.
-      const int x = warp - 8;
-      if ((tid & 31) == 0 && (x == 0 || has_b)) {
+      const int xw = warp - 8;  // this warp's tile (bf16 storage)
+      if ((tid & 31) == 0 && (kSepP ? (xw == 0 || has_b) : xw == 0)) {
         constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
         constexpr uint32_t idO = idesc_bf16(128, D, 0, 1);
-        const uint32_t sQ = smem_u32(smem + (x ? L::kQB : L::kQA));
-        const int my_nkv = x ? nkv_b : nkv_a;
-        auto issue_s = [&](int j) {
+        const int n_x[2] = {nkv_a, nkv_b};
+        auto issue_s = [&](int x, int j) {
+          const uint32_t sQ = smem_u32(smem + (x ? L::kQB : L::kQA));
           const uint32_t sK = smem_u32(smem + L::kK0 + (j % NK) * L::kKStage);
           const uint32_t dS = tbase + 256 * x;
 #pragma unroll
@@ -373,33 +381,10 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
             }
           }
           tc_commit(&bar_s[x]);
+          tc_commit(&bar_kempty[j % NK]);
         };
-        bool ok = wait_thread(bar_qtma, 0, wc, kErrWaitProducer) &&
-                  wait_thread(&bar_ktma[0], 0, wc, kErrWaitProducer);
-        if (ok) {
-          tc_fence_after();
-          issue_s(0);
-          tc_commit(&bar_kempty[0]);
-        }
-        for (int j = 0; ok && j < my_nkv; ++j) {
+        auto issue_pv = [&](int x, int j) {
           const int sv = j % NV;
-          if (kSepP && j + 1 < my_nkv) {
-            // S_X(j+1) as soon as the softmax holds S_X(j) in registers
-            const int sk = (j + 1) % NK;
-            if (!wait_thread(&bar_sread[x], j & 1, wc, kErrWaitSoftmax) ||
-                !wait_thread(&bar_ktma[sk], ((j + 1) / NK) & 1, wc, kErrWaitProducer))
-              break;
-            NEA_TRACE_STAMP(p, 44 + min(j, 7), x == 0);
-            tc_fence_after();
-            issue_s(j + 1);
-            tc_commit(&bar_kempty[sk]);
-          }
-          if (!wait_thread(&bar_p[x], j & 1, wc, kErrWaitSoftmax) ||
-              !wait_thread(&bar_vtma[sv], (j / NV) & 1, wc, kErrWaitProducer))
-            break;
-          NEA_TRACE_STAMP(p, 36 + min(j, 7), x == 0);
-          NEA_TRACE_STAMP(p, 36 + min(j, 7), x == 0);
-          tc_fence_after();
           const uint32_t sV = smem_u32(smem + L::kV0 + sv * L::kVStage);
           const uint32_t phi = tbase + 256 * x, plo = tbase + 256 * x + 192, dO = tbase + 256 * x + 128;
 #pragma unroll
@@ -414,21 +399,60 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
           }
           tc_commit(&bar_o[x]);
           tc_commit(&bar_vempty[sv]);
-          NEA_TRACE_STAMP(p, 68 + min(j, 7), x == 0);
-          if (!kSepP && j + 1 < my_nkv) {
-            // S_X(j+1) overwrites P_X(j): wait until PV_X(j) has read it
-            const int sk = (j + 1) % NK;
-            if (!wait_thread(&bar_o[x], j & 1, wc, kErrWaitMma) ||
-                !wait_thread(&bar_ktma[sk], ((j + 1) / NK) & 1, wc, kErrWaitProducer))
-              break;
-            NEA_TRACE_STAMP(p, 44 + min(j, 7), x == 0);
+        };
+        // S_X(j+1): key tile landed, and S_X(j) no longer needed
+        auto next_s = [&](int x, int j) {
+          const bool free = kSepP ? wait_thread(&bar_sread[x], j & 1, wc, kErrWaitSoftmax)
+                                  : wait_thread(&bar_o[x], j & 1, wc, kErrWaitMma);
+          if (!free || !wait_thread(&bar_ktma[(j + 1) % NK], ((j + 1) / NK) & 1, wc, kErrWaitProducer))
+            return false;
+          NEA_TRACE_STAMP(p, 44 + min(j, 7), x == 0);
+          tc_fence_after();
+          issue_s(x, j + 1);
+          return true;
+        };
+        // PV_X(j): P_X(j) written and value tile landed
+        auto next_pv = [&](int x, int j) {
+          if (!wait_thread(&bar_p[x], j & 1, wc, kErrWaitSoftmax) ||
+              !wait_thread(&bar_vtma[j % NV], (j / NV) & 1, wc, kErrWaitProducer))
+            return false;
+          NEA_TRACE_STAMP(p, 36 + min(j, 7), x == 0);
+          tc_fence_after();
+          issue_pv(x, j);
+          return true;
+        };
+        bool ok = wait_thread(bar_qtma, 0, wc, kErrWaitProducer) &&
+                  wait_thread(&bar_ktma[0], 0, wc, kErrWaitProducer);
+        if constexpr (kSepP) {
+          // one tile: S(0); per key tile j, S(j+1) once the softmax holds S(j),
+          // then PV(j) once P(j) is written
+          if (ok) {
             tc_fence_after();
-            issue_s(j + 1);
-            tc_commit(&bar_kempty[sk]);
+            issue_s(xw, 0);
+          }
+          for (int j = 0; ok && j < n_x[xw]; ++j) {
+            if (j + 1 < n_x[xw] && !(ok = next_s(xw, j))) break;
+            if (!(ok = next_pv(xw, j))) break;
+          }
+        } else {
+          if (ok) {
+            tc_fence_after();
+            issue_s(0, 0);
+            ok = next_pv(0, 0);
+            if (ok && n_x[1] > 0) issue_s(1, 0);
+          }
+          for (int j = 0; ok; ++j) {
+            if (j + 1 < n_x[0] && !(ok = next_s(0, j))) break;
+            if (j < n_x[1]) {
+              if (!(ok = next_pv(1, j))) break;
+              if (j + 1 < n_x[1] && !(ok = next_s(1, j))) break;
+            }
+            if (j + 1 < n_x[0] && !(ok = next_pv(0, j + 1))) break;
+            if (j + 1 >= n_x[0] && j + 1 >= n_x[1]) break;
           }
         }
-        tc_commit(&bar_fin[x]);
-        drain_wait(&bar_fin[x], 0, wc);
+        tc_commit(&bar_fin[kSepP ? xw : 0]);
+        drain_wait(&bar_fin[kSepP ? xw : 0], 0, wc);
       }
       __syncwarp();
     }
