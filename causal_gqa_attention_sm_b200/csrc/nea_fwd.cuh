@@ -23,16 +23,15 @@
 //              arithmetic; the running max m moves only when it grows by more
 //              than 2^8 (O rescaled in TMEM then); the epilogue writes O / l
 //              and LSE.
-//   8, 9       MMA issuers.  bfloat16 storage: warp 8 for tile A, warp 9 for
-//              tile B, each issuing S_X(j+1) as soon as its softmax holds
-//              S_X(j) in registers, so S_X(j+1) runs under the exponentials
-//              of step j.  float32 storage (S_X(j+1) must wait for PV_X(j),
-//              which reads P over S): warp 8 alone, for both tiles, in a
-//              fixed ping-pong order -- S_A(0); PV_A(0), S_B(0); then per key
-//              tile j S_A(j+1), PV_B(j), S_B(j+1), PV_A(j+1) -- so that tile
-//              B runs half a step behind tile A and each tile's softmax
-//              overlaps the other tile's products (issued per tile, the two
-//              tiles fall into step and share the exponential unit).
+//   8, 9       MMA issuers, one thread each: warp 8 for tile A, warp 9 for
+//              tile B.  bfloat16 storage: S_X(j+1) as soon as the softmax
+//              holds S_X(j) in registers, so it runs under the exponentials
+//              of step j; then PV_X(j).  float32 storage (S_X(j+1) must wait
+//              for PV_X(j), which reads P over S): PV_X(j), then S_X(j+1),
+//              and tile B starts only once tile A has written its first P, so
+//              B runs about half a step behind A and each tile's softmax
+//              overlaps the other tile's products (started together, the two
+//              tiles stay in step and share the exponential unit).
 //   10         TMA: query tiles, then K and V tiles into two rings (K stages
 //              free as soon as S is computed, V stages after PV).
 // TMEM per tile X: S [256X, 256X+128), O [256X+128, +D), and
@@ -355,14 +354,14 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
       __syncwarp();
     } else if (warp < 10) {
       // ------------------------------------------------------------ MMA issuers (warps 8, 9)
-      // Fixed ping-pong order over the two tiles (see the header).  S_X(j+1)
-      // may overwrite S_X(j) once the softmax holds S_X(j) in registers
-      // (bf16 storage: P in its own columns) or once PV_X(j) has read P_X(j)
-      // (float32 storage: P hi over S).  Stage releases count one commit per
-      // tile; the last key tile of a causal pair is used by B alone, but its
-      // stages are never refilled, so no one waits for that release.
-      const int xw = warp - 8;  // this warp's tile (bf16 storage)
-      if ((tid & 31) == 0 && (kSepP ? (xw == 0 || has_b) : xw == 0)) {
+      // S_X(j+1) may overwrite S_X(j) once the softmax holds S_X(j) in
+      // registers (bf16 storage: P in its own columns) or once PV_X(j) has
+      // read P_X(j) (float32 storage: P hi over S).  Stage releases count one
+      // commit per tile; the last key tile of a causal pair is used by B
+      // alone, but its stages are never refilled, so no one waits for that
+      // release.
+      const int xw = warp - 8;  // this warp's tile
+      if ((tid & 31) == 0 && (xw == 0 || has_b)) {
         constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
         constexpr uint32_t idO = idesc_bf16(128, D, 0, 1);
         const int n_x[2] = {nkv_a, nkv_b};
@@ -423,36 +422,19 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
         };
         bool ok = wait_thread(bar_qtma, 0, wc, kErrWaitProducer) &&
                   wait_thread(&bar_ktma[0], 0, wc, kErrWaitProducer);
-        if constexpr (kSepP) {
-          // one tile: S(0); per key tile j, S(j+1) once the softmax holds S(j),
-          // then PV(j) once P(j) is written
-          if (ok) {
-            tc_fence_after();
-            issue_s(xw, 0);
-          }
-          for (int j = 0; ok && j < n_x[xw]; ++j) {
-            if (j + 1 < n_x[xw] && !(ok = next_s(xw, j))) break;
-            if (!(ok = next_pv(xw, j))) break;
-          }
-        } else {
-          if (ok) {
-            tc_fence_after();
-            issue_s(0, 0);
-            ok = next_pv(0, 0);
-            if (ok && n_x[1] > 0) issue_s(1, 0);
-          }
-          for (int j = 0; ok; ++j) {
-            if (j + 1 < n_x[0] && !(ok = next_s(0, j))) break;
-            if (j < n_x[1]) {
-              if (!(ok = next_pv(1, j))) break;
-              if (j + 1 < n_x[1] && !(ok = next_s(1, j))) break;
-            }
-            if (j + 1 < n_x[0] && !(ok = next_pv(0, j + 1))) break;
-            if (j + 1 >= n_x[0] && j + 1 >= n_x[1]) break;
-          }
+        // float32 storage: tile B waits for tile A's first P (half a step)
+        if (!kSepP && xw == 1) ok = ok && wait_thread(&bar_p[0], 0, wc, kErrWaitSoftmax);
+        if (ok) {
+          tc_fence_after();
+          issue_s(xw, 0);
         }
-        tc_commit(&bar_fin[kSepP ? xw : 0]);
-        drain_wait(&bar_fin[kSepP ? xw : 0], 0, wc);
+        for (int j = 0; ok && j < n_x[xw]; ++j) {
+          if (kSepP && j + 1 < n_x[xw] && !(ok = next_s(xw, j))) break;
+          if (!(ok = next_pv(xw, j))) break;
+          if (!kSepP && j + 1 < n_x[xw] && !(ok = next_s(xw, j))) break;
+        }
+        tc_commit(&bar_fin[xw]);
+        drain_wait(&bar_fin[xw], 0, wc);
       }
       __syncwarp();
     }
