@@ -283,15 +283,16 @@ def measure_tf32_peak(dev, sustain_s=4.0):
 # ---------------------------------------------------------------- ncu traffic records
 # The sources that make up each kernel: its own header plus the shared device
 # helpers, tile geometry and the host code that sets up its launch.
-KERNEL_SOURCES = {"attn_fwd_prologue": "nea_prep.cuh", "attn_bwd_prologue": "nea_prep.cuh",
-                  "attn_fwd": "nea_fwd.cuh", "attn_bwd": "nea_bwd.cuh", "attn_decode": "nea_decode.cuh"}
+KERNEL_SOURCES = {"attn_fwd_prologue": ("nea_prep.cuh",), "attn_bwd_prologue": ("nea_prep.cuh",),
+                  "attn_fwd": ("nea_fwd.cuh",), "attn_bwd": ("nea_bwd.cuh", "nea_bwd_f32.cuh"),
+                  "attn_decode": ("nea_decode.cuh",)}
 SHARED_SOURCES = ("nea_attn.cu", "nea_device.cuh", "nea_tiles.cuh")
 
 
 def kernel_source_hash(kernel):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "causal_gqa_attention_sm_b200", "csrc")
-    for name in sorted(SHARED_SOURCES + (KERNEL_SOURCES[kernel],)):
+    for name in sorted(SHARED_SOURCES + KERNEL_SOURCES[kernel]):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]

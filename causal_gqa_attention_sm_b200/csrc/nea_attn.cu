@@ -371,8 +371,8 @@ int launch_fwd(uint32_t& attr_done, const nea::FwdParams& p, cudaStream_t stream
 template <int D, bool F32IO>
 int launch_bwd(uint32_t& attr_done, const nea::BwdParams& p, cudaStream_t stream, bool ev) {
   cudaError_t e;
-  using L = std::conditional_t<F32IO, nea::Bwd32Smem<D>, nea::BwdSmem<D, false>>;
-  auto kern = F32IO ? nea::attn_bwd_f32_kernel<D> : nea::attn_bwd_kernel<D, false>;
+  using L = std::conditional_t<F32IO, nea::Bwd32Smem<D>, nea::BwdSmem<D>>;
+  auto kern = F32IO ? nea::attn_bwd_f32_kernel<D> : nea::attn_bwd_kernel<D>;
   int rc = set_smem(attr_done, 4 + (D == 64) * 2 + F32IO, kern, L::kAlloc);
   if (rc) return rc;
   e = launch_dependent(kern, unsigned(p.n_dkdv + p.B * p.Hq * p.n_tiles), L::kThreads, L::kAlloc, stream, p);

@@ -19,11 +19,9 @@
 //         over the GQA group needs no extra pass or atomics.
 //   DQ    row = query tile i of head h (Q'_i, dO_i), columns = key tiles
 //         j <= i (K'_j, V_j).
-// Operands arrive by TMA in the swizzled operand layout, already rotated by
-// the operand prologue (nea_prep.cuh): bf16 storage reads rotated copies of Q
-// and K and the inputs V, dO; float32 storage reads the bf16 hi/lo planes and
-// forms S and dP from three bf16 products, the gradient products from the hi
-// parts.
+// This kernel serves bfloat16 storage (float32 storage: nea_bwd_f32.cuh).
+// Operands arrive by TMA in the swizzled operand layout: rotated copies of Q
+// and K from the operand prologue (nea_prep.cuh) and the inputs V, dO.
 // Warps: 0-7 elementwise work, warp w on TMEM lanes 32 (w % 4) .. + 31 (its
 // rows) and columns 64 (w / 4) .. + 63 of the tile; 8 issues the MMAs; 9
 // issues TMA (resident tiles, then column tiles and, for DKDV, the LSE/Dv
@@ -48,6 +46,8 @@
 namespace nea {
 
 // ---------------------------------------------------------------- main kernel
+// Parameters of both gradient kernels (bfloat16 storage here, float32 storage
+// in nea_bwd_f32.cuh).
 struct BwdParams {
   // bf16 storage: rotated Q, K (the inputs when the rotation is off), V, dO.
   // float32 storage: the hi planes.
@@ -80,10 +80,10 @@ struct BwdParams {
   unsigned long long* trace;  // per-CTA phase stamps (NEA_TRACE builds only)
 };
 
-template <int D, bool F32IO>
+template <int D>
 struct BwdSmem {
-  static constexpr int kStages = F32IO ? 2 : 3;
-  static constexpr uint32_t kTile = Stage<D, F32IO>::kBytes;
+  static constexpr int kStages = 3;
+  static constexpr uint32_t kTile = TileGeom<D>::kOpBytes;
   static constexpr uint32_t kR1 = 0;
   static constexpr uint32_t kR2 = kR1 + kTile;
   static constexpr uint32_t kStage0 = kR2 + kTile;
@@ -130,13 +130,11 @@ __device__ __forceinline__ void tmem_ld_n(uint32_t taddr, float* v) {
 // One unit (a dK/dV unit when DKDV, else a dQ unit; `bid` its index among
 // units of its kind), specialised per pass so that neither pays for the
 // other's branches.
-template <int D, bool F32IO, bool DKDV>
+template <int D, bool DKDV>
 __device__ __forceinline__ void attn_bwd_unit(const BwdParams& p, int bid) {
-  using L = BwdSmem<D, F32IO>;
+  using L = BwdSmem<D>;
   constexpr uint32_t RB = TileGeom<D>::kRowBytes;
-  constexpr uint32_t OPB = TileGeom<D>::kOpBytes;
   constexpr int NS = L::kStages;
-  constexpr int kTerms = F32IO ? 3 : 1;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
@@ -217,26 +215,20 @@ __device__ __forceinline__ void attn_bwd_unit(const BwdParams& p, int bid) {
       const CUtensorMap* m_r2 = DKDV ? &p.tm_v : &p.tm_do;
       const CUtensorMap* m_c1 = DKDV ? &p.tm_q : &p.tm_k;
       const CUtensorMap* m_c2 = DKDV ? &p.tm_do : &p.tm_v;
-      const CUtensorMap* m_r1l = DKDV ? &p.tm_k_lo : &p.tm_q_lo;
-      const CUtensorMap* m_r2l = DKDV ? &p.tm_v_lo : &p.tm_do_lo;
-      const CUtensorMap* m_c1l = DKDV ? &p.tm_q_lo : &p.tm_k_lo;
-      const CUtensorMap* m_c2l = DKDV ? &p.tm_do_lo : &p.tm_v_lo;
       prefetch_tmap(m_r1);
       prefetch_tmap(m_r2);
       prefetch_tmap(m_c1);
       prefetch_tmap(m_c2);
-      auto load_tile = [&](uint8_t* dst, const CUtensorMap* hi, const CUtensorMap* lo, int head, int row0,
-                           uint64_t* bar) {
-        tma_load_4d(dst, hi, 0, head, row0, b, bar);
-        if (F32IO) tma_load_4d(dst + OPB, lo, 0, head, row0, b, bar);
+      auto load_tile = [&](uint8_t* dst, const CUtensorMap* m, int head, int row0, uint64_t* bar) {
+        tma_load_4d(dst, m, 0, head, row0, b, bar);
       };
       // fault-injection hook: withhold the resident tiles so every wait on
       // them runs into its limit
       const bool r_armed = !(p.debug & 2);
       if (r_armed) {
         mbar_arrive_expect_tx(bar_rtma, 2 * L::kTile);
-        load_tile(smem + L::kR1, m_r1, m_r1l, head_r, rt * kTileRows, bar_rtma);
-        load_tile(smem + L::kR2, m_r2, m_r2l, head_r, rt * kTileRows, bar_rtma);
+        load_tile(smem + L::kR1, m_r1, head_r, rt * kTileRows, bar_rtma);
+        load_tile(smem + L::kR2, m_r2, head_r, rt * kTileRows, bar_rtma);
       }
       int armed = 0;
       for (int k = 0; k < n_items; ++k) {
@@ -245,8 +237,8 @@ __device__ __forceinline__ void attn_bwd_unit(const BwdParams& p, int bid) {
         uint8_t* st = smem + L::kStage0 + s * L::kStageBytes;
         const int ch = item_head(k), ct = item_tile(k);
         mbar_arrive_expect_tx(&bar_tma[s], 2 * L::kTile + (DKDV ? 1024 : 0));
-        load_tile(st, m_c1, m_c1l, ch, ct * kTileRows, &bar_tma[s]);
-        load_tile(st + L::kTile, m_c2, m_c2l, ch, ct * kTileRows, &bar_tma[s]);
+        load_tile(st, m_c1, ch, ct * kTileRows, &bar_tma[s]);
+        load_tile(st + L::kTile, m_c2, ch, ct * kTileRows, &bar_tma[s]);
         if (DKDV)  // -LSE*log2e then Dv of the 128 queries of this column tile
           tma_load_3d(st + L::kColVec, &p.tm_ws, ct * kTileRows, 0, b * p.Hq + ch, &bar_tma[s]);
         armed = k + 1;
@@ -269,10 +261,7 @@ __device__ __forceinline__ void attn_bwd_unit(const BwdParams& p, int bid) {
         const uint32_t sC1 = stage_c1(k);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-#pragma unroll
-          for (int term = 0; term < kTerms; ++term)
-            mma_ss(tbase + kColS, smem_desc(sR1 + (term == 2 ? OPB : 0) + kk * 32, RB, 16),
-                   smem_desc(sC1 + (term == 1 ? OPB : 0) + kk * 32, RB, 16), idSS, (kk | term) != 0);
+          mma_ss(tbase + kColS, smem_desc(sR1 + kk * 32, RB, 16), smem_desc(sC1 + kk * 32, RB, 16), idSS, kk != 0);
         tc_commit(bar_s);
       };
       bool ok = wait_thread(bar_rtma, 0, wc, kErrWaitProducer) &&
@@ -286,10 +275,7 @@ __device__ __forceinline__ void attn_bwd_unit(const BwdParams& p, int bid) {
         // dP(k) overwrites dP(k-1), which the rows read before dS(k-1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-#pragma unroll
-          for (int term = 0; term < kTerms; ++term)
-            mma_ss(tbase + kColDP, smem_desc(sR2 + (term == 2 ? OPB : 0) + kk * 32, RB, 16),
-                   smem_desc(sC2 + (term == 1 ? OPB : 0) + kk * 32, RB, 16), idSS, (kk | term) != 0);
+          mma_ss(tbase + kColDP, smem_desc(sR2 + kk * 32, RB, 16), smem_desc(sC2 + kk * 32, RB, 16), idSS, kk != 0);
         tc_commit(bar_dp);
         NEA_TRACE_STAMP(p, 36 + min(k, 7), true);
         if (k + 1 < n_items) {
@@ -456,7 +442,7 @@ __device__ __forceinline__ void attn_bwd_unit(const BwdParams& p, int bid) {
             }
           }
           const size_t off = ((size_t(b) * p.T + row) * p.Hkv + head_r) * D;
-          store_span<D, F32IO>(hf ? p.dK : p.dV, off, acc);
+          store_span<D, false>(hf ? p.dK : p.dV, off, acc);
         }
       } else {
         // half h writes columns [h D/2, h D/2 + D/2) of the row of dQ
@@ -475,7 +461,7 @@ __device__ __forceinline__ void attn_bwd_unit(const BwdParams& p, int bid) {
             }
           }
           const size_t off = ((size_t(b) * p.T + row) * p.Hq + head_r) * D + DH * hf;
-          store_span<DH, F32IO>(p.dQ, off, acc);
+          store_span<DH, false>(p.dQ, off, acc);
         }
       }
     }
@@ -489,14 +475,14 @@ __device__ __forceinline__ void attn_bwd_unit(const BwdParams& p, int bid) {
   NEA_TRACE_STAMP(p, 78, tid == 0);
 }
 
-template <int D, bool F32IO>
-__global__ void __launch_bounds__(BwdSmem<D, F32IO>::kThreads, 1)
+template <int D>
+__global__ void __launch_bounds__(BwdSmem<D>::kThreads, 1)
     attn_bwd_kernel(const __grid_constant__ BwdParams p) {
   const int unit = p.unit0 + int(blockIdx.x);
   if (unit < p.n_dkdv)
-    attn_bwd_unit<D, F32IO, true>(p, unit);
+    attn_bwd_unit<D, true>(p, unit);
   else
-    attn_bwd_unit<D, F32IO, false>(p, unit - p.n_dkdv);
+    attn_bwd_unit<D, false>(p, unit - p.n_dkdv);
 }
 
 }  // namespace nea
