@@ -1,9 +1,10 @@
 """Throughput of causal GQA attention forward+backward on B200.
 
-One step = nea_attn_fwd + nea_attn_bwd (four kernels: the forward operand
-prologue, the forward, the backward prologue with the row terms, and the
-gradient kernel with its dK/dV and dQ units) over one batch of synthetic
-inputs already resident in HBM.
+One step = nea_attn_fwd_save + nea_attn_bwd_saved, the save-for-backward pair
+(four kernels: the forward operand prologue, which keeps its planes for the
+backward; the forward; the backward prologue, which converts dO and writes the
+row terms; and the gradient kernel with its dK/dV and dQ units) over one batch
+of synthetic inputs already resident in HBM.
 Default workload: B=4, T=1024, Hq=12, Hkv=4, D=64, float32 storage, causal,
 RoPE base 10000, Q,K ~ N(0, 9), V, dO ~ N(0, 1) -- the longer-context
 configuration of the NanoEuler GPU model shape.
@@ -44,14 +45,16 @@ L2_FLUSH_BYTES = 256 << 20
 
 def prologue_bytes(w, kernel):
     """Algorithmic HBM bytes of one operand-prologue launch: every input
-    element read once and every output element written once."""
+    element read once and every output element written once.  The forward's
+    prologue converts Q, K, V (bf16 storage: rotates Q, K); the backward's, fed
+    the saved planes, converts only dO (nothing for bf16 storage)."""
     nq, nk = w.B * w.T * w.Hq * w.D, w.B * w.T * w.Hkv * w.D
     rope = w.rope_base > 0
     if w.dtype == "f32":  # fp32 in, bf16 hi + lo out
-        conv = (nq + 2 * nk) if kernel == "attn_fwd_prologue" else (2 * nq + 2 * nk)
+        conv = (nq + 2 * nk) if kernel == "attn_fwd_prologue" else nq
         b = conv * (4 + 4)
-    else:  # rotated bf16 copies of Q, K
-        b = (nq + nk) * (2 + 2) if rope else 0
+    else:  # rotated bf16 copies of Q, K in the forward
+        b = (nq + nk) * (2 + 2) if rope and kernel == "attn_fwd_prologue" else 0
     if kernel == "attn_bwd_prologue":  # row terms: read O, dO, LSE; write ws[B*Hq][2][Tp]
         e = 4 if w.dtype == "f32" else 2
         tp = -(-w.T // 128) * 128
@@ -548,8 +551,10 @@ def main():
     for L in layers:
         o = torch.empty_like(L["q"])
         lse = torch.empty((w.B, w.Hq, w.T), dtype=torch.float32, device=dev)
+        saved = torch.empty(nea.nea_attn_saved_bytes(w.B, w.T, w.Hq, w.Hkv, w.D, w.torch_dtype, w.rope_base),
+                            dtype=torch.uint8, device=dev)
         outs.append({"o": o, "lse": lse, "dq": torch.empty_like(L["q"]), "dk": torch.empty_like(L["k"]),
-                     "dv": torch.empty_like(L["v"])})
+                     "dv": torch.empty_like(L["v"]), "saved": saved})
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     drain = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     drain_sum = torch.empty((), dtype=torch.float32, device=dev)
@@ -558,11 +563,15 @@ def main():
         flush.fill_(float(i))
         torch.sum(drain, dim=0, out=drain_sum)
 
+    def layer_step(L, O, s=None):
+        nea.nea_attn_fwd_save(L["q"], L["k"], L["v"], w.rope_base, w.causal, o=O["o"], lse=O["lse"],
+                              saved=O["saved"], stream=s)
+        nea.nea_attn_bwd_saved(L["q"], L["k"], L["v"], O["o"], O["lse"], L["do"], O["saved"], w.rope_base,
+                               w.causal, dq=O["dq"], dk=O["dk"], dv=O["dv"], stream=s)
+
     def step():
         for L, O in zip(layers, outs):
-            nea.nea_attn_fwd(L["q"], L["k"], L["v"], w.rope_base, w.causal, o=O["o"], lse=O["lse"])
-            nea.nea_attn_bwd(L["q"], L["k"], L["v"], O["o"], O["lse"], L["do"], w.rope_base, w.causal,
-                             dq=O["dq"], dk=O["dk"], dv=O["dv"])
+            layer_step(L, O)
 
     for _ in range(a.warmup):
         flush_l2(1)
@@ -608,9 +617,7 @@ def main():
         flush_l2(i)
         for li, (L, O) in enumerate(zip(layers, outs)):
             nea.nea_set_profile_events(ev_k[i][li])
-            nea.nea_attn_fwd(L["q"], L["k"], L["v"], w.rope_base, w.causal, o=O["o"], lse=O["lse"])
-            nea.nea_attn_bwd(L["q"], L["k"], L["v"], O["o"], O["lse"], L["do"], w.rope_base, w.causal,
-                             dq=O["dq"], dk=O["dk"], dv=O["dv"])
+            layer_step(L, O)
         nea.nea_set_profile_events(None)
     torch.cuda.synchronize(dev)
     status = nea.nea_device_status()
@@ -678,8 +685,9 @@ def main():
         host_in = [{n: t.cpu().pin_memory() for n, t in L.items()} for L in layers]
         dev_in = [[{n: torch.empty_like(t) for n, t in L.items()} for L in layers] for _ in range(NB)]
         dev_out = [[{"o": torch.empty_like(L["q"]), "lse": torch.empty((w.B, w.Hq, w.T), dtype=torch.float32, device=dev),
-                     "dq": torch.empty_like(L["q"]), "dk": torch.empty_like(L["k"]), "dv": torch.empty_like(L["v"])}
-                    for L in layers] for _ in range(NB)]
+                     "dq": torch.empty_like(L["q"]), "dk": torch.empty_like(L["k"]), "dv": torch.empty_like(L["v"]),
+                     "saved": O["saved"]}
+                    for L, O in zip(layers, outs)] for _ in range(NB)]
         host_out = [[{n: torch.empty(O[n].shape, dtype=O[n].dtype, pin_memory=True) for n in ("o", "dq", "dk", "dv")}
                      for O in dev_out[0]] for _ in range(NB)]
         h2d = sum(t.numel() * t.element_size() for H in host_in for t in H.values())
@@ -700,10 +708,7 @@ def main():
             stream.wait_event(ev_in[bi])
             stream.wait_event(ev_out[bi])  # the read-back that last used these outputs
             for Dv, O in zip(dev_in[bi], dev_out[bi]):
-                nea.nea_attn_fwd(Dv["q"], Dv["k"], Dv["v"], w.rope_base, w.causal, o=O["o"], lse=O["lse"],
-                                 stream=stream)
-                nea.nea_attn_bwd(Dv["q"], Dv["k"], Dv["v"], O["o"], O["lse"], Dv["do"], w.rope_base, w.causal,
-                                 dq=O["dq"], dk=O["dk"], dv=O["dv"], stream=stream)
+                layer_step(Dv, O, stream)
             ev_comp[bi].record(stream)
             s_out.wait_event(ev_comp[bi])
             with torch.cuda.stream(s_out):

@@ -18,7 +18,7 @@ __all__ = [
     "nea_attn_fwd", "nea_attn_bwd", "nea_device_status", "nea_set_wait_limit_ns", "nea_debug_inject",
     "nea_status_string", "nea_version", "nea_set_profile_events", "NeaError", "LIB_PATH", "NEA_OK", "NEA_ERR_ARG", "NEA_ERR_CUDA",
     "NEA_ERR_TIMEOUT", "NEA_ERR_UNSUPPORTED", "NEA_ERR_NOMEM", "NEA_ERR_SCRATCH_LIMIT", "NEA_F32", "NEA_BF16",
-    "nea_attn_bwd_noalloc", "nea_attn_decode",
+    "nea_attn_bwd_noalloc", "nea_attn_decode", "nea_attn_saved_bytes", "nea_attn_fwd_save", "nea_attn_bwd_saved",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnea.so")
@@ -49,6 +49,12 @@ _lib.nea_attn_bwd_noalloc.argtypes = list(_lib.nea_attn_bwd.argtypes)
 _lib.nea_attn_bwd_noalloc.restype = _i
 _lib.nea_attn_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp]
 _lib.nea_attn_decode.restype = _i
+_lib.nea_attn_saved_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _f]
+_lib.nea_attn_saved_bytes.restype = _ll
+_lib.nea_attn_fwd_save.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp]
+_lib.nea_attn_fwd_save.restype = _i
+_lib.nea_attn_bwd_saved.argtypes = [_vp] * 10 + [_i, _i, _i, _i, _i, _i, _f, _i, _vp]
+_lib.nea_attn_bwd_saved.restype = _i
 _lib.nea_version.argtypes = []
 _lib.nea_version.restype = _i
 
@@ -179,6 +185,84 @@ def nea_attn_bwd_noalloc(q, k, v, o, lse, do, dq, dk, dv, rope_base: float = 100
                                    _stream(stream))
     if rc != NEA_OK:
         raise NeaError(rc, "nea_attn_bwd_noalloc")
+    return dq, dk, dv
+
+
+def nea_attn_saved_bytes(B: int, T: int, Hq: int, Hkv: int, D: int, dtype, rope_base: float = 10000.0) -> int:
+    """Bytes of the save-for-backward buffer (``dtype`` a torch dtype or NEA_F32/NEA_BF16)."""
+    import torch
+
+    code = dtype if isinstance(dtype, int) else {torch.float32: NEA_F32, torch.bfloat16: NEA_BF16}[dtype]
+    n = int(_lib.nea_attn_saved_bytes(B, T, Hq, Hkv, D, code, float(rope_base)))
+    if n < 0:
+        raise NeaError(NEA_ERR_ARG, "nea_attn_saved_bytes")
+    return n
+
+
+def _check_saved(saved, need, device):
+    if need == 0:
+        return
+    if saved is None or not saved.is_cuda or saved.device != device or not saved.is_contiguous():
+        raise ValueError(f"saved must be a contiguous CUDA tensor on {device}")
+    if saved.numel() * saved.element_size() < need:
+        raise ValueError(f"saved holds {saved.numel() * saved.element_size()} bytes, needs {need}")
+
+
+def nea_attn_fwd_save(q, k, v, rope_base: float = 10000.0, causal: bool = True, o=None, lse=None, saved=None,
+                      stream=None):
+    """Forward that keeps its operand planes for the backward: returns
+    ``(o, lse, saved)``; ``saved`` (a uint8 CUDA tensor of
+    ``nea_attn_saved_bytes`` bytes) is passed to ``nea_attn_bwd_saved``."""
+    import torch
+
+    B, T, Hq, Hkv, D = _shapes(q, k, v)
+    dev, dt = q.device, q.dtype
+    code = _dtype_code(q)
+    _check(q, "q", (B, T, Hq, D), dt, dev)
+    _check(k, "k", (B, T, Hkv, D), dt, dev)
+    _check(v, "v", (B, T, Hkv, D), dt, dev)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, T), dtype=torch.float32, device=dev)
+    _check(o, "o", (B, T, Hq, D), dt, dev)
+    _check(lse, "lse", (B, Hq, T), torch.float32, dev)
+    need = nea_attn_saved_bytes(B, T, Hq, Hkv, D, code, rope_base)
+    if saved is None:
+        saved = torch.empty(need, dtype=torch.uint8, device=dev)
+    _check_saved(saved, need, dev)
+    rc = _lib.nea_attn_fwd_save(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(saved), B, T, Hq, Hkv, D, code,
+                                float(rope_base), int(bool(causal)), _stream(stream))
+    if rc != NEA_OK:
+        raise NeaError(rc, "nea_attn_fwd_save")
+    return o, lse, saved
+
+
+def nea_attn_bwd_saved(q, k, v, o, lse, do, saved, rope_base: float = 10000.0, causal: bool = True,
+                       dq=None, dk=None, dv=None, stream=None):
+    """Backward reading Q, K, V operands from ``saved`` (what ``nea_attn_fwd_save``
+    wrote for the same q, k, v and rope_base): returns ``(dq, dk, dv)``."""
+    import torch
+
+    B, T, Hq, Hkv, D = _shapes(q, k, v)
+    dev, dt = q.device, q.dtype
+    code = _dtype_code(q)
+    for t, n, shp in ((q, "q", (B, T, Hq, D)), (k, "k", (B, T, Hkv, D)), (v, "v", (B, T, Hkv, D)),
+                      (o, "o", (B, T, Hq, D)), (do, "do", (B, T, Hq, D))):
+        _check(t, n, shp, dt, dev)
+    _check(lse, "lse", (B, Hq, T), torch.float32, dev)
+    _check_saved(saved, nea_attn_saved_bytes(B, T, Hq, Hkv, D, code, rope_base), dev)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check(dq, "dq", (B, T, Hq, D), dt, dev)
+    _check(dk, "dk", (B, T, Hkv, D), dt, dev)
+    _check(dv, "dv", (B, T, Hkv, D), dt, dev)
+    rc = _lib.nea_attn_bwd_saved(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(saved), _ptr(dq),
+                                 _ptr(dk), _ptr(dv), B, T, Hq, Hkv, D, code, float(rope_base), int(bool(causal)),
+                                 _stream(stream))
+    if rc != NEA_OK:
+        raise NeaError(rc, "nea_attn_bwd_saved")
     return dq, dk, dv
 
 

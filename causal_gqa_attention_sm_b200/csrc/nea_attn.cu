@@ -297,26 +297,13 @@ size_t prep_bytes(const size_t* elems, const int* rot, int n, bool f32, bool rop
   return b;
 }
 
-// Carves the prologue's outputs out of `base` (prep_bytes() bytes) and runs
-// it.  jobs_out[i].hi (and .lo for float32 storage) are the operand tensors
-// the attention kernels read: for bfloat16 storage the rotated copy or, for
-// tensors left as they are, the input itself.
-int run_prep(uint8_t* base, const void* const* src, const size_t* elems, const int* H, const int* rot, int n,
-             int T, int D, bool f32, const float2* table, nea::PrepJob* jobs_out, cudaStream_t stream,
-             const nea::PrepParams* rowterm = nullptr) {
-  nea::PrepParams pp{};
-  if (rowterm) pp = *rowterm;  // row-term fields of the backward
-  pp.n_jobs = 0;
-  pp.total = 0;
-  pp.prep_blocks = 0;
+// Carves the prologue's outputs for `n` tensors out of `base` (prep_bytes()
+// bytes, same order).  jobs[i].hi (and .lo for float32 storage) are the
+// operand tensors the attention kernels read: for bfloat16 storage the
+// rotated copy or, for tensors left as they are, the input itself.
+void carve_planes(uint8_t* base, const void* const* src, const size_t* elems, const int* H, const int* rot, int n,
+                  int D, bool f32, const float2* table, nea::PrepJob* jobs) {
   size_t off = 0;
-  pp.T = T;
-  pp.rope = table;
-  pp.divT = nea::make_fastdiv(uint32_t(T));
-  if (pp.rt_threads) {
-    pp.divTp = nea::make_fastdiv(uint32_t(pp.Tp));
-    pp.divHq = nea::make_fastdiv(uint32_t(pp.Hq));
-  }
   for (int i = 0; i < n; ++i) {
     nea::PrepJob j{};
     j.src = src[i];
@@ -325,7 +312,7 @@ int run_prep(uint8_t* base, const void* const* src, const size_t* elems, const i
     j.rope = rot[i] && table != nullptr;
     if (!f32 && !j.rope) {  // read in place
       j.hi = static_cast<__nv_bfloat16*>(const_cast<void*>(src[i]));
-      jobs_out[i] = j;
+      jobs[i] = j;
       continue;
     }
     j.hi = reinterpret_cast<__nv_bfloat16*>(base + off);
@@ -336,12 +323,34 @@ int run_prep(uint8_t* base, const void* const* src, const size_t* elems, const i
     }
     j.chunks = static_cast<long long>(elems[i] / (f32 ? 4 : 8));
     j.rows = static_cast<int>(elems[i] / D);
-    const int rows_per_block = 256 / (D * (f32 ? 4 : 2) / 16) * nea::kPrepUnroll;
+    jobs[i] = j;
+  }
+}
+
+// Runs the prologue over the jobs with run[i] set that have planes to write
+// (and, with `rowterm`, the backward row terms in the same launch).
+int launch_prep(const nea::PrepJob* jobs, const bool* run, int n, int T, int D, bool f32, const float2* table,
+                cudaStream_t stream, const nea::PrepParams* rowterm = nullptr) {
+  nea::PrepParams pp{};
+  if (rowterm) pp = *rowterm;  // row-term fields of the backward
+  pp.n_jobs = 0;
+  pp.total = 0;
+  pp.prep_blocks = 0;
+  pp.T = T;
+  pp.rope = table;
+  pp.divT = nea::make_fastdiv(uint32_t(T));
+  if (pp.rt_threads) {
+    pp.divTp = nea::make_fastdiv(uint32_t(pp.Tp));
+    pp.divHq = nea::make_fastdiv(uint32_t(pp.Hq));
+  }
+  const int rows_per_block = 256 / (D * (f32 ? 4 : 2) / 16) * nea::kPrepUnroll;
+  for (int i = 0; i < n; ++i) {
+    if (!run[i] || jobs[i].rows == 0) continue;  // nothing to write (in place, or planes made elsewhere)
+    nea::PrepJob j = jobs[i];
     j.block0 = pp.prep_blocks;
     pp.prep_blocks += (j.rows + rows_per_block - 1) / rows_per_block;
     pp.job[pp.n_jobs++] = j;
     pp.total += j.chunks;
-    jobs_out[i] = j;
   }
   const long long blocks = pp.prep_blocks + (pp.rt_threads + 255) / 256;
   if (blocks == 0) return NEA_OK;
@@ -350,6 +359,15 @@ int run_prep(uint8_t* base, const void* const* src, const size_t* elems, const i
                       : (f32 ? nea::attn_prep_kernel<32, true> : nea::attn_prep_kernel<32, false>);
   const cudaError_t e = launch_dependent(kern, g, 256, 0, stream, pp);
   return e == cudaSuccess ? NEA_OK : cuda_fail(e);
+}
+
+// Carves and runs the prologue for all `n` tensors.
+int run_prep(uint8_t* base, const void* const* src, const size_t* elems, const int* H, const int* rot, int n,
+             int T, int D, bool f32, const float2* table, nea::PrepJob* jobs_out, cudaStream_t stream,
+             const nea::PrepParams* rowterm = nullptr) {
+  carve_planes(base, src, elems, H, rot, n, D, f32, table, jobs_out);
+  const bool run[4] = {true, true, true, true};
+  return launch_prep(jobs_out, run, n, T, D, f32, table, stream, rowterm);
 }
 
 // ----------------------------------------------------------------- forward
@@ -398,20 +416,26 @@ int check_bwd_args(const void* Q, const void* K, const void* V, const void* O, c
 // Bytes of backward workspace: the padded row terms, then the operand
 // prologue's output (fp32: planes of Q, K, V, dO; bf16 with the rotation on:
 // rotated Q and K).
-size_t bwd_ws_bytes(int B, int T, int Hq, int Hkv, int D, bool f32, bool rope_on, size_t* rowterm_bytes) {
+// With `saved` planes only dO's share of the prologue output is needed.
+size_t bwd_ws_bytes(int B, int T, int Hq, int Hkv, int D, bool f32, bool rope_on, size_t* rowterm_bytes,
+                    bool saved = false) {
   const size_t Tp = round_up(size_t(T), nea::kTileRows);
   *rowterm_bytes = round_up(size_t(B) * Hq * 2 * Tp * sizeof(float), 256);
   const size_t nq = size_t(B) * T * Hq * D, nk = size_t(B) * T * Hkv * D;
   const size_t elems[4] = {nq, nk, nk, nq};
   const int rot[4] = {1, 1, 0, 0};
+  if (saved) return *rowterm_bytes + prep_bytes(elems + 3, rot + 3, 1, f32, rope_on);
   return *rowterm_bytes + prep_bytes(elems, rot, 4, f32, rope_on);
 }
 
 // The backward after argument checks, given a workspace of bwd_ws_bytes()
 // bytes, a rotary table (or nullptr) and a status word.
+// With `saved` (the planes nea_attn_fwd_save wrote), the prologue converts
+// only dO and writes the row terms; Q, K, V operands come from `saved`.
 int run_bwd(uint32_t& attr_done, uint8_t* ws, const float2* rope, int* status, const void* Q, const void* K,
             const void* V, const void* O, const float* LSE, const void* dO, void* dQ, void* dK, void* dV, int B,
-            int T, int Hq, int Hkv, int D, int dtype, int causal, cudaStream_t stream, bool ev) {
+            int T, int Hq, int Hkv, int D, int dtype, int causal, cudaStream_t stream, bool ev,
+            const uint8_t* saved = nullptr) {
   const bool f32 = dtype == NEA_F32;
   size_t rowterm_bytes = 0;
   (void)bwd_ws_bytes(B, T, Hq, Hkv, D, f32, rope != nullptr, &rowterm_bytes);
@@ -437,7 +461,14 @@ int run_bwd(uint32_t& attr_done, uint8_t* ws, const float2* rope, int* status, c
     rt.Tp = p.Tp;
     rt.Hq = Hq;
     rt.rt_threads = static_cast<long long>(B) * p.Tp * Hq * (D / (f32 ? 4 : 8));
-    if ((rc = run_prep(ws + rowterm_bytes, src, elems, H, rot, 4, T, D, f32, rope, jobs, stream, &rt))) return rc;
+    if (saved) {  // Q, K, V planes from the forward; dO planes in the workspace
+      carve_planes(const_cast<uint8_t*>(saved), src, elems, H, rot, 3, D, f32, rope, jobs);
+      carve_planes(ws + rowterm_bytes, src + 3, elems + 3, H + 3, rot + 3, 1, D, f32, rope, jobs + 3);
+      const bool run[4] = {false, false, false, true};
+      if ((rc = launch_prep(jobs, run, 4, T, D, f32, rope, stream, &rt))) return rc;
+    } else if ((rc = run_prep(ws + rowterm_bytes, src, elems, H, rot, 4, T, D, f32, rope, jobs, stream, &rt))) {
+      return rc;
+    }
     if (ev) prof_record(3, stream);
     if ((rc = make_tile_map(&p.tm_q, jobs[0].hi, B, T, Hq, D)) ||
         (rc = make_tile_map(&p.tm_k, jobs[1].hi, B, T, Hkv, D)) ||
@@ -477,22 +508,32 @@ int run_bwd(uint32_t& attr_done, uint8_t* ws, const float2* rope, int* status, c
   });
 }
 
-}  // namespace
+// Bytes of the forward's operand planes: float32 storage, hi/lo planes of
+// the rotated Q, K and of V; bfloat16 storage with the rotation on, rotated
+// Q and K; otherwise none.
+size_t fwd_plane_bytes(int B, int T, int Hq, int Hkv, int D, bool f32, bool rope_on) {
+  const size_t nq = size_t(B) * T * Hq * D, nk = size_t(B) * T * Hkv * D;
+  const size_t elems[3] = {nq, nk, nk};
+  const int rot[3] = {1, 1, 0};
+  return prep_bytes(elems, rot, 3, f32, rope_on);
+}
 
-extern "C" {
-
-int nea_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int T, int Hq, int Hkv,
-                 int D, int dtype, float rope_base, int causal, void* stream_) {
-  bool empty = false;
-  int rc = check_shape(B, T, Hq, Hkv, D, dtype, causal, &empty);
-  if (rc) return rc;
-  if (empty) return NEA_OK;
+int check_fwd_args(const void* Q, const void* K, const void* V, const void* O, const float* LSE, int B, int T,
+                   int Hq, int Hkv, int D, int dtype, float rope_base, int causal, bool* empty) {
+  int rc = check_shape(B, T, Hq, Hkv, D, dtype, causal, empty);
+  if (rc || *empty) return rc;
   if (!Q || !K || !V || !O || !LSE) return NEA_ERR_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE)) return NEA_ERR_ARG;
   if (!std::isfinite(rope_base)) return NEA_ERR_ARG;
-  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-  const bool f32 = dtype == NEA_F32;
+  return NEA_OK;
+}
 
+// The forward after argument checks; its operand planes go to `saved` when
+// given, else to the device workspace.
+int run_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int T, int Hq, int Hkv, int D,
+            int dtype, float rope_base, int causal, cudaStream_t stream, uint8_t* saved) {
+  const bool f32 = dtype == NEA_F32;
+  int rc;
   std::lock_guard<std::mutex> lock(g_mu);
   DeviceState* st = nullptr;
   if ((rc = device_state(&st))) return rc;
@@ -507,9 +548,13 @@ int nea_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
     const void* src[3] = {Q, K, V};
     const size_t elems[3] = {nq, nk, nk};
     const int H[3] = {Hq, Hkv, Hkv}, rot[3] = {1, 1, 0};
-    if ((rc = ensure_ws(*st, prep_bytes(elems, rot, 3, f32, rope != nullptr)))) return rc;
+    uint8_t* planes = saved;
+    if (!planes) {
+      if ((rc = ensure_ws(*st, fwd_plane_bytes(B, T, Hq, Hkv, D, f32, rope != nullptr)))) return rc;
+      planes = st->ws;
+    }
     nea::PrepJob jobs[3];
-    if ((rc = run_prep(st->ws, src, elems, H, rot, 3, T, D, f32, rope, jobs, stream))) return rc;
+    if ((rc = run_prep(planes, src, elems, H, rot, 3, T, D, f32, rope, jobs, stream))) return rc;
     prof_record(6, stream);
     if ((rc = make_tile_map(&p.tm_q, jobs[0].hi, B, T, Hq, D)) ||
         (rc = make_tile_map(&p.tm_k, jobs[1].hi, B, T, Hkv, D)) ||
@@ -545,6 +590,37 @@ int nea_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
   return rc;
 }
 
+}  // namespace
+
+extern "C" {
+
+int nea_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int T, int Hq, int Hkv,
+                 int D, int dtype, float rope_base, int causal, void* stream) {
+  bool empty = false;
+  int rc = check_fwd_args(Q, K, V, O, LSE, B, T, Hq, Hkv, D, dtype, rope_base, causal, &empty);
+  if (rc || empty) return rc;
+  return run_fwd(Q, K, V, O, LSE, B, T, Hq, Hkv, D, dtype, rope_base, causal, static_cast<cudaStream_t>(stream),
+                 nullptr);
+}
+
+long long nea_attn_saved_bytes(int B, int T, int Hq, int Hkv, int D, int dtype, float rope_base) {
+  bool empty = false;
+  if (check_shape(B, T, Hq, Hkv, D, dtype, 1, &empty) || !std::isfinite(rope_base)) return -1;
+  if (empty) return 0;
+  return static_cast<long long>(fwd_plane_bytes(B, T, Hq, Hkv, D, dtype == NEA_F32, rope_base > 0.f));
+}
+
+int nea_attn_fwd_save(const void* Q, const void* K, const void* V, void* O, float* LSE, void* saved, int B, int T,
+                      int Hq, int Hkv, int D, int dtype, float rope_base, int causal, void* stream) {
+  bool empty = false;
+  int rc = check_fwd_args(Q, K, V, O, LSE, B, T, Hq, Hkv, D, dtype, rope_base, causal, &empty);
+  if (rc || empty) return rc;
+  const bool need = fwd_plane_bytes(B, T, Hq, Hkv, D, dtype == NEA_F32, rope_base > 0.f) > 0;
+  if (need && (!saved || !aligned16(saved))) return NEA_ERR_ARG;
+  return run_fwd(Q, K, V, O, LSE, B, T, Hq, Hkv, D, dtype, rope_base, causal, static_cast<cudaStream_t>(stream),
+                 need ? static_cast<uint8_t*>(saved) : nullptr);
+}
+
 int nea_attn_bwd(const void* Q, const void* K, const void* V, const void* O, const float* LSE, const void* dO,
                  void* dQ, void* dK, void* dV, int B, int T, int Hq, int Hkv, int D, int dtype, float rope_base,
                  int causal, void* stream_) {
@@ -563,6 +639,29 @@ int nea_attn_bwd(const void* Q, const void* K, const void* V, const void* O, con
     return rc;
   return run_bwd(st->attr_done, st->ws, rope, st->err, Q, K, V, O, LSE, dO, dQ, dK, dV, B, T, Hq, Hkv, D, dtype,
                  causal, stream, true);
+}
+
+int nea_attn_bwd_saved(const void* Q, const void* K, const void* V, const void* O, const float* LSE, const void* dO,
+                       const void* saved, void* dQ, void* dK, void* dV, int B, int T, int Hq, int Hkv, int D,
+                       int dtype, float rope_base, int causal, void* stream_) {
+  bool empty = false;
+  int rc = check_bwd_args(Q, K, V, O, LSE, dO, dQ, dK, dV, B, T, Hq, Hkv, D, dtype, rope_base, causal, &empty);
+  if (rc || empty) return rc;
+  const bool f32 = dtype == NEA_F32, rope_on = rope_base > 0.f;
+  if (fwd_plane_bytes(B, T, Hq, Hkv, D, f32, rope_on) == 0)  // nothing was saved: the regular backward
+    return nea_attn_bwd(Q, K, V, O, LSE, dO, dQ, dK, dV, B, T, Hq, Hkv, D, dtype, rope_base, causal, stream_);
+  if (!saved || !aligned16(saved)) return NEA_ERR_ARG;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&st))) return rc;
+  const float2* rope = nullptr;
+  if ((rc = rope_table(*st, T, D, rope_base, stream, &rope))) return rc;
+  size_t rowterm_bytes = 0;
+  if ((rc = ensure_ws(*st, bwd_ws_bytes(B, T, Hq, Hkv, D, f32, rope_on, &rowterm_bytes, true)))) return rc;
+  return run_bwd(st->attr_done, st->ws, rope, st->err, Q, K, V, O, LSE, dO, dQ, dK, dV, B, T, Hq, Hkv, D, dtype,
+                 causal, stream, true, static_cast<const uint8_t*>(saved));
 }
 
 int nea_attn_decode(const void* Q, const void* Kc, const void* Vc, const int* lens, void* O, float* LSE, int B,

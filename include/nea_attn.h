@@ -118,6 +118,42 @@ int nea_attn_bwd(const void* Q, const void* K, const void* V, const void* O, con
                  int causal, void* stream);
 
 /*
+ * Save-for-backward pair.  The forward's operand prologue (rotated Q and K;
+ * for NEA_F32 also the bf16 hi/lo planes of Q, K and V) produces exactly the
+ * operands the backward needs again.  nea_attn_fwd_save writes them into a
+ * caller-owned buffer `saved` instead of the library workspace, and
+ * nea_attn_bwd_saved reads them from there, so the backward's prologue only
+ * converts dO and writes the row terms.
+ *
+ * nea_attn_saved_bytes: the size of `saved` for these arguments (the same for
+ * either value of causal): NEA_F32 4*(B*T*(Hq + 2*Hkv)*D) bytes, each plane
+ * rounded up to 256 bytes; NEA_BF16 with the rotation on, the rotated Q and K
+ * (2*B*T*(Hq + Hkv)*D bytes, rounded likewise); NEA_BF16 with the rotation
+ * off, 0.  Returns -1 for arguments the forward would reject.
+ *
+ * nea_attn_fwd_save: nea_attn_fwd with the planes written to `saved` (device
+ * memory, 16-byte aligned, at least nea_attn_saved_bytes bytes, owned by the
+ * caller; may be NULL when that size is 0).  O and LSE are bit-identical to
+ * nea_attn_fwd's.
+ *
+ * nea_attn_bwd_saved: nea_attn_bwd with Q, K and V operands taken from
+ * `saved`.  `saved` must hold what nea_attn_fwd_save wrote for the same Q, K,
+ * V, B, T, Hq, Hkv, D, dtype and rope_base, and must not have been written
+ * since; Q, K and V are still passed (and checked) but their values are not
+ * read.  With those inputs dQ, dK, dV are bit-identical to nea_attn_bwd's.
+ * The library cannot check the contents of `saved`: stale planes give
+ * gradients of the tensors they were made from.  When the saved size is 0
+ * this is nea_attn_bwd.  Errors as for nea_attn_bwd, plus NEA_ERR_ARG for a
+ * NULL or unaligned `saved` of nonzero size.
+ */
+long long nea_attn_saved_bytes(int B, int T, int Hq, int Hkv, int D, int dtype, float rope_base);
+int nea_attn_fwd_save(const void* Q, const void* K, const void* V, void* O, float* LSE, void* saved, int B, int T,
+                      int Hq, int Hkv, int D, int dtype, float rope_base, int causal, void* stream);
+int nea_attn_bwd_saved(const void* Q, const void* K, const void* V, const void* O, const float* LSE, const void* dO,
+                       const void* saved, void* dQ, void* dK, void* dV, int B, int T, int Hq, int Hkv, int D,
+                       int dtype, float rope_base, int causal, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device status words of the
  * current device: the one the regular entry points write and the one inside
  * the fixed scratch of nea_attn_bwd_noalloc.  Returns NEA_OK, NEA_ERR_TIMEOUT

@@ -72,6 +72,44 @@ def test_empty_problem_is_a_noop(lib):
     assert _bwd(lib, B=0, ptr=None) == 0
 
 
+def _saved_bytes(lib, B=2, T=100, Hq=6, Hkv=2, D=64, dtype=0, base=10000.0):
+    f = lib.nea_attn_saved_bytes
+    f.argtypes = [ctypes.c_int] * 6 + [ctypes.c_float]
+    f.restype = ctypes.c_longlong
+    return f(B, T, Hq, Hkv, D, dtype, base)
+
+
+def test_saved_bytes_closed_form(lib):
+    def r256(x):
+        return (x + 255) // 256 * 256
+
+    nq, nk = 2 * 100 * 6 * 64, 2 * 100 * 2 * 64
+    # float32: hi and lo bf16 planes of rotated Q, K and of V
+    assert _saved_bytes(lib) == 2 * (r256(2 * nq) + 2 * r256(2 * nk))
+    # bfloat16 with the rotation on: rotated Q and K only
+    assert _saved_bytes(lib, dtype=1) == r256(2 * nq) + r256(2 * nk)
+    # bfloat16 without rotation: nothing to save; float32 keeps its planes
+    assert _saved_bytes(lib, dtype=1, base=0.0) == 0
+    assert _saved_bytes(lib, base=0.0) == _saved_bytes(lib)
+    assert _saved_bytes(lib, B=0) == 0
+    assert _saved_bytes(lib, D=48) == -1
+    assert _saved_bytes(lib, base=float("inf")) == -1
+
+
+def test_saved_pair_rejects_missing_buffer(lib):
+    vp = ctypes.c_void_p
+    f = lib.nea_attn_fwd_save
+    f.argtypes = [vp] * 6 + [ctypes.c_int] * 6 + [ctypes.c_float, ctypes.c_int, vp]
+    p = vp(16)
+    assert f(p, p, p, p, p, None, 1, 4, 4, 2, 64, 0, 10000.0, 1, None) == 1   # saved needed, NULL
+    assert f(p, p, p, p, p, vp(24), 1, 4, 4, 2, 64, 0, 10000.0, 1, None) == 1  # misaligned
+    g = lib.nea_attn_bwd_saved
+    g.argtypes = [vp] * 10 + [ctypes.c_int] * 6 + [ctypes.c_float, ctypes.c_int, vp]
+    assert g(p, p, p, p, p, p, None, p, p, p, 1, 4, 4, 2, 64, 0, 10000.0, 1, None) == 1
+    assert g(p, p, p, p, p, p, p, p, p, p, 1, 4, 4, 2, 48, 0, 10000.0, 1, None) == 1
+    assert g(*([None] * 10), 0, 4, 4, 2, 64, 0, 10000.0, 1, None) == 0  # empty: no-op
+
+
 def test_status_strings(lib):
     lib.nea_status_string.restype = ctypes.c_char_p
     for code in range(6):
