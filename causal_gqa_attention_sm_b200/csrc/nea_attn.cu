@@ -55,7 +55,7 @@ struct DeviceState {
   // runs, so in-flight kernels on any stream keep valid pointers
   std::map<std::tuple<int, int, uint32_t>, float2*> rope;
   uint32_t attr_done = 0;      // bitmask of kernels whose smem attribute is set
-  uint64_t attr_dec = 0;       // the same for the decode split kernels
+  uint64_t attr_dec = 0;       // the same for the decode kernels
   int n_sm = 148;              // streaming multiprocessors
 };
 
@@ -103,21 +103,26 @@ int make_tile_map(CUtensorMap* m, const void* base, int B, int T, int H, int D) 
   return r == CUDA_SUCCESS ? NEA_OK : NEA_ERR_CUDA;
 }
 
-// Descriptor of a decode cache [B][Tc][Hkv][D] (fp32 or bf16), box
-// {D, 1, 128, 1}: 128 consecutive positions of one kv head, rows contiguous
-// in shared memory (no swizzle), positions past Tc read as zero.
-int make_cache_map(CUtensorMap* m, const void* base, int B, int Tc, int Hkv, int D, bool f32) {
+// Descriptor of a decode cache [B][Tc][Hkv][D] (fp32 or bf16), described
+// with its dimensions in the order (D, position, kv head, sequence), box
+// {min(D, 128 bytes), rows, heads, 1}: `rows` consecutive positions of
+// `heads` neighbouring kv heads, landing in shared memory head-major (fp32
+// with D = 64 takes two boxes per piece, one per column half), each
+// (head, position) line 128 bytes with the 128-byte swizzle or 64 bytes with
+// the 64-byte swizzle; positions past Tc read as zero.
+int make_cache_map(CUtensorMap* m, const void* base, int B, int Tc, int Hkv, int D, bool f32, int heads, int rows) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (!enc) return NEA_ERR_CUDA;
   const cuuint64_t e = f32 ? 4 : 2;
-  const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(Hkv), cuuint64_t(Tc), cuuint64_t(B)};
-  const cuuint64_t strides[3] = {D * e, cuuint64_t(Hkv) * D * e, cuuint64_t(Tc) * Hkv * D * e};
-  const cuuint32_t box[4] = {cuuint32_t(D), 1, cuuint32_t(nea::kDecChunk), 1};
+  const cuuint32_t row_bytes = D * e < 128 ? cuuint32_t(D * e) : 128u;  // one swizzle atom row
+  const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(Tc), cuuint64_t(Hkv), cuuint64_t(B)};
+  const cuuint64_t strides[3] = {cuuint64_t(Hkv) * D * e, D * e, cuuint64_t(Tc) * Hkv * D * e};
+  const cuuint32_t box[4] = {cuuint32_t(row_bytes / e), cuuint32_t(rows), cuuint32_t(heads), 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   const CUresult r = enc(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
                          const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                         CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                         row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? NEA_OK : NEA_ERR_CUDA;
 }
 
@@ -677,9 +682,12 @@ int nea_attn_decode(const void* Q, const void* Kc, const void* Vc, const int* le
   if (!aligned16(Q) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(O) || !aligned16(LSE) ||
       (reinterpret_cast<uintptr_t>(lens) & 3u))
     return NEA_ERR_ARG;
-  const int n_split = (Tc + nea::kDecChunk - 1) / nea::kDecChunk;
-  const size_t part_bytes = round_up(size_t(B) * Hq * n_split * (D + 2) * sizeof(float), 256);
-  const size_t count_bytes = size_t(B) * Hkv * sizeof(int);
+  const int G = Hq / Hkv;
+  const int HP = nea::dec_heads_per_piece(Hkv, G, D, dtype == NEA_F32);
+  const int R = nea::dec_lines(G, D, dtype == NEA_F32) / HP;
+  const int NP = (Tc + R - 1) / R;
+  const unsigned long long n_pieces = static_cast<unsigned long long>(B) * (Hkv / HP) * NP;
+  const size_t part_bytes = round_up(size_t(n_pieces) * nea::kDecWarps * G * (D + 2) * sizeof(float), 256);
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
 
   std::lock_guard<std::mutex> lock(g_mu);
@@ -688,56 +696,69 @@ int nea_attn_decode(const void* Q, const void* Kc, const void* Vc, const int* le
   if (rc) return rc;
   nea::DecodeParams p{};
   if ((rc = rope_table(*st, Tc, D, rope_base, stream, &p.rope))) return rc;
-  if ((rc = ensure_ws(*st, part_bytes + count_bytes))) return rc;
+  if ((rc = ensure_ws(*st, part_bytes))) return rc;
   p.Q = Q;
   p.lens = lens;
   p.O = O;
   p.LSE = LSE;
   p.part = reinterpret_cast<float*>(st->ws);
-  p.count = reinterpret_cast<int*>(st->ws + part_bytes);
-  cudaError_t em = cudaMemsetAsync(p.count, 0, count_bytes, stream);
-  if (em != cudaSuccess) return cuda_fail(em);
   p.B = B;
   p.Tc = Tc;
   p.Hq = Hq;
   p.Hkv = Hkv;
-  p.G = Hq / Hkv;
-  p.n_split = n_split;
+  p.G = G;
+  p.HP = HP;
+  p.NHG = Hkv / HP;
+  p.WPH = nea::kDecWarps / HP;
+  p.R = R;
+  p.NP = NP;
+  p.n_pieces = n_pieces;
+  p.n_cta = static_cast<int>(std::min<unsigned long long>(
+      n_pieces, static_cast<unsigned long long>(std::min(st->n_sm, nea::kDecMaxSeg - 1))));
   p.scale_log2 = float(1.4426950408889634 / std::sqrt(double(D)));
   p.err = st->err;
   p.wait_limit = static_cast<unsigned long long>(t_wait_limit_ns);
-  if ((rc = make_cache_map(&p.tm_k, Kc, B, Tc, Hkv, D, dtype == NEA_F32)) ||
-      (rc = make_cache_map(&p.tm_v, Vc, B, Tc, Hkv, D, dtype == NEA_F32)))
+  if ((rc = make_cache_map(&p.tm_k, Kc, B, Tc, Hkv, D, dtype == NEA_F32, HP, R)) ||
+      (rc = make_cache_map(&p.tm_v, Vc, B, Tc, Hkv, D, dtype == NEA_F32, HP, R)))
     return rc;
-  const dim3 grid(static_cast<unsigned>(n_split), static_cast<unsigned>(Hkv), static_cast<unsigned>(B));
   rc = dispatch(D, dtype, [&](auto d, auto f) {
     constexpr int DD = decltype(d)::value;
     constexpr bool FF = decltype(f)::value;
-    using S = nea::DecSmem<DD, FF>;
     auto launch = [&](auto gtag) -> int {
       constexpr int GG = decltype(gtag)::value;
-      auto kern = nea::attn_decode_split_kernel<DD, FF, GG>;
+      using L = nea::DecLayout<DD, FF, GG>;
+      auto kern = nea::attn_decode_kernel<DD, FF, GG>;
       const int bit = ((DD == 64) * 2 + FF) * 8 + (GG - 1);
       if (!(st->attr_dec >> bit & 1)) {
-        const cudaError_t ea = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(S::kBytes));
+        // both kernels ask for the largest shared-memory carveout, so that
+        // the SMs keep one configuration from the stream to the merge
+        cudaError_t ea = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(L::kAlloc));
+        if (ea == cudaSuccess)
+          ea = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, int(cudaSharedmemCarveoutMaxShared));
+        if (ea == cudaSuccess)
+          ea = cudaFuncSetAttribute(nea::attn_decode_merge_kernel<DD, FF, GG>,
+                                    cudaFuncAttributePreferredSharedMemoryCarveout, int(cudaSharedmemCarveoutMaxShared));
         if (ea != cudaSuccess) return cuda_fail(ea);
         st->attr_dec |= uint64_t(1) << bit;
       }
-      kern<<<grid, 128, S::kBytes, stream>>>(p);
-      return NEA_OK;
+      kern<<<unsigned(p.n_cta), nea::kDecThreads, L::kAlloc, stream>>>(p);
+      const cudaError_t ek = cudaGetLastError();
+      if (ek != cudaSuccess) return cuda_fail(ek);
+      // the merge, one CTA per (sequence, kv head), resident while the stream drains
+      const cudaError_t em = launch_dependent(nea::attn_decode_merge_kernel<DD, FF, GG>, unsigned(B * Hkv),
+                                              unsigned(nea::dec_merge_groups(GG, DD) * GG * DD), 0, stream, p);
+      return em == cudaSuccess ? NEA_OK : cuda_fail(em);
     };
-    int r2;
     switch (p.G) {
-      case 1: r2 = launch(std::integral_constant<int, 1>{}); break;
-      case 2: r2 = launch(std::integral_constant<int, 2>{}); break;
-      case 3: r2 = launch(std::integral_constant<int, 3>{}); break;
-      case 4: r2 = launch(std::integral_constant<int, 4>{}); break;
-      case 5: r2 = launch(std::integral_constant<int, 5>{}); break;
-      case 6: r2 = launch(std::integral_constant<int, 6>{}); break;
-      case 7: r2 = launch(std::integral_constant<int, 7>{}); break;
-      default: r2 = launch(std::integral_constant<int, 8>{}); break;
+      case 1: return launch(std::integral_constant<int, 1>{});
+      case 2: return launch(std::integral_constant<int, 2>{});
+      case 3: return launch(std::integral_constant<int, 3>{});
+      case 4: return launch(std::integral_constant<int, 4>{});
+      case 5: return launch(std::integral_constant<int, 5>{});
+      case 6: return launch(std::integral_constant<int, 6>{});
+      case 7: return launch(std::integral_constant<int, 7>{});
+      default: return launch(std::integral_constant<int, 8>{});
     }
-    return r2;
   });
   if (rc) return rc;
   const cudaError_t e = cudaGetLastError();

@@ -87,6 +87,17 @@ CASES = [
     (2, 257, 4, 2, 32, "f32", [257, 256]),
     (2, 257, 8, 1, 32, "bf16", [1, 200]),
     (4, 128, 6, 6, 64, "bf16", [128, 127, 64, 0]),
+    # G = 4 .. 7 (lanes per row 4 or 8, pieces of 64 or 32 rows)
+    (2, 190, 8, 2, 64, "f32", [190, 31]),
+    (2, 190, 10, 2, 64, "bf16", [33, 190]),
+    (2, 150, 12, 2, 32, "f32", [150, 65]),
+    (2, 150, 14, 2, 32, "bf16", [1, 150]),
+    # one (sequence, kv head) spread over every CTA (ranges of a few pieces each)
+    (1, 20000, 3, 1, 64, "bf16", [19999]),
+    (1, 9000, 3, 1, 64, "f32", [9000]),
+    # many short sequences: one CTA's range crosses several (sequence, kv head) pairs
+    (300, 70, 6, 2, 32, "bf16", [(7 * i) % 71 for i in range(300)]),
+    (40, 5, 8, 2, 64, "f32", [i % 6 for i in range(40)]),
 ]
 
 
@@ -97,6 +108,19 @@ def test_decode_parity(cuda_lib, case):
     q, kc, v, ln, base, o_ref, lse_ref = _case(B, Tc, Hq, Hkv, D, dtype, lens, seed=sum(lens) + Tc)
     o, lse = _run(cuda_lib, q, kc, v, ln, base)
     _compare(o, lse, o_ref, lse_ref, dtype)
+
+
+@pytest.mark.gpu
+def test_decode_calls_of_different_shapes_in_turn(cuda_lib):
+    """The per-(sequence, kv head) piece counts are left at zero by every call:
+    calls of different shapes, one after another on one stream, each match the
+    oracle."""
+    cases = [(3, 300, 12, 4, 64, "f32", [300, 1, 0]), (9, 1000, 6, 3, 64, "bf16", [1000, 999, 500] * 3),
+             (3, 300, 12, 4, 64, "f32", [300, 1, 0]), (1, 64, 2, 2, 32, "f32", [64])]
+    prepared = [_case(*c, seed=17 + i) for i, c in enumerate(cases)]
+    for c, (q, kc, v, ln, base, o_ref, lse_ref) in zip(cases, prepared):
+        o, lse = _run(cuda_lib, q, kc, v, ln, base)
+        _compare(o, lse, o_ref, lse_ref, c[5])
 
 
 @pytest.mark.gpu
