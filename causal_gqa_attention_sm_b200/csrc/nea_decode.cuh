@@ -169,6 +169,23 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
       : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
 }
 
+// A 4-D tile copy like tma_load_4d, with an L2 eviction policy: the cache is
+// read once, so its lines are marked evict-first and do not push out what
+// the call reads again (partials, queries, lengths).
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void tma_load_4d_hint(void* dst, const void* tmap, int c0, int c1, int c2, int c3,
+                                                 uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(smem_u32(dst)),
+      "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
 // Partial of consumer warp `warp`, query head gi of its kv head, for the
 // range of (sequence, head group) bhg that starts at piece k0.
 __device__ __forceinline__ float* dec_partial(const DecodeParams& p, int bhg, int k0, int warp, int gi, int D) {
@@ -304,6 +321,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
   if (warp == kDecWarps) {
     if (lane != 0) return;
     const uint32_t q_bytes = uint32_t(p.HP) * G * D * L::E;
+    const uint64_t stream_policy = l2_evict_first_policy();
     uint32_t it = 0;
     bool ok = true;
     for (unsigned long long q = lo; q < hi && ok;) {
@@ -323,8 +341,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
         mbar_arrive_expect_tx(&full[s], L::kAuxOff + aux);
 #pragma unroll
         for (int a = 0; a < L::NA; ++a) {
-          tma_load_4d(st + a * L::kArray, &p.tm_k, a * L::EPA, k * p.R, hg * p.HP, b, &full[s]);
-          tma_load_4d(st + (L::NA + a) * L::kArray, &p.tm_v, a * L::EPA, k * p.R, hg * p.HP, b, &full[s]);
+          tma_load_4d_hint(st + a * L::kArray, &p.tm_k, a * L::EPA, k * p.R, hg * p.HP, b, &full[s], stream_policy);
+          tma_load_4d_hint(st + (L::NA + a) * L::kArray, &p.tm_v, a * L::EPA, k * p.R, hg * p.HP, b, &full[s],
+                           stream_policy);
         }
         if (first) {  // the head group's query rows and the rotary row of position len - 1
           bulk_load(st + L::kAuxOff,
