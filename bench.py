@@ -47,18 +47,20 @@ def prologue_bytes(w, kernel):
     """Algorithmic HBM bytes of one operand-prologue launch: every input
     element read once and every output element written once.  The forward's
     prologue converts Q, K, V (bf16 storage: rotates Q, K); the backward's, fed
-    the saved planes, converts only dO (nothing for bf16 storage)."""
+    the saved planes, writes the row terms and (fp32 storage) dO's planes."""
     nq, nk = w.B * w.T * w.Hq * w.D, w.B * w.T * w.Hkv * w.D
     rope = w.rope_base > 0
-    if w.dtype == "f32":  # fp32 in, bf16 hi + lo out
-        conv = (nq + 2 * nk) if kernel == "attn_fwd_prologue" else nq
-        b = conv * (4 + 4)
-    else:  # rotated bf16 copies of Q, K in the forward
-        b = (nq + nk) * (2 + 2) if rope and kernel == "attn_fwd_prologue" else 0
-    if kernel == "attn_bwd_prologue":  # row terms: read O, dO, LSE; write ws[B*Hq][2][Tp]
-        e = 4 if w.dtype == "f32" else 2
-        tp = -(-w.T // 128) * 128
-        b += 2 * nq * e + 4 * w.B * w.Hq * w.T + 8 * w.B * w.Hq * tp
+    e = 4 if w.dtype == "f32" else 2
+    if kernel == "attn_fwd_prologue":
+        if w.dtype == "f32":  # fp32 in, bf16 hi + lo out
+            return (nq + 2 * nk) * (4 + 4)
+        return (nq + nk) * (2 + 2) if rope else 0  # rotated bf16 copies of Q, K
+    # backward: row terms read O, dO (once) and LSE and write ws[B*Hq][2][Tp];
+    # for fp32 storage the same pass writes dO's bf16 hi + lo planes
+    tp = -(-w.T // 128) * 128
+    b = 2 * nq * e + 4 * w.B * w.Hq * w.T + 8 * w.B * w.Hq * tp
+    if w.dtype == "f32":
+        b += nq * 4
     return b
 
 

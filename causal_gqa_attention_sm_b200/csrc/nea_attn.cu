@@ -344,7 +344,7 @@ int launch_prep(const nea::PrepJob* jobs, const bool* run, int n, int T, int D, 
   pp.T = T;
   pp.rope = table;
   pp.divT = nea::make_fastdiv(uint32_t(T));
-  if (pp.rt_threads) {
+  if (pp.rt_rows) {
     pp.divTp = nea::make_fastdiv(uint32_t(pp.Tp));
     pp.divHq = nea::make_fastdiv(uint32_t(pp.Hq));
   }
@@ -357,7 +357,11 @@ int launch_prep(const nea::PrepJob* jobs, const bool* run, int n, int T, int D, 
     pp.job[pp.n_jobs++] = j;
     pp.total += j.chunks;
   }
-  const long long blocks = pp.prep_blocks + (pp.rt_threads + 255) / 256;
+  const long long rt_blocks = D == 64 ? (f32 ? nea::rowterm_blocks<64, true>(pp.rt_rows)
+                                                : nea::rowterm_blocks<64, false>(pp.rt_rows))
+                                      : (f32 ? nea::rowterm_blocks<32, true>(pp.rt_rows)
+                                             : nea::rowterm_blocks<32, false>(pp.rt_rows));
+  const long long blocks = pp.prep_blocks + rt_blocks;
   if (blocks == 0) return NEA_OK;
   const unsigned g = unsigned(blocks);
   auto kern = D == 64 ? (f32 ? nea::attn_prep_kernel<64, true> : nea::attn_prep_kernel<64, false>)
@@ -465,15 +469,17 @@ int run_bwd(uint32_t& attr_done, uint8_t* ws, const float2* rope, int* status, c
     rt.B = B;
     rt.Tp = p.Tp;
     rt.Hq = Hq;
-    rt.rt_threads = static_cast<long long>(B) * p.Tp * Hq * (D / (f32 ? 4 : 8));
-    if (saved) {  // Q, K, V planes from the forward; dO planes in the workspace
-      carve_planes(const_cast<uint8_t*>(saved), src, elems, H, rot, 3, D, f32, rope, jobs);
-      carve_planes(ws + rowterm_bytes, src + 3, elems + 3, H + 3, rot + 3, 1, D, f32, rope, jobs + 3);
-      const bool run[4] = {false, false, false, true};
-      if ((rc = launch_prep(jobs, run, 4, T, D, f32, rope, stream, &rt))) return rc;
-    } else if ((rc = run_prep(ws + rowterm_bytes, src, elems, H, rot, 4, T, D, f32, rope, jobs, stream, &rt))) {
-      return rc;
-    }
+    rt.rt_rows = static_cast<long long>(B) * p.Tp * Hq;
+    // Q, K, V planes from the forward (`saved`) or made here; dO's planes
+    // (float32 storage) are written by the row-term threads, which read dO
+    if (saved) carve_planes(const_cast<uint8_t*>(saved), src, elems, H, rot, 3, D, f32, rope, jobs);
+    else carve_planes(ws + rowterm_bytes, src, elems, H, rot, 3, D, f32, rope, jobs);
+    const size_t q_planes = saved ? 0 : prep_bytes(elems, rot, 3, f32, rope != nullptr);
+    carve_planes(ws + rowterm_bytes + q_planes, src + 3, elems + 3, H + 3, rot + 3, 1, D, f32, rope, jobs + 3);
+    rt.do_hi = f32 ? jobs[3].hi : nullptr;
+    rt.do_lo = f32 ? jobs[3].lo : nullptr;
+    const bool run[4] = {!saved, !saved, !saved, false};
+    if ((rc = launch_prep(jobs, run, 4, T, D, f32, rope, stream, &rt))) return rc;
     if (ev) prof_record(3, stream);
     if ((rc = make_tile_map(&p.tm_q, jobs[0].hi, B, T, Hq, D)) ||
         (rc = make_tile_map(&p.tm_k, jobs[1].hi, B, T, Hkv, D)) ||

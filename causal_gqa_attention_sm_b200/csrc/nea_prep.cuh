@@ -9,7 +9,9 @@
 //   - bfloat16 storage: Q and K are rotated into bf16 copies (V and dO are
 //     read in place).  Reads 2 bytes and writes 2 per element.
 // In the backward the same launch also writes the per-row terms of every
-// query row (below).  Everything here is bound by HBM bandwidth.
+// query row (below); for float32 storage the threads that read dO for them
+// also write its hi/lo planes, so dO is read once.  Everything here is bound
+// by HBM bandwidth.
 #pragma once
 
 #include "nea_device.cuh"
@@ -35,13 +37,15 @@ struct PrepParams {
   const float2* rope;     // [T][D/2] (cos, sin) or nullptr
   long long total;        // sum of chunks
   int prep_blocks;        // blocks [0, prep_blocks) rotate/split, kPrepUnroll rows' chunks per thread
-  // backward row terms (rt_threads == 0: none), blocks from prep_blocks on
+  // backward row terms (rt_rows == 0: none), blocks from prep_blocks on
   const void* O;
   const void* dO;
   const float* LSE;
   float* ws;
+  __nv_bfloat16* do_hi;   // float32 storage: dO's bf16 planes, written with the row terms
+  __nv_bfloat16* do_lo;
   int B, Tp, Hq;
-  long long rt_threads;
+  long long rt_rows;      // B * Tp * Hq
   FastDiv divT, divTp, divHq;
 };
 
@@ -52,48 +56,85 @@ constexpr int kPrepUnroll = 4;  // 16-byte chunks in flight per thread
 // rounded up to whole 128-row tiles, so a tile of it is one TMA box):
 //   ws[bh][0][t] = -LSE[b][h][t] * log2(e)          (-inf for t >= T)
 //   ws[bh][1][t] = Dv = sum_d dO[b][t][h][d] O[b][t][h][d]   (0 for t >= T)
-// The padding makes P = exp2(s*c + ws0) vanish for queries past T.  One group
-// of D/ELEMS lanes per (b, t, h) row, t over [0, Tp).
+// The padding makes P = exp2(s*c + ws0) vanish for queries past T.  A group
+// of D/ELEMS consecutive lanes takes one (b, t, h) row, t over [0, Tp), one
+// 16-byte chunk of O and dO per lane; each thread takes kPrepUnroll rows of
+// the block (kSlots rows apart) with all their loads in flight at once.
 template <int D, bool F32IO>
-__device__ __forceinline__ void rowterm_lane(const PrepParams& p, long long gtid) {
+__device__ __forceinline__ void rowterm_block(const PrepParams& p, long long rb) {
   constexpr int kElems = F32IO ? 4 : 8;    // elements per 16-byte chunk
   constexpr int kLanes = D / kElems;       // lanes per row: 4, 8 or 16
-  if (gtid >= p.rt_threads) return;        // whole groups of lanes leave together
-  const uint32_t prow = uint32_t(gtid / kLanes);  // (b, t, h) over t in [0, Tp)
-  const int c = int(gtid % kLanes);
-  const uint32_t bt = fdiv(prow, p.divHq);
-  const int h = int(prow - bt * uint32_t(p.Hq));
-  const uint32_t bq = fdiv(bt, p.divTp);
-  const int t = int(bt - bq * uint32_t(p.Tp));
-  const long long b = bq;
-  float* out = p.ws + (b * p.Hq + h) * 2 * (long long)p.Tp + t;
-  if (t >= p.T) {
-    if (c == 0) {
-      out[0] = -INFINITY;
-      out[p.Tp] = 0.f;
-    }
-    return;
+  constexpr int kSlots = 256 / kLanes;     // rows per block step
+  constexpr int kRowBytes = D * (F32IO ? 4 : 2);
+  const int c = int(threadIdx.x) % kLanes, slot = int(threadIdx.x) / kLanes;
+  uint4 a[kPrepUnroll], z[kPrepUnroll];
+  long long row[kPrepUnroll];  // (b, t, h) row of O and dO; -1: padding row (t >= T); -2: past the end
+  float* out[kPrepUnroll];
+  int bh_t[kPrepUnroll];
+#pragma unroll
+  for (int u = 0; u < kPrepUnroll; ++u) {
+    const long long prow = (rb * kPrepUnroll + u) * kSlots + slot;  // (b, t, h) over t in [0, Tp)
+    row[u] = -2;
+    if (prow >= p.rt_rows) continue;
+    const uint32_t bt = fdiv(uint32_t(prow), p.divHq);
+    const int h = int(uint32_t(prow) - bt * uint32_t(p.Hq));
+    const uint32_t bq = fdiv(bt, p.divTp);
+    const int t = int(bt - bq * uint32_t(p.Tp));
+    const long long b = bq;
+    out[u] = p.ws + (b * p.Hq + h) * 2 * (long long)p.Tp + t;
+    bh_t[u] = int((b * p.Hq + h) * (long long)p.T + t);
+    row[u] = -1;
+    if (t >= p.T) continue;
+    row[u] = (b * p.T + t) * p.Hq + h;
+    a[u] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.O) + row[u] * kRowBytes) + c);
+    z[u] = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.dO) + row[u] * kRowBytes) + c);
   }
-  const long long row = (b * p.T + t) * p.Hq + h;
-  const uint4 a = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.O) + row * D * (F32IO ? 4 : 2)) + c);
-  const uint4 z = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.dO) + row * D * (F32IO ? 4 : 2)) + c);
-  float acc;
-  if constexpr (F32IO) {
-    acc = __uint_as_float(a.x) * __uint_as_float(z.x) + __uint_as_float(a.y) * __uint_as_float(z.y) +
-          __uint_as_float(a.z) * __uint_as_float(z.z) + __uint_as_float(a.w) * __uint_as_float(z.w);
-  } else {
-    acc = bf16_lo_f(a.x) * bf16_lo_f(z.x) + bf16_hi_f(a.x) * bf16_hi_f(z.x) + bf16_lo_f(a.y) * bf16_lo_f(z.y) +
-          bf16_hi_f(a.y) * bf16_hi_f(z.y) + bf16_lo_f(a.z) * bf16_lo_f(z.z) + bf16_hi_f(a.z) * bf16_hi_f(z.z) +
-          bf16_lo_f(a.w) * bf16_lo_f(z.w) + bf16_hi_f(a.w) * bf16_hi_f(z.w);
-  }
-  // the kLanes lanes of a row are consecutive and leave or stay together
+  // the kLanes lanes of a row are consecutive and share its row index
   const unsigned group = (kLanes == 32 ? kFullMask : ((1u << kLanes) - 1u) << (threadIdx.x & 31 & ~(kLanes - 1)));
 #pragma unroll
-  for (int off = kLanes / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(group, acc, off);
-  if (c == 0) {
-    out[0] = __ldg(p.LSE + (b * p.Hq + h) * (long long)p.T + t) * -1.4426950408889634f;
-    out[p.Tp] = acc;
+  for (int u = 0; u < kPrepUnroll; ++u) {
+    if (row[u] == -2) continue;
+    if (row[u] == -1) {
+      if (c == 0) {
+        out[u][0] = -INFINITY;
+        out[u][p.Tp] = 0.f;
+      }
+      continue;
+    }
+    float acc;
+    if constexpr (F32IO) {
+      const float4 x = make_float4(__uint_as_float(a[u].x), __uint_as_float(a[u].y), __uint_as_float(a[u].z),
+                                   __uint_as_float(a[u].w));
+      const float4 y = make_float4(__uint_as_float(z[u].x), __uint_as_float(z[u].y), __uint_as_float(z[u].z),
+                                   __uint_as_float(z[u].w));
+      acc = x.x * y.x + x.y * y.y + x.z * y.z + x.w * y.w;
+      if (p.do_hi) {  // dO's planes for the gradient kernel
+        uint2 hi, lo;
+        split_bf16(y.x, y.y, hi.x, lo.x);
+        split_bf16(y.z, y.w, hi.y, lo.y);
+        const size_t ci = size_t(row[u]) * kLanes + c;
+        reinterpret_cast<uint2*>(p.do_hi)[ci] = hi;
+        reinterpret_cast<uint2*>(p.do_lo)[ci] = lo;
+      }
+    } else {
+      acc = bf16_lo_f(a[u].x) * bf16_lo_f(z[u].x) + bf16_hi_f(a[u].x) * bf16_hi_f(z[u].x) +
+            bf16_lo_f(a[u].y) * bf16_lo_f(z[u].y) + bf16_hi_f(a[u].y) * bf16_hi_f(z[u].y) +
+            bf16_lo_f(a[u].z) * bf16_lo_f(z[u].z) + bf16_hi_f(a[u].z) * bf16_hi_f(z[u].z) +
+            bf16_lo_f(a[u].w) * bf16_lo_f(z[u].w) + bf16_hi_f(a[u].w) * bf16_hi_f(z[u].w);
+    }
+#pragma unroll
+    for (int off = kLanes / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(group, acc, off);
+    if (c == 0) {
+      out[u][0] = __ldg(p.LSE + bh_t[u]) * -1.4426950408889634f;
+      out[u][p.Tp] = acc;
+    }
   }
+}
+
+// Blocks of the row-term pass for `rows` (b, t, h) rows.
+template <int D, bool F32IO>
+__host__ __device__ constexpr long long rowterm_blocks(long long rows) {
+  return (rows + (256 / (D / (F32IO ? 4 : 8))) * kPrepUnroll - 1) / ((256 / (D / (F32IO ? 4 : 8))) * kPrepUnroll);
 }
 
 // One 16-byte chunk (chunk c of a head vector at position t) of job tensor
@@ -134,27 +175,20 @@ __device__ __forceinline__ void prep_chunk(const PrepParams& p, const PrepJob& j
   }
 }
 
-// Blocks [0, prep_blocks) cover the jobs' head vectors in memory order, the
-// job chosen once per block: thread t takes chunk t % CPR of kPrepUnroll rows
-// (CPR chunks per row), so a warp reads and writes contiguous 512-byte runs
-// and the position of each row is found once per row, not per element.  The
-// remaining blocks write the row terms.
+// Work blocks [0, prep_blocks) cover the jobs' head vectors in memory order,
+// the job chosen once per block: thread t takes chunk t % CPR of kPrepUnroll
+// rows (CPR chunks per row), so a warp reads and writes contiguous 512-byte
+// runs and the position of each row is found once per row, not per element.
+// The remaining work blocks write the row terms.
 template <int D, bool F32IO>
-__global__ void __launch_bounds__(256) attn_prep_kernel(const __grid_constant__ PrepParams p) {
-  grid_dep_wait();
-  grid_dep_launch();
-  if (int(blockIdx.x) >= p.prep_blocks) {
-    const long long g = (long long)(blockIdx.x - p.prep_blocks) * blockDim.x + threadIdx.x;
-    if (g < p.rt_threads) rowterm_lane<D, F32IO>(p, g);
-    return;
-  }
+__device__ __forceinline__ void prep_block(const PrepParams& p, int vb) {
   constexpr int CPR = D * (F32IO ? 4 : 2) / 16;   // 16-byte chunks per head vector
   constexpr int kSlots = 256 / CPR;               // rows per block step
   int j = 0;
-  while (j + 1 < p.n_jobs && int(blockIdx.x) >= p.job[j + 1].block0) ++j;
+  while (j + 1 < p.n_jobs && vb >= p.job[j + 1].block0) ++j;
   const PrepJob& job = p.job[j];
   const int c = threadIdx.x % CPR;
-  const int row0 = (int(blockIdx.x) - job.block0) * kSlots * kPrepUnroll + threadIdx.x / CPR;
+  const int row0 = (vb - job.block0) * kSlots * kPrepUnroll + threadIdx.x / CPR;
   uint4 raw[kPrepUnroll];
 #pragma unroll
   for (int u = 0; u < kPrepUnroll; ++u) {
@@ -169,6 +203,15 @@ __global__ void __launch_bounds__(256) attn_prep_kernel(const __grid_constant__ 
     const int t = int(bt - fdiv(bt, p.divT) * uint32_t(p.T));
     prep_chunk<D, F32IO>(p, job, size_t(ri) * CPR + c, c, t, raw[u]);
   }
+}
+
+// One CTA per work block.
+template <int D, bool F32IO>
+__global__ void __launch_bounds__(256) attn_prep_kernel(const __grid_constant__ PrepParams p) {
+  grid_dep_wait();
+  grid_dep_launch();
+  if (int(blockIdx.x) >= p.prep_blocks) rowterm_block<D, F32IO>(p, (long long)(blockIdx.x - p.prep_blocks));
+  else prep_block<D, F32IO>(p, int(blockIdx.x));
 }
 
 }  // namespace nea

@@ -29,8 +29,9 @@ def test_prologue_bytes_count_each_element_once():
     assert bench.prologue_bytes(w, "attn_fwd_prologue") == (nq + 2 * nk) * 8
     tp = 1024
     rowterm = 2 * nq * 4 + 4 * 4 * 12 * 1024 + 8 * 4 * 12 * tp
-    # the backward prologue gets the forward's saved planes: only dO is split
-    assert bench.prologue_bytes(w, "attn_bwd_prologue") == nq * 8 + rowterm
+    # the backward prologue gets the forward's saved planes: dO is read once,
+    # for the row terms, and split into its planes in the same pass
+    assert bench.prologue_bytes(w, "attn_bwd_prologue") == nq * 4 + rowterm
     b = WORKLOADS["sweep1024"]  # bf16: rotated copies of Q and K only
     nq, nk = 16 * 1024 * 12 * 64, 16 * 1024 * 4 * 64
     assert bench.prologue_bytes(b, "attn_fwd_prologue") == (nq + nk) * 4
