@@ -19,6 +19,7 @@ __all__ = [
     "nea_status_string", "nea_version", "nea_set_profile_events", "NeaError", "LIB_PATH", "NEA_OK", "NEA_ERR_ARG", "NEA_ERR_CUDA",
     "NEA_ERR_TIMEOUT", "NEA_ERR_UNSUPPORTED", "NEA_ERR_NOMEM", "NEA_ERR_SCRATCH_LIMIT", "NEA_F32", "NEA_BF16",
     "nea_attn_bwd_noalloc", "nea_attn_decode", "nea_attn_saved_bytes", "nea_attn_fwd_save", "nea_attn_bwd_saved",
+    "nea_block_qkv_fwd", "nea_block_qkv_bwd", "nea_block_out_fwd", "nea_block_out_bwd",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnea.so")
@@ -55,6 +56,14 @@ _lib.nea_attn_fwd_save.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
 _lib.nea_attn_fwd_save.restype = _i
 _lib.nea_attn_bwd_saved.argtypes = [_vp] * 10 + [_i, _i, _i, _i, _i, _i, _f, _i, _vp]
 _lib.nea_attn_bwd_saved.restype = _i
+_lib.nea_block_qkv_fwd.argtypes = [_vp] * 8 + [_i] * 6 + [_vp]
+_lib.nea_block_qkv_fwd.restype = _i
+_lib.nea_block_qkv_bwd.argtypes = [_vp] * 14 + [_i] * 6 + [_vp]
+_lib.nea_block_qkv_bwd.restype = _i
+_lib.nea_block_out_fwd.argtypes = [_vp] * 4 + [_i] * 5 + [_vp]
+_lib.nea_block_out_fwd.restype = _i
+_lib.nea_block_out_bwd.argtypes = [_vp] * 5 + [_i] * 5 + [_vp]
+_lib.nea_block_out_bwd.restype = _i
 _lib.nea_version.argtypes = []
 _lib.nea_version.restype = _i
 
@@ -264,6 +273,97 @@ def nea_attn_bwd_saved(q, k, v, o, lse, do, saved, rope_base: float = 10000.0, c
     if rc != NEA_OK:
         raise NeaError(rc, "nea_attn_bwd_saved")
     return dq, dk, dv
+
+
+def _block_check(name, t, shape, dt, dev):
+    _check(t, name, shape, dt, dev)
+
+
+def nea_block_qkv_fwd(x, g, Wq, Wk, Wv, Hq: int, Hkv: int, D: int, q=None, k=None, v=None, stream=None):
+    """Pre-norm and projections: returns ``(q, k, v)`` as ``[B, T, H, D]`` for
+    ``x`` of shape ``[B, T, C]`` (RMSNorm with gain ``g`` applied inside)."""
+    import torch
+
+    B, T, C = x.shape
+    dev, dt = x.device, x.dtype
+    code = _dtype_code(x)
+    for t, n, shp in ((x, "x", (B, T, C)), (g, "g", (C,)), (Wq, "Wq", (C, Hq * D)), (Wk, "Wk", (C, Hkv * D)),
+                      (Wv, "Wv", (C, Hkv * D))):
+        _block_check(n, t, shp, dt, dev)
+    q = torch.empty((B, T, Hq, D), dtype=dt, device=dev) if q is None else q
+    k = torch.empty((B, T, Hkv, D), dtype=dt, device=dev) if k is None else k
+    v = torch.empty((B, T, Hkv, D), dtype=dt, device=dev) if v is None else v
+    for t, n, shp in ((q, "q", (B, T, Hq, D)), (k, "k", (B, T, Hkv, D)), (v, "v", (B, T, Hkv, D))):
+        _block_check(n, t, shp, dt, dev)
+    rc = _lib.nea_block_qkv_fwd(_ptr(x), _ptr(g), _ptr(Wq), _ptr(Wk), _ptr(Wv), _ptr(q), _ptr(k), _ptr(v), B * T, C,
+                                Hq, Hkv, D, code, _stream(stream))
+    if rc != NEA_OK:
+        raise NeaError(rc, "nea_block_qkv_fwd")
+    return q, k, v
+
+
+def nea_block_qkv_bwd(x, g, Wq, Wk, Wv, dq, dk, dv, dres=None, stream=None):
+    """Backward of ``nea_block_qkv_fwd``: returns ``(dx, dg, dWq, dWk, dWv)``;
+    ``dres`` (the residual branch's gradient) is added to ``dx`` when given."""
+    import torch
+
+    B, T, C = x.shape
+    Hq, D = dq.shape[2], dq.shape[3]
+    Hkv = dk.shape[2]
+    dev, dt = x.device, x.dtype
+    code = _dtype_code(x)
+    for t, n, shp in ((x, "x", (B, T, C)), (g, "g", (C,)), (Wq, "Wq", (C, Hq * D)), (Wk, "Wk", (C, Hkv * D)),
+                      (Wv, "Wv", (C, Hkv * D)), (dq, "dq", (B, T, Hq, D)), (dk, "dk", (B, T, Hkv, D)),
+                      (dv, "dv", (B, T, Hkv, D))):
+        _block_check(n, t, shp, dt, dev)
+    if dres is not None:
+        _block_check("dres", dres, (B, T, C), dt, dev)
+    dx, dg = torch.empty_like(x), torch.empty_like(g)
+    dWq, dWk, dWv = torch.empty_like(Wq), torch.empty_like(Wk), torch.empty_like(Wv)
+    rc = _lib.nea_block_qkv_bwd(_ptr(x), _ptr(g), _ptr(Wq), _ptr(Wk), _ptr(Wv), _ptr(dq), _ptr(dk), _ptr(dv),
+                                _ptr(dres), _ptr(dx), _ptr(dg), _ptr(dWq), _ptr(dWk), _ptr(dWv), B * T, C, Hq, Hkv, D,
+                                code, _stream(stream))
+    if rc != NEA_OK:
+        raise NeaError(rc, "nea_block_qkv_bwd")
+    return dx, dg, dWq, dWk, dWv
+
+
+def nea_block_out_fwd(x, o, Wo, h=None, stream=None):
+    """Output projection with the residual: ``h = x + o Wo`` for ``o`` of shape
+    ``[B, T, Hq, D]``."""
+    import torch
+
+    B, T, C = x.shape
+    Hq, D = o.shape[2], o.shape[3]
+    dev, dt = x.device, x.dtype
+    code = _dtype_code(x)
+    for t, n, shp in ((x, "x", (B, T, C)), (o, "o", (B, T, Hq, D)), (Wo, "Wo", (Hq * D, C))):
+        _block_check(n, t, shp, dt, dev)
+    h = torch.empty_like(x) if h is None else h
+    _block_check("h", h, (B, T, C), dt, dev)
+    rc = _lib.nea_block_out_fwd(_ptr(x), _ptr(o), _ptr(Wo), _ptr(h), B * T, C, Hq, D, code, _stream(stream))
+    if rc != NEA_OK:
+        raise NeaError(rc, "nea_block_out_fwd")
+    return h
+
+
+def nea_block_out_bwd(o, Wo, dh, stream=None):
+    """Backward of ``nea_block_out_fwd``: returns ``(do, dWo)`` (the residual's
+    gradient is ``dh``)."""
+    import torch
+
+    B, T, Hq, D = o.shape
+    C = dh.shape[2]
+    dev, dt = o.device, o.dtype
+    code = _dtype_code(o)
+    for t, n, shp in ((o, "o", (B, T, Hq, D)), (Wo, "Wo", (Hq * D, C)), (dh, "dh", (B, T, C))):
+        _block_check(n, t, shp, dt, dev)
+    do, dWo = torch.empty_like(o), torch.empty_like(Wo)
+    rc = _lib.nea_block_out_bwd(_ptr(o), _ptr(Wo), _ptr(dh), _ptr(do), _ptr(dWo), B * T, C, Hq, D, code,
+                                _stream(stream))
+    if rc != NEA_OK:
+        raise NeaError(rc, "nea_block_out_bwd")
+    return do, dWo
 
 
 def nea_device_status(stream=None) -> int:

@@ -11,7 +11,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libnea.so")
-SOURCES = [os.path.join(HERE, "csrc", "nea_attn.cu")]
+SOURCES = [os.path.join(HERE, "csrc", "nea_attn.cu"), os.path.join(HERE, "csrc", "nea_block.cu")]
 DEPS = [os.path.join(HERE, "csrc", f) for f in os.listdir(os.path.join(HERE, "csrc"))] + [
     os.path.join(ROOT, "include", "nea_attn.h")]
 

@@ -18,6 +18,7 @@
 #include <vector>
 
 #include "nea_attn.h"
+#include "nea_internal.h"
 #include "nea_bwd.cuh"
 #include "nea_bwd_f32.cuh"
 #include "nea_decode.cuh"
@@ -602,6 +603,22 @@ int run_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, in
 }
 
 }  // namespace
+
+namespace nea_internal {
+
+int device_status_word(int** err, int* n_sm) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState* st = nullptr;
+  const int rc = device_state(&st);
+  if (rc) return rc;
+  *err = st->err;
+  *n_sm = st->n_sm;
+  return NEA_OK;
+}
+
+long long wait_limit_ns() { return t_wait_limit_ns; }
+
+}  // namespace nea_internal
 
 extern "C" {
 

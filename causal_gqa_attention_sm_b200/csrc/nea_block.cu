@@ -1,0 +1,382 @@
+// C ABI of the decoder-block steps beside the attention (include/nea_attn.h,
+// "Decoder-block steps"): the RMSNorm pre-norm with the Q/K/V projections
+// and the output projection with the residual add, forward and backward.
+// Every product runs on nea::gemm_kernel (tcgen05, TMA, TMEM accumulators);
+// the host side here chooses operand orientations, makes the operand planes
+// and sequences the launches on the caller's stream.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <mutex>
+
+#include "nea_attn.h"
+#include "nea_block.cuh"
+#include "nea_internal.h"
+
+namespace {
+
+std::mutex g_block_mu;
+
+// Per-device workspace of the block steps (operand planes, the fp32 input
+// gradient of the norm, the dg partial sums), grown when a call needs more.
+struct BlockState {
+  uint8_t* ws = nullptr;
+  size_t ws_bytes = 0;
+  uint32_t attr_done = 0;
+};
+BlockState g_block[64];
+
+int fail(cudaError_t e) {
+  (void)cudaGetLastError();
+  return e == cudaErrorMemoryAllocation ? NEA_ERR_NOMEM : NEA_ERR_CUDA;
+}
+
+size_t rup(size_t n) { return (n + 255) / 256 * 256; }
+bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* f = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  return fn;
+}
+
+// A bf16 row-major matrix [rows][cols] as a GEMM operand tile source.
+// k_major: the reduction runs along `cols` (box 64 cols x 128 rows);
+// otherwise along `rows` (box 64 cols x 64 rows, two per tile).
+int mat_map(CUtensorMap* m, const void* base, long long rows, long long cols, bool k_major) {
+  auto enc = encoder();
+  if (!enc) return NEA_ERR_CUDA;
+  const cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(cols) * 2};
+  const cuuint32_t box[2] = {64, k_major ? 128u : 64u};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? NEA_OK : NEA_ERR_CUDA;
+}
+
+// An operand in the form the GEMM reads: bf16 hi (and, for float32 storage,
+// lo) planes of a row-major matrix.
+struct Operand {
+  const void* hi = nullptr;
+  const void* lo = nullptr;
+  long long rows = 0, cols = 0;
+};
+
+struct Ctx {
+  cudaStream_t stream;
+  bool f32;
+  int* err;
+  int n_sm;
+  BlockState* st;
+  unsigned long long wait_limit;
+};
+
+int setup(Ctx& c, int dtype, void* stream) {
+  c.stream = static_cast<cudaStream_t>(stream);
+  c.f32 = dtype == NEA_F32;
+  int rc = nea_internal::device_status_word(&c.err, &c.n_sm);
+  if (rc) return rc;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(e);
+  if (dev < 0 || dev >= 64) return NEA_ERR_UNSUPPORTED;
+  c.st = &g_block[dev];
+  c.wait_limit = static_cast<unsigned long long>(nea_internal::wait_limit_ns());
+  return NEA_OK;
+}
+
+int ensure(Ctx& c, size_t bytes) {
+  if (bytes <= c.st->ws_bytes) return NEA_OK;
+  cudaError_t e = cudaDeviceSynchronize();  // in-flight kernels may still use the old buffer
+  if (e != cudaSuccess) return fail(e);
+  if (c.st->ws) cudaFree(c.st->ws);
+  c.st->ws = nullptr;
+  c.st->ws_bytes = 0;
+  if ((e = cudaMalloc(&c.st->ws, bytes)) != cudaSuccess) return fail(e);
+  c.st->ws_bytes = bytes;
+  return NEA_OK;
+}
+
+// Bump allocator over the workspace (256-byte aligned pieces).
+struct Carve {
+  uint8_t* base;
+  size_t off = 0;
+  void* take(size_t bytes) {
+    void* p = base + off;
+    off += rup(bytes);
+    return p;
+  }
+};
+
+template <typename K, typename... A>
+cudaError_t launch_pdl(K kern, unsigned grid, unsigned block, size_t smem, cudaStream_t stream, A... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+// fp32 [n] -> hi/lo planes (float32 storage); bfloat16 storage reads the
+// tensor itself.
+int make_operand(Ctx& c, Carve& w, const void* src, long long rows, long long cols, Operand* op) {
+  op->rows = rows;
+  op->cols = cols;
+  if (!c.f32) {
+    op->hi = src;
+    return NEA_OK;
+  }
+  const size_t n = size_t(rows) * cols;
+  auto* hi = static_cast<__nv_bfloat16*>(w.take(n * 2));
+  auto* lo = static_cast<__nv_bfloat16*>(w.take(n * 2));
+  const long long n4 = static_cast<long long>(n / 4);
+  const unsigned grid = unsigned(std::min<long long>((n4 + 255) / 256, (long long)c.n_sm * 8));
+  const cudaError_t e = launch_pdl(nea::split_planes_kernel, grid, 256u, size_t(0), c.stream,
+                                   static_cast<const float*>(src), hi, lo, n4);
+  if (e != cudaSuccess) return fail(e);
+  op->hi = hi;
+  op->lo = lo;
+  return NEA_OK;
+}
+
+// out[M][N] (ldo) (+)= A B, A [M x K] and B [K x N] given as operands whose
+// stored matrices are read K-major or MN-major as the flags say.
+int gemm(Ctx& c, const Operand& A, bool a_mn, const Operand& B, bool b_mn, int M, int N, int K, void* out,
+         long long ldo, bool out_f32, bool accumulate, const void* res) {
+  nea::GemmParams p{};
+  int rc;
+  // A [M x K]: stored [M][K] (K-major) or [K][M] (MN-major); B [K x N]:
+  // stored [N][K] (K-major) or [K][N] (MN-major)
+  if ((rc = mat_map(&p.a_hi, A.hi, A.rows, A.cols, !a_mn)) || (rc = mat_map(&p.b_hi, B.hi, B.rows, B.cols, !b_mn)))
+    return rc;
+  if (c.f32 && ((rc = mat_map(&p.a_lo, A.lo, A.rows, A.cols, !a_mn)) ||
+                (rc = mat_map(&p.b_lo, B.lo, B.rows, B.cols, !b_mn))))
+    return rc;
+  p.out = out;
+  p.res = res;
+  p.ldo = ldo;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.out_f32 = out_f32;
+  p.accumulate = accumulate;
+  p.n_m = (M + nea::kGemmBM - 1) / nea::kGemmBM;
+  p.n_n = (N + nea::kGemmBN - 1) / nea::kGemmBN;
+  p.n_k = (K + nea::kGemmBK - 1) / nea::kGemmBK;
+  p.n_tiles = p.n_m * p.n_n;
+  p.err = c.err;
+  p.wait_limit = c.wait_limit;
+  if (p.n_tiles == 0 || K == 0) return NEA_OK;
+  const unsigned grid = unsigned(std::min(p.n_tiles, c.n_sm));
+  auto run = [&](auto kern, uint32_t smem, int bit) -> int {
+    if (!(c.st->attr_done & (1u << bit))) {
+      const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+      if (e != cudaSuccess) return fail(e);
+      c.st->attr_done |= 1u << bit;
+    }
+    const cudaError_t e = launch_pdl(kern, grid, unsigned(nea::kGemmThreads), size_t(smem), c.stream, p);
+    return e == cudaSuccess ? NEA_OK : fail(e);
+  };
+  const int form = (a_mn ? 2 : 0) + (b_mn ? 1 : 0);
+  if (c.f32) {
+    constexpr uint32_t sm = nea::GemmSmem<true>::kAlloc;
+    switch (form) {
+      case 0: return run(nea::gemm_kernel<false, false, true>, sm, 0);
+      case 1: return run(nea::gemm_kernel<false, true, true>, sm, 1);
+      case 2: return run(nea::gemm_kernel<true, false, true>, sm, 2);
+      default: return run(nea::gemm_kernel<true, true, true>, sm, 3);
+    }
+  }
+  constexpr uint32_t sm = nea::GemmSmem<false>::kAlloc;
+  switch (form) {
+    case 0: return run(nea::gemm_kernel<false, false, false>, sm, 4);
+    case 1: return run(nea::gemm_kernel<false, true, false>, sm, 5);
+    case 2: return run(nea::gemm_kernel<true, false, false>, sm, 6);
+    default: return run(nea::gemm_kernel<true, true, false>, sm, 7);
+  }
+}
+
+// y = x rstd g as an operand (planes), rstd into `rstd`.
+int norm_rows(Ctx& c, Carve& w, const void* x, const void* g, int M, int C, float eps, Operand* y, float* rstd) {
+  const size_t n = size_t(M) * C;
+  auto* hi = static_cast<__nv_bfloat16*>(w.take(n * 2));
+  auto* lo = c.f32 ? static_cast<__nv_bfloat16*>(w.take(n * 2)) : nullptr;
+  const unsigned grid = unsigned((M + 7) / 8);
+  const cudaError_t e = c.f32 ? launch_pdl(nea::rmsnorm_rows_kernel<true>, grid, 256u, size_t(0), c.stream, x, g, hi,
+                                           lo, rstd, M, C, eps)
+                              : launch_pdl(nea::rmsnorm_rows_kernel<false>, grid, 256u, size_t(0), c.stream, x, g, hi,
+                                           lo, rstd, M, C, eps);
+  if (e != cudaSuccess) return fail(e);
+  y->hi = hi;
+  y->lo = lo;
+  y->rows = M;
+  y->cols = C;
+  return NEA_OK;
+}
+
+// Widths (C, Hkv D, hence Hq D) in whole 64-column operand boxes.
+int check_dims(int M, int C, int Hq, int Hkv, int D, int dtype) {
+  if (M < 0 || C < 64 || C % 64 != 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return NEA_ERR_ARG;
+  if (D < 8 || (Hkv * D) % 64 != 0 || (dtype != NEA_F32 && dtype != NEA_BF16)) return NEA_ERR_ARG;
+  if (static_cast<long long>(M) * std::max(C, Hq * D) > (1LL << 31)) return NEA_ERR_ARG;
+  return NEA_OK;
+}
+
+constexpr float kNormEps = 1e-5f;
+
+}  // namespace
+
+extern "C" {
+
+int nea_block_qkv_fwd(const void* x, const void* g, const void* Wq, const void* Wk, const void* Wv, void* q, void* k,
+                      void* v, int M, int C, int Hq, int Hkv, int D, int dtype, void* stream) {
+  int rc = check_dims(M, C, Hq, Hkv, D, dtype);
+  if (rc) return rc;
+  if (M == 0) return NEA_OK;
+  for (const void* ptr : {x, g, Wq, Wk, Wv, static_cast<const void*>(q), static_cast<const void*>(k),
+                          static_cast<const void*>(v)})
+    if (!ptr || !al16(ptr)) return NEA_ERR_ARG;
+  std::lock_guard<std::mutex> lock(g_block_mu);
+  Ctx c;
+  if ((rc = setup(c, dtype, stream))) return rc;
+  const int Nq = Hq * D, Nk = Hkv * D;
+  const int e = c.f32 ? 4 : 2;
+  const size_t need = rup(size_t(M) * 4) + rup(size_t(M) * C * e) +
+                      (c.f32 ? rup(size_t(C) * Nq * 4) + 2 * rup(size_t(C) * Nk * 4) : 0) + 4096;
+  if ((rc = ensure(c, need))) return rc;
+  Carve w{c.st->ws};
+  auto* rstd = static_cast<float*>(w.take(size_t(M) * 4));
+  Operand y, bq, bk, bv;
+  if ((rc = norm_rows(c, w, x, g, M, C, kNormEps, &y, rstd))) return rc;
+  if ((rc = make_operand(c, w, Wq, C, Nq, &bq)) || (rc = make_operand(c, w, Wk, C, Nk, &bk)) ||
+      (rc = make_operand(c, w, Wv, C, Nk, &bv)))
+    return rc;
+  // q = y Wq: A = y [M][C] K-major; B = Wq [C][Nq], N contiguous: MN-major
+  if ((rc = gemm(c, y, false, bq, true, M, Nq, C, q, Nq, c.f32, false, nullptr)) ||
+      (rc = gemm(c, y, false, bk, true, M, Nk, C, k, Nk, c.f32, false, nullptr)) ||
+      (rc = gemm(c, y, false, bv, true, M, Nk, C, v, Nk, c.f32, false, nullptr)))
+    return rc;
+  return NEA_OK;
+}
+
+int nea_block_qkv_bwd(const void* x, const void* g, const void* Wq, const void* Wk, const void* Wv, const void* dq,
+                      const void* dk, const void* dv, const void* dres, void* dx, void* dg, void* dWq, void* dWk,
+                      void* dWv, int M, int C, int Hq, int Hkv, int D, int dtype, void* stream) {
+  int rc = check_dims(M, C, Hq, Hkv, D, dtype);
+  if (rc) return rc;
+  if (M == 0) return NEA_OK;
+  for (const void* ptr : {x, g, Wq, Wk, Wv, dq, dk, dv, static_cast<const void*>(dx), static_cast<const void*>(dg),
+                          static_cast<const void*>(dWq), static_cast<const void*>(dWk), static_cast<const void*>(dWv)})
+    if (!ptr || !al16(ptr)) return NEA_ERR_ARG;
+  if (dres && !al16(dres)) return NEA_ERR_ARG;
+  std::lock_guard<std::mutex> lock(g_block_mu);
+  Ctx c;
+  if ((rc = setup(c, dtype, stream))) return rc;
+  const int Nq = Hq * D, Nk = Hkv * D;
+  const int e = c.f32 ? 4 : 2;
+  const int n_part = std::min((M + 7) / 8, c.n_sm * 2);
+  const size_t need = rup(size_t(M) * 4) + rup(size_t(M) * C * e) + rup(size_t(M) * C * 4) +
+                      rup(size_t(n_part) * C * 4) +
+                      (c.f32 ? rup(size_t(C) * Nq * 4) + 2 * rup(size_t(C) * Nk * 4) + rup(size_t(M) * Nq * 4) +
+                                   2 * rup(size_t(M) * Nk * 4)
+                             : 0) +
+                      4096;
+  if ((rc = ensure(c, need))) return rc;
+  Carve w{c.st->ws};
+  auto* rstd = static_cast<float*>(w.take(size_t(M) * 4));
+  auto* dy = static_cast<float*>(w.take(size_t(M) * C * 4));
+  auto* dg_part = static_cast<float*>(w.take(size_t(n_part) * C * 4));
+  Operand y, bq, bk, bv, gq, gk, gv;
+  if ((rc = norm_rows(c, w, x, g, M, C, kNormEps, &y, rstd))) return rc;
+  if ((rc = make_operand(c, w, Wq, C, Nq, &bq)) || (rc = make_operand(c, w, Wk, C, Nk, &bk)) ||
+      (rc = make_operand(c, w, Wv, C, Nk, &bv)) || (rc = make_operand(c, w, dq, M, Nq, &gq)) ||
+      (rc = make_operand(c, w, dk, M, Nk, &gk)) || (rc = make_operand(c, w, dv, M, Nk, &gv)))
+    return rc;
+  // dW* = y^T d*: A = y^T (y [M][C], C contiguous: MN-major); B = d* [M][N*], MN-major
+  if ((rc = gemm(c, y, true, gq, true, C, Nq, M, dWq, Nq, c.f32, false, nullptr)) ||
+      (rc = gemm(c, y, true, gk, true, C, Nk, M, dWk, Nk, c.f32, false, nullptr)) ||
+      (rc = gemm(c, y, true, gv, true, C, Nk, M, dWv, Nk, c.f32, false, nullptr)))
+    return rc;
+  // dy = dq Wq^T + dk Wk^T + dv Wv^T (fp32): A = d* K-major; B = W*^T, i.e. W* [C][N*] read K-major
+  if ((rc = gemm(c, gq, false, bq, false, M, C, Nq, dy, C, true, false, nullptr)) ||
+      (rc = gemm(c, gk, false, bk, false, M, C, Nk, dy, C, true, true, nullptr)) ||
+      (rc = gemm(c, gv, false, bv, false, M, C, Nk, dy, C, true, true, nullptr)))
+    return rc;
+  cudaError_t err = c.f32 ? launch_pdl(nea::rmsnorm_bwd_rows_kernel<true>, unsigned(n_part), 256u, size_t(C) * 4,
+                                       c.stream, x, g, static_cast<const float*>(rstd), static_cast<const float*>(dy),
+                                       dres, dx, dg_part, M, C)
+                          : launch_pdl(nea::rmsnorm_bwd_rows_kernel<false>, unsigned(n_part), 256u, size_t(C) * 4,
+                                       c.stream, x, g, static_cast<const float*>(rstd), static_cast<const float*>(dy),
+                                       dres, dx, dg_part, M, C);
+  if (err != cudaSuccess) return fail(err);
+  const unsigned cg = unsigned((C + 255) / 256);
+  err = c.f32 ? launch_pdl(nea::colsum_kernel<true>, cg, 256u, size_t(0), c.stream,
+                           static_cast<const float*>(dg_part), n_part, C, dg)
+              : launch_pdl(nea::colsum_kernel<false>, cg, 256u, size_t(0), c.stream,
+                           static_cast<const float*>(dg_part), n_part, C, dg);
+  return err == cudaSuccess ? NEA_OK : fail(err);
+}
+
+int nea_block_out_fwd(const void* x, const void* o, const void* Wo, void* h, int M, int C, int Hq, int D, int dtype,
+                      void* stream) {
+  int rc = check_dims(M, C, Hq, Hq, D, dtype);
+  if (rc) return rc;
+  if (M == 0) return NEA_OK;
+  for (const void* ptr : {x, o, Wo, static_cast<const void*>(h)})
+    if (!ptr || !al16(ptr)) return NEA_ERR_ARG;
+  std::lock_guard<std::mutex> lock(g_block_mu);
+  Ctx c;
+  if ((rc = setup(c, dtype, stream))) return rc;
+  const int Nq = Hq * D;
+  const size_t need = (c.f32 ? rup(size_t(M) * Nq * 4) + rup(size_t(Nq) * C * 4) : 0) + 4096;
+  if ((rc = ensure(c, need))) return rc;
+  Carve w{c.st->ws};
+  Operand a, b;
+  if ((rc = make_operand(c, w, o, M, Nq, &a)) || (rc = make_operand(c, w, Wo, Nq, C, &b))) return rc;
+  // h = x + o Wo: A = o [M][Nq] K-major; B = Wo [Nq][C], C contiguous: MN-major
+  return gemm(c, a, false, b, true, M, C, Nq, h, C, c.f32, false, x);
+}
+
+int nea_block_out_bwd(const void* o, const void* Wo, const void* dh, void* do_, void* dWo, int M, int C, int Hq,
+                      int D, int dtype, void* stream) {
+  int rc = check_dims(M, C, Hq, Hq, D, dtype);
+  if (rc) return rc;
+  if (M == 0) return NEA_OK;
+  for (const void* ptr : {o, Wo, dh, static_cast<const void*>(do_), static_cast<const void*>(dWo)})
+    if (!ptr || !al16(ptr)) return NEA_ERR_ARG;
+  std::lock_guard<std::mutex> lock(g_block_mu);
+  Ctx c;
+  if ((rc = setup(c, dtype, stream))) return rc;
+  const int Nq = Hq * D;
+  const size_t need =
+      (c.f32 ? rup(size_t(M) * Nq * 4) + rup(size_t(Nq) * C * 4) + rup(size_t(M) * C * 4) : 0) + 4096;
+  if ((rc = ensure(c, need))) return rc;
+  Carve w{c.st->ws};
+  Operand a, b, d;
+  if ((rc = make_operand(c, w, o, M, Nq, &a)) || (rc = make_operand(c, w, Wo, Nq, C, &b)) ||
+      (rc = make_operand(c, w, dh, M, C, &d)))
+    return rc;
+  // do = dh Wo^T: A = dh [M][C] K-major; B = Wo^T, i.e. Wo [Nq][C] read K-major
+  if ((rc = gemm(c, d, false, b, false, M, Nq, C, do_, Nq, c.f32, false, nullptr))) return rc;
+  // dWo = o^T dh: A = o^T (o [M][Nq]: MN-major); B = dh [M][C], MN-major
+  return gemm(c, a, true, d, true, Nq, C, M, dWo, C, c.f32, false, nullptr);
+}
+
+}  // extern "C"

@@ -1,0 +1,357 @@
+// The steps on either side of the attention in a pre-norm decoder block
+// ("NanoEuler" write-up, aimsg.uk, section 1 "Architecture design" and
+// section 2 "Model components": RMSNorm pre-norm, bias-free projections,
+// residual update x <- x + f(x)):
+//   forward   y = x rstd g (rstd = (mean_j x_j^2 + eps)^-1/2 per token),
+//             q = y Wq, k = y Wk, v = y Wv;   h = x + o Wo
+//   backward  dWo = o^T dh, do = dh Wo^T;  dW* = y^T d*, dy = sum d* W*^T,
+//             dx = rstd g dy - x rstd^3 / C sum_j (g dy)_j x_j (+ dh), dg = sum_tokens dy x rstd
+// The products run on one tcgen05 GEMM kernel, C = A B with A [M x K] and B
+// [K x N] stored row-major in either orientation (an operand whose reduction
+// index is the contiguous one is "K-major", else "MN-major"); operands are
+// bf16 (bfloat16 storage) or bf16 hi/lo planes (float32 storage: every
+// product hi*hi + hi*lo + lo*hi, fp32 accumulation, as in the attention).
+// RMSNorm's reductions are row kernels that write the GEMM operands.
+#pragma once
+
+#include "nea_device.cuh"
+
+namespace nea {
+
+constexpr int kGemmBM = 128, kGemmBN = 128, kGemmBK = 64;
+constexpr int kGemmThreads = 192;  // warp 0: TMA, warp 1: MMA, warps 2-5: epilogue
+
+struct GemmParams {
+  // operands: hi planes (bf16 storage: the tensors themselves), lo planes
+  // (float32 storage); K-major maps have box {64, 128}, MN-major {64, 64}
+  CUtensorMap a_hi, a_lo, b_hi, b_lo;
+  void* out;          // [M][ldo] row-major, fp32 or bf16
+  const void* res;    // residual added to the result (same layout as out), or nullptr
+  long long ldo;
+  int M, N, K;
+  int out_f32;        // 1: fp32 output, 0: bf16
+  int accumulate;     // 1: out += A B (fp32 output)
+  int n_m, n_n, n_k, n_tiles;
+  int* err;
+  unsigned long long wait_limit;
+};
+
+template <bool SPLIT>
+struct GemmSmem {
+  static constexpr uint32_t kOp = 128 * 128;             // one 128 x 64 bf16 operand tile (16 KB)
+  static constexpr int kPlanes = SPLIT ? 2 : 1;
+  static constexpr uint32_t kStage = 2 * kPlanes * kOp;  // A planes, then B planes
+  static constexpr int ST = SPLIT ? 3 : 6;
+  static constexpr uint32_t kBars = ST * kStage;         // full[ST], empty[ST], acc_full[2], acc_empty[2]
+  static constexpr uint32_t kMisc = kBars + (2 * ST + 4) * 8;  // TMEM base, abort flag
+  static constexpr uint32_t kBytes = kMisc + 16;
+  static constexpr uint32_t kAlloc = kBytes + 1024;
+};
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int c0, int c1, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(tmap), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// One 128 x 64 operand tile (rows of the M or N extent, 64 of K) into
+// shared memory: K-major, one box of 128 rows x 128 bytes; MN-major, two
+// boxes of 64 K-rows x 64 MN-elements (the two MN halves 8 KB apart).
+template <bool MN>
+__device__ __forceinline__ void gemm_load_tile(uint8_t* dst, const CUtensorMap* map, int mn0, int k0, uint64_t* bar) {
+  if constexpr (MN) {
+    tma_load_2d(dst, map, mn0, k0, bar);
+    tma_load_2d(dst + 8192, map, mn0 + 64, k0, bar);
+  } else {
+    tma_load_2d(dst, map, k0, mn0, bar);
+  }
+}
+
+// Descriptor of the 16-wide K slice kk of a tile.  K-major: rows of 128
+// bytes, the slice 32 bytes on.  MN-major: K rows of 128 bytes (64 MN
+// elements), the slice 16 rows on, the second MN half 8 KB on.
+template <bool MN>
+__device__ __forceinline__ uint64_t gemm_desc(uint32_t tile, int kk) {
+  return MN ? smem_desc(tile + kk * 2048, 128, 8192) : smem_desc(tile + kk * 32, 128, 16);
+}
+
+template <bool AMN, bool BMN, bool SPLIT>
+__global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
+  using L = GemmSmem<SPLIT>;
+  extern __shared__ uint8_t raw[];
+  uint8_t* sm = raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + L::kBars);
+  uint64_t* empty = full + L::ST;
+  uint64_t* acc_full = empty + L::ST;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kMisc + 4);
+  const WaitCtl wc{p.err, p.wait_limit, abort_flag};
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int s = 0; s < L::ST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);  // one arrival per epilogue warp
+    }
+    mbar_init_fence();
+  }
+  if (warp == 1) tmem_alloc(tmem_holder, 256);  // two 128-column fp32 accumulators
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_holder;
+  grid_dep_wait();
+  grid_dep_launch();
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA
+    if (lane == 0) {
+      prefetch_tmap(&p.a_hi);
+      prefetch_tmap(&p.b_hi);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x) {
+        const int mi = t % p.n_m, ni = t / p.n_m;
+        for (int ks = 0; ks < p.n_k; ++ks, ++it) {
+          const int s = it % L::ST;
+          if (it >= uint32_t(L::ST) && !(ok = wait_thread(&empty[s], ((it / L::ST) - 1) & 1, wc, kErrWaitEmpty)))
+            break;
+          uint8_t* st = sm + s * L::kStage;
+          mbar_arrive_expect_tx(&full[s], L::kStage);
+          gemm_load_tile<AMN>(st, &p.a_hi, mi * kGemmBM, ks * kGemmBK, &full[s]);
+          gemm_load_tile<BMN>(st + L::kPlanes * L::kOp, &p.b_hi, ni * kGemmBN, ks * kGemmBK, &full[s]);
+          if constexpr (SPLIT) {
+            gemm_load_tile<AMN>(st + L::kOp, &p.a_lo, mi * kGemmBM, ks * kGemmBK, &full[s]);
+            gemm_load_tile<BMN>(st + 3 * L::kOp, &p.b_lo, ni * kGemmBN, ks * kGemmBK, &full[s]);
+          }
+        }
+      }
+      // never exit with copies in flight
+      for (uint32_t i = it > uint32_t(L::ST) ? it - L::ST : 0; i < it; ++i)
+        drain_wait(&full[i % L::ST], (i / L::ST) & 1, wc);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA
+    constexpr uint32_t idesc = idesc_bf16(kGemmBM, kGemmBN, AMN, BMN);
+    uint32_t it = 0, last = 0xffffffffu;  // the last stage use committed
+    int lt = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x, ++lt) {
+      const int ab = lt & 1;
+      if (lt >= 2) ok = wait_warp(&acc_empty[ab], ((lt >> 1) - 1) & 1, wc, kErrWaitSoftmax);
+      tc_fence_after();
+      for (int ks = 0; ks < p.n_k && ok; ++ks, ++it) {
+        const int s = it % L::ST;
+        if (!(ok = wait_warp(&full[s], (it / L::ST) & 1, wc, kErrWaitProducer))) break;
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t a = smem_u32(sm + s * L::kStage);
+          const uint32_t b = a + L::kPlanes * L::kOp;
+#pragma unroll
+          for (int kk = 0; kk < kGemmBK / 16; ++kk) {
+#pragma unroll
+            for (int term = 0; term < (SPLIT ? 3 : 1); ++term) {
+              // hi*hi, hi*lo, lo*hi
+              const uint32_t ap = a + (term == 2 ? L::kOp : 0), bp = b + (term == 1 ? L::kOp : 0);
+              mma_ss(tbase + ab * kGemmBN, gemm_desc<AMN>(ap, kk), gemm_desc<BMN>(bp, kk), idesc,
+                     (ks | kk | term) != 0);
+            }
+          }
+          tc_commit(&empty[s]);
+          if (ks == p.n_k - 1) tc_commit(&acc_full[ab]);
+          last = it;
+        }
+        __syncwarp();
+      }
+    }
+    // commits complete in order: once the last has, no product is in flight
+    if (lane == 0 && last != 0xffffffffu) drain_wait(&empty[last % L::ST], (last / L::ST) & 1, wc);
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int q4 = warp & 3;  // TMEM lanes 32 q4 .. 32 q4 + 31
+    int lt = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x, ++lt) {
+      const int ab = lt & 1;
+      if (!(ok = wait_warp(&acc_full[ab], (lt >> 1) & 1, wc, kErrWaitMma))) break;
+      tc_fence_after();
+      const int mi = t % p.n_m, ni = t / p.n_m;
+      const int row = mi * kGemmBM + q4 * 32 + lane;
+#pragma unroll 1
+      for (int c = 0; c < kGemmBN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem_addr(tbase, q4 * 32, ab * kGemmBN + c * 32), r);
+        const int col0 = ni * kGemmBN + c * 32;
+        if (row >= p.M || col0 >= p.N) continue;
+        const bool whole = col0 + 32 <= p.N;
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+        const size_t o0 = size_t(row) * p.ldo + col0;
+        if (p.out_f32) {
+          float* out = static_cast<float*>(p.out) + o0;
+          const float* res = p.res ? static_cast<const float*>(p.res) + o0 : nullptr;
+          if (whole) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              float4 w = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+              if (p.accumulate) {
+                const float4 u = *reinterpret_cast<const float4*>(out + j);
+                w.x += u.x, w.y += u.y, w.z += u.z, w.w += u.w;
+              }
+              if (res) {
+                const float4 u = *reinterpret_cast<const float4*>(res + j);
+                w.x += u.x, w.y += u.y, w.z += u.z, w.w += u.w;
+              }
+              *reinterpret_cast<float4*>(out + j) = w;
+            }
+          } else {
+            for (int j = 0; j < 32 && col0 + j < p.N; ++j)
+              out[j] = v[j] + (p.accumulate ? out[j] : 0.f) + (res ? res[j] : 0.f);
+          }
+        } else {
+          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + o0;
+          const __nv_bfloat16* res = p.res ? static_cast<const __nv_bfloat16*>(p.res) + o0 : nullptr;
+          if (whole) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) {
+              float w[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) w[i] = v[j + i];
+              if (res) {
+                const uint4 u = *reinterpret_cast<const uint4*>(res + j);
+                const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) w[2 * i] += bf16_lo_f(uw[i]), w[2 * i + 1] += bf16_hi_f(uw[i]);
+              }
+              *reinterpret_cast<uint4*>(out + j) =
+                  make_uint4(pack_bf16(w[0], w[1]), pack_bf16(w[2], w[3]), pack_bf16(w[4], w[5]), pack_bf16(w[6], w[7]));
+            }
+          } else {
+            for (int j = 0; j < 32 && col0 + j < p.N; ++j)
+              out[j] = __float2bfloat16_rn(v[j] + (res ? __bfloat162float(res[j]) : 0.f));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[ab]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 256);
+  }
+}
+
+// ------------------------------------------------------------------ RMSNorm rows
+// One warp per token row of x [M][C] (C a multiple of 8): rstd = (mean x^2 +
+// eps)^-1/2, y = x rstd g written as the GEMM operand (bfloat16 storage:
+// y in bf16; float32 storage: bf16 hi and lo planes of y).
+template <bool F32IO>
+__global__ void __launch_bounds__(256) rmsnorm_rows_kernel(const void* x, const void* g, __nv_bfloat16* y_hi,
+                                                           __nv_bfloat16* y_lo, float* rstd, int M, int C,
+                                                           float eps) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  grid_dep_wait();
+  grid_dep_launch();
+  if (row >= M) return;
+  auto load = [&](const void* base, size_t i) {
+    return F32IO ? static_cast<const float*>(base)[i] : __bfloat162float(static_cast<const __nv_bfloat16*>(base)[i]);
+  };
+  const size_t r0 = size_t(row) * C;
+  float ss = 0.f;
+  for (int j = lane; j < C; j += 32) {
+    const float v = load(x, r0 + j);
+    ss = fmaf(v, v, ss);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(kFullMask, ss, off);
+  const float rs = 1.f / sqrtf(ss / float(C) + eps);
+  if (lane == 0) rstd[row] = rs;
+  for (int j = lane; j < C; j += 32) {
+    const float yv = load(x, r0 + j) * rs * load(g, j);
+    const __nv_bfloat16 h = __float2bfloat16_rn(yv);
+    y_hi[r0 + j] = h;
+    if (F32IO) y_lo[r0 + j] = __float2bfloat16_rn(yv - __bfloat162float(h));
+  }
+}
+
+// fp32 tensor of n elements (n a multiple of 4) -> bf16 hi and lo planes.
+__global__ void __launch_bounds__(256) split_planes_kernel(const float* src, __nv_bfloat16* hi, __nv_bfloat16* lo,
+                                                           long long n4) {
+  grid_dep_wait();
+  grid_dep_launch();
+  for (long long i = blockIdx.x * 256ll + threadIdx.x; i < n4; i += 256ll * gridDim.x) {
+    const float4 v = reinterpret_cast<const float4*>(src)[i];
+    uint2 h, l;
+    split_bf16(v.x, v.y, h.x, l.x);
+    split_bf16(v.z, v.w, h.y, l.y);
+    reinterpret_cast<uint2*>(hi)[i] = h;
+    reinterpret_cast<uint2*>(lo)[i] = l;
+  }
+}
+
+// RMSNorm backward, one warp per token row (rows grid-stride): from
+// dy [M][C] (fp32) and the forward's x, g, rstd,
+//   dx = rstd g dy - x rstd^3 / C sum_j (g dy)_j x_j  (+ dres),
+// and this CTA's share of dg = sum_tokens dy x rstd, written to
+// dg_part[blockIdx.x][C] (fp32).
+template <bool F32IO>
+__global__ void __launch_bounds__(256) rmsnorm_bwd_rows_kernel(const void* x, const void* g, const float* rstd,
+                                                               const float* dy, const void* dres, void* dx,
+                                                               float* dg_part, int M, int C) {
+  extern __shared__ float dg_s[];  // [C]
+  grid_dep_wait();
+  grid_dep_launch();
+  for (int j = threadIdx.x; j < C; j += 256) dg_s[j] = 0.f;
+  __syncthreads();
+  auto load = [&](const void* base, size_t i) {
+    return F32IO ? static_cast<const float*>(base)[i] : __bfloat162float(static_cast<const __nv_bfloat16*>(base)[i]);
+  };
+  const int lane = threadIdx.x & 31;
+  for (int row = blockIdx.x * 8 + (threadIdx.x >> 5); row < M; row += gridDim.x * 8) {
+    const size_t r0 = size_t(row) * C;
+    const float rs = rstd[row];
+    float dot = 0.f;
+    for (int j = lane; j < C; j += 32) dot = fmaf(load(g, j) * dy[r0 + j], load(x, r0 + j), dot);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(kFullMask, dot, off);
+    const float c2 = rs * rs * rs * dot / float(C);
+    for (int j = lane; j < C; j += 32) {
+      const float xv = load(x, r0 + j), d = dy[r0 + j];
+      float v = rs * load(g, j) * d - xv * c2;
+      if (dres) v += load(dres, r0 + j);
+      if (F32IO) static_cast<float*>(dx)[r0 + j] = v;
+      else static_cast<__nv_bfloat16*>(dx)[r0 + j] = __float2bfloat16_rn(v);
+      atomicAdd(&dg_s[j], d * xv * rs);
+    }
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < C; j += 256) dg_part[size_t(blockIdx.x) * C + j] = dg_s[j];
+}
+
+// dg[j] = sum over the parts of dg_part[.][j], in the storage type.
+template <bool F32IO>
+__global__ void __launch_bounds__(256) colsum_kernel(const float* part, int n_part, int C, void* dg) {
+  grid_dep_wait();
+  grid_dep_launch();
+  const int j = blockIdx.x * 256 + threadIdx.x;
+  if (j >= C) return;
+  float s = 0.f;
+  for (int i = 0; i < n_part; ++i) s += part[size_t(i) * C + j];
+  if (F32IO) static_cast<float*>(dg)[j] = s;
+  else static_cast<__nv_bfloat16*>(dg)[j] = __float2bfloat16_rn(s);
+}
+
+}  // namespace nea

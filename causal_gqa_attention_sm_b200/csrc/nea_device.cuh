@@ -102,7 +102,7 @@ __device__ __forceinline__ void raise_error(const WaitCtl& c, int code) {
 // Wait of a single thread for the phase of `bar` with the given parity to
 // complete.  Returns false, after recording `code`, once the CTA aborted or
 // the wait exceeded its limit.
-__device__ __noinline__ bool wait_thread_slow(uint64_t* bar, uint32_t parity, const WaitCtl& c, int code) {
+static __device__ __noinline__ bool wait_thread_slow(uint64_t* bar, uint32_t parity, const WaitCtl& c, int code) {
   const uint64_t t0 = global_timer_ns();
   for (;;) {
 #pragma unroll 1
@@ -119,7 +119,7 @@ __device__ __noinline__ bool wait_thread_slow(uint64_t* bar, uint32_t parity, co
 // Same wait, taken by all 32 lanes of a warp with a warp-uniform outcome, so
 // that warp-collective tcgen05 loads/stores after it stay converged.  Every
 // lane performs its own successful try_wait (acquire) before proceeding.
-__device__ __noinline__ bool wait_warp_slow(uint64_t* bar, uint32_t parity, const WaitCtl& c, int code) {
+static __device__ __noinline__ bool wait_warp_slow(uint64_t* bar, uint32_t parity, const WaitCtl& c, int code) {
   bool done = false;
   const uint64_t t0 = global_timer_ns();
   for (;;) {
@@ -145,7 +145,7 @@ __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, const 
 
 // Wait that ignores the CTA's abort flag (still bounded by the limit, records
 // nothing): used before exit so that no copy or MMA is left in flight.
-__device__ __noinline__ bool drain_wait(uint64_t* bar, uint32_t parity, const WaitCtl& c) {
+static __device__ __noinline__ bool drain_wait(uint64_t* bar, uint32_t parity, const WaitCtl& c) {
   const uint64_t t0 = global_timer_ns();
   while (!mbar_try_wait(bar, parity))
     if (global_timer_ns() - t0 > c.limit) return false;

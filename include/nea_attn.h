@@ -154,6 +154,51 @@ int nea_attn_bwd_saved(const void* Q, const void* K, const void* V, const void* 
                        int dtype, float rope_base, int causal, void* stream);
 
 /*
+ * Decoder-block steps beside the attention ("NanoEuler" write-up, aimsg.uk,
+ * section 1 "Architecture design" and section 2 "Model components": a
+ * pre-norm block x <- x + Attn(RMSNorm(x)), RMSNorm without bias, no bias in
+ * any projection):
+ *
+ *   rstd_m = (mean_c x_mc^2 + 1e-5)^(-1/2),  y = x rstd g
+ *   q = y Wq,  k = y Wk,  v = y Wv           (the attention's inputs, un-rotated)
+ *   h = x + o Wo                             (o: the attention's output)
+ *
+ * Layouts (row-major, contiguous, element type `dtype` as for the attention;
+ * M = B*T tokens):
+ *   x, h, dx, dh : [M][C];   g, dg : [C]
+ *   Wq, dWq      : [C][Hq*D];   Wk, Wv, dWk, dWv : [C][Hkv*D]
+ *   Wo, dWo      : [Hq*D][C]
+ *   q, dq, o, do : [M][Hq*D] (= [B][T][Hq][D]);  k, v, dk, dv : [M][Hkv*D]
+ * C and Hkv*D must be multiples of 64; D a multiple of 8; Hq % Hkv == 0.
+ * Every product runs on the library's tcgen05 GEMM: bf16 operands with fp32
+ * accumulation for NEA_BF16; for NEA_F32 each operand as bf16 hi and lo
+ * planes and each product as hi*hi + hi*lo + lo*hi (as in the attention).
+ * The steps keep a per-device workspace of their own (operand planes, the
+ * norm's fp32 input gradient), grown when a call needs more.  Errors and
+ * streams as for the attention; nothing is launched on NEA_ERR_ARG.
+ *
+ * nea_block_qkv_fwd: q, k, v from x (the norm is applied inside).
+ * nea_block_qkv_bwd: from the forward's inputs and the upstream gradients dq,
+ *   dk, dv (gradients of the un-rotated q, k, v -- nea_attn_bwd's outputs):
+ *   dWq = y^T dq (likewise dWk, dWv), dy = dq Wq^T + dk Wk^T + dv Wv^T,
+ *   dx = rstd g dy - x rstd^3 / C sum_c (g dy)_c x_c, plus `dres` when it is
+ *   not NULL (the residual branch's gradient, dh), and dg = sum_m dy x rstd.
+ *   The norm is recomputed from x.
+ * nea_block_out_fwd: h = x + o Wo.
+ * nea_block_out_bwd: do = dh Wo^T and dWo = o^T dh (the residual's gradient
+ *   is dh itself).
+ */
+int nea_block_qkv_fwd(const void* x, const void* g, const void* Wq, const void* Wk, const void* Wv, void* q, void* k,
+                      void* v, int M, int C, int Hq, int Hkv, int D, int dtype, void* stream);
+int nea_block_qkv_bwd(const void* x, const void* g, const void* Wq, const void* Wk, const void* Wv, const void* dq,
+                      const void* dk, const void* dv, const void* dres, void* dx, void* dg, void* dWq, void* dWk,
+                      void* dWv, int M, int C, int Hq, int Hkv, int D, int dtype, void* stream);
+int nea_block_out_fwd(const void* x, const void* o, const void* Wo, void* h, int M, int C, int Hq, int D, int dtype,
+                      void* stream);
+int nea_block_out_bwd(const void* o, const void* Wo, const void* dh, void* do_, void* dWo, int M, int C, int Hq,
+                      int D, int dtype, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device status words of the
  * current device: the one the regular entry points write and the one inside
  * the fixed scratch of nea_attn_bwd_noalloc.  Returns NEA_OK, NEA_ERR_TIMEOUT
