@@ -156,19 +156,47 @@ int make_operand(Ctx& c, Carve& w, const void* src, long long rows, long long co
   return NEA_OK;
 }
 
-// out[M][N] (ldo) (+)= A B, A [M x K] and B [K x N] given as operands whose
-// stored matrices are read K-major or MN-major as the flags say.
-int gemm(Ctx& c, const Operand& A, bool a_mn, const Operand& B, bool b_mn, int M, int N, int K, void* out,
-         long long ldo, bool out_f32, bool accumulate, const void* res) {
+// One operand segment of a product: A and B operands (read K-major or
+// MN-major as the product's flags say), and for N segments the output.
+struct Seg {
+  Operand A, B;
+  void* out = nullptr;
+  long long width = 0;  // K extent (K segments) or N extent = output columns (N segments)
+};
+
+// out = sum_s A_s B_s (kseg: segments along K, one output `out` [M][ldo]) or
+// out_s = A_0 B_s (segments along N, output s [M][width_s]); A [M x K] is
+// stored [M][K] (K-major) or [K][M] (MN-major), B [K x N] stored [N][K]
+// (K-major) or [K][N] (MN-major).
+int gemm_seg(Ctx& c, const Seg* segs, int n_seg, bool kseg, bool a_mn, bool b_mn, int M, void* out, long long ldo,
+             bool out_f32, const void* res) {
   nea::GemmParams p{};
   int rc;
-  // A [M x K]: stored [M][K] (K-major) or [K][M] (MN-major); B [K x N]:
-  // stored [N][K] (K-major) or [K][N] (MN-major)
-  if ((rc = mat_map(&p.a_hi, A.hi, A.rows, A.cols, !a_mn)) || (rc = mat_map(&p.b_hi, B.hi, B.rows, B.cols, !b_mn)))
-    return rc;
-  if (c.f32 && ((rc = mat_map(&p.a_lo, A.lo, A.rows, A.cols, !a_mn)) ||
-                (rc = mat_map(&p.b_lo, B.lo, B.rows, B.cols, !b_mn))))
-    return rc;
+  int N = 0, K = 0, begin = 0;
+  for (int i = 0; i < n_seg; ++i) {
+    const Seg& g = segs[i];
+    nea::GemmSeg& q = p.seg[i];
+    if ((rc = mat_map(&q.a_hi, g.A.hi, g.A.rows, g.A.cols, !a_mn)) ||
+        (rc = mat_map(&q.b_hi, g.B.hi, g.B.rows, g.B.cols, !b_mn)))
+      return rc;
+    if (c.f32 && ((rc = mat_map(&q.a_lo, g.A.lo, g.A.rows, g.A.cols, !a_mn)) ||
+                  (rc = mat_map(&q.b_lo, g.B.lo, g.B.rows, g.B.cols, !b_mn))))
+      return rc;
+    q.out = g.out;
+    q.ldo = g.width;
+    q.begin = begin;
+    if (kseg) {
+      begin += int(g.width / nea::kGemmBK);
+      K += int(g.width);
+    } else {
+      begin += int((g.width + nea::kGemmBN - 1) / nea::kGemmBN);
+      N += int(g.width);
+    }
+  }
+  if (kseg) N = int(ldo);
+  else K = int(a_mn ? segs[0].A.rows : segs[0].A.cols);
+  p.n_seg = n_seg;
+  p.kseg = kseg;
   p.out = out;
   p.res = res;
   p.ldo = ldo;
@@ -176,9 +204,8 @@ int gemm(Ctx& c, const Operand& A, bool a_mn, const Operand& B, bool b_mn, int M
   p.N = N;
   p.K = K;
   p.out_f32 = out_f32;
-  p.accumulate = accumulate;
   p.n_m = (M + nea::kGemmBM - 1) / nea::kGemmBM;
-  p.n_n = (N + nea::kGemmBN - 1) / nea::kGemmBN;
+  p.n_n = kseg ? (N + nea::kGemmBN - 1) / nea::kGemmBN : begin;
   p.n_k = (K + nea::kGemmBK - 1) / nea::kGemmBK;
   p.n_tiles = p.n_m * p.n_n;
   p.err = c.err;
@@ -211,6 +238,17 @@ int gemm(Ctx& c, const Operand& A, bool a_mn, const Operand& B, bool b_mn, int M
     case 2: return run(nea::gemm_kernel<true, false, false>, sm, 6);
     default: return run(nea::gemm_kernel<true, true, false>, sm, 7);
   }
+}
+
+// out[M][N] = A B (+ res), one segment.
+int gemm(Ctx& c, const Operand& A, bool a_mn, const Operand& B, bool b_mn, int M, int N, void* out, bool out_f32,
+         const void* res) {
+  Seg g;
+  g.A = A;
+  g.B = B;
+  g.out = out;
+  g.width = N;
+  return gemm_seg(c, &g, 1, false, a_mn, b_mn, M, out, N, out_f32, res);
 }
 
 // y = x rstd g as an operand (planes), rstd into `rstd`.
@@ -269,9 +307,16 @@ int nea_block_qkv_fwd(const void* x, const void* g, const void* Wq, const void* 
       (rc = make_operand(c, w, Wv, C, Nk, &bv)))
     return rc;
   // q = y Wq: A = y [M][C] K-major; B = Wq [C][Nq], N contiguous: MN-major
-  if ((rc = gemm(c, y, false, bq, true, M, Nq, C, q, Nq, c.f32, false, nullptr)) ||
-      (rc = gemm(c, y, false, bk, true, M, Nk, C, k, Nk, c.f32, false, nullptr)) ||
-      (rc = gemm(c, y, false, bv, true, M, Nk, C, v, Nk, c.f32, false, nullptr)))
+  if (Nq % nea::kGemmBN == 0 && Nk % nea::kGemmBN == 0) {  // one launch, q | k | v side by side along N
+    Seg g[3];
+    g[0].A = y, g[0].B = bq, g[0].out = q, g[0].width = Nq;
+    g[1].A = y, g[1].B = bk, g[1].out = k, g[1].width = Nk;
+    g[2].A = y, g[2].B = bv, g[2].out = v, g[2].width = Nk;
+    return gemm_seg(c, g, 3, false, false, true, M, nullptr, 0, c.f32, nullptr);
+  }
+  if ((rc = gemm(c, y, false, bq, true, M, Nq, q, c.f32, nullptr)) ||
+      (rc = gemm(c, y, false, bk, true, M, Nk, k, c.f32, nullptr)) ||
+      (rc = gemm(c, y, false, bv, true, M, Nk, v, c.f32, nullptr)))
     return rc;
   return NEA_OK;
 }
@@ -310,15 +355,26 @@ int nea_block_qkv_bwd(const void* x, const void* g, const void* Wq, const void* 
       (rc = make_operand(c, w, dk, M, Nk, &gk)) || (rc = make_operand(c, w, dv, M, Nk, &gv)))
     return rc;
   // dW* = y^T d*: A = y^T (y [M][C], C contiguous: MN-major); B = d* [M][N*], MN-major
-  if ((rc = gemm(c, y, true, gq, true, C, Nq, M, dWq, Nq, c.f32, false, nullptr)) ||
-      (rc = gemm(c, y, true, gk, true, C, Nk, M, dWk, Nk, c.f32, false, nullptr)) ||
-      (rc = gemm(c, y, true, gv, true, C, Nk, M, dWv, Nk, c.f32, false, nullptr)))
+  if (Nq % nea::kGemmBN == 0 && Nk % nea::kGemmBN == 0) {  // one launch, side by side along N
+    Seg g[3];
+    g[0].A = y, g[0].B = gq, g[0].out = dWq, g[0].width = Nq;
+    g[1].A = y, g[1].B = gk, g[1].out = dWk, g[1].width = Nk;
+    g[2].A = y, g[2].B = gv, g[2].out = dWv, g[2].width = Nk;
+    if ((rc = gemm_seg(c, g, 3, false, true, true, C, nullptr, 0, c.f32, nullptr))) return rc;
+  } else if ((rc = gemm(c, y, true, gq, true, C, Nq, dWq, c.f32, nullptr)) ||
+             (rc = gemm(c, y, true, gk, true, C, Nk, dWk, c.f32, nullptr)) ||
+             (rc = gemm(c, y, true, gv, true, C, Nk, dWv, c.f32, nullptr))) {
     return rc;
-  // dy = dq Wq^T + dk Wk^T + dv Wv^T (fp32): A = d* K-major; B = W*^T, i.e. W* [C][N*] read K-major
-  if ((rc = gemm(c, gq, false, bq, false, M, C, Nq, dy, C, true, false, nullptr)) ||
-      (rc = gemm(c, gk, false, bk, false, M, C, Nk, dy, C, true, true, nullptr)) ||
-      (rc = gemm(c, gv, false, bv, false, M, C, Nk, dy, C, true, true, nullptr)))
-    return rc;
+  }
+  // dy = dq Wq^T + dk Wk^T + dv Wv^T (fp32), one product chained along K:
+  // A = d* K-major; B = W*^T, i.e. W* [C][N*] read K-major
+  {
+    Seg g[3];
+    g[0].A = gq, g[0].B = bq, g[0].width = Nq;
+    g[1].A = gk, g[1].B = bk, g[1].width = Nk;
+    g[2].A = gv, g[2].B = bv, g[2].width = Nk;
+    if ((rc = gemm_seg(c, g, 3, true, false, false, M, dy, C, true, nullptr))) return rc;
+  }
   cudaError_t err = c.f32 ? launch_pdl(nea::rmsnorm_bwd_rows_kernel<true>, unsigned(n_part), 256u, size_t(C) * 4,
                                        c.stream, x, g, static_cast<const float*>(rstd), static_cast<const float*>(dy),
                                        dres, dx, dg_part, M, C)
@@ -351,7 +407,7 @@ int nea_block_out_fwd(const void* x, const void* o, const void* Wo, void* h, int
   Operand a, b;
   if ((rc = make_operand(c, w, o, M, Nq, &a)) || (rc = make_operand(c, w, Wo, Nq, C, &b))) return rc;
   // h = x + o Wo: A = o [M][Nq] K-major; B = Wo [Nq][C], C contiguous: MN-major
-  return gemm(c, a, false, b, true, M, C, Nq, h, C, c.f32, false, x);
+  return gemm(c, a, false, b, true, M, C, h, c.f32, x);
 }
 
 int nea_block_out_bwd(const void* o, const void* Wo, const void* dh, void* do_, void* dWo, int M, int C, int Hq,
@@ -374,9 +430,9 @@ int nea_block_out_bwd(const void* o, const void* Wo, const void* dh, void* do_, 
       (rc = make_operand(c, w, dh, M, C, &d)))
     return rc;
   // do = dh Wo^T: A = dh [M][C] K-major; B = Wo^T, i.e. Wo [Nq][C] read K-major
-  if ((rc = gemm(c, d, false, b, false, M, Nq, C, do_, Nq, c.f32, false, nullptr))) return rc;
+  if ((rc = gemm(c, d, false, b, false, M, Nq, do_, c.f32, nullptr))) return rc;
   // dWo = o^T dh: A = o^T (o [M][Nq]: MN-major); B = dh [M][C], MN-major
-  return gemm(c, a, true, d, true, Nq, C, M, dWo, C, c.f32, false, nullptr);
+  return gemm(c, a, true, d, true, Nq, C, dWo, c.f32, nullptr);
 }
 
 }  // extern "C"

@@ -21,20 +21,38 @@ namespace nea {
 constexpr int kGemmBM = 128, kGemmBN = 128, kGemmBK = 64;
 constexpr int kGemmThreads = 192;  // warp 0: TMA, warp 1: MMA, warps 2-5: epilogue
 
-struct GemmParams {
-  // operands: hi planes (bf16 storage: the tensors themselves), lo planes
-  // (float32 storage); K-major maps have box {64, 128}, MN-major {64, 64}
+// Up to three operand segments.  Chained along K (kseg): out = sum_s A_s B_s,
+// segment s owning k-steps [begin_s, begin_{s+1}).  Side by side along N:
+// out_s = A B_s for the N tiles [begin_s, begin_{s+1}), A taken from
+// segment 0.  Operands: hi planes (bf16 storage: the tensors themselves), lo
+// planes (float32 storage); K-major maps have box {64, 128}, MN-major {64, 64}.
+constexpr int kGemmMaxSeg = 3;
+struct GemmSeg {
   CUtensorMap a_hi, a_lo, b_hi, b_lo;
-  void* out;          // [M][ldo] row-major, fp32 or bf16
+  void* out;          // N segments: this segment's output [M][ldo]
+  long long ldo;
+  int begin;          // first k-step (K segments) or first N tile (N segments)
+};
+struct GemmParams {
+  GemmSeg seg[kGemmMaxSeg];
+  int n_seg;
+  int kseg;           // 1: segments along K; 0: along N (one segment: either)
+  void* out;          // K segments: [M][ldo] row-major, fp32 or bf16
   const void* res;    // residual added to the result (same layout as out), or nullptr
   long long ldo;
   int M, N, K;
   int out_f32;        // 1: fp32 output, 0: bf16
-  int accumulate;     // 1: out += A B (fp32 output)
   int n_m, n_n, n_k, n_tiles;
   int* err;
   unsigned long long wait_limit;
 };
+
+// Segment holding index i (a k-step or an N tile).
+__device__ __forceinline__ int gemm_seg_of(const GemmParams& p, int i) {
+  int s = 0;
+  while (s + 1 < p.n_seg && i >= p.seg[s + 1].begin) ++s;
+  return s;
+}
 
 template <bool SPLIT>
 struct GemmSmem {
@@ -114,23 +132,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA
     if (lane == 0) {
-      prefetch_tmap(&p.a_hi);
-      prefetch_tmap(&p.b_hi);
       uint32_t it = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x) {
         const int mi = t % p.n_m, ni = t / p.n_m;
+        const int ns = p.kseg ? 0 : gemm_seg_of(p, ni);  // N segment of the tile
+        const GemmSeg& sa = p.seg[0];
+        const int n0 = (ni - (p.kseg ? 0 : p.seg[ns].begin)) * kGemmBN;
         for (int ks = 0; ks < p.n_k; ++ks, ++it) {
           const int s = it % L::ST;
           if (it >= uint32_t(L::ST) && !(ok = wait_thread(&empty[s], ((it / L::ST) - 1) & 1, wc, kErrWaitEmpty)))
             break;
+          const int kq = p.kseg ? gemm_seg_of(p, ks) : 0;  // K segment of the step
+          const GemmSeg& g = p.kseg ? p.seg[kq] : p.seg[ns];
+          const GemmSeg& ga = p.kseg ? p.seg[kq] : sa;
+          const int k0 = (ks - (p.kseg ? p.seg[kq].begin : 0)) * kGemmBK;
           uint8_t* st = sm + s * L::kStage;
           mbar_arrive_expect_tx(&full[s], L::kStage);
-          gemm_load_tile<AMN>(st, &p.a_hi, mi * kGemmBM, ks * kGemmBK, &full[s]);
-          gemm_load_tile<BMN>(st + L::kPlanes * L::kOp, &p.b_hi, ni * kGemmBN, ks * kGemmBK, &full[s]);
+          gemm_load_tile<AMN>(st, &ga.a_hi, mi * kGemmBM, k0, &full[s]);
+          gemm_load_tile<BMN>(st + L::kPlanes * L::kOp, &g.b_hi, n0, k0, &full[s]);
           if constexpr (SPLIT) {
-            gemm_load_tile<AMN>(st + L::kOp, &p.a_lo, mi * kGemmBM, ks * kGemmBK, &full[s]);
-            gemm_load_tile<BMN>(st + 3 * L::kOp, &p.b_lo, ni * kGemmBN, ks * kGemmBK, &full[s]);
+            gemm_load_tile<AMN>(st + L::kOp, &ga.a_lo, mi * kGemmBM, k0, &full[s]);
+            gemm_load_tile<BMN>(st + 3 * L::kOp, &g.b_lo, n0, k0, &full[s]);
           }
         }
       }
@@ -185,28 +208,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       tc_fence_after();
       const int mi = t % p.n_m, ni = t / p.n_m;
       const int row = mi * kGemmBM + q4 * 32 + lane;
+      // the tile's output: its N segment's tensor, or the one output
+      const int ns = p.kseg ? 0 : gemm_seg_of(p, ni);
+      void* const out_base = p.kseg ? p.out : p.seg[ns].out;
+      const long long ldo = p.kseg ? p.ldo : p.seg[ns].ldo;
+      const int ncol0 = (ni - (p.kseg ? 0 : p.seg[ns].begin)) * kGemmBN;  // first column in that tensor
+      const int nlim = p.kseg ? p.N : int(ldo);                           // its column count
 #pragma unroll 1
       for (int c = 0; c < kGemmBN / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(tmem_addr(tbase, q4 * 32, ab * kGemmBN + c * 32), r);
-        const int col0 = ni * kGemmBN + c * 32;
-        if (row >= p.M || col0 >= p.N) continue;
-        const bool whole = col0 + 32 <= p.N;
+        const int col0 = ncol0 + c * 32;
+        if (row >= p.M || col0 >= nlim) continue;
+        const bool whole = col0 + 32 <= nlim;
         float v[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-        const size_t o0 = size_t(row) * p.ldo + col0;
+        const size_t o0 = size_t(row) * ldo + col0;
         if (p.out_f32) {
-          float* out = static_cast<float*>(p.out) + o0;
+          float* out = static_cast<float*>(out_base) + o0;
           const float* res = p.res ? static_cast<const float*>(p.res) + o0 : nullptr;
           if (whole) {
 #pragma unroll
             for (int j = 0; j < 32; j += 4) {
               float4 w = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-              if (p.accumulate) {
-                const float4 u = *reinterpret_cast<const float4*>(out + j);
-                w.x += u.x, w.y += u.y, w.z += u.z, w.w += u.w;
-              }
               if (res) {
                 const float4 u = *reinterpret_cast<const float4*>(res + j);
                 w.x += u.x, w.y += u.y, w.z += u.z, w.w += u.w;
@@ -214,11 +239,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
               *reinterpret_cast<float4*>(out + j) = w;
             }
           } else {
-            for (int j = 0; j < 32 && col0 + j < p.N; ++j)
-              out[j] = v[j] + (p.accumulate ? out[j] : 0.f) + (res ? res[j] : 0.f);
+            for (int j = 0; j < 32 && col0 + j < nlim; ++j) out[j] = v[j] + (res ? res[j] : 0.f);
           }
         } else {
-          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + o0;
+          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(out_base) + o0;
           const __nv_bfloat16* res = p.res ? static_cast<const __nv_bfloat16*>(p.res) + o0 : nullptr;
           if (whole) {
 #pragma unroll
@@ -236,7 +260,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
                   make_uint4(pack_bf16(w[0], w[1]), pack_bf16(w[2], w[3]), pack_bf16(w[4], w[5]), pack_bf16(w[6], w[7]));
             }
           } else {
-            for (int j = 0; j < 32 && col0 + j < p.N; ++j)
+            for (int j = 0; j < 32 && col0 + j < nlim; ++j)
               out[j] = __float2bfloat16_rn(v[j] + (res ? __bfloat162float(res[j]) : 0.f));
           }
         }
