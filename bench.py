@@ -105,6 +105,10 @@ def config_of(w, world):
         return {"workload": w.name, "B": w.B, "Tc": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "storage": storage,
                 "rope_base": w.rope_base, "lens": "all Tc", "l2": decode_l2_note(w),
                 "parallelism": f"dp{world} (independent sequences per GPU)"}
+    if w.block:
+        return {"workload": w.name, "B": w.B, "T": w.T, "C": w.Hq * w.D, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+                "storage": storage, "rmsnorm_eps": 1e-5, "l2": L2_NOTE,
+                "parallelism": f"dp{world} (independent batches per GPU)"}
     return {"workload": w.name, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "storage": storage,
             "causal": w.causal, "rope_base": w.rope_base, "layers": w.layers, "qk_std": w.qk_std, "l2": L2_NOTE,
             "parallelism": f"dp{world} (independent batches per GPU)"}
@@ -544,11 +548,212 @@ def reference_decode(a, w):
     return 0
 
 
+# ---------------------------------------------------------------- block workload
+BLOCK_METRIC = ("decoder-block steps beside the attention (RMSNorm + q/k/v projections, output projection + "
+                "residual), fwd+bwd TFLOP/s (% of tensor-core peak)")
+BLOCK_STEPS = ("qkv_fwd", "out_fwd", "out_bwd", "qkv_bwd")
+
+
+def block_step_flops(w):
+    M, C, Nqkv, Nq = w.B * w.T, w.Hq * w.D, (w.Hq + 2 * w.Hkv) * w.D, w.Hq * w.D
+    return {"qkv_fwd": 2.0 * M * C * Nqkv, "out_fwd": 2.0 * M * Nq * C, "out_bwd": 4.0 * M * Nq * C,
+            "qkv_bwd": 4.0 * M * C * Nqkv}
+
+
+def run_oracle_block(w, rows=None, min_seconds=0.0):
+    """Times the fp64 oracle (numpy) on the block steps for the first `rows`
+    tokens (all by default), repeated until `min_seconds` have passed.
+    Returns (seconds, FLOPs, threads, description)."""
+    from oracle import block_ref
+
+    inp = load_workloads().make_block_inputs(w)
+    a = {n: t.float().double().numpy() for n, t in inp.items()}
+    B = w.B if rows is None else max(1, rows // w.T)
+    for n in ("x", "o", "dh", "dq", "dk", "dv"):
+        a[n] = a[n][:B]
+    sub = load_workloads().replace(w, B=B)
+    reps, dt = 0, 0.0
+    while reps == 0 or dt < min_seconds:
+        t0 = time.perf_counter()
+        q, k, v, y, rstd = block_ref.qkv_fwd(a["x"], a["g"], a["Wq"], a["Wk"], a["Wv"], w.Hq, w.Hkv, w.D)
+        block_ref.out_fwd(a["x"], a["o"], a["Wo"])
+        block_ref.out_bwd(a["o"], a["Wo"], a["dh"])
+        block_ref.qkv_bwd(a["x"], a["g"], a["Wq"], a["Wk"], a["Wv"], y, rstd, a["dq"], a["dk"], a["dv"])
+        dt += time.perf_counter() - t0
+        reps += 1
+    threads = len(os.sched_getaffinity(0))
+    desc = f"block steps on {B} x {w.T} tokens (of {w.B} x {w.T}), fp64 numpy, {reps} repetitions"
+    return dt, sub.block_flops() * reps, threads, desc
+
+
+def reference_block(a, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    run_oracle_block(w, rows=w.T)  # untimed warm-up of the same sample
+    secs, flops, threads, desc = 0.0, 0.0, None, None
+    for _ in range(a.steps):
+        dt, fl, threads, desc = run_oracle_block(w, rows=w.T)
+        secs += dt
+        flops += fl
+    value = flops / secs / 1e12
+    line = {
+        "impl": "reference", "metric": BLOCK_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": a.gpus,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": secs / a.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, a.gpus),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def block_main(a, w, rank, world, local):
+    import torch
+
+    import causal_gqa_attention_sm_b200 as nea
+
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    d = {n: t.to(dev) for n, t in load_workloads().make_block_inputs(w).items()}
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    drain = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    drain_sum = torch.empty((), dtype=torch.float32, device=dev)
+
+    def flush_l2(i):
+        flush.fill_(float(i))
+        torch.sum(drain, dim=0, out=drain_sum)
+
+    def call(name, inp):
+        if name == "qkv_fwd":
+            return nea.nea_block_qkv_fwd(inp["x"], inp["g"], inp["Wq"], inp["Wk"], inp["Wv"], w.Hq, w.Hkv, w.D)
+        if name == "out_fwd":
+            return (nea.nea_block_out_fwd(inp["x"], inp["o"], inp["Wo"]),)
+        if name == "out_bwd":
+            return nea.nea_block_out_bwd(inp["o"], inp["Wo"], inp["dh"])
+        return nea.nea_block_qkv_bwd(inp["x"], inp["g"], inp["Wq"], inp["Wk"], inp["Wv"], inp["dq"], inp["dk"],
+                                     inp["dv"], dres=inp["dh"])
+
+    def step(inp=d, evs=None):
+        outs = []
+        for i, n in enumerate(BLOCK_STEPS):
+            if evs:
+                evs[i].record(stream)
+            outs.extend(call(n, inp))
+        if evs:
+            evs[-1].record(stream)
+        return outs
+
+    for i in range(a.warmup):
+        flush_l2(i)
+        step()
+    torch.cuda.synchronize(dev)
+    if nea.nea_device_status() != nea.NEA_OK:
+        raise SystemExit("device status after warm-up")
+    K = a.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    clocks = ClockSampler(local, a.clocks_csv)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with clocks:
+        window = None if a.profile else clock_window(step, flush_l2, stream, dev, 1.2)
+        for i in range(K):
+            flush_l2(i)
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    # per-step durations: the same steps again with events between the calls
+    ev_k = [[torch.cuda.Event(enable_timing=True) for _ in range(len(BLOCK_STEPS) + 1)] for _ in range(K)]
+    for i in range(K):
+        flush_l2(i)
+        step(evs=ev_k[i])
+    torch.cuda.synchronize(dev)
+    if nea.nea_device_status() != nea.NEA_OK:
+        raise SystemExit("device status after timing")
+    total_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in ev), world)
+    flops = w.block_flops()
+    value = flops * K * world / (total_ms * 1e-3) / 1e12
+    sf = block_step_flops(w)
+    kern_ms = {n: sum(e[j].elapsed_time(e[j + 1]) for e in ev_k) / K for j, n in enumerate(BLOCK_STEPS)}
+    kernels = {n: {"ms_per_call": kern_ms[n], "tflops": sf[n] / (kern_ms[n] * 1e-3) / 1e12,
+                   "share": kern_ms[n] / sum(kern_ms.values())} for n in BLOCK_STEPS}
+    dominant = max(kern_ms, key=kern_ms.get)
+    pk = peaks()
+    tf32 = measure_tf32_peak(dev) if (w.dtype == "f32" and not a.profile) else None
+    achieved = sf[dominant] / (kern_ms[dominant] * 1e-3) / 1e12
+    if tf32:
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tf32["tf32_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / tf32["tf32_tflops"], "traffic": None,
+                "kernel": dominant + " (its GEMMs with the norm and operand-plane kernels)",
+                "peak_kind": "tf32 dense burst (measured in this run: " + tf32["how"] + ")",
+                "frac_of_bf16_peak": achieved / pk["bf16_tflops"], "bf16_peak_kind": f"bf16 dense burst ({pk['source']})"}
+    else:
+        roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / pk["bf16_tflops"], "traffic": None,
+                "kernel": dominant + " (its GEMMs with the norm and operand-plane kernels)",
+                "peak_kind": f"bf16 dense burst ({pk['source']})"}
+    e2e = None
+    if not a.no_e2e:
+        act = ("x", "o", "dh", "dq", "dk", "dv")
+        host = {n: d[n].cpu().pin_memory() for n in act}
+        dev_in = {n: torch.empty_like(d[n]) for n in act}
+        inp = dict(d)
+        inp.update(dev_in)
+        outs = step(inp)
+        host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = sum(t.numel() * t.element_size() for t in host_out)
+
+        def e2e_step():
+            for n in act:
+                dev_in[n].copy_(host[n], non_blocking=True)
+            for t, ho in zip(step(inp), host_out):
+                ho.copy_(t, non_blocking=True)
+
+        for _ in range(a.warmup):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(K):
+            e2e_step()
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(s0.elapsed_time(s1), world)
+        e2e = {"value": flops * K * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h}
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        dt, fl, threads, desc = run_oracle_block(w, rows=w.T, min_seconds=10.0)
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc,
+               "seconds": dt}
+    if rank == 0:
+        line = {
+            "metric": BLOCK_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": a.warmup, "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16x3" if w.dtype == "f32" else "bf16", "data": "synthetic",
+            "config": config_of(w, world), "tokens_per_s": w.B * w.T * K * world / (total_ms * 1e-3),
+            "kernels": kernels, "roofline": roof, "tf32_peak": tf32, "cpu_baseline": cpu, "e2e": e2e,
+            "clocks": clocks.summary(), "clock_window": window,
+            # per step: norm rows, q|k|v GEMM; out GEMM; do and dWo GEMMs; norm
+            # rows, dW and dy GEMMs, norm backward, dg sum; float32 storage adds
+            # the operand-plane kernels (3 + 2 + 3 + 6)
+            "gpu_launches": K * (24 if w.dtype == "f32" else 10),
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 # ---------------------------------------------------------------- GPU arm
 def main():
     a = parse()
     w = load_workloads().WORKLOADS[a.workload]
     if a.impl == "reference":
+        if w.block:
+            return reference_block(a, w)
         return reference_decode(a, w) if w.decode else reference_arm(a, w)
 
     import torch
@@ -558,8 +763,8 @@ def main():
 
     rank, world, local = dist_init(a.gpus)
     torch.cuda.set_device(local)
-    if w.decode:
-        rc = decode_main(a, w, rank, world, local)
+    if w.decode or w.block:
+        rc = (decode_main if w.decode else block_main)(a, w, rank, world, local)
         if world > 1:
             import torch.distributed as dist
 

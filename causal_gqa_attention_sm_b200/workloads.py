@@ -33,6 +33,7 @@ class Workload:
     layers: int = 1     # independent attention layers per step
     seed: int = 0
     decode: bool = False  # one query per sequence over a cache of T positions
+    block: bool = False   # the decoder-block steps beside the attention (model dim C = Hq D)
 
     @property
     def torch_dtype(self):
@@ -49,6 +50,14 @@ class Workload:
         if not self.causal:
             f *= 2.0
         return f * self.layers
+
+    def block_flops(self) -> float:
+        """Algorithmic FLOPs of the block steps' forward and backward on M = B T
+        tokens, C = Hq D: q/k/v projections 2 M C (Hq + 2 Hkv) D forward and
+        twice that backward; output projection 2 M (Hq D) C forward, twice that
+        backward (the norms' elementwise work is not counted)."""
+        M, C = self.B * self.T, self.Hq * self.D
+        return 6.0 * M * C * (self.Hq + 2 * self.Hkv) * self.D + 6.0 * M * self.Hq * self.D * C
 
     def tokens(self) -> int:
         return self.B * (1 if self.decode else self.T) * self.layers
@@ -75,6 +84,8 @@ WORKLOADS = {
     # generation over a key/value cache: 16 sequences, one new token each
     "decode1024": Workload("decode1024", 16, 1024, 12, 4, 64, "f32", seed=6000, decode=True),
     "decode4096": Workload("decode4096", 16, 4096, 12, 4, 64, "bf16", seed=6001, decode=True),
+    # the decoder-block steps of the GPU model layer (dim 768 = 12 x 64)
+    "block": Workload("block", 8, 512, 12, 4, 64, "f32", seed=7000, block=True),
 }
 
 
@@ -105,6 +116,21 @@ def make_decode_inputs(w: Workload, device="cpu"):
     out = {n: t.to(w.torch_dtype).to(device).contiguous() for n, t in {"q": q, "kc": kc, "vc": vc}.items()}
     out["lens"] = torch.full((w.B,), w.T, dtype=torch.int32, device=device)
     return out
+
+
+def make_block_inputs(w: Workload, device="cpu"):
+    """Inputs of the block steps for C = Hq D: x [B, T, C], gain g [C] ~ 1 +
+    N(0, 0.01), weights ~ N(0, 1/fan_in) (Wq [C, Hq D], Wk, Wv [C, Hkv D],
+    Wo [Hq D, C]), the attention output o and the upstream gradients dh, dq,
+    dk, dv ~ N(0, 1); drawn like ``make_inputs``."""
+    g = torch.Generator(device="cpu").manual_seed(int(w.seed))
+    C = w.Hq * w.D
+    r = lambda *shape, std=1.0: torch.randn(shape, generator=g, dtype=torch.float32) * std
+    out = dict(x=r(w.B, w.T, C), g=1.0 + r(C, std=0.1), Wq=r(C, w.Hq * w.D, std=C ** -0.5),
+               Wk=r(C, w.Hkv * w.D, std=C ** -0.5), Wv=r(C, w.Hkv * w.D, std=C ** -0.5),
+               Wo=r(w.Hq * w.D, C, std=(w.Hq * w.D) ** -0.5), o=r(w.B, w.T, w.Hq, w.D), dh=r(w.B, w.T, C),
+               dq=r(w.B, w.T, w.Hq, w.D), dk=r(w.B, w.T, w.Hkv, w.D), dv=r(w.B, w.T, w.Hkv, w.D))
+    return {n: t.to(w.torch_dtype).to(device).contiguous() for n, t in out.items()}
 
 
 def custom(name="custom", **kw) -> Workload:
