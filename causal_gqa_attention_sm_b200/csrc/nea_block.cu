@@ -80,7 +80,13 @@ struct Ctx {
   int n_sm;
   BlockState* st;
   unsigned long long wait_limit;
+  float* part = nullptr;  // split-K partial tiles (a piece of the workspace)
+  size_t part_bytes = 0;
 };
+
+// Bytes set aside for split-K partial tiles: up to 4 chunks of every tile of
+// a product with fewer tiles than SMs.
+size_t part_reserve(int n_sm) { return size_t(n_sm) * 128 * 128 * 4 * 4; }
 
 int setup(Ctx& c, int dtype, void* stream) {
   c.stream = static_cast<cudaStream_t>(stream);
@@ -211,14 +217,29 @@ int gemm_seg(Ctx& c, const Seg* segs, int n_seg, bool kseg, bool a_mn, bool b_mn
   p.err = c.err;
   p.wait_limit = c.wait_limit;
   if (p.n_tiles == 0 || K == 0) return NEA_OK;
-  const unsigned grid = unsigned(std::min(p.n_tiles, c.n_sm));
+  // split K when the tiles leave SMs idle: the chunk count (at most 4, each
+  // of two k-steps or more) that minimises the per-CTA share of work
+  p.split = 1;
+  if (p.n_tiles < c.n_sm && c.part) {
+    double best = double((p.n_tiles + c.n_sm - 1) / c.n_sm);
+    for (int sp = 2; sp <= 4 && p.n_k >= 2 * sp; ++sp) {
+      const double share = double((p.n_tiles * sp + c.n_sm - 1) / c.n_sm) / sp;
+      if (share < best - 1e-9 && size_t(p.n_tiles) * sp * 128 * 128 * 4 <= c.part_bytes) best = share, p.split = sp;
+    }
+  }
+  p.k_per = (p.n_k + p.split - 1) / p.split;
+  p.split = (p.n_k + p.k_per - 1) / p.k_per;
+  p.part = p.split > 1 ? c.part : nullptr;
+  const unsigned grid = unsigned(std::min(p.n_tiles * p.split, c.n_sm));
   auto run = [&](auto kern, uint32_t smem, int bit) -> int {
     if (!(c.st->attr_done & (1u << bit))) {
       const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
       if (e != cudaSuccess) return fail(e);
       c.st->attr_done |= 1u << bit;
     }
-    const cudaError_t e = launch_pdl(kern, grid, unsigned(nea::kGemmThreads), size_t(smem), c.stream, p);
+    cudaError_t e = launch_pdl(kern, grid, unsigned(nea::kGemmThreads), size_t(smem), c.stream, p);
+    if (e == cudaSuccess && p.split > 1)
+      e = launch_pdl(nea::gemm_reduce_kernel, unsigned(p.n_tiles * 16), 256u, size_t(0), c.stream, p);
     return e == cudaSuccess ? NEA_OK : fail(e);
   };
   const int form = (a_mn ? 2 : 0) + (b_mn ? 1 : 0);
@@ -271,7 +292,7 @@ int norm_rows(Ctx& c, Carve& w, const void* x, const void* g, int M, int C, floa
 
 // Widths (C, Hkv D, hence Hq D) in whole 64-column operand boxes.
 int check_dims(int M, int C, int Hq, int Hkv, int D, int dtype) {
-  if (M < 0 || C < 64 || C % 64 != 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return NEA_ERR_ARG;
+  if (M < 0 || C < 64 || C > 4096 || C % 64 != 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return NEA_ERR_ARG;
   if (D < 8 || (Hkv * D) % 64 != 0 || (dtype != NEA_F32 && dtype != NEA_BF16)) return NEA_ERR_ARG;
   if (static_cast<long long>(M) * std::max(C, Hq * D) > (1LL << 31)) return NEA_ERR_ARG;
   return NEA_OK;
@@ -296,10 +317,12 @@ int nea_block_qkv_fwd(const void* x, const void* g, const void* Wq, const void* 
   if ((rc = setup(c, dtype, stream))) return rc;
   const int Nq = Hq * D, Nk = Hkv * D;
   const int e = c.f32 ? 4 : 2;
-  const size_t need = rup(size_t(M) * 4) + rup(size_t(M) * C * e) +
+  const size_t need = part_reserve(c.n_sm) + rup(size_t(M) * 4) + rup(size_t(M) * C * e) +
                       (c.f32 ? rup(size_t(C) * Nq * 4) + 2 * rup(size_t(C) * Nk * 4) : 0) + 4096;
   if ((rc = ensure(c, need))) return rc;
   Carve w{c.st->ws};
+  c.part_bytes = part_reserve(c.n_sm);
+  c.part = static_cast<float*>(w.take(c.part_bytes));
   auto* rstd = static_cast<float*>(w.take(size_t(M) * 4));
   Operand y, bq, bk, bv;
   if ((rc = norm_rows(c, w, x, g, M, C, kNormEps, &y, rstd))) return rc;
@@ -337,7 +360,7 @@ int nea_block_qkv_bwd(const void* x, const void* g, const void* Wq, const void* 
   const int Nq = Hq * D, Nk = Hkv * D;
   const int e = c.f32 ? 4 : 2;
   const int n_part = std::min((M + 7) / 8, c.n_sm * 2);
-  const size_t need = rup(size_t(M) * 4) + rup(size_t(M) * C * e) + rup(size_t(M) * C * 4) +
+  const size_t need = part_reserve(c.n_sm) + rup(size_t(M) * 4) + rup(size_t(M) * C * e) + rup(size_t(M) * C * 4) +
                       rup(size_t(n_part) * C * 4) +
                       (c.f32 ? rup(size_t(C) * Nq * 4) + 2 * rup(size_t(C) * Nk * 4) + rup(size_t(M) * Nq * 4) +
                                    2 * rup(size_t(M) * Nk * 4)
@@ -345,6 +368,8 @@ int nea_block_qkv_bwd(const void* x, const void* g, const void* Wq, const void* 
                       4096;
   if ((rc = ensure(c, need))) return rc;
   Carve w{c.st->ws};
+  c.part_bytes = part_reserve(c.n_sm);
+  c.part = static_cast<float*>(w.take(c.part_bytes));
   auto* rstd = static_cast<float*>(w.take(size_t(M) * 4));
   auto* dy = static_cast<float*>(w.take(size_t(M) * C * 4));
   auto* dg_part = static_cast<float*>(w.take(size_t(n_part) * C * 4));
@@ -375,14 +400,23 @@ int nea_block_qkv_bwd(const void* x, const void* g, const void* Wq, const void* 
     g[2].A = gv, g[2].B = bv, g[2].width = Nk;
     if ((rc = gemm_seg(c, g, 3, true, false, false, M, dy, C, true, nullptr))) return rc;
   }
-  cudaError_t err = c.f32 ? launch_pdl(nea::rmsnorm_bwd_rows_kernel<true>, unsigned(n_part), 256u, size_t(C) * 4,
+  const size_t nb_smem = size_t(C) * 4 * 8;  // the eight warps' dg rows
+  if (nb_smem > 48 * 1024) {
+    const cudaError_t ea =
+        c.f32 ? cudaFuncSetAttribute(nea::rmsnorm_bwd_rows_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     int(nb_smem))
+              : cudaFuncSetAttribute(nea::rmsnorm_bwd_rows_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     int(nb_smem));
+    if (ea != cudaSuccess) return fail(ea);
+  }
+  cudaError_t err = c.f32 ? launch_pdl(nea::rmsnorm_bwd_rows_kernel<true>, unsigned(n_part), 256u, nb_smem,
                                        c.stream, x, g, static_cast<const float*>(rstd), static_cast<const float*>(dy),
                                        dres, dx, dg_part, M, C)
-                          : launch_pdl(nea::rmsnorm_bwd_rows_kernel<false>, unsigned(n_part), 256u, size_t(C) * 4,
+                          : launch_pdl(nea::rmsnorm_bwd_rows_kernel<false>, unsigned(n_part), 256u, nb_smem,
                                        c.stream, x, g, static_cast<const float*>(rstd), static_cast<const float*>(dy),
                                        dres, dx, dg_part, M, C);
   if (err != cudaSuccess) return fail(err);
-  const unsigned cg = unsigned((C + 255) / 256);
+  const unsigned cg = unsigned((C + 31) / 32);
   err = c.f32 ? launch_pdl(nea::colsum_kernel<true>, cg, 256u, size_t(0), c.stream,
                            static_cast<const float*>(dg_part), n_part, C, dg)
               : launch_pdl(nea::colsum_kernel<false>, cg, 256u, size_t(0), c.stream,
@@ -401,9 +435,11 @@ int nea_block_out_fwd(const void* x, const void* o, const void* Wo, void* h, int
   Ctx c;
   if ((rc = setup(c, dtype, stream))) return rc;
   const int Nq = Hq * D;
-  const size_t need = (c.f32 ? rup(size_t(M) * Nq * 4) + rup(size_t(Nq) * C * 4) : 0) + 4096;
+  const size_t need = part_reserve(c.n_sm) + (c.f32 ? rup(size_t(M) * Nq * 4) + rup(size_t(Nq) * C * 4) : 0) + 4096;
   if ((rc = ensure(c, need))) return rc;
   Carve w{c.st->ws};
+  c.part_bytes = part_reserve(c.n_sm);
+  c.part = static_cast<float*>(w.take(c.part_bytes));
   Operand a, b;
   if ((rc = make_operand(c, w, o, M, Nq, &a)) || (rc = make_operand(c, w, Wo, Nq, C, &b))) return rc;
   // h = x + o Wo: A = o [M][Nq] K-major; B = Wo [Nq][C], C contiguous: MN-major
@@ -421,10 +457,12 @@ int nea_block_out_bwd(const void* o, const void* Wo, const void* dh, void* do_, 
   Ctx c;
   if ((rc = setup(c, dtype, stream))) return rc;
   const int Nq = Hq * D;
-  const size_t need =
+  const size_t need = part_reserve(c.n_sm) +
       (c.f32 ? rup(size_t(M) * Nq * 4) + rup(size_t(Nq) * C * 4) + rup(size_t(M) * C * 4) : 0) + 4096;
   if ((rc = ensure(c, need))) return rc;
   Carve w{c.st->ws};
+  c.part_bytes = part_reserve(c.n_sm);
+  c.part = static_cast<float*>(w.take(c.part_bytes));
   Operand a, b, d;
   if ((rc = make_operand(c, w, o, M, Nq, &a)) || (rc = make_operand(c, w, Wo, Nq, C, &b)) ||
       (rc = make_operand(c, w, dh, M, C, &d)))

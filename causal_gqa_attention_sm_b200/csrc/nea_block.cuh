@@ -43,6 +43,11 @@ struct GemmParams {
   int M, N, K;
   int out_f32;        // 1: fp32 output, 0: bf16
   int n_m, n_n, n_k, n_tiles;
+  // split K: work unit u is tile u % n_tiles over k-steps of chunk u /
+  // n_tiles; with split > 1 each unit writes an fp32 partial tile to
+  // part[u][128][128] and gemm_reduce_kernel sums them into the output
+  int split, k_per;   // chunks, k-steps per chunk
+  float* part;
   int* err;
   unsigned long long wait_limit;
 };
@@ -52,6 +57,42 @@ __device__ __forceinline__ int gemm_seg_of(const GemmParams& p, int i) {
   int s = 0;
   while (s + 1 < p.n_seg && i >= p.seg[s + 1].begin) ++s;
   return s;
+}
+
+// Writes value v of output element (row, tile column c) of tile `ni`: the
+// tile's N segment (or the one output), residual added, fp32 or bf16.
+__device__ __forceinline__ void gemm_store(const GemmParams& p, int row, int ni, int c, float v) {
+  const int ns = p.kseg ? 0 : gemm_seg_of(p, ni);
+  void* const out = p.kseg ? p.out : p.seg[ns].out;
+  const long long ldo = p.kseg ? p.ldo : p.seg[ns].ldo;
+  const int col = (ni - (p.kseg ? 0 : p.seg[ns].begin)) * 128 + c;
+  if (row >= p.M || col >= (p.kseg ? p.N : int(ldo))) return;
+  const size_t o = size_t(row) * ldo + col;
+  if (p.out_f32) {
+    static_cast<float*>(out)[o] = v + (p.res ? static_cast<const float*>(p.res)[o] : 0.f);
+  } else {
+    const float r = p.res ? __bfloat162float(static_cast<const __nv_bfloat16*>(p.res)[o]) : 0.f;
+    static_cast<__nv_bfloat16*>(out)[o] = __float2bfloat16_rn(v + r);
+  }
+}
+
+// Sums the split partial tiles in chunk order (deterministic) and stores
+// the output: 16 CTAs per tile, four consecutive elements per thread.
+__global__ void __launch_bounds__(256) gemm_reduce_kernel(const __grid_constant__ GemmParams p) {
+  grid_dep_wait();
+  grid_dep_launch();
+  const int t = blockIdx.x >> 4, mi = t % p.n_m, ni = t / p.n_m;
+  const int e = ((blockIdx.x & 15) * 256 + threadIdx.x) * 4;  // element of the 128 x 128 tile
+  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s < p.split; ++s) {
+    const float4 u = *reinterpret_cast<const float4*>(p.part + (size_t(s) * p.n_tiles + t) * 128 * 128 + e);
+    v.x += u.x, v.y += u.y, v.z += u.z, v.w += u.w;
+  }
+  const int row = mi * 128 + e / 128, c = e % 128;
+  gemm_store(p, row, ni, c, v.x);
+  gemm_store(p, row, ni, c + 1, v.y);
+  gemm_store(p, row, ni, c + 2, v.z);
+  gemm_store(p, row, ni, c + 3, v.w);
 }
 
 template <bool SPLIT>
@@ -134,12 +175,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x) {
+      for (int u = blockIdx.x; u < p.n_tiles * p.split && ok; u += gridDim.x) {
+        const int t = u % p.n_tiles, kb = (u / p.n_tiles) * p.k_per, ke = min(p.n_k, kb + p.k_per);
         const int mi = t % p.n_m, ni = t / p.n_m;
         const int ns = p.kseg ? 0 : gemm_seg_of(p, ni);  // N segment of the tile
         const GemmSeg& sa = p.seg[0];
         const int n0 = (ni - (p.kseg ? 0 : p.seg[ns].begin)) * kGemmBN;
-        for (int ks = 0; ks < p.n_k; ++ks, ++it) {
+        for (int ks = kb; ks < ke; ++ks, ++it) {
           const int s = it % L::ST;
           if (it >= uint32_t(L::ST) && !(ok = wait_thread(&empty[s], ((it / L::ST) - 1) & 1, wc, kErrWaitEmpty)))
             break;
@@ -167,11 +209,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     uint32_t it = 0, last = 0xffffffffu;  // the last stage use committed
     int lt = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x, ++lt) {
+    for (int u = blockIdx.x; u < p.n_tiles * p.split && ok; u += gridDim.x, ++lt) {
+      const int kb = (u / p.n_tiles) * p.k_per, ke = min(p.n_k, kb + p.k_per);
       const int ab = lt & 1;
       if (lt >= 2) ok = wait_warp(&acc_empty[ab], ((lt >> 1) - 1) & 1, wc, kErrWaitSoftmax);
       tc_fence_after();
-      for (int ks = 0; ks < p.n_k && ok; ++ks, ++it) {
+      for (int ks = kb; ks < ke && ok; ++ks, ++it) {
         const int s = it % L::ST;
         if (!(ok = wait_warp(&full[s], (it / L::ST) & 1, wc, kErrWaitProducer))) break;
         tc_fence_after();
@@ -185,11 +228,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
               // hi*hi, hi*lo, lo*hi
               const uint32_t ap = a + (term == 2 ? L::kOp : 0), bp = b + (term == 1 ? L::kOp : 0);
               mma_ss(tbase + ab * kGemmBN, gemm_desc<AMN>(ap, kk), gemm_desc<BMN>(bp, kk), idesc,
-                     (ks | kk | term) != 0);
+                     ((ks - kb) | kk | term) != 0);
             }
           }
           tc_commit(&empty[s]);
-          if (ks == p.n_k - 1) tc_commit(&acc_full[ab]);
+          if (ks == ke - 1) tc_commit(&acc_full[ab]);
           last = it;
         }
         __syncwarp();
@@ -202,10 +245,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     const int q4 = warp & 3;  // TMEM lanes 32 q4 .. 32 q4 + 31
     int lt = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x, ++lt) {
+    for (int u = blockIdx.x; u < p.n_tiles * p.split && ok; u += gridDim.x, ++lt) {
+      const int t = u % p.n_tiles;
       const int ab = lt & 1;
       if (!(ok = wait_warp(&acc_full[ab], (lt >> 1) & 1, wc, kErrWaitMma))) break;
       tc_fence_after();
+      if (p.split > 1) {  // this chunk's partial tile, row-major 128 x 128 fp32
+        float* dst = p.part + size_t(u) * 128 * 128 + size_t(q4 * 32 + lane) * 128;
+#pragma unroll 1
+        for (int c = 0; c < kGemmBN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tmem_addr(tbase, q4 * 32, ab * kGemmBN + c * 32), r);
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4*>(dst + c * 32 + j) = make_float4(
+                __uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[ab]);
+        continue;
+      }
       const int mi = t % p.n_m, ni = t / p.n_m;
       const int row = mi * kGemmBM + q4 * 32 + lane;
       // the tile's output: its N segment's tensor, or the one output
@@ -279,35 +339,74 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
 }
 
 // ------------------------------------------------------------------ RMSNorm rows
-// One warp per token row of x [M][C] (C a multiple of 8): rstd = (mean x^2 +
-// eps)^-1/2, y = x rstd g written as the GEMM operand (bfloat16 storage:
-// y in bf16; float32 storage: bf16 hi and lo planes of y).
+// Elements of a row handled as 16-byte chunks: 4 fp32 or 8 bf16 values.
+template <bool F32IO>
+struct RowChunk {
+  static constexpr int N = F32IO ? 4 : 8;
+  float v[N];
+  __device__ __forceinline__ void load(const void* base, size_t elem) {
+    const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(base) + elem * (F32IO ? 4 : 2));
+    if constexpr (F32IO) {
+      v[0] = __uint_as_float(u.x), v[1] = __uint_as_float(u.y), v[2] = __uint_as_float(u.z), v[3] = __uint_as_float(u.w);
+    } else {
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) v[2 * k] = bf16_lo_f(w[k]), v[2 * k + 1] = bf16_hi_f(w[k]);
+    }
+  }
+  __device__ __forceinline__ void store(void* base, size_t elem) const {
+    uint4 u;
+    if constexpr (F32IO) {
+      u = make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]), __float_as_uint(v[3]));
+    } else {
+      u = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+    }
+    *reinterpret_cast<uint4*>(static_cast<uint8_t*>(base) + elem * (F32IO ? 4 : 2)) = u;
+  }
+};
+
+// One warp per token row of x [M][C] (C a multiple of 64): rstd = (mean x^2
+// + eps)^-1/2, y = x rstd g written as the GEMM operand (bfloat16 storage:
+// y in bf16; float32 storage: bf16 hi and lo planes of y).  Lanes take
+// 16-byte chunks of the row.
 template <bool F32IO>
 __global__ void __launch_bounds__(256) rmsnorm_rows_kernel(const void* x, const void* g, __nv_bfloat16* y_hi,
                                                            __nv_bfloat16* y_lo, float* rstd, int M, int C,
                                                            float eps) {
+  using RC = RowChunk<F32IO>;
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   grid_dep_wait();
   grid_dep_launch();
   if (row >= M) return;
-  auto load = [&](const void* base, size_t i) {
-    return F32IO ? static_cast<const float*>(base)[i] : __bfloat162float(static_cast<const __nv_bfloat16*>(base)[i]);
-  };
   const size_t r0 = size_t(row) * C;
   float ss = 0.f;
-  for (int j = lane; j < C; j += 32) {
-    const float v = load(x, r0 + j);
-    ss = fmaf(v, v, ss);
+  for (int j = lane * RC::N; j < C; j += 32 * RC::N) {
+    RC a;
+    a.load(x, r0 + j);
+#pragma unroll
+    for (int k = 0; k < RC::N; ++k) ss = fmaf(a.v[k], a.v[k], ss);
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(kFullMask, ss, off);
   const float rs = 1.f / sqrtf(ss / float(C) + eps);
   if (lane == 0) rstd[row] = rs;
-  for (int j = lane; j < C; j += 32) {
-    const float yv = load(x, r0 + j) * rs * load(g, j);
-    const __nv_bfloat16 h = __float2bfloat16_rn(yv);
-    y_hi[r0 + j] = h;
-    if (F32IO) y_lo[r0 + j] = __float2bfloat16_rn(yv - __bfloat162float(h));
+  for (int j = lane * RC::N; j < C; j += 32 * RC::N) {
+    RC a, gg;
+    a.load(x, r0 + j);
+    gg.load(g, j);
+    float yv[RC::N];
+#pragma unroll
+    for (int k = 0; k < RC::N; ++k) yv[k] = a.v[k] * rs * gg.v[k];
+    if constexpr (F32IO) {
+      uint2 h, l;
+      split_bf16(yv[0], yv[1], h.x, l.x);
+      split_bf16(yv[2], yv[3], h.y, l.y);
+      *reinterpret_cast<uint2*>(y_hi + r0 + j) = h;
+      *reinterpret_cast<uint2*>(y_lo + r0 + j) = l;
+    } else {
+      *reinterpret_cast<uint4*>(y_hi + r0 + j) =
+          make_uint4(pack_bf16(yv[0], yv[1]), pack_bf16(yv[2], yv[3]), pack_bf16(yv[4], yv[5]), pack_bf16(yv[6], yv[7]));
+    }
   }
 }
 
@@ -330,52 +429,89 @@ __global__ void __launch_bounds__(256) split_planes_kernel(const float* src, __n
 // dy [M][C] (fp32) and the forward's x, g, rstd,
 //   dx = rstd g dy - x rstd^3 / C sum_j (g dy)_j x_j  (+ dres),
 // and this CTA's share of dg = sum_tokens dy x rstd, written to
-// dg_part[blockIdx.x][C] (fp32).
+// dg_part[blockIdx.x][C] (fp32).  Each warp sums its rows' dg terms in its
+// own shared-memory row (every column owned by one lane), the CTA adds the
+// eight rows at the end.
 template <bool F32IO>
 __global__ void __launch_bounds__(256) rmsnorm_bwd_rows_kernel(const void* x, const void* g, const float* rstd,
                                                                const float* dy, const void* dres, void* dx,
                                                                float* dg_part, int M, int C) {
-  extern __shared__ float dg_s[];  // [C]
+  using RC = RowChunk<F32IO>;
+  extern __shared__ float dg_s[];  // [8 warps][C]
   grid_dep_wait();
   grid_dep_launch();
-  for (int j = threadIdx.x; j < C; j += 256) dg_s[j] = 0.f;
-  __syncthreads();
-  auto load = [&](const void* base, size_t i) {
-    return F32IO ? static_cast<const float*>(base)[i] : __bfloat162float(static_cast<const __nv_bfloat16*>(base)[i]);
-  };
-  const int lane = threadIdx.x & 31;
-  for (int row = blockIdx.x * 8 + (threadIdx.x >> 5); row < M; row += gridDim.x * 8) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* mine = dg_s + size_t(warp) * C;
+  for (int j = lane; j < C; j += 32) mine[j] = 0.f;
+  for (int row = blockIdx.x * 8 + warp; row < M; row += gridDim.x * 8) {
     const size_t r0 = size_t(row) * C;
     const float rs = rstd[row];
     float dot = 0.f;
-    for (int j = lane; j < C; j += 32) dot = fmaf(load(g, j) * dy[r0 + j], load(x, r0 + j), dot);
+    for (int j = lane * RC::N; j < C; j += 32 * RC::N) {
+      RC a, gg;
+      a.load(x, r0 + j);
+      gg.load(g, j);
+#pragma unroll
+      for (int k = 0; k < RC::N; k += 4) {
+        const float4 d = *reinterpret_cast<const float4*>(dy + r0 + j + k);
+        dot = fmaf(gg.v[k] * d.x, a.v[k], dot);
+        dot = fmaf(gg.v[k + 1] * d.y, a.v[k + 1], dot);
+        dot = fmaf(gg.v[k + 2] * d.z, a.v[k + 2], dot);
+        dot = fmaf(gg.v[k + 3] * d.w, a.v[k + 3], dot);
+      }
+    }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(kFullMask, dot, off);
     const float c2 = rs * rs * rs * dot / float(C);
-    for (int j = lane; j < C; j += 32) {
-      const float xv = load(x, r0 + j), d = dy[r0 + j];
-      float v = rs * load(g, j) * d - xv * c2;
-      if (dres) v += load(dres, r0 + j);
-      if (F32IO) static_cast<float*>(dx)[r0 + j] = v;
-      else static_cast<__nv_bfloat16*>(dx)[r0 + j] = __float2bfloat16_rn(v);
-      atomicAdd(&dg_s[j], d * xv * rs);
+    for (int j = lane * RC::N; j < C; j += 32 * RC::N) {
+      RC a, gg, out;
+      a.load(x, r0 + j);
+      gg.load(g, j);
+      RC rr;
+      if (dres) rr.load(dres, r0 + j);
+#pragma unroll
+      for (int k = 0; k < RC::N; k += 4) {
+        const float4 d = *reinterpret_cast<const float4*>(dy + r0 + j + k);
+        const float dd[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          out.v[k + q] = rs * gg.v[k + q] * dd[q] - a.v[k + q] * c2 + (dres ? rr.v[k + q] : 0.f);
+          mine[j + k + q] += dd[q] * a.v[k + q] * rs;
+        }
+      }
+      out.store(dx, r0 + j);
     }
   }
   __syncthreads();
-  for (int j = threadIdx.x; j < C; j += 256) dg_part[size_t(blockIdx.x) * C + j] = dg_s[j];
+  for (int j = threadIdx.x; j < C; j += 256) {
+    float acc = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) acc += dg_s[size_t(w) * C + j];
+    dg_part[size_t(blockIdx.x) * C + j] = acc;
+  }
 }
 
-// dg[j] = sum over the parts of dg_part[.][j], in the storage type.
+// dg[j] = sum over the parts of dg_part[.][j], in the storage type: a CTA
+// per 32 columns, its eight warps summing every eighth part, then the warps'
+// sums added in a fixed order.
 template <bool F32IO>
 __global__ void __launch_bounds__(256) colsum_kernel(const float* part, int n_part, int C, void* dg) {
+  __shared__ float red[8][32];
   grid_dep_wait();
   grid_dep_launch();
-  const int j = blockIdx.x * 256 + threadIdx.x;
-  if (j >= C) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j = blockIdx.x * 32 + lane;
   float s = 0.f;
-  for (int i = 0; i < n_part; ++i) s += part[size_t(i) * C + j];
-  if (F32IO) static_cast<float*>(dg)[j] = s;
-  else static_cast<__nv_bfloat16*>(dg)[j] = __float2bfloat16_rn(s);
+  if (j < C)
+    for (int i = warp; i < n_part; i += 8) s += part[size_t(i) * C + j];
+  red[warp][lane] = s;
+  __syncthreads();
+  if (warp != 0 || j >= C) return;
+  float t = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) t += red[w][lane];
+  if (F32IO) static_cast<float*>(dg)[j] = t;
+  else static_cast<__nv_bfloat16*>(dg)[j] = __float2bfloat16_rn(t);
 }
 
 }  // namespace nea
