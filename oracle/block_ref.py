@@ -1,6 +1,7 @@
 """fp64 CPU oracle for the steps on either side of the attention: the RMSNorm
 pre-norm feeding the Q/K/V projections, and the output projection with the
-residual add, forward and backward.
+residual add, forward and backward; and the block's other half, the
+pre-norm SwiGLU feed-forward with its residual add.
 
 TEST INFRASTRUCTURE ONLY: imported by ``tests/``, never by the product
 package.  Plain numpy in float64; a matrix product is the only library step.
@@ -20,6 +21,11 @@ Readings where the pages are silent:
     the Hq*D outputs of a token are Hq heads of D consecutive values (the
     attention layout [B, T, Hq, D]); likewise K, V with Hkv heads;
   * the block output is h = x + o @ Wo with o in [B, T, Hq*D], Wo [Hq*D, C].
+  * SwiGLU feed-forward (the pages: down(silu(gate(x)) * up(x)), silu(z) =
+    z * sigmoid(z), inside a residual branch with its own pre-norm):
+    h = x + (silu(y @ Wg) * (y @ Wu)) @ Wd with y = RMSNorm(x) * g, Wg and Wu
+    of shape [C, F], Wd [F, C]; the pages give no width F: F = 4 C (the
+    GPT-2-small MLP width of the configuration they name).
 
 Arrays: x, h, dh [B, T, C]; g [C]; Wq [C, Hq*D]; Wk, Wv [C, Hkv*D];
 Wo [Hq*D, C]; q, o [B, T, Hq, D]; k, v [B, T, Hkv, D].
@@ -93,6 +99,43 @@ def out_bwd(o, Wo, dh):
     dh2 = np.asarray(dh, np.float64).reshape(B * T, -1)
     o2 = o.reshape(B * T, -1)
     return np.asarray(dh, np.float64).copy(), (dh2 @ Wo.T).reshape(o.shape), o2.T @ dh2
+
+
+# ----------------------------------------------------------------- SwiGLU feed-forward
+def silu(z):
+    z = np.asarray(z, np.float64)
+    return z / (1.0 + np.exp(-z))
+
+
+def ffn_fwd(x, g, Wg, Wu, Wd, eps=EPS):
+    """h = x + (silu(y Wg) * (y Wu)) Wd, y = RMSNorm(x) g.  Returns h and the
+    saved (y, rstd, a, b) with a = y Wg, b = y Wu."""
+    B, T, C = x.shape
+    y, rstd = rmsnorm_fwd(x, g, eps)
+    y2 = y.reshape(B * T, C)
+    a, b = y2 @ Wg, y2 @ Wu
+    h = np.asarray(x, np.float64) + ((silu(a) * b) @ Wd).reshape(B, T, C)
+    return h, dict(y=y, rstd=rstd, a=a, b=b)
+
+
+def ffn_bwd(x, g, Wg, Wu, Wd, saved, dh):
+    """Backward of ffn_fwd for the upstream gradient dh: returns (dx, dg, dWg,
+    dWu, dWd); dx includes the residual branch's dh.  With s = sigmoid(a):
+    d silu(a)/da = s (1 + a (1 - s))."""
+    B, T, C = x.shape
+    y2 = saved["y"].reshape(B * T, C)
+    a, b = saved["a"], saved["b"]
+    dh2 = np.asarray(dh, np.float64).reshape(B * T, C)
+    act = silu(a) * b
+    dWd = act.T @ dh2
+    dact = dh2 @ Wd.T
+    s = 1.0 / (1.0 + np.exp(-a))
+    da = dact * b * s * (1.0 + a * (1.0 - s))
+    db = dact * silu(a)
+    dWg, dWu = y2.T @ da, y2.T @ db
+    dy = (da @ Wg.T + db @ Wu.T).reshape(B, T, C)
+    dx, dg = rmsnorm_bwd(x, g, saved["rstd"], dy)
+    return dx + np.asarray(dh, np.float64), dg, dWg, dWu, dWd
 
 
 # ----------------------------------------------------------------- whole block

@@ -1,7 +1,7 @@
 """Pins of the fp64 block oracle (oracle/block_ref.py): the RMSNorm pre-norm,
-the Q/K/V projections and the output projection with the residual, forward
-and backward, checked against closed forms, brute-force sums and central
-finite differences (no GPU)."""
+the Q/K/V projections and the output projection with the residual, and the
+SwiGLU feed-forward, forward and backward, checked against closed forms,
+brute-force sums and central finite differences (no GPU)."""
 import numpy as np
 import pytest
 
@@ -123,3 +123,59 @@ def test_whole_block_backward_against_finite_differences(causal):
     grads = br.block_bwd(x, g, Wq, Wk, Wv, Wo, saved, dh, base, causal)
     _fd(lambda: float(np.sum(dh * br.block_fwd(x, g, Wq, Wk, Wv, Wo, Hq, Hkv, D, base, causal)[0])),
         [x, g, Wq, Wk, Wv, Wo], list(grads))
+
+
+# ----------------------------------------------------------------- SwiGLU feed-forward
+def test_silu_closed_forms():
+    assert br.silu(0.0) == 0.0
+    assert abs(br.silu(1.0) - 1.0 / (1.0 + np.exp(-1.0))) < 1e-15
+    z = np.linspace(-30, 30, 61)
+    assert np.allclose(br.silu(z) - br.silu(-z), z, rtol=0, atol=1e-12)  # silu(z) - silu(-z) = z
+    assert np.all(np.abs(br.silu(z[z < -20])) < 1e-6)                    # vanishes for large negative z
+    assert np.allclose(br.silu(z[z > 20]), z[z > 20], rtol=0, atol=1e-6)  # tends to z for large positive z
+
+
+def test_ffn_matches_brute_force_sums():
+    rng = np.random.default_rng(7)
+    B, T, C, F = 1, 2, 4, 6
+    x, g = rng.standard_normal((B, T, C)), rng.standard_normal(C)
+    Wg, Wu, Wd = rng.standard_normal((C, F)), rng.standard_normal((C, F)), rng.standard_normal((F, C))
+    h, sv = br.ffn_fwd(x, g, Wg, Wu, Wd)
+    for t in range(T):
+        ms = sum(x[0, t, c] ** 2 for c in range(C)) / C
+        y = [x[0, t, c] / (ms + br.EPS) ** 0.5 * g[c] for c in range(C)]
+        act = []
+        for f in range(F):
+            a = sum(y[c] * Wg[c, f] for c in range(C))
+            b = sum(y[c] * Wu[c, f] for c in range(C))
+            act.append(a / (1.0 + np.exp(-a)) * b)
+        for c in range(C):
+            ref = x[0, t, c] + sum(act[f] * Wd[f, c] for f in range(F))
+            assert abs(h[0, t, c] - ref) < 1e-12
+
+
+def test_ffn_backward_against_finite_differences():
+    rng = np.random.default_rng(8)
+    B, T, C, F = 1, 3, 4, 5
+    x, g = rng.standard_normal((B, T, C)), rng.standard_normal(C)
+    Wg, Wu, Wd = rng.standard_normal((C, F)), rng.standard_normal((C, F)), rng.standard_normal((F, C))
+    dh = rng.standard_normal((B, T, C))
+    _, sv = br.ffn_fwd(x, g, Wg, Wu, Wd)
+    dx, dg, dWg, dWu, dWd = br.ffn_bwd(x, g, Wg, Wu, Wd, sv, dh)
+    _fd(lambda: float(np.sum(dh * br.ffn_fwd(x, g, Wg, Wu, Wd)[0])), [x, g, Wg, Wu, Wd], [dx, dg, dWg, dWu, dWd])
+
+
+def test_ffn_backward_pin_catches_a_dropped_term():
+    """A plausible mistake -- d silu(a)/da taken as sigmoid(a) -- fails the
+    finite-difference pin."""
+    rng = np.random.default_rng(9)
+    B, T, C, F = 1, 2, 3, 4
+    x, g = rng.standard_normal((B, T, C)), rng.standard_normal(C)
+    Wg, Wu, Wd = rng.standard_normal((C, F)), rng.standard_normal((C, F)), rng.standard_normal((F, C))
+    dh = rng.standard_normal((B, T, C))
+    _, sv = br.ffn_fwd(x, g, Wg, Wu, Wd)
+    a, b = sv["a"], sv["b"]
+    dact = dh.reshape(B * T, C) @ Wd.T
+    wrong = (sv["y"].reshape(B * T, C).T @ (dact * b / (1.0 + np.exp(-a))))
+    with pytest.raises(AssertionError):
+        _fd(lambda: float(np.sum(dh * br.ffn_fwd(x, g, Wg, Wu, Wd)[0])), [Wg], [wrong])
