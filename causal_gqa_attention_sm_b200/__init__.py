@@ -19,7 +19,8 @@ __all__ = [
     "nea_status_string", "nea_version", "nea_set_profile_events", "NeaError", "LIB_PATH", "NEA_OK", "NEA_ERR_ARG", "NEA_ERR_CUDA",
     "NEA_ERR_TIMEOUT", "NEA_ERR_UNSUPPORTED", "NEA_ERR_NOMEM", "NEA_ERR_SCRATCH_LIMIT", "NEA_F32", "NEA_BF16",
     "nea_attn_bwd_noalloc", "nea_attn_decode", "nea_attn_saved_bytes", "nea_attn_fwd_save", "nea_attn_bwd_saved",
-    "nea_block_qkv_fwd", "nea_block_qkv_bwd", "nea_block_out_fwd", "nea_block_out_bwd",
+    "nea_block_qkv_fwd", "nea_block_qkv_bwd", "nea_block_out_fwd", "nea_block_out_bwd", "nea_block_ffn_fwd",
+    "nea_block_ffn_bwd",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnea.so")
@@ -64,6 +65,10 @@ _lib.nea_block_out_fwd.argtypes = [_vp] * 4 + [_i] * 5 + [_vp]
 _lib.nea_block_out_fwd.restype = _i
 _lib.nea_block_out_bwd.argtypes = [_vp] * 5 + [_i] * 5 + [_vp]
 _lib.nea_block_out_bwd.restype = _i
+_lib.nea_block_ffn_fwd.argtypes = [_vp] * 8 + [_i] * 4 + [_vp]
+_lib.nea_block_ffn_fwd.restype = _i
+_lib.nea_block_ffn_bwd.argtypes = [_vp] * 13 + [_i] * 4 + [_vp]
+_lib.nea_block_ffn_bwd.restype = _i
 _lib.nea_version.argtypes = []
 _lib.nea_version.restype = _i
 
@@ -364,6 +369,55 @@ def nea_block_out_bwd(o, Wo, dh, stream=None):
     if rc != NEA_OK:
         raise NeaError(rc, "nea_block_out_bwd")
     return do, dWo
+
+
+def nea_block_ffn_fwd(x, g, Wg, Wu, Wd, h=None, save=True, stream=None):
+    """Pre-norm SwiGLU feed-forward with the residual: ``h = x + (silu(y Wg) *
+    (y Wu)) Wd`` for ``x`` of shape ``[B, T, C]``, ``y`` the RMSNorm of ``x``
+    with gain ``g``.  Returns ``(h, a, b)``, ``a = y Wg`` and ``b = y Wu`` of
+    shape ``[B, T, F]`` saved for the backward (``None`` when ``save`` is
+    false)."""
+    import torch
+
+    B, T, C = x.shape
+    F = Wg.shape[1]
+    dev, dt = x.device, x.dtype
+    code = _dtype_code(x)
+    for t, n, shp in ((x, "x", (B, T, C)), (g, "g", (C,)), (Wg, "Wg", (C, F)), (Wu, "Wu", (C, F)),
+                      (Wd, "Wd", (F, C))):
+        _block_check(n, t, shp, dt, dev)
+    h = torch.empty_like(x) if h is None else h
+    _block_check("h", h, (B, T, C), dt, dev)
+    a = torch.empty((B, T, F), dtype=dt, device=dev) if save else None
+    b = torch.empty((B, T, F), dtype=dt, device=dev) if save else None
+    rc = _lib.nea_block_ffn_fwd(_ptr(x), _ptr(g), _ptr(Wg), _ptr(Wu), _ptr(Wd), _ptr(h), _ptr(a), _ptr(b), B * T,
+                                C, F, code, _stream(stream))
+    if rc != NEA_OK:
+        raise NeaError(rc, "nea_block_ffn_fwd")
+    return h, a, b
+
+
+def nea_block_ffn_bwd(x, g, Wg, Wu, Wd, a, b, dh, stream=None):
+    """Backward of ``nea_block_ffn_fwd`` from its saved ``a`` and ``b``:
+    returns ``(dx, dg, dWg, dWu, dWd)``, ``dx`` including the residual's
+    ``dh``."""
+    import torch
+
+    B, T, C = x.shape
+    F = Wg.shape[1]
+    dev, dt = x.device, x.dtype
+    code = _dtype_code(x)
+    for t, n, shp in ((x, "x", (B, T, C)), (g, "g", (C,)), (Wg, "Wg", (C, F)), (Wu, "Wu", (C, F)),
+                      (Wd, "Wd", (F, C)), (a, "a", (B, T, F)), (b, "b", (B, T, F)), (dh, "dh", (B, T, C))):
+        _block_check(n, t, shp, dt, dev)
+    dx, dg = torch.empty_like(x), torch.empty_like(g)
+    dWg, dWu, dWd = torch.empty_like(Wg), torch.empty_like(Wu), torch.empty_like(Wd)
+    rc = _lib.nea_block_ffn_bwd(_ptr(x), _ptr(g), _ptr(Wg), _ptr(Wu), _ptr(Wd), _ptr(a), _ptr(b), _ptr(dh),
+                                _ptr(dx), _ptr(dg), _ptr(dWg), _ptr(dWu), _ptr(dWd), B * T, C, F, code,
+                                _stream(stream))
+    if rc != NEA_OK:
+        raise NeaError(rc, "nea_block_ffn_bwd")
+    return dx, dg, dWg, dWu, dWd
 
 
 def nea_device_status(stream=None) -> int:

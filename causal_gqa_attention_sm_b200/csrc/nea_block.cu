@@ -1,6 +1,7 @@
 // C ABI of the decoder-block steps beside the attention (include/nea_attn.h,
 // "Decoder-block steps"): the RMSNorm pre-norm with the Q/K/V projections
-// and the output projection with the residual add, forward and backward.
+// and the output projection with the residual add, and the pre-norm SwiGLU
+// feed-forward with its residual add, forward and backward.
 // Every product runs on nea::gemm_kernel (tcgen05, TMA, TMEM accumulators);
 // the host side here chooses operand orientations, makes the operand planes
 // and sequences the launches on the caller's stream.
@@ -173,9 +174,10 @@ struct Seg {
 // out = sum_s A_s B_s (kseg: segments along K, one output `out` [M][ldo]) or
 // out_s = A_0 B_s (segments along N, output s [M][width_s]); A [M x K] is
 // stored [M][K] (K-major) or [K][M] (MN-major), B [K x N] stored [N][K]
-// (K-major) or [K][N] (MN-major).
+// (K-major) or [K][N] (MN-major).  `mode`, `pl` and `ab` select a SwiGLU
+// epilogue (nea::GemmParams::mode); those products run unsplit.
 int gemm_seg(Ctx& c, const Seg* segs, int n_seg, bool kseg, bool a_mn, bool b_mn, int M, void* out, long long ldo,
-             bool out_f32, const void* res) {
+             bool out_f32, const void* res, int mode = 0, void* const* pl = nullptr, const void* const* ab = nullptr) {
   nea::GemmParams p{};
   int rc;
   int N = 0, K = 0, begin = 0;
@@ -214,13 +216,16 @@ int gemm_seg(Ctx& c, const Seg* segs, int n_seg, bool kseg, bool a_mn, bool b_mn
   p.n_n = kseg ? (N + nea::kGemmBN - 1) / nea::kGemmBN : begin;
   p.n_k = (K + nea::kGemmBK - 1) / nea::kGemmBK;
   p.n_tiles = p.n_m * p.n_n;
+  p.mode = mode;
+  for (int i = 0; i < 6 && pl; ++i) p.pl[i] = pl[i];
+  for (int i = 0; i < 2 && ab; ++i) p.ab[i] = ab[i];
   p.err = c.err;
   p.wait_limit = c.wait_limit;
   if (p.n_tiles == 0 || K == 0) return NEA_OK;
   // split K when the tiles leave SMs idle: the chunk count (at most 4, each
   // of two k-steps or more) that minimises the per-CTA share of work
   p.split = 1;
-  if (p.n_tiles < c.n_sm && c.part) {
+  if (p.n_tiles < c.n_sm && c.part && mode == 0) {
     double best = double((p.n_tiles + c.n_sm - 1) / c.n_sm);
     for (int sp = 2; sp <= 4 && p.n_k >= 2 * sp; ++sp) {
       const double share = double((p.n_tiles * sp + c.n_sm - 1) / c.n_sm) / sp;
@@ -299,6 +304,51 @@ int check_dims(int M, int C, int Hq, int Hkv, int D, int dtype) {
 }
 
 constexpr float kNormEps = 1e-5f;
+
+// The feed-forward's widths: C and F in whole 64-column operand boxes.
+int check_ffn(int M, int C, int F, int dtype) {
+  if (M < 0 || C < 64 || C > 4096 || C % 64 != 0 || F < 64 || F % 64 != 0) return NEA_ERR_ARG;
+  if (dtype != NEA_F32 && dtype != NEA_BF16) return NEA_ERR_ARG;
+  if (static_cast<long long>(M) * std::max(C, F) > (1LL << 31) || static_cast<long long>(C) * F > (1LL << 31))
+    return NEA_ERR_ARG;
+  return NEA_OK;
+}
+
+// dx (with dres) and dg of the RMSNorm from dy: the rows kernel writes dx
+// and per-CTA dg sums, the column kernel adds those.
+int norm_bwd(Ctx& c, const void* x, const void* g, const float* rstd, const float* dy, const void* dres, void* dx,
+             void* dg, float* dg_part, int n_part, int M, int C) {
+  const size_t nb_smem = size_t(C) * 4 * 8;  // the eight warps' dg rows
+  if (nb_smem > 48 * 1024) {
+    const cudaError_t ea =
+        c.f32 ? cudaFuncSetAttribute(nea::rmsnorm_bwd_rows_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     int(nb_smem))
+              : cudaFuncSetAttribute(nea::rmsnorm_bwd_rows_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     int(nb_smem));
+    if (ea != cudaSuccess) return fail(ea);
+  }
+  cudaError_t err = c.f32 ? launch_pdl(nea::rmsnorm_bwd_rows_kernel<true>, unsigned(n_part), 256u, nb_smem,
+                                       c.stream, x, g, rstd, dy, dres, dx, dg_part, M, C)
+                          : launch_pdl(nea::rmsnorm_bwd_rows_kernel<false>, unsigned(n_part), 256u, nb_smem,
+                                       c.stream, x, g, rstd, dy, dres, dx, dg_part, M, C);
+  if (err != cudaSuccess) return fail(err);
+  const unsigned cg = unsigned((C + 31) / 32);
+  err = c.f32 ? launch_pdl(nea::colsum_kernel<true>, cg, 256u, size_t(0), c.stream,
+                           static_cast<const float*>(dg_part), n_part, C, dg)
+              : launch_pdl(nea::colsum_kernel<false>, cg, 256u, size_t(0), c.stream,
+                           static_cast<const float*>(dg_part), n_part, C, dg);
+  return err == cudaSuccess ? NEA_OK : fail(err);
+}
+
+// bf16 planes of an [rows][cols] intermediate: hi, and lo for float32 storage.
+Operand planes(Ctx& c, Carve& w, long long rows, long long cols) {
+  Operand o;
+  o.rows = rows;
+  o.cols = cols;
+  o.hi = w.take(size_t(rows) * cols * 2);
+  o.lo = c.f32 ? w.take(size_t(rows) * cols * 2) : nullptr;
+  return o;
+}
 
 }  // namespace
 
@@ -400,28 +450,7 @@ int nea_block_qkv_bwd(const void* x, const void* g, const void* Wq, const void* 
     g[2].A = gv, g[2].B = bv, g[2].width = Nk;
     if ((rc = gemm_seg(c, g, 3, true, false, false, M, dy, C, true, nullptr))) return rc;
   }
-  const size_t nb_smem = size_t(C) * 4 * 8;  // the eight warps' dg rows
-  if (nb_smem > 48 * 1024) {
-    const cudaError_t ea =
-        c.f32 ? cudaFuncSetAttribute(nea::rmsnorm_bwd_rows_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     int(nb_smem))
-              : cudaFuncSetAttribute(nea::rmsnorm_bwd_rows_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     int(nb_smem));
-    if (ea != cudaSuccess) return fail(ea);
-  }
-  cudaError_t err = c.f32 ? launch_pdl(nea::rmsnorm_bwd_rows_kernel<true>, unsigned(n_part), 256u, nb_smem,
-                                       c.stream, x, g, static_cast<const float*>(rstd), static_cast<const float*>(dy),
-                                       dres, dx, dg_part, M, C)
-                          : launch_pdl(nea::rmsnorm_bwd_rows_kernel<false>, unsigned(n_part), 256u, nb_smem,
-                                       c.stream, x, g, static_cast<const float*>(rstd), static_cast<const float*>(dy),
-                                       dres, dx, dg_part, M, C);
-  if (err != cudaSuccess) return fail(err);
-  const unsigned cg = unsigned((C + 31) / 32);
-  err = c.f32 ? launch_pdl(nea::colsum_kernel<true>, cg, 256u, size_t(0), c.stream,
-                           static_cast<const float*>(dg_part), n_part, C, dg)
-              : launch_pdl(nea::colsum_kernel<false>, cg, 256u, size_t(0), c.stream,
-                           static_cast<const float*>(dg_part), n_part, C, dg);
-  return err == cudaSuccess ? NEA_OK : fail(err);
+  return norm_bwd(c, x, g, rstd, dy, dres, dx, dg, dg_part, n_part, M, C);
 }
 
 int nea_block_out_fwd(const void* x, const void* o, const void* Wo, void* h, int M, int C, int Hq, int D, int dtype,
@@ -471,6 +500,108 @@ int nea_block_out_bwd(const void* o, const void* Wo, const void* dh, void* do_, 
   if ((rc = gemm(c, d, false, b, false, M, Nq, do_, c.f32, nullptr))) return rc;
   // dWo = o^T dh: A = o^T (o [M][Nq]: MN-major); B = dh [M][C], MN-major
   return gemm(c, a, true, d, true, Nq, C, dWo, c.f32, nullptr);
+}
+
+int nea_block_ffn_fwd(const void* x, const void* g, const void* Wg, const void* Wu, const void* Wd, void* h, void* a,
+                      void* b, int M, int C, int F, int dtype, void* stream) {
+  int rc = check_ffn(M, C, F, dtype);
+  if (rc) return rc;
+  if (M == 0) return NEA_OK;
+  for (const void* ptr : {x, g, Wg, Wu, Wd, static_cast<const void*>(h)})
+    if (!ptr || !al16(ptr)) return NEA_ERR_ARG;
+  if ((a && !al16(a)) || (b && !al16(b))) return NEA_ERR_ARG;
+  std::lock_guard<std::mutex> lock(g_block_mu);
+  Ctx c;
+  if ((rc = setup(c, dtype, stream))) return rc;
+  const int e = c.f32 ? 4 : 2;  // bytes of an operand element's planes
+  const size_t need = part_reserve(c.n_sm) + rup(size_t(M) * 4) + rup(size_t(M) * C * e) + rup(size_t(M) * F * e) +
+                      (c.f32 ? 3 * rup(size_t(C) * F * 4) : 0) + 4096;
+  if ((rc = ensure(c, need))) return rc;
+  Carve w{c.st->ws};
+  c.part_bytes = part_reserve(c.n_sm);
+  c.part = static_cast<float*>(w.take(c.part_bytes));
+  auto* rstd = static_cast<float*>(w.take(size_t(M) * 4));
+  Operand y, bg, bu, bd;
+  if ((rc = norm_rows(c, w, x, g, M, C, kNormEps, &y, rstd))) return rc;
+  if ((rc = make_operand(c, w, Wg, C, F, &bg)) || (rc = make_operand(c, w, Wu, C, F, &bu)) ||
+      (rc = make_operand(c, w, Wd, F, C, &bd)))
+    return rc;
+  const Operand act = planes(c, w, M, F);
+  // a = y Wg and b = y Wu side by side in TMEM (two K segments), the
+  // epilogue writing a, b and act = silu(a) b: A = y K-major; B = Wg, Wu
+  // [C][F], F contiguous: MN-major
+  {
+    Seg s[2];
+    s[0].A = y, s[0].B = bg, s[0].out = a, s[0].width = C;
+    s[1].A = y, s[1].B = bu, s[1].out = b, s[1].width = C;
+    void* const pl[6] = {const_cast<void*>(act.hi), const_cast<void*>(act.lo), nullptr, nullptr, nullptr, nullptr};
+    if ((rc = gemm_seg(c, s, 2, true, false, true, M, nullptr, F, c.f32, nullptr, 1, pl))) return rc;
+  }
+  // h = x + act Wd: A = act [M][F] K-major; B = Wd [F][C], C contiguous: MN-major
+  return gemm(c, act, false, bd, true, M, C, h, c.f32, x);
+}
+
+int nea_block_ffn_bwd(const void* x, const void* g, const void* Wg, const void* Wu, const void* Wd, const void* a,
+                      const void* b, const void* dh, void* dx, void* dg, void* dWg, void* dWu, void* dWd, int M, int C,
+                      int F, int dtype, void* stream) {
+  int rc = check_ffn(M, C, F, dtype);
+  if (rc) return rc;
+  if (M == 0) return NEA_OK;
+  for (const void* ptr : {x, g, Wg, Wu, Wd, a, b, dh, static_cast<const void*>(dx), static_cast<const void*>(dg),
+                          static_cast<const void*>(dWg), static_cast<const void*>(dWu), static_cast<const void*>(dWd)})
+    if (!ptr || !al16(ptr)) return NEA_ERR_ARG;
+  std::lock_guard<std::mutex> lock(g_block_mu);
+  Ctx c;
+  if ((rc = setup(c, dtype, stream))) return rc;
+  const int e = c.f32 ? 4 : 2;
+  const int n_part = std::min((M + 7) / 8, c.n_sm * 2);
+  const size_t need = part_reserve(c.n_sm) + rup(size_t(M) * 4) + rup(size_t(M) * C * e) + rup(size_t(M) * C * 4) +
+                      rup(size_t(n_part) * C * 4) + 3 * rup(size_t(M) * F * e) +
+                      (c.f32 ? 3 * rup(size_t(C) * F * 4) + rup(size_t(M) * C * 4) : 0) + 4096;
+  if ((rc = ensure(c, need))) return rc;
+  Carve w{c.st->ws};
+  c.part_bytes = part_reserve(c.n_sm);
+  c.part = static_cast<float*>(w.take(c.part_bytes));
+  auto* rstd = static_cast<float*>(w.take(size_t(M) * 4));
+  auto* dy = static_cast<float*>(w.take(size_t(M) * C * 4));
+  auto* dg_part = static_cast<float*>(w.take(size_t(n_part) * C * 4));
+  Operand y, bg, bu, bd, gh;
+  if ((rc = norm_rows(c, w, x, g, M, C, kNormEps, &y, rstd))) return rc;
+  if ((rc = make_operand(c, w, Wg, C, F, &bg)) || (rc = make_operand(c, w, Wu, C, F, &bu)) ||
+      (rc = make_operand(c, w, Wd, F, C, &bd)) || (rc = make_operand(c, w, dh, M, C, &gh)))
+    return rc;
+  const Operand da = planes(c, w, M, F), db = planes(c, w, M, F), act = planes(c, w, M, F);
+  // dact = dh Wd^T, combined in the epilogue with a and b into da, db and
+  // act: A = dh [M][C] K-major; B = Wd^T, i.e. Wd [F][C] read K-major
+  {
+    Seg s;
+    s.A = gh, s.B = bd, s.width = F;
+    void* const pl[6] = {const_cast<void*>(da.hi), const_cast<void*>(da.lo), const_cast<void*>(db.hi),
+                         const_cast<void*>(db.lo), const_cast<void*>(act.hi), const_cast<void*>(act.lo)};
+    const void* const ab[2] = {a, b};
+    if ((rc = gemm_seg(c, &s, 1, false, false, false, M, nullptr, F, c.f32, nullptr, 2, pl, ab))) return rc;
+  }
+  // dWd = act^T dh: A = act^T (act [M][F]: MN-major); B = dh [M][C], MN-major
+  if ((rc = gemm(c, act, true, gh, true, F, C, dWd, c.f32, nullptr))) return rc;
+  // dWg = y^T da, dWu = y^T db: A = y^T (MN-major); B = da, db [M][F], MN-major
+  if (F % nea::kGemmBN == 0) {  // one launch, side by side along N
+    Seg s[2];
+    s[0].A = y, s[0].B = da, s[0].out = dWg, s[0].width = F;
+    s[1].A = y, s[1].B = db, s[1].out = dWu, s[1].width = F;
+    if ((rc = gemm_seg(c, s, 2, false, true, true, C, nullptr, 0, c.f32, nullptr))) return rc;
+  } else if ((rc = gemm(c, y, true, da, true, C, F, dWg, c.f32, nullptr)) ||
+             (rc = gemm(c, y, true, db, true, C, F, dWu, c.f32, nullptr))) {
+    return rc;
+  }
+  // dy = da Wg^T + db Wu^T (fp32), chained along K: A = da, db K-major;
+  // B = Wg^T, Wu^T, i.e. Wg, Wu [C][F] read K-major
+  {
+    Seg s[2];
+    s[0].A = da, s[0].B = bg, s[0].width = F;
+    s[1].A = db, s[1].B = bu, s[1].width = F;
+    if ((rc = gemm_seg(c, s, 2, true, false, false, M, dy, C, true, nullptr))) return rc;
+  }
+  return norm_bwd(c, x, g, rstd, dy, dh, dx, dg, dg_part, n_part, M, C);
 }
 
 }  // extern "C"

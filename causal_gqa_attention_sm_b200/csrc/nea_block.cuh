@@ -6,6 +6,13 @@
 //             q = y Wq, k = y Wk, v = y Wv;   h = x + o Wo
 //   backward  dWo = o^T dh, do = dh Wo^T;  dW* = y^T d*, dy = sum d* W*^T,
 //             dx = rstd g dy - x rstd^3 / C sum_j (g dy)_j x_j (+ dh), dg = sum_tokens dy x rstd
+// and the block's feed-forward half, a pre-norm SwiGLU ("NanoEuler" write-up,
+// section 2, "SwiGLU feed-forward": down(silu(gate(x)) * up(x)), silu(z) =
+// z sigmoid(z)), F its inner width:
+//   forward   a = y Wg, b = y Wu, act = silu(a) b, h = x + act Wd
+//   backward  dact = dh Wd^T, da = dact b silu'(a), db = dact silu(a),
+//             dWd = act^T dh, dWg = y^T da, dWu = y^T db, dy = da Wg^T + db Wu^T,
+//             silu'(a) = s (1 + a (1 - s)) with s = sigmoid(a)
 // The products run on one tcgen05 GEMM kernel, C = A B with A [M x K] and B
 // [K x N] stored row-major in either orientation (an operand whose reduction
 // index is the contiguous one is "K-major", else "MN-major"); operands are
@@ -48,6 +55,17 @@ struct GemmParams {
   // part[u][128][128] and gemm_reduce_kernel sums them into the output
   int split, k_per;   // chunks, k-steps per chunk
   float* part;
+  // epilogue mode: 0 the plain store above; 1 the SwiGLU forward, two K
+  // segments (y Wg, then y Wu) accumulated side by side in TMEM, the tile
+  // writing a and b (seg[0].out, seg[1].out, each optional) and the operand
+  // planes of act = silu(a) b (pl[0] hi, pl[1] lo); 2 the SwiGLU backward,
+  // the product dact = dh Wd^T combined with the forward's a and b (ab[0],
+  // ab[1]) into the planes of da (pl[0], pl[1]), db (pl[2], pl[3]) and act
+  // (pl[4], pl[5]).  Lo planes (float32 storage) may be null; modes 1 and 2
+  // write [M][ldo] tensors and run unsplit.
+  int mode;
+  void* pl[6];
+  const void* ab[2];
   int* err;
   unsigned long long wait_limit;
 };
@@ -94,6 +112,84 @@ __global__ void __launch_bounds__(256) gemm_reduce_kernel(const __grid_constant_
   gemm_store(p, row, ni, c + 2, v.z);
   gemm_store(p, row, ni, c + 3, v.w);
 }
+
+// n (<= 32) consecutive values of a row, starting at element o of a tensor
+// in the storage type (fp32, or bf16 when !f32).  Full runs of 32 move as
+// 16-byte vectors (o is a multiple of 32 in a row of a multiple of 64).
+__device__ __forceinline__ void row_load32(const void* src, size_t o, bool f32, int n, float* v) {
+  if (n == 32) {
+    if (f32) {
+#pragma unroll
+      for (int j = 0; j < 32; j += 4) {
+        const float4 u = *reinterpret_cast<const float4*>(static_cast<const float*>(src) + o + j);
+        v[j] = u.x, v[j + 1] = u.y, v[j + 2] = u.z, v[j + 3] = u.w;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; j += 8) {
+        const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(src) + o + j);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[j + 2 * i] = bf16_lo_f(w[i]), v[j + 2 * i + 1] = bf16_hi_f(w[i]);
+      }
+    }
+    return;
+  }
+#pragma unroll
+  for (int j = 0; j < 32; ++j)  // a ragged run: static indices keep v in registers
+    if (j < n)
+      v[j] = f32 ? static_cast<const float*>(src)[o + j] : __bfloat162float(static_cast<const __nv_bfloat16*>(src)[o + j]);
+}
+
+__device__ __forceinline__ void row_store32(void* dst, size_t o, bool f32, int n, const float* v) {
+  if (n == 32) {
+    if (f32) {
+#pragma unroll
+      for (int j = 0; j < 32; j += 4)
+        *reinterpret_cast<float4*>(static_cast<float*>(dst) + o + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; j += 8)
+        *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dst) + o + j) =
+            make_uint4(pack_bf16(v[j], v[j + 1]), pack_bf16(v[j + 2], v[j + 3]), pack_bf16(v[j + 4], v[j + 5]),
+                       pack_bf16(v[j + 6], v[j + 7]));
+    }
+    return;
+  }
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    if (j >= n) break;
+    if (f32) static_cast<float*>(dst)[o + j] = v[j];
+    else static_cast<__nv_bfloat16*>(dst)[o + j] = __float2bfloat16_rn(v[j]);
+  }
+}
+
+// The same values as GEMM operand planes: bf16 hi, and when `lo` is given
+// the bf16 rounding remainder.
+__device__ __forceinline__ void row_planes32(void* hi, void* lo, size_t o, int n, const float* v) {
+  auto* h = static_cast<__nv_bfloat16*>(hi) + o;
+  auto* l = static_cast<__nv_bfloat16*>(lo) + o;
+  if (n == 32) {
+#pragma unroll
+    for (int j = 0; j < 32; j += 8) {
+      uint32_t hh[4], ll[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) split_bf16(v[j + 2 * i], v[j + 2 * i + 1], hh[i], ll[i]);
+      *reinterpret_cast<uint4*>(h + j) = make_uint4(hh[0], hh[1], hh[2], hh[3]);
+      if (lo) *reinterpret_cast<uint4*>(l + j) = make_uint4(ll[0], ll[1], ll[2], ll[3]);
+    }
+    return;
+  }
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    if (j >= n) break;
+    const __nv_bfloat16 b = __float2bfloat16_rn(v[j]);
+    h[j] = b;
+    if (lo) l[j] = __float2bfloat16_rn(v[j] - __bfloat162float(b));
+  }
+}
+
+__device__ __forceinline__ float sigmoid_f(float z) { return 1.f / (1.f + expf(-z)); }
 
 template <bool SPLIT>
 struct GemmSmem {
@@ -162,7 +258,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     }
     mbar_init_fence();
   }
-  if (warp == 1) tmem_alloc(tmem_holder, 256);  // two 128-column fp32 accumulators
+  // two accumulators of 128 fp32 columns, or (SwiGLU forward) two pairs
+  const uint32_t tcols = p.mode == 1 ? 512 : 256, acc_cols = tcols / 2;
+  if (warp == 1) tmem_alloc(tmem_holder, tcols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -218,6 +316,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         const int s = it % L::ST;
         if (!(ok = wait_warp(&full[s], (it / L::ST) & 1, wc, kErrWaitProducer))) break;
         tc_fence_after();
+        // SwiGLU forward: the second K segment accumulates beside the first
+        const int kq = p.mode == 1 && ks >= p.seg[1].begin ? 1 : 0;
+        const int kfirst = p.mode == 1 ? p.seg[kq].begin : kb;
         if (lane == 0) {
           const uint32_t a = smem_u32(sm + s * L::kStage);
           const uint32_t b = a + L::kPlanes * L::kOp;
@@ -227,8 +328,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             for (int term = 0; term < (SPLIT ? 3 : 1); ++term) {
               // hi*hi, hi*lo, lo*hi
               const uint32_t ap = a + (term == 2 ? L::kOp : 0), bp = b + (term == 1 ? L::kOp : 0);
-              mma_ss(tbase + ab * kGemmBN, gemm_desc<AMN>(ap, kk), gemm_desc<BMN>(bp, kk), idesc,
-                     ((ks - kb) | kk | term) != 0);
+              mma_ss(tbase + ab * acc_cols + kq * kGemmBN, gemm_desc<AMN>(ap, kk), gemm_desc<BMN>(bp, kk), idesc,
+                     ((ks - kfirst) | kk | term) != 0);
             }
           }
           tc_commit(&empty[s]);
@@ -255,7 +356,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
 #pragma unroll 1
         for (int c = 0; c < kGemmBN / 32; ++c) {
           uint32_t r[32];
-          tmem_ld32(tmem_addr(tbase, q4 * 32, ab * kGemmBN + c * 32), r);
+          tmem_ld32(tmem_addr(tbase, q4 * 32, ab * acc_cols + c * 32), r);
 #pragma unroll
           for (int j = 0; j < 32; j += 4)
             *reinterpret_cast<float4*>(dst + c * 32 + j) = make_float4(
@@ -268,6 +369,48 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       }
       const int mi = t % p.n_m, ni = t / p.n_m;
       const int row = mi * kGemmBM + q4 * 32 + lane;
+      if (p.mode != 0) {  // SwiGLU epilogues, 32 columns of a row per pass
+#pragma unroll 1
+        for (int c = 0; c < kGemmBN / 32; ++c) {
+          uint32_t r0[32], r1[32];
+          const uint32_t tc = ab * acc_cols + c * 32;
+          tmem_ld32(tmem_addr(tbase, q4 * 32, tc), r0);
+          if (p.mode == 1) tmem_ld32(tmem_addr(tbase, q4 * 32, tc + kGemmBN), r1);
+          const int col0 = ni * kGemmBN + c * 32;
+          if (row >= p.M || col0 >= p.N) continue;
+          const int n = min(32, p.N - col0);
+          const size_t o = size_t(row) * p.ldo + col0;
+          float a[32], b[32], act[32];
+          if (p.mode == 1) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              a[j] = __uint_as_float(r0[j]), b[j] = __uint_as_float(r1[j]);
+              act[j] = a[j] * sigmoid_f(a[j]) * b[j];
+            }
+            if (p.seg[0].out) row_store32(p.seg[0].out, o, p.out_f32, n, a);
+            if (p.seg[1].out) row_store32(p.seg[1].out, o, p.out_f32, n, b);
+            row_planes32(p.pl[0], p.pl[1], o, n, act);
+          } else {
+            row_load32(p.ab[0], o, p.out_f32, n, a);
+            row_load32(p.ab[1], o, p.out_f32, n, b);
+            float da[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float d = __uint_as_float(r0[j]), sg = sigmoid_f(a[j]), si = a[j] * sg;
+              da[j] = d * b[j] * sg * (1.f + a[j] * (1.f - sg));
+              act[j] = si * b[j];
+              b[j] = d * si;  // db
+            }
+            row_planes32(p.pl[0], p.pl[1], o, n, da);
+            row_planes32(p.pl[2], p.pl[3], o, n, b);
+            row_planes32(p.pl[4], p.pl[5], o, n, act);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[ab]);
+        continue;
+      }
       // the tile's output: its N segment's tensor, or the one output
       const int ns = p.kseg ? 0 : gemm_seg_of(p, ni);
       void* const out_base = p.kseg ? p.out : p.seg[ns].out;
@@ -277,7 +420,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
 #pragma unroll 1
       for (int c = 0; c < kGemmBN / 32; ++c) {
         uint32_t r[32];
-        tmem_ld32(tmem_addr(tbase, q4 * 32, ab * kGemmBN + c * 32), r);
+        tmem_ld32(tmem_addr(tbase, q4 * 32, ab * acc_cols + c * 32), r);
         const int col0 = ncol0 + c * 32;
         if (row >= p.M || col0 >= nlim) continue;
         const bool whole = col0 + 32 <= nlim;
@@ -334,7 +477,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tbase, 256);
+    tmem_dealloc(tbase, tcols);
   }
 }
 

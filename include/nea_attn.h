@@ -199,6 +199,39 @@ int nea_block_out_bwd(const void* o, const void* Wo, const void* dh, void* do_, 
                       int D, int dtype, void* stream);
 
 /*
+ * The block's feed-forward half, a pre-norm SwiGLU with its residual add
+ * ("NanoEuler" write-up, section 2 "Model components", SwiGLU feed-forward:
+ * down(silu(gate(x)) * up(x)) with silu(z) = z / (1 + e^-z)):
+ *
+ *   y = x rstd g (the RMSNorm above),  a = y Wg,  b = y Wu,
+ *   h = x + (silu(a) * b) Wd             (* elementwise)
+ *
+ * Layouts (row-major, contiguous, element type `dtype`; M = B*T tokens):
+ *   x, h, dx, dh : [M][C];   g, dg : [C];   a, b : [M][F]
+ *   Wg, Wu, dWg, dWu : [C][F];   Wd, dWd : [F][C]
+ * C and F must be multiples of 64, C <= 4096.  Products, precision,
+ * workspace, errors and streams as for the steps above.
+ *
+ * nea_block_ffn_fwd: h from x; the gate and up pre-activations a and b are
+ *   written to the caller's buffers for the backward (save for backward;
+ *   either may be NULL when no backward follows).  silu(a) b is formed in
+ *   the epilogue of the gate/up product and never stored in the storage
+ *   type: the down product reads it in fp32 precision (NEA_F32) or bf16.
+ * nea_block_ffn_bwd: from the forward's inputs, its a and b, and the
+ *   upstream gradient dh: with s = sigmoid(a), dact = dh Wd^T,
+ *   da = dact b s (1 + a (1 - s)), db = dact silu(a),
+ *   dWd = (silu(a) b)^T dh,  dWg = y^T da,  dWu = y^T db,
+ *   dy = da Wg^T + db Wu^T, and dx, dg from dy through the norm as in
+ *   nea_block_qkv_bwd, dx including the residual's dh.  The norm is
+ *   recomputed from x.
+ */
+int nea_block_ffn_fwd(const void* x, const void* g, const void* Wg, const void* Wu, const void* Wd, void* h, void* a,
+                      void* b, int M, int C, int F, int dtype, void* stream);
+int nea_block_ffn_bwd(const void* x, const void* g, const void* Wg, const void* Wu, const void* Wd, const void* a,
+                      const void* b, const void* dh, void* dx, void* dg, void* dWg, void* dWu, void* dWd, int M, int C,
+                      int F, int dtype, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device status words of the
  * current device: the one the regular entry points write and the one inside
  * the fixed scratch of nea_attn_bwd_noalloc.  Returns NEA_OK, NEA_ERR_TIMEOUT
