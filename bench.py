@@ -105,6 +105,9 @@ def config_of(w, world):
         return {"workload": w.name, "B": w.B, "Tc": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "storage": storage,
                 "rope_base": w.rope_base, "lens": "all Tc", "l2": decode_l2_note(w),
                 "parallelism": f"dp{world} (independent sequences per GPU)"}
+    if w.block and w.ffn:
+        return {"workload": w.name, "B": w.B, "T": w.T, "C": w.Hq * w.D, "F": w.ffn, "storage": storage,
+                "rmsnorm_eps": 1e-5, "l2": L2_NOTE, "parallelism": f"dp{world} (independent batches per GPU)"}
     if w.block:
         return {"workload": w.name, "B": w.B, "T": w.T, "C": w.Hq * w.D, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
                 "storage": storage, "rmsnorm_eps": 1e-5, "l2": L2_NOTE,
@@ -552,10 +555,22 @@ def reference_decode(a, w):
 BLOCK_METRIC = ("decoder-block steps beside the attention (RMSNorm + q/k/v projections, output projection + "
                 "residual), fwd+bwd TFLOP/s (% of tensor-core peak)")
 BLOCK_STEPS = ("qkv_fwd", "out_fwd", "out_bwd", "qkv_bwd")
+FFN_METRIC = "pre-norm SwiGLU feed-forward with residual, fwd+bwd TFLOP/s (% of tensor-core peak)"
+FFN_STEPS = ("ffn_fwd", "ffn_bwd")
+
+
+def block_metric(w):
+    return FFN_METRIC if w.ffn else BLOCK_METRIC
+
+
+def block_steps(w):
+    return FFN_STEPS if w.ffn else BLOCK_STEPS
 
 
 def block_step_flops(w):
     M, C, Nqkv, Nq = w.B * w.T, w.Hq * w.D, (w.Hq + 2 * w.Hkv) * w.D, w.Hq * w.D
+    if w.ffn:
+        return {"ffn_fwd": 6.0 * M * C * w.ffn, "ffn_bwd": 12.0 * M * C * w.ffn}
     return {"qkv_fwd": 2.0 * M * C * Nqkv, "out_fwd": 2.0 * M * Nq * C, "out_bwd": 4.0 * M * Nq * C,
             "qkv_bwd": 4.0 * M * C * Nqkv}
 
@@ -570,19 +585,25 @@ def run_oracle_block(w, rows=None, min_seconds=0.0):
     a = {n: t.float().double().numpy() for n, t in inp.items()}
     B = w.B if rows is None else max(1, rows // w.T)
     for n in ("x", "o", "dh", "dq", "dk", "dv"):
-        a[n] = a[n][:B]
+        if n in a:
+            a[n] = a[n][:B]
     sub = load_workloads().replace(w, B=B)
     reps, dt = 0, 0.0
     while reps == 0 or dt < min_seconds:
         t0 = time.perf_counter()
-        q, k, v, y, rstd = block_ref.qkv_fwd(a["x"], a["g"], a["Wq"], a["Wk"], a["Wv"], w.Hq, w.Hkv, w.D)
-        block_ref.out_fwd(a["x"], a["o"], a["Wo"])
-        block_ref.out_bwd(a["o"], a["Wo"], a["dh"])
-        block_ref.qkv_bwd(a["x"], a["g"], a["Wq"], a["Wk"], a["Wv"], y, rstd, a["dq"], a["dk"], a["dv"])
+        if w.ffn:
+            _, sv = block_ref.ffn_fwd(a["x"], a["g"], a["Wg"], a["Wu"], a["Wd"])
+            block_ref.ffn_bwd(a["x"], a["g"], a["Wg"], a["Wu"], a["Wd"], sv, a["dh"])
+        else:
+            q, k, v, y, rstd = block_ref.qkv_fwd(a["x"], a["g"], a["Wq"], a["Wk"], a["Wv"], w.Hq, w.Hkv, w.D)
+            block_ref.out_fwd(a["x"], a["o"], a["Wo"])
+            block_ref.out_bwd(a["o"], a["Wo"], a["dh"])
+            block_ref.qkv_bwd(a["x"], a["g"], a["Wq"], a["Wk"], a["Wv"], y, rstd, a["dq"], a["dk"], a["dv"])
         dt += time.perf_counter() - t0
         reps += 1
     threads = len(os.sched_getaffinity(0))
-    desc = f"block steps on {B} x {w.T} tokens (of {w.B} x {w.T}), fp64 numpy, {reps} repetitions"
+    what = "feed-forward" if w.ffn else "block steps"
+    desc = f"{what} on {B} x {w.T} tokens (of {w.B} x {w.T}), fp64 numpy, {reps} repetitions"
     return dt, sub.block_flops() * reps, threads, desc
 
 
@@ -598,7 +619,7 @@ def reference_block(a, w):
         flops += fl
     value = flops / secs / 1e12
     line = {
-        "impl": "reference", "metric": BLOCK_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": a.gpus,
+        "impl": "reference", "metric": block_metric(w), "value": value, "unit": "TFLOP/s", "n_gpus": a.gpus,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": secs / a.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_of(w, a.gpus),
@@ -607,6 +628,12 @@ def reference_block(a, w):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def block_launches(w):
+    if w.ffn:
+        return 17 if w.dtype == "f32" else 10
+    return 24 if w.dtype == "f32" else 10
 
 
 def block_main(a, w, rank, world, local):
@@ -625,7 +652,16 @@ def block_main(a, w, rank, world, local):
         flush.fill_(float(i))
         torch.sum(drain, dim=0, out=drain_sum)
 
+    steps = block_steps(w)
+    saved = {}
+
     def call(name, inp):
+        if name == "ffn_fwd":
+            h, saved["a"], saved["b"] = nea.nea_block_ffn_fwd(inp["x"], inp["g"], inp["Wg"], inp["Wu"], inp["Wd"])
+            return (h,)
+        if name == "ffn_bwd":
+            return nea.nea_block_ffn_bwd(inp["x"], inp["g"], inp["Wg"], inp["Wu"], inp["Wd"], saved["a"],
+                                         saved["b"], inp["dh"])
         if name == "qkv_fwd":
             return nea.nea_block_qkv_fwd(inp["x"], inp["g"], inp["Wq"], inp["Wk"], inp["Wv"], w.Hq, w.Hkv, w.D)
         if name == "out_fwd":
@@ -637,7 +673,7 @@ def block_main(a, w, rank, world, local):
 
     def step(inp=d, evs=None):
         outs = []
-        for i, n in enumerate(BLOCK_STEPS):
+        for i, n in enumerate(steps):
             if evs:
                 evs[i].record(stream)
             outs.extend(call(n, inp))
@@ -666,7 +702,7 @@ def block_main(a, w, rank, world, local):
         torch.cuda.synchronize(dev)
     barrier(world)
     # per-step durations: the same steps again with events between the calls
-    ev_k = [[torch.cuda.Event(enable_timing=True) for _ in range(len(BLOCK_STEPS) + 1)] for _ in range(K)]
+    ev_k = [[torch.cuda.Event(enable_timing=True) for _ in range(len(steps) + 1)] for _ in range(K)]
     for i in range(K):
         flush_l2(i)
         step(evs=ev_k[i])
@@ -677,9 +713,9 @@ def block_main(a, w, rank, world, local):
     flops = w.block_flops()
     value = flops * K * world / (total_ms * 1e-3) / 1e12
     sf = block_step_flops(w)
-    kern_ms = {n: sum(e[j].elapsed_time(e[j + 1]) for e in ev_k) / K for j, n in enumerate(BLOCK_STEPS)}
+    kern_ms = {n: sum(e[j].elapsed_time(e[j + 1]) for e in ev_k) / K for j, n in enumerate(steps)}
     kernels = {n: {"ms_per_call": kern_ms[n], "tflops": sf[n] / (kern_ms[n] * 1e-3) / 1e12,
-                   "share": kern_ms[n] / sum(kern_ms.values())} for n in BLOCK_STEPS}
+                   "share": kern_ms[n] / sum(kern_ms.values())} for n in steps}
     dominant = max(kern_ms, key=kern_ms.get)
     pk = peaks()
     tf32 = measure_tf32_peak(dev) if (w.dtype == "f32" and not a.profile) else None
@@ -697,7 +733,7 @@ def block_main(a, w, rank, world, local):
                 "peak_kind": f"bf16 dense burst ({pk['source']})"}
     e2e = None
     if not a.no_e2e:
-        act = ("x", "o", "dh", "dq", "dk", "dv")
+        act = ("x", "dh") if w.ffn else ("x", "o", "dh", "dq", "dk", "dv")
         host = {n: d[n].cpu().pin_memory() for n in act}
         dev_in = {n: torch.empty_like(d[n]) for n in act}
         inp = dict(d)
@@ -732,7 +768,7 @@ def block_main(a, w, rank, world, local):
                "seconds": dt}
     if rank == 0:
         line = {
-            "metric": BLOCK_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "metric": block_metric(w), "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
             "warmup": a.warmup, "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16x3" if w.dtype == "f32" else "bf16", "data": "synthetic",
             "config": config_of(w, world), "tokens_per_s": w.B * w.T * K * world / (total_ms * 1e-3),
@@ -740,8 +776,10 @@ def block_main(a, w, rank, world, local):
             "clocks": clocks.summary(), "clock_window": window,
             # per step: norm rows, q|k|v GEMM; out GEMM; do and dWo GEMMs; norm
             # rows, dW and dy GEMMs, norm backward, dg sum; float32 storage adds
-            # the operand-plane kernels (3 + 2 + 3 + 6)
-            "gpu_launches": K * (24 if w.dtype == "f32" else 10),
+            # the operand-plane kernels (3 + 2 + 3 + 6).  Feed-forward: norm
+            # rows, gate|up and down GEMMs; norm rows, dact, dWd, dWg|dWu and
+            # dy GEMMs, norm backward, dg sum; float32 storage adds 3 + 4
+            "gpu_launches": K * block_launches(w),
         }
         print(json.dumps(line), flush=True)
     return 0

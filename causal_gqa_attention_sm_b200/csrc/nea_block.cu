@@ -163,6 +163,21 @@ int make_operand(Ctx& c, Carve& w, const void* src, long long rows, long long co
   return NEA_OK;
 }
 
+// Launches the kernel instance of an operand orientation (form = 2 a_mn +
+// b_mn) for a plane count and tile width; `bit` indexes the instances whose
+// shared-memory limit is already raised.
+template <bool SPLIT, int BN, typename Run>
+int launch_form(Run& run, int form) {
+  constexpr uint32_t sm = nea::GemmSmem<SPLIT, BN>::kAlloc;
+  constexpr int base = (SPLIT ? 0 : 4) + (BN == 256 ? 8 : 0);
+  switch (form) {
+    case 0: return run(nea::gemm_kernel<false, false, SPLIT, BN>, sm, base + 0);
+    case 1: return run(nea::gemm_kernel<false, true, SPLIT, BN>, sm, base + 1);
+    case 2: return run(nea::gemm_kernel<true, false, SPLIT, BN>, sm, base + 2);
+    default: return run(nea::gemm_kernel<true, true, SPLIT, BN>, sm, base + 3);
+  }
+}
+
 // One operand segment of a product: A and B operands (read K-major or
 // MN-major as the product's flags say), and for N segments the output.
 struct Seg {
@@ -180,7 +195,7 @@ int gemm_seg(Ctx& c, const Seg* segs, int n_seg, bool kseg, bool a_mn, bool b_mn
              bool out_f32, const void* res, int mode = 0, void* const* pl = nullptr, const void* const* ab = nullptr) {
   nea::GemmParams p{};
   int rc;
-  int N = 0, K = 0, begin = 0;
+  const bool pair = mode == 1;  // segments 0 and 1 are the two halves of one 256-wide B tile
   for (int i = 0; i < n_seg; ++i) {
     const Seg& g = segs[i];
     nea::GemmSeg& q = p.seg[i];
@@ -192,16 +207,44 @@ int gemm_seg(Ctx& c, const Seg* segs, int n_seg, bool kseg, bool a_mn, bool b_mn
       return rc;
     q.out = g.out;
     q.ldo = g.width;
-    q.begin = begin;
-    if (kseg) {
+  }
+  // the N tiles of a tile width: N segments each start on a tile of their own
+  auto n_tiles_n = [&](int bn) {
+    if (kseg || pair) return int((ldo + bn - 1) / bn);
+    int n = 0;
+    for (int i = 0; i < n_seg; ++i) n += int((segs[i].width + bn - 1) / bn);
+    return n;
+  };
+  const int n_m = (M + nea::kGemmBM - 1) / nea::kGemmBM;
+  // tile width: 256 where the tiles still fill the SMs about as well -- a
+  // wave of 256-wide tiles is taken to cost 1.4 waves of 128-wide ones with
+  // bf16 operands (they stream from L2, and the wider tile reads A once for
+  // twice the columns) and 1.8 with hi/lo planes (whose 96 KB stages leave
+  // room for two in flight, against three); measured on the block's
+  // products.  The SwiGLU forward pairs Wg and Wu in one 256-wide tile.
+  int bn = 128;
+  if (pair) {
+    bn = 256;
+  } else {
+    const long long w128 = (static_cast<long long>(n_m) * n_tiles_n(128) + c.n_sm - 1) / c.n_sm;
+    const long long w256 = (static_cast<long long>(n_m) * n_tiles_n(256) + c.n_sm - 1) / c.n_sm;
+    if (w128 > 1 && (c.f32 ? 1.8 : 1.4) * double(w256) < double(w128)) bn = 256;
+  }
+  int N = 0, K = 0, begin = 0;
+  for (int i = 0; i < n_seg; ++i) {
+    const Seg& g = segs[i];
+    p.seg[i].begin = begin;
+    if (pair) {
+      K = int(g.width);
+    } else if (kseg) {
       begin += int(g.width / nea::kGemmBK);
       K += int(g.width);
     } else {
-      begin += int((g.width + nea::kGemmBN - 1) / nea::kGemmBN);
+      begin += int((g.width + bn - 1) / bn);
       N += int(g.width);
     }
   }
-  if (kseg) N = int(ldo);
+  if (kseg || pair) N = int(ldo);
   else K = int(a_mn ? segs[0].A.rows : segs[0].A.cols);
   p.n_seg = n_seg;
   p.kseg = kseg;
@@ -212,8 +255,8 @@ int gemm_seg(Ctx& c, const Seg* segs, int n_seg, bool kseg, bool a_mn, bool b_mn
   p.N = N;
   p.K = K;
   p.out_f32 = out_f32;
-  p.n_m = (M + nea::kGemmBM - 1) / nea::kGemmBM;
-  p.n_n = kseg ? (N + nea::kGemmBN - 1) / nea::kGemmBN : begin;
+  p.n_m = n_m;
+  p.n_n = pair ? (N + 127) / 128 : (kseg ? (N + bn - 1) / bn : begin);
   p.n_k = (K + nea::kGemmBK - 1) / nea::kGemmBK;
   p.n_tiles = p.n_m * p.n_n;
   p.mode = mode;
@@ -222,10 +265,11 @@ int gemm_seg(Ctx& c, const Seg* segs, int n_seg, bool kseg, bool a_mn, bool b_mn
   p.err = c.err;
   p.wait_limit = c.wait_limit;
   if (p.n_tiles == 0 || K == 0) return NEA_OK;
-  // split K when the tiles leave SMs idle: the chunk count (at most 4, each
-  // of two k-steps or more) that minimises the per-CTA share of work
+  // split K (128-wide tiles, plain epilogue) when the tiles leave SMs idle:
+  // the chunk count (at most 4, each of two k-steps or more) that minimises
+  // the per-CTA share of work
   p.split = 1;
-  if (p.n_tiles < c.n_sm && c.part && mode == 0) {
+  if (bn == 128 && p.n_tiles < c.n_sm && c.part && mode == 0) {
     double best = double((p.n_tiles + c.n_sm - 1) / c.n_sm);
     for (int sp = 2; sp <= 4 && p.n_k >= 2 * sp; ++sp) {
       const double share = double((p.n_tiles * sp + c.n_sm - 1) / c.n_sm) / sp;
@@ -248,22 +292,8 @@ int gemm_seg(Ctx& c, const Seg* segs, int n_seg, bool kseg, bool a_mn, bool b_mn
     return e == cudaSuccess ? NEA_OK : fail(e);
   };
   const int form = (a_mn ? 2 : 0) + (b_mn ? 1 : 0);
-  if (c.f32) {
-    constexpr uint32_t sm = nea::GemmSmem<true>::kAlloc;
-    switch (form) {
-      case 0: return run(nea::gemm_kernel<false, false, true>, sm, 0);
-      case 1: return run(nea::gemm_kernel<false, true, true>, sm, 1);
-      case 2: return run(nea::gemm_kernel<true, false, true>, sm, 2);
-      default: return run(nea::gemm_kernel<true, true, true>, sm, 3);
-    }
-  }
-  constexpr uint32_t sm = nea::GemmSmem<false>::kAlloc;
-  switch (form) {
-    case 0: return run(nea::gemm_kernel<false, false, false>, sm, 4);
-    case 1: return run(nea::gemm_kernel<false, true, false>, sm, 5);
-    case 2: return run(nea::gemm_kernel<true, false, false>, sm, 6);
-    default: return run(nea::gemm_kernel<true, true, false>, sm, 7);
-  }
+  return c.f32 ? (bn == 256 ? launch_form<true, 256>(run, form) : launch_form<true, 128>(run, form))
+               : (bn == 256 ? launch_form<false, 256>(run, form) : launch_form<false, 128>(run, form));
 }
 
 // out[M][N] = A B (+ res), one segment.
@@ -527,15 +557,15 @@ int nea_block_ffn_fwd(const void* x, const void* g, const void* Wg, const void* 
       (rc = make_operand(c, w, Wd, F, C, &bd)))
     return rc;
   const Operand act = planes(c, w, M, F);
-  // a = y Wg and b = y Wu side by side in TMEM (two K segments), the
-  // epilogue writing a, b and act = silu(a) b: A = y K-major; B = Wg, Wu
-  // [C][F], F contiguous: MN-major
+  // a = y Wg and b = y Wu side by side in one accumulator (the halves of a
+  // 256-wide B tile), the epilogue writing a, b and act = silu(a) b: A = y
+  // K-major; B = Wg, Wu [C][F], F contiguous: MN-major
   {
     Seg s[2];
     s[0].A = y, s[0].B = bg, s[0].out = a, s[0].width = C;
     s[1].A = y, s[1].B = bu, s[1].out = b, s[1].width = C;
     void* const pl[6] = {const_cast<void*>(act.hi), const_cast<void*>(act.lo), nullptr, nullptr, nullptr, nullptr};
-    if ((rc = gemm_seg(c, s, 2, true, false, true, M, nullptr, F, c.f32, nullptr, 1, pl))) return rc;
+    if ((rc = gemm_seg(c, s, 2, false, false, true, M, nullptr, F, c.f32, nullptr, 1, pl))) return rc;
   }
   // h = x + act Wd: A = act [M][F] K-major; B = Wd [F][C], C contiguous: MN-major
   return gemm(c, act, false, bd, true, M, C, h, c.f32, x);

@@ -25,8 +25,15 @@
 
 namespace nea {
 
+// Tiles are 128 rows (M) by BN = 128 or 256 columns (N); a k-step covers 64
+// of K.  A 256-wide tile halves the A traffic per FLOP, which matters because
+// the operands stream from L2 for every tile: the host takes it where the
+// tile count still fills the SMs.
 constexpr int kGemmBM = 128, kGemmBN = 128, kGemmBK = 64;
-constexpr int kGemmThreads = 192;  // warp 0: TMA, warp 1: MMA, warps 2-5: epilogue
+// warp 0: TMA, warp 1: MMA, warps 2-9: epilogue (two warps per 32-lane TMEM
+// quarter, each taking half of the tile's columns)
+constexpr int kGemmThreads = 320;
+constexpr int kGemmEpiWarps = 8;
 
 // Up to three operand segments.  Chained along K (kseg): out = sum_s A_s B_s,
 // segment s owning k-steps [begin_s, begin_{s+1}).  Side by side along N:
@@ -49,16 +56,17 @@ struct GemmParams {
   long long ldo;
   int M, N, K;
   int out_f32;        // 1: fp32 output, 0: bf16
-  int n_m, n_n, n_k, n_tiles;
+  int n_m, n_n, n_k, n_tiles;  // tiles of 128 x BN (mode 1: 128 output columns of each of a, b)
   // split K: work unit u is tile u % n_tiles over k-steps of chunk u /
   // n_tiles; with split > 1 each unit writes an fp32 partial tile to
   // part[u][128][128] and gemm_reduce_kernel sums them into the output
   int split, k_per;   // chunks, k-steps per chunk
   float* part;
-  // epilogue mode: 0 the plain store above; 1 the SwiGLU forward, two K
-  // segments (y Wg, then y Wu) accumulated side by side in TMEM, the tile
-  // writing a and b (seg[0].out, seg[1].out, each optional) and the operand
-  // planes of act = silu(a) b (pl[0] hi, pl[1] lo); 2 the SwiGLU backward,
+  // epilogue mode: 0 the plain store above; 1 the SwiGLU forward: a 256-wide
+  // tile whose B halves are the same 128 columns of seg[0].b (Wg) and
+  // seg[1].b (Wu), so that one accumulator holds a = y Wg beside b = y Wu;
+  // the tile writes a and b (seg[0].out, seg[1].out, each optional) and the
+  // operand planes of act = silu(a) b (pl[0] hi, pl[1] lo); 2 the SwiGLU backward,
   // the product dact = dh Wd^T combined with the forward's a and b (ab[0],
   // ab[1]) into the planes of da (pl[0], pl[1]), db (pl[2], pl[3]) and act
   // (pl[4], pl[5]).  Lo planes (float32 storage) may be null; modes 1 and 2
@@ -113,51 +121,43 @@ __global__ void __launch_bounds__(256) gemm_reduce_kernel(const __grid_constant_
   gemm_store(p, row, ni, c + 3, v.w);
 }
 
-// n (<= 32) consecutive values of a row, starting at element o of a tensor
-// in the storage type (fp32, or bf16 when !f32).  Full runs of 32 move as
-// 16-byte vectors (o is a multiple of 32 in a row of a multiple of 64).
-__device__ __forceinline__ void row_load32(const void* src, size_t o, bool f32, int n, float* v) {
-  if (n == 32) {
+// n (<= 8) consecutive values of a row, starting at element o of a tensor
+// in the storage type (fp32, or bf16 when !f32).  Full runs of 8 move as
+// 16-byte vectors (o is then a multiple of 8).
+__device__ __forceinline__ void row_load8(const void* src, size_t o, bool f32, int n, float* v) {
+  if (n >= 8) {
     if (f32) {
-#pragma unroll
-      for (int j = 0; j < 32; j += 4) {
-        const float4 u = *reinterpret_cast<const float4*>(static_cast<const float*>(src) + o + j);
-        v[j] = u.x, v[j + 1] = u.y, v[j + 2] = u.z, v[j + 3] = u.w;
-      }
+      const float4 u0 = *reinterpret_cast<const float4*>(static_cast<const float*>(src) + o);
+      const float4 u1 = *reinterpret_cast<const float4*>(static_cast<const float*>(src) + o + 4);
+      v[0] = u0.x, v[1] = u0.y, v[2] = u0.z, v[3] = u0.w, v[4] = u1.x, v[5] = u1.y, v[6] = u1.z, v[7] = u1.w;
     } else {
+      const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(src) + o);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-      for (int j = 0; j < 32; j += 8) {
-        const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(src) + o + j);
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[j + 2 * i] = bf16_lo_f(w[i]), v[j + 2 * i + 1] = bf16_hi_f(w[i]);
-      }
+      for (int i = 0; i < 4; ++i) v[2 * i] = bf16_lo_f(w[i]), v[2 * i + 1] = bf16_hi_f(w[i]);
     }
     return;
   }
 #pragma unroll
-  for (int j = 0; j < 32; ++j)  // a ragged run: static indices keep v in registers
-    if (j < n)
-      v[j] = f32 ? static_cast<const float*>(src)[o + j] : __bfloat162float(static_cast<const __nv_bfloat16*>(src)[o + j]);
+  for (int j = 0; j < 8; ++j)  // a ragged run: static indices keep v in registers
+    v[j] = j >= n ? 0.f
+                  : f32 ? static_cast<const float*>(src)[o + j]
+                        : __bfloat162float(static_cast<const __nv_bfloat16*>(src)[o + j]);
 }
 
-__device__ __forceinline__ void row_store32(void* dst, size_t o, bool f32, int n, const float* v) {
-  if (n == 32) {
+__device__ __forceinline__ void row_store8(void* dst, size_t o, bool f32, int n, const float* v) {
+  if (n >= 8) {
     if (f32) {
-#pragma unroll
-      for (int j = 0; j < 32; j += 4)
-        *reinterpret_cast<float4*>(static_cast<float*>(dst) + o + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+      *reinterpret_cast<float4*>(static_cast<float*>(dst) + o) = make_float4(v[0], v[1], v[2], v[3]);
+      *reinterpret_cast<float4*>(static_cast<float*>(dst) + o + 4) = make_float4(v[4], v[5], v[6], v[7]);
     } else {
-#pragma unroll
-      for (int j = 0; j < 32; j += 8)
-        *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dst) + o + j) =
-            make_uint4(pack_bf16(v[j], v[j + 1]), pack_bf16(v[j + 2], v[j + 3]), pack_bf16(v[j + 4], v[j + 5]),
-                       pack_bf16(v[j + 6], v[j + 7]));
+      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dst) + o) =
+          make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
     }
     return;
   }
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
+  for (int j = 0; j < 8; ++j) {
     if (j >= n) break;
     if (f32) static_cast<float*>(dst)[o + j] = v[j];
     else static_cast<__nv_bfloat16*>(dst)[o + j] = __float2bfloat16_rn(v[j]);
@@ -166,22 +166,19 @@ __device__ __forceinline__ void row_store32(void* dst, size_t o, bool f32, int n
 
 // The same values as GEMM operand planes: bf16 hi, and when `lo` is given
 // the bf16 rounding remainder.
-__device__ __forceinline__ void row_planes32(void* hi, void* lo, size_t o, int n, const float* v) {
+__device__ __forceinline__ void row_planes8(void* hi, void* lo, size_t o, int n, const float* v) {
   auto* h = static_cast<__nv_bfloat16*>(hi) + o;
   auto* l = static_cast<__nv_bfloat16*>(lo) + o;
-  if (n == 32) {
+  if (n >= 8) {
+    uint32_t hh[4], ll[4];
 #pragma unroll
-    for (int j = 0; j < 32; j += 8) {
-      uint32_t hh[4], ll[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) split_bf16(v[j + 2 * i], v[j + 2 * i + 1], hh[i], ll[i]);
-      *reinterpret_cast<uint4*>(h + j) = make_uint4(hh[0], hh[1], hh[2], hh[3]);
-      if (lo) *reinterpret_cast<uint4*>(l + j) = make_uint4(ll[0], ll[1], ll[2], ll[3]);
-    }
+    for (int i = 0; i < 4; ++i) split_bf16(v[2 * i], v[2 * i + 1], hh[i], ll[i]);
+    *reinterpret_cast<uint4*>(h) = make_uint4(hh[0], hh[1], hh[2], hh[3]);
+    if (lo) *reinterpret_cast<uint4*>(l) = make_uint4(ll[0], ll[1], ll[2], ll[3]);
     return;
   }
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
+  for (int j = 0; j < 8; ++j) {
     if (j >= n) break;
     const __nv_bfloat16 b = __float2bfloat16_rn(v[j]);
     h[j] = b;
@@ -189,14 +186,18 @@ __device__ __forceinline__ void row_planes32(void* hi, void* lo, size_t o, int n
   }
 }
 
-__device__ __forceinline__ float sigmoid_f(float z) { return 1.f / (1.f + expf(-z)); }
+// 1 / (1 + e^-z) with the fast exponential and division intrinsics; z is
+// clamped at -80 so that e^-z stays below 2^126 (the divide's range), which
+// changes the result only where it is below 2e-35.
+__device__ __forceinline__ float sigmoid_f(float z) { return __fdividef(1.f, 1.f + __expf(-fmaxf(z, -80.f))); }
 
-template <bool SPLIT>
+template <bool SPLIT, int BN>
 struct GemmSmem {
   static constexpr uint32_t kOp = 128 * 128;             // one 128 x 64 bf16 operand tile (16 KB)
+  static constexpr uint32_t kOpB = BN * 128;             // the B tile: BN x 64
   static constexpr int kPlanes = SPLIT ? 2 : 1;
-  static constexpr uint32_t kStage = 2 * kPlanes * kOp;  // A planes, then B planes
-  static constexpr int ST = SPLIT ? 3 : 6;
+  static constexpr uint32_t kStage = kPlanes * (kOp + kOpB);  // A planes, then B planes
+  static constexpr int ST = (200 * 1024) / kStage;       // 6, 4 (bf16); 3, 2 (split)
   static constexpr uint32_t kBars = ST * kStage;         // full[ST], empty[ST], acc_full[2], acc_empty[2]
   static constexpr uint32_t kMisc = kBars + (2 * ST + 4) * 8;  // TMEM base, abort flag
   static constexpr uint32_t kBytes = kMisc + 16;
@@ -232,9 +233,10 @@ __device__ __forceinline__ uint64_t gemm_desc(uint32_t tile, int kk) {
   return MN ? smem_desc(tile + kk * 2048, 128, 8192) : smem_desc(tile + kk * 32, 128, 16);
 }
 
-template <bool AMN, bool BMN, bool SPLIT>
+template <bool AMN, bool BMN, bool SPLIT, int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
-  using L = GemmSmem<SPLIT>;
+  using L = GemmSmem<SPLIT, BN>;
+  static_assert(BN == 128 || BN == 256, "tile width");
   extern __shared__ uint8_t raw[];
   uint8_t* sm = raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + L::kBars);
@@ -254,12 +256,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 4);  // one arrival per epilogue warp
+      mbar_init(&acc_empty[i], kGemmEpiWarps);  // one arrival per epilogue warp
     }
     mbar_init_fence();
   }
-  // two accumulators of 128 fp32 columns, or (SwiGLU forward) two pairs
-  const uint32_t tcols = p.mode == 1 ? 512 : 256, acc_cols = tcols / 2;
+  // two accumulators of BN fp32 columns
+  constexpr uint32_t tcols = 2 * BN, acc_cols = BN;
   if (warp == 1) tmem_alloc(tmem_holder, tcols);
   tc_fence_before();
   __syncthreads();
@@ -276,9 +278,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       for (int u = blockIdx.x; u < p.n_tiles * p.split && ok; u += gridDim.x) {
         const int t = u % p.n_tiles, kb = (u / p.n_tiles) * p.k_per, ke = min(p.n_k, kb + p.k_per);
         const int mi = t % p.n_m, ni = t / p.n_m;
-        const int ns = p.kseg ? 0 : gemm_seg_of(p, ni);  // N segment of the tile
+        const int ns = (p.kseg || p.mode == 1) ? 0 : gemm_seg_of(p, ni);  // N segment of the tile
         const GemmSeg& sa = p.seg[0];
-        const int n0 = (ni - (p.kseg ? 0 : p.seg[ns].begin)) * kGemmBN;
+        const int n0 = p.mode == 1 ? ni * 128 : (ni - (p.kseg ? 0 : p.seg[ns].begin)) * BN;
         for (int ks = kb; ks < ke; ++ks, ++it) {
           const int s = it % L::ST;
           if (it >= uint32_t(L::ST) && !(ok = wait_thread(&empty[s], ((it / L::ST) - 1) & 1, wc, kErrWaitEmpty)))
@@ -290,10 +292,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
           uint8_t* st = sm + s * L::kStage;
           mbar_arrive_expect_tx(&full[s], L::kStage);
           gemm_load_tile<AMN>(st, &ga.a_hi, mi * kGemmBM, k0, &full[s]);
-          gemm_load_tile<BMN>(st + L::kPlanes * L::kOp, &g.b_hi, n0, k0, &full[s]);
-          if constexpr (SPLIT) {
-            gemm_load_tile<AMN>(st + L::kOp, &ga.a_lo, mi * kGemmBM, k0, &full[s]);
-            gemm_load_tile<BMN>(st + 3 * L::kOp, &g.b_lo, n0, k0, &full[s]);
+          if constexpr (SPLIT) gemm_load_tile<AMN>(st + L::kOp, &ga.a_lo, mi * kGemmBM, k0, &full[s]);
+          uint8_t* const sb = st + L::kPlanes * L::kOp;  // B planes: hi, then lo
+#pragma unroll
+          for (int h = 0; h < BN / 128; ++h) {  // 128-column halves (mode 1: Wg, then Wu)
+            const GemmSeg& gb = p.mode == 1 ? p.seg[h] : g;
+            const int nb = p.mode == 1 ? n0 : n0 + h * 128;
+            gemm_load_tile<BMN>(sb + h * L::kOp, &gb.b_hi, nb, k0, &full[s]);
+            if constexpr (SPLIT) gemm_load_tile<BMN>(sb + L::kOpB + h * L::kOp, &gb.b_lo, nb, k0, &full[s]);
           }
         }
       }
@@ -303,7 +309,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA
-    constexpr uint32_t idesc = idesc_bf16(kGemmBM, kGemmBN, AMN, BMN);
+    constexpr uint32_t idesc = idesc_bf16(kGemmBM, BN, AMN, BMN);
     uint32_t it = 0, last = 0xffffffffu;  // the last stage use committed
     int lt = 0;
     bool ok = true;
@@ -316,9 +322,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         const int s = it % L::ST;
         if (!(ok = wait_warp(&full[s], (it / L::ST) & 1, wc, kErrWaitProducer))) break;
         tc_fence_after();
-        // SwiGLU forward: the second K segment accumulates beside the first
-        const int kq = p.mode == 1 && ks >= p.seg[1].begin ? 1 : 0;
-        const int kfirst = p.mode == 1 ? p.seg[kq].begin : kb;
         if (lane == 0) {
           const uint32_t a = smem_u32(sm + s * L::kStage);
           const uint32_t b = a + L::kPlanes * L::kOp;
@@ -327,9 +330,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
 #pragma unroll
             for (int term = 0; term < (SPLIT ? 3 : 1); ++term) {
               // hi*hi, hi*lo, lo*hi
-              const uint32_t ap = a + (term == 2 ? L::kOp : 0), bp = b + (term == 1 ? L::kOp : 0);
-              mma_ss(tbase + ab * acc_cols + kq * kGemmBN, gemm_desc<AMN>(ap, kk), gemm_desc<BMN>(bp, kk), idesc,
-                     ((ks - kfirst) | kk | term) != 0);
+              const uint32_t ap = a + (term == 2 ? L::kOp : 0), bp = b + (term == 1 ? L::kOpB : 0);
+              mma_ss(tbase + ab * acc_cols, gemm_desc<AMN>(ap, kk), gemm_desc<BMN>(bp, kk), idesc,
+                     ((ks - kb) | kk | term) != 0);
             }
           }
           tc_commit(&empty[s]);
@@ -343,7 +346,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     if (lane == 0 && last != 0xffffffffu) drain_wait(&empty[last % L::ST], (last / L::ST) & 1, wc);
   } else {
     // ---------------------------------------------------------------- epilogue
-    const int q4 = warp & 3;  // TMEM lanes 32 q4 .. 32 q4 + 31
+    const int q4 = warp & 3;         // TMEM lanes 32 q4 .. 32 q4 + 31
+    const int ch = (warp - 2) >> 2;  // column half of the tile
     int lt = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < p.n_tiles * p.split && ok; u += gridDim.x, ++lt) {
@@ -351,10 +355,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       const int ab = lt & 1;
       if (!(ok = wait_warp(&acc_full[ab], (lt >> 1) & 1, wc, kErrWaitMma))) break;
       tc_fence_after();
-      if (p.split > 1) {  // this chunk's partial tile, row-major 128 x 128 fp32
+      if (BN == 128 && p.split > 1) {  // this chunk's partial tile, row-major 128 x 128 fp32
         float* dst = p.part + size_t(u) * 128 * 128 + size_t(q4 * 32 + lane) * 128;
 #pragma unroll 1
-        for (int c = 0; c < kGemmBN / 32; ++c) {
+        for (int c = ch * 2; c < ch * 2 + 2; ++c) {
           uint32_t r[32];
           tmem_ld32(tmem_addr(tbase, q4 * 32, ab * acc_cols + c * 32), r);
 #pragma unroll
@@ -369,41 +373,56 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       }
       const int mi = t % p.n_m, ni = t / p.n_m;
       const int row = mi * kGemmBM + q4 * 32 + lane;
-      if (p.mode != 0) {  // SwiGLU epilogues, 32 columns of a row per pass
+      if (p.mode != 0) {  // SwiGLU epilogues, 32 columns of a row per pass, 8 at a time
+        const int nc = p.mode == 1 ? 2 : BN / 64;  // 32-column chunks per warp
 #pragma unroll 1
-        for (int c = 0; c < kGemmBN / 32; ++c) {
+        for (int c = ch * nc; c < ch * nc + nc; ++c) {
           uint32_t r0[32], r1[32];
           const uint32_t tc = ab * acc_cols + c * 32;
           tmem_ld32(tmem_addr(tbase, q4 * 32, tc), r0);
-          if (p.mode == 1) tmem_ld32(tmem_addr(tbase, q4 * 32, tc + kGemmBN), r1);
-          const int col0 = ni * kGemmBN + c * 32;
+          if (p.mode == 1) tmem_ld32(tmem_addr(tbase, q4 * 32, tc + 128), r1);  // b beside a
+          const int col0 = (p.mode == 1 ? ni * 128 : ni * BN) + c * 32;
           if (row >= p.M || col0 >= p.N) continue;
-          const int n = min(32, p.N - col0);
-          const size_t o = size_t(row) * p.ldo + col0;
-          float a[32], b[32], act[32];
+          const size_t o0 = size_t(row) * p.ldo + col0;
           if (p.mode == 1) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              a[j] = __uint_as_float(r0[j]), b[j] = __uint_as_float(r1[j]);
-              act[j] = a[j] * sigmoid_f(a[j]) * b[j];
-            }
-            if (p.seg[0].out) row_store32(p.seg[0].out, o, p.out_f32, n, a);
-            if (p.seg[1].out) row_store32(p.seg[1].out, o, p.out_f32, n, b);
-            row_planes32(p.pl[0], p.pl[1], o, n, act);
-          } else {
-            row_load32(p.ab[0], o, p.out_f32, n, a);
-            row_load32(p.ab[1], o, p.out_f32, n, b);
-            float da[32];
+            for (int j = 0; j < 32; j += 8) {
+              const int n = min(8, p.N - col0 - j);
+              if (n <= 0) break;
+              float a[8], b[8], x[8];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float d = __uint_as_float(r0[j]), sg = sigmoid_f(a[j]), si = a[j] * sg;
-              da[j] = d * b[j] * sg * (1.f + a[j] * (1.f - sg));
-              act[j] = si * b[j];
-              b[j] = d * si;  // db
+              for (int i = 0; i < 8; ++i) {
+                a[i] = __uint_as_float(r0[j + i]), b[i] = __uint_as_float(r1[j + i]);
+                x[i] = a[i] * sigmoid_f(a[i]) * b[i];  // act
+              }
+              if (p.seg[0].out) row_store8(p.seg[0].out, o0 + j, p.out_f32, n, a);
+              if (p.seg[1].out) row_store8(p.seg[1].out, o0 + j, p.out_f32, n, b);
+              row_planes8(p.pl[0], p.pl[1], o0 + j, n, x);
             }
-            row_planes32(p.pl[0], p.pl[1], o, n, da);
-            row_planes32(p.pl[2], p.pl[3], o, n, b);
-            row_planes32(p.pl[4], p.pl[5], o, n, act);
+          } else {
+            float a[32], b[32];  // the chunk's a and b, all loads in flight together
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) {
+              row_load8(p.ab[0], o0 + j, p.out_f32, p.N - col0 - j, a + j);
+              row_load8(p.ab[1], o0 + j, p.out_f32, p.N - col0 - j, b + j);
+            }
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) {
+              const int n = min(8, p.N - col0 - j);
+              if (n <= 0) break;
+              float x[8], y[8], z[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float d = __uint_as_float(r0[j + i]), aa = a[j + i], bb = b[j + i];
+                const float sg = sigmoid_f(aa), si = aa * sg;
+                x[i] = d * bb * sg * (1.f + aa * (1.f - sg));  // da
+                y[i] = d * si;                                 // db
+                z[i] = si * bb;                                // act
+              }
+              row_planes8(p.pl[0], p.pl[1], o0 + j, n, x);
+              row_planes8(p.pl[2], p.pl[3], o0 + j, n, y);
+              row_planes8(p.pl[4], p.pl[5], o0 + j, n, z);
+            }
           }
         }
         tc_fence_before();
@@ -415,10 +434,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       const int ns = p.kseg ? 0 : gemm_seg_of(p, ni);
       void* const out_base = p.kseg ? p.out : p.seg[ns].out;
       const long long ldo = p.kseg ? p.ldo : p.seg[ns].ldo;
-      const int ncol0 = (ni - (p.kseg ? 0 : p.seg[ns].begin)) * kGemmBN;  // first column in that tensor
+      const int ncol0 = (ni - (p.kseg ? 0 : p.seg[ns].begin)) * BN;  // first column in that tensor
       const int nlim = p.kseg ? p.N : int(ldo);                           // its column count
 #pragma unroll 1
-      for (int c = 0; c < kGemmBN / 32; ++c) {
+      for (int c = ch * (BN / 64); c < (ch + 1) * (BN / 64); ++c) {
         uint32_t r[32];
         tmem_ld32(tmem_addr(tbase, q4 * 32, ab * acc_cols + c * 32), r);
         const int col0 = ncol0 + c * 32;

@@ -34,6 +34,7 @@ class Workload:
     seed: int = 0
     decode: bool = False  # one query per sequence over a cache of T positions
     block: bool = False   # the decoder-block steps beside the attention (model dim C = Hq D)
+    ffn: int = 0          # block workloads: the SwiGLU feed-forward of inner width F = ffn instead
 
     @property
     def torch_dtype(self):
@@ -57,6 +58,8 @@ class Workload:
         twice that backward; output projection 2 M (Hq D) C forward, twice that
         backward (the norms' elementwise work is not counted)."""
         M, C = self.B * self.T, self.Hq * self.D
+        if self.ffn:  # gate, up and down products: 6 M C F forward, 12 M C F backward
+            return 18.0 * M * C * self.ffn
         return 6.0 * M * C * (self.Hq + 2 * self.Hkv) * self.D + 6.0 * M * self.Hq * self.D * C
 
     def tokens(self) -> int:
@@ -86,6 +89,8 @@ WORKLOADS = {
     "decode4096": Workload("decode4096", 16, 4096, 12, 4, 64, "bf16", seed=6001, decode=True),
     # the decoder-block steps of the GPU model layer (dim 768 = 12 x 64)
     "block": Workload("block", 8, 512, 12, 4, 64, "f32", seed=7000, block=True),
+    # its SwiGLU feed-forward, inner width F = 4 x 768
+    "ffn": Workload("ffn", 8, 512, 12, 4, 64, "f32", seed=7100, block=True, ffn=3072),
 }
 
 
@@ -122,10 +127,16 @@ def make_block_inputs(w: Workload, device="cpu"):
     """Inputs of the block steps for C = Hq D: x [B, T, C], gain g [C] ~ 1 +
     N(0, 0.01), weights ~ N(0, 1/fan_in) (Wq [C, Hq D], Wk, Wv [C, Hkv D],
     Wo [Hq D, C]), the attention output o and the upstream gradients dh, dq,
-    dk, dv ~ N(0, 1); drawn like ``make_inputs``."""
+    dk, dv ~ N(0, 1); drawn like ``make_inputs``.  Feed-forward workloads:
+    x, g, Wg, Wu [C, F], Wd [F, C] and dh, drawn the same way."""
     g = torch.Generator(device="cpu").manual_seed(int(w.seed))
     C = w.Hq * w.D
     r = lambda *shape, std=1.0: torch.randn(shape, generator=g, dtype=torch.float32) * std
+    if w.ffn:
+        F = w.ffn
+        out = dict(x=r(w.B, w.T, C), g=1.0 + r(C, std=0.1), Wg=r(C, F, std=C ** -0.5), Wu=r(C, F, std=C ** -0.5),
+                   Wd=r(F, C, std=F ** -0.5), dh=r(w.B, w.T, C))
+        return {n: t.to(w.torch_dtype).to(device).contiguous() for n, t in out.items()}
     out = dict(x=r(w.B, w.T, C), g=1.0 + r(C, std=0.1), Wq=r(C, w.Hq * w.D, std=C ** -0.5),
                Wk=r(C, w.Hkv * w.D, std=C ** -0.5), Wv=r(C, w.Hkv * w.D, std=C ** -0.5),
                Wo=r(w.Hq * w.D, C, std=(w.Hq * w.D) ** -0.5), o=r(w.B, w.T, w.Hq, w.D), dh=r(w.B, w.T, C),

@@ -77,7 +77,7 @@ def test_traffic_is_withheld_when_the_kernel_changed(tmp_path, monkeypatch):
     assert bench.ncu_traffic("attn_bwd", "long") is None  # sources changed since the capture
 
 
-@pytest.mark.parametrize("workload", ["tiny", "decode1024", "block"])
+@pytest.mark.parametrize("workload", ["tiny", "decode1024", "block", "ffn"])
 def test_reference_arm_prints_the_contract_line(workload):
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
                           workload, "--steps", "1", "--warmup", "3"], capture_output=True, text=True, timeout=600,
