@@ -631,9 +631,15 @@ def reference_block(a, w):
 
 
 def block_launches(w):
+    """Library kernels per step (as the ncu launch lists count them).  Block:
+    norm rows, q|k|v GEMM; out GEMM; do GEMM, dWo GEMM + split-K reduce; norm
+    rows, dWq|dWk|dWv GEMM + reduce, dy GEMM, norm backward, dg sum (12).
+    Feed-forward: norm rows, gate|up and down GEMMs; norm rows, dact, dWd,
+    dWg|dWu and dy GEMMs, norm backward, dg sum (10).  Float32 storage adds
+    one operand-plane launch per call (4 and 2)."""
     if w.ffn:
-        return 17 if w.dtype == "f32" else 10
-    return 24 if w.dtype == "f32" else 10
+        return 12 if w.dtype == "f32" else 10
+    return 16 if w.dtype == "f32" else 12
 
 
 def block_main(a, w, rank, world, local):
@@ -774,11 +780,6 @@ def block_main(a, w, rank, world, local):
             "config": config_of(w, world), "tokens_per_s": w.B * w.T * K * world / (total_ms * 1e-3),
             "kernels": kernels, "roofline": roof, "tf32_peak": tf32, "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clocks.summary(), "clock_window": window,
-            # per step: norm rows, q|k|v GEMM; out GEMM; do and dWo GEMMs; norm
-            # rows, dW and dy GEMMs, norm backward, dg sum; float32 storage adds
-            # the operand-plane kernels (3 + 2 + 3 + 6).  Feed-forward: norm
-            # rows, gate|up and down GEMMs; norm rows, dact, dWd, dWg|dWu and
-            # dy GEMMs, norm backward, dg sum; float32 storage adds 3 + 4
             "gpu_launches": K * block_launches(w),
         }
         print(json.dumps(line), flush=True)

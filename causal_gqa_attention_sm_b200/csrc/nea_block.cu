@@ -83,6 +83,7 @@ struct Ctx {
   unsigned long long wait_limit;
   float* part = nullptr;  // split-K partial tiles (a piece of the workspace)
   size_t part_bytes = 0;
+  nea::SplitParams planes{};  // operand-plane splits not launched yet
 };
 
 // Bytes set aside for split-K partial tiles: up to 4 chunks of every tile of
@@ -141,8 +142,19 @@ cudaError_t launch_pdl(K kern, unsigned grid, unsigned block, size_t smem, cudaS
   return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
-// fp32 [n] -> hi/lo planes (float32 storage); bfloat16 storage reads the
-// tensor itself.
+// Launches the pending operand-plane splits, if any, as one kernel.
+int flush_planes(Ctx& c) {
+  nea::SplitParams& sp = c.planes;
+  if (sp.n == 0) return NEA_OK;
+  const unsigned grid = unsigned(std::min<long long>((sp.total + 255) / 256, (long long)c.n_sm * 8));
+  const cudaError_t e = launch_pdl(nea::split_planes_kernel, grid, 256u, size_t(0), c.stream, sp);
+  sp = nea::SplitParams{};
+  return e == cudaSuccess ? NEA_OK : fail(e);
+}
+
+// fp32 [rows][cols] -> hi/lo planes (float32 storage), queued: every product
+// launch first flushes the queue, so one kernel splits all the operands a
+// call needs.  bfloat16 storage reads the tensor itself.
 int make_operand(Ctx& c, Carve& w, const void* src, long long rows, long long cols, Operand* op) {
   op->rows = rows;
   op->cols = cols;
@@ -153,11 +165,14 @@ int make_operand(Ctx& c, Carve& w, const void* src, long long rows, long long co
   const size_t n = size_t(rows) * cols;
   auto* hi = static_cast<__nv_bfloat16*>(w.take(n * 2));
   auto* lo = static_cast<__nv_bfloat16*>(w.take(n * 2));
-  const long long n4 = static_cast<long long>(n / 4);
-  const unsigned grid = unsigned(std::min<long long>((n4 + 255) / 256, (long long)c.n_sm * 8));
-  const cudaError_t e = launch_pdl(nea::split_planes_kernel, grid, 256u, size_t(0), c.stream,
-                                   static_cast<const float*>(src), hi, lo, n4);
-  if (e != cudaSuccess) return fail(e);
+  if (c.planes.n == nea::kSplitJobs) {
+    const int rc = flush_planes(c);
+    if (rc) return rc;
+  }
+  nea::SplitParams& sp = c.planes;
+  sp.job[sp.n] = nea::SplitJob{static_cast<const float*>(src), hi, lo, sp.total};
+  sp.n += 1;
+  sp.total += static_cast<long long>(n / 4);
   op->hi = hi;
   op->lo = lo;
   return NEA_OK;
@@ -194,7 +209,8 @@ struct Seg {
 int gemm_seg(Ctx& c, const Seg* segs, int n_seg, bool kseg, bool a_mn, bool b_mn, int M, void* out, long long ldo,
              bool out_f32, const void* res, int mode = 0, void* const* pl = nullptr, const void* const* ab = nullptr) {
   nea::GemmParams p{};
-  int rc;
+  int rc = flush_planes(c);  // the operands' planes first
+  if (rc) return rc;
   const bool pair = mode == 1;  // segments 0 and 1 are the two halves of one 256-wide B tile
   for (int i = 0; i < n_seg; ++i) {
     const Seg& g = segs[i];

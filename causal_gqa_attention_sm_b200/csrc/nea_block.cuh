@@ -572,18 +572,35 @@ __global__ void __launch_bounds__(256) rmsnorm_rows_kernel(const void* x, const 
   }
 }
 
-// fp32 tensor of n elements (n a multiple of 4) -> bf16 hi and lo planes.
-__global__ void __launch_bounds__(256) split_planes_kernel(const float* src, __nv_bfloat16* hi, __nv_bfloat16* lo,
-                                                           long long n4) {
+// fp32 tensors -> bf16 hi and lo planes, up to kSplitJobs tensors in one
+// launch (the operands of one call), 16 bytes per thread per step.
+constexpr int kSplitJobs = 6;
+struct SplitJob {
+  const float* src;
+  __nv_bfloat16* hi;
+  __nv_bfloat16* lo;
+  long long start;  // first 4-element chunk of this tensor in the launch's range
+};
+struct SplitParams {
+  SplitJob job[kSplitJobs];
+  int n;
+  long long total;  // 4-element chunks of all tensors
+};
+
+__global__ void __launch_bounds__(256) split_planes_kernel(const __grid_constant__ SplitParams p) {
   grid_dep_wait();
   grid_dep_launch();
-  for (long long i = blockIdx.x * 256ll + threadIdx.x; i < n4; i += 256ll * gridDim.x) {
-    const float4 v = reinterpret_cast<const float4*>(src)[i];
+  for (long long i = blockIdx.x * 256ll + threadIdx.x; i < p.total; i += 256ll * gridDim.x) {
+    int j = 0;
+    while (j + 1 < p.n && i >= p.job[j + 1].start) ++j;
+    const SplitJob& q = p.job[j];
+    const long long k = i - q.start;
+    const float4 v = reinterpret_cast<const float4*>(q.src)[k];
     uint2 h, l;
     split_bf16(v.x, v.y, h.x, l.x);
     split_bf16(v.z, v.w, h.y, l.y);
-    reinterpret_cast<uint2*>(hi)[i] = h;
-    reinterpret_cast<uint2*>(lo)[i] = l;
+    reinterpret_cast<uint2*>(q.hi)[k] = h;
+    reinterpret_cast<uint2*>(q.lo)[k] = l;
   }
 }
 
