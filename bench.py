@@ -519,7 +519,7 @@ def decode_main(a, w, rank, world, local):
         line = {
             "metric": DECODE_METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
             "warmup": a.warmup, "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
             "config": config_of(w, world),
             "tokens_per_s": w.B * K * world / (total_ms * 1e-3),
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks.summary(),
