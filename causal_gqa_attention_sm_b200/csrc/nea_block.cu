@@ -232,19 +232,42 @@ int gemm_seg(Ctx& c, const Seg* segs, int n_seg, bool kseg, bool a_mn, bool b_mn
     return n;
   };
   const int n_m = (M + nea::kGemmBM - 1) / nea::kGemmBM;
-  // tile width: 256 where the tiles still fill the SMs about as well -- a
-  // wave of 256-wide tiles is taken to cost 1.4 waves of 128-wide ones with
-  // bf16 operands (they stream from L2, and the wider tile reads A once for
-  // twice the columns) and 1.8 with hi/lo planes (whose 96 KB stages leave
-  // room for two in flight, against three); measured on the block's
-  // products.  The SwiGLU forward pairs Wg and Wu in one 256-wide tile.
-  int bn = 128;
-  if (pair) {
-    bn = 256;
-  } else {
-    const long long w128 = (static_cast<long long>(n_m) * n_tiles_n(128) + c.n_sm - 1) / c.n_sm;
-    const long long w256 = (static_cast<long long>(n_m) * n_tiles_n(256) + c.n_sm - 1) / c.n_sm;
-    if (w128 > 1 && (c.f32 ? 1.8 : 1.4) * double(w256) < double(w128)) bn = 256;
+  int n_k_all = 0;  // k-steps of the whole product
+  for (int i = 0; i < n_seg; ++i)
+    n_k_all += (kseg || (pair && i == 0)) ? int((segs[i].width + nea::kGemmBK - 1) / nea::kGemmBK) : 0;
+  if (!kseg && !pair) n_k_all = int(((a_mn ? segs[0].A.rows : segs[0].A.cols) + nea::kGemmBK - 1) / nea::kGemmBK);
+  // Tile width and split-K chunk count from a cost model in k-steps of a
+  // 128-wide tile: waves of units x (k-steps per unit + 4 for a unit's ramp
+  // and epilogue), a 256-wide unit counted as 1.4 such units with bf16
+  // operands (they stream from L2, and the wider tile reads A once for twice
+  // the columns) and 1.8 with hi/lo planes (whose 96 KB stages leave room
+  // for two in flight, against three), plus 4 for the partial-tile reduce;
+  // factors measured on the block's products.  A split writes fp32 partial
+  // tiles (at most 4 chunks of two k-steps or more, within the reserve);
+  // with hi/lo planes it pays on the feed-forward's down and dy products
+  // (96 tiles of 256 columns, 48 and 96 k-steps: a 3-way split took the
+  // forward from 250 to 238 us and the backward from 509 to 485 us).
+  // The SwiGLU epilogues run unsplit; the forward pairs Wg and Wu in one
+  // 256-wide tile.
+  int bn = pair ? 256 : 128, split = 1;
+  if (!pair && n_k_all > 0) {
+    double best = 1e300;
+    for (int w = 128; w <= 256; w += 128) {
+      const long long tiles = static_cast<long long>(n_m) * n_tiles_n(w);
+      for (int sp = 1; sp <= (mode == 0 && c.part ? 4 : 1); ++sp) {
+        // bf16 products are fast enough that the partial tiles' traffic only
+        // pays for 128-wide tiles that alone leave SMs idle (a 3-way split of
+        // the feed-forward's down product, 96 tiles of 256 columns, took its
+        // forward from 103 to 124 us)
+        if (sp > 1 && (n_k_all < 2 * sp || size_t(tiles) * sp * 128 * w * 4 > c.part_bytes ||
+                       (!c.f32 && (w == 256 || tiles >= c.n_sm))))
+          break;
+        const int k_per = (n_k_all + sp - 1) / sp;
+        const long long waves = (tiles * sp + c.n_sm - 1) / c.n_sm;
+        const double cost = double(waves) * (k_per + 4) * (w == 256 ? (c.f32 ? 1.8 : 1.4) : 1.0) + (sp > 1 ? 4 : 0);
+        if (cost < best - 1e-9) best = cost, bn = w, split = sp;
+      }
+    }
   }
   int N = 0, K = 0, begin = 0;
   for (int i = 0; i < n_seg; ++i) {
@@ -281,17 +304,8 @@ int gemm_seg(Ctx& c, const Seg* segs, int n_seg, bool kseg, bool a_mn, bool b_mn
   p.err = c.err;
   p.wait_limit = c.wait_limit;
   if (p.n_tiles == 0 || K == 0) return NEA_OK;
-  // split K (128-wide tiles, plain epilogue) when the tiles leave SMs idle:
-  // the chunk count (at most 4, each of two k-steps or more) that minimises
-  // the per-CTA share of work
-  p.split = 1;
-  if (bn == 128 && p.n_tiles < c.n_sm && c.part && mode == 0) {
-    double best = double((p.n_tiles + c.n_sm - 1) / c.n_sm);
-    for (int sp = 2; sp <= 4 && p.n_k >= 2 * sp; ++sp) {
-      const double share = double((p.n_tiles * sp + c.n_sm - 1) / c.n_sm) / sp;
-      if (share < best - 1e-9 && size_t(p.n_tiles) * sp * 128 * 128 * 4 <= c.part_bytes) best = share, p.split = sp;
-    }
-  }
+  p.split = split;
+  p.bn = bn;
   p.k_per = (p.n_k + p.split - 1) / p.split;
   p.split = (p.n_k + p.k_per - 1) / p.k_per;
   p.part = p.split > 1 ? c.part : nullptr;
@@ -304,7 +318,7 @@ int gemm_seg(Ctx& c, const Seg* segs, int n_seg, bool kseg, bool a_mn, bool b_mn
     }
     cudaError_t e = launch_pdl(kern, grid, unsigned(nea::kGemmThreads), size_t(smem), c.stream, p);
     if (e == cudaSuccess && p.split > 1)
-      e = launch_pdl(nea::gemm_reduce_kernel, unsigned(p.n_tiles * 16), 256u, size_t(0), c.stream, p);
+      e = launch_pdl(nea::gemm_reduce_kernel, unsigned(p.n_tiles * (bn / 8)), 256u, size_t(0), c.stream, p);
     return e == cudaSuccess ? NEA_OK : fail(e);
   };
   const int form = (a_mn ? 2 : 0) + (b_mn ? 1 : 0);

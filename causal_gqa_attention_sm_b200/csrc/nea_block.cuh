@@ -59,8 +59,9 @@ struct GemmParams {
   int n_m, n_n, n_k, n_tiles;  // tiles of 128 x BN (mode 1: 128 output columns of each of a, b)
   // split K: work unit u is tile u % n_tiles over k-steps of chunk u /
   // n_tiles; with split > 1 each unit writes an fp32 partial tile to
-  // part[u][128][128] and gemm_reduce_kernel sums them into the output
+  // part[u][128][bn] and gemm_reduce_kernel sums them into the output
   int split, k_per;   // chunks, k-steps per chunk
+  int bn;             // the launch's tile width
   float* part;
   // epilogue mode: 0 the plain store above; 1 the SwiGLU forward: a 256-wide
   // tile whose B halves are the same 128 columns of seg[0].b (Wg) and
@@ -91,7 +92,7 @@ __device__ __forceinline__ void gemm_store(const GemmParams& p, int row, int ni,
   const int ns = p.kseg ? 0 : gemm_seg_of(p, ni);
   void* const out = p.kseg ? p.out : p.seg[ns].out;
   const long long ldo = p.kseg ? p.ldo : p.seg[ns].ldo;
-  const int col = (ni - (p.kseg ? 0 : p.seg[ns].begin)) * 128 + c;
+  const int col = (ni - (p.kseg ? 0 : p.seg[ns].begin)) * p.bn + c;
   if (row >= p.M || col >= (p.kseg ? p.N : int(ldo))) return;
   const size_t o = size_t(row) * ldo + col;
   if (p.out_f32) {
@@ -103,18 +104,21 @@ __device__ __forceinline__ void gemm_store(const GemmParams& p, int row, int ni,
 }
 
 // Sums the split partial tiles in chunk order (deterministic) and stores
-// the output: 16 CTAs per tile, four consecutive elements per thread.
+// the output: bn / 8 CTAs per 128 x bn tile, four consecutive elements per
+// thread.
 __global__ void __launch_bounds__(256) gemm_reduce_kernel(const __grid_constant__ GemmParams p) {
   grid_dep_wait();
   grid_dep_launch();
-  const int t = blockIdx.x >> 4, mi = t % p.n_m, ni = t / p.n_m;
-  const int e = ((blockIdx.x & 15) * 256 + threadIdx.x) * 4;  // element of the 128 x 128 tile
+  const int per = p.bn / 8;  // CTAs per tile
+  const int t = int(blockIdx.x) / per, mi = t % p.n_m, ni = t / p.n_m;
+  const int e = ((int(blockIdx.x) % per) * 256 + threadIdx.x) * 4;  // element of the 128 x bn tile
+  const size_t tile = size_t(128) * p.bn;
   float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int s = 0; s < p.split; ++s) {
-    const float4 u = *reinterpret_cast<const float4*>(p.part + (size_t(s) * p.n_tiles + t) * 128 * 128 + e);
+    const float4 u = *reinterpret_cast<const float4*>(p.part + (size_t(s) * p.n_tiles + t) * tile + e);
     v.x += u.x, v.y += u.y, v.z += u.z, v.w += u.w;
   }
-  const int row = mi * 128 + e / 128, c = e % 128;
+  const int row = mi * 128 + e / p.bn, c = e % p.bn;
   gemm_store(p, row, ni, c, v.x);
   gemm_store(p, row, ni, c + 1, v.y);
   gemm_store(p, row, ni, c + 2, v.z);
@@ -355,10 +359,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       const int ab = lt & 1;
       if (!(ok = wait_warp(&acc_full[ab], (lt >> 1) & 1, wc, kErrWaitMma))) break;
       tc_fence_after();
-      if (BN == 128 && p.split > 1) {  // this chunk's partial tile, row-major 128 x 128 fp32
-        float* dst = p.part + size_t(u) * 128 * 128 + size_t(q4 * 32 + lane) * 128;
+      if (p.split > 1) {  // this chunk's partial tile, row-major 128 x BN fp32
+        float* dst = p.part + size_t(u) * 128 * BN + size_t(q4 * 32 + lane) * BN;
 #pragma unroll 1
-        for (int c = ch * 2; c < ch * 2 + 2; ++c) {
+        for (int c = ch * (BN / 64); c < (ch + 1) * (BN / 64); ++c) {
           uint32_t r[32];
           tmem_ld32(tmem_addr(tbase, q4 * 32, ab * acc_cols + c * 32), r);
 #pragma unroll
