@@ -190,6 +190,26 @@ __device__ __forceinline__ void row_planes8(void* hi, void* lo, size_t o, int n,
   }
 }
 
+// Single elements of a tensor in the storage type (fp32, or bf16 when
+// !f32), and of a GEMM operand's bf16 planes (hi, and when `lo` is given the
+// rounding remainder), for the transposed SwiGLU epilogues, whose lanes hold
+// consecutive columns of one row.
+__device__ __forceinline__ float elem_load(const void* src, size_t o, bool f32) {
+  if (f32) return __ldg(static_cast<const float*>(src) + o);
+  return __uint_as_float(uint32_t(__ldg(static_cast<const unsigned short*>(src) + o)) << 16);
+}
+
+__device__ __forceinline__ void elem_store(void* dst, size_t o, bool f32, float v) {
+  if (f32) static_cast<float*>(dst)[o] = v;
+  else static_cast<__nv_bfloat16*>(dst)[o] = __float2bfloat16_rn(v);
+}
+
+__device__ __forceinline__ void elem_planes(void* hi, void* lo, size_t o, float v) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(v);
+  static_cast<__nv_bfloat16*>(hi)[o] = h;
+  if (lo) static_cast<__nv_bfloat16*>(lo)[o] = __float2bfloat16_rn(v - __bfloat162float(h));
+}
+
 // 1 / (1 + e^-z) with the fast exponential and division intrinsics; z is
 // clamped at -80 so that e^-z stays below 2^126 (the divide's range), which
 // changes the result only where it is below 2e-35.
@@ -201,11 +221,13 @@ struct GemmSmem {
   static constexpr uint32_t kOpB = BN * 128;             // the B tile: BN x 64
   static constexpr int kPlanes = SPLIT ? 2 : 1;
   static constexpr uint32_t kStage = kPlanes * (kOp + kOpB);  // A planes, then B planes
-  static constexpr int ST = (200 * 1024) / kStage;       // 6, 4 (bf16); 3, 2 (split)
-  static constexpr uint32_t kBars = ST * kStage;         // full[ST], empty[ST], acc_full[2], acc_empty[2]
+  static constexpr int ST = (200 * 1024) / kStage;       // 6, 4 (bf16); 3, 2 (split): 192 KB
+  static constexpr uint32_t kEpi = ST * kStage;          // each epilogue warp's 32 x 33 fp32 staging rows
+  static constexpr uint32_t kBars = kEpi + kGemmEpiWarps * 32 * 33 * 4;  // full[ST], empty[ST], acc_full[2], acc_empty[2]
   static constexpr uint32_t kMisc = kBars + (2 * ST + 4) * 8;  // TMEM base, abort flag
   static constexpr uint32_t kBytes = kMisc + 16;
   static constexpr uint32_t kAlloc = kBytes + 1024;
+  static_assert(kAlloc <= 232448, "shared memory");
 };
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int c0, int c1, uint64_t* bar) {
@@ -352,6 +374,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     // ---------------------------------------------------------------- epilogue
     const int q4 = warp & 3;         // TMEM lanes 32 q4 .. 32 q4 + 31
     const int ch = (warp - 2) >> 2;  // column half of the tile
+    // float32 storage, SwiGLU epilogues: a 32-column chunk of the warp's 32
+    // TMEM lanes goes through the warp's staging rows in shared memory
+    // (padded to 33 words: no bank conflicts either way), so that lane l then
+    // holds column l of the 32 rows and every global access is one row's 32
+    // consecutive elements.  The per-row 16-byte accesses these epilogues
+    // would otherwise make (fp32 a and b, hi/lo planes: 12 to 20 bytes per
+    // element in 16-byte pieces of 32 rows per warp instruction) cost more
+    // than the staging; for the plain stores and for bf16 storage the
+    // staging's shared-memory traffic, which competes with the MMAs' operand
+    // reads, costs more than it saves.
+    float* const stage_rows = reinterpret_cast<float*>(sm + L::kEpi) + (warp - 2) * (32 * 33);
+    // the chunk at TMEM column `col`: v[r] = row r of this lane's column
+    auto load_chunk = [&](uint32_t col, float* v) {
+      uint32_t r[32];
+      tmem_ld32(tmem_addr(tbase, q4 * 32, col), r);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) stage_rows[lane * 33 + j] = __uint_as_float(r[j]);
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = stage_rows[i * 33 + lane];
+      __syncwarp();
+    };
     int lt = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < p.n_tiles * p.split && ok; u += gridDim.x, ++lt) {
@@ -376,8 +420,63 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         continue;
       }
       const int mi = t % p.n_m, ni = t / p.n_m;
-      const int row = mi * kGemmBM + q4 * 32 + lane;
-      if (p.mode != 0) {  // SwiGLU epilogues, 32 columns of a row per pass, 8 at a time
+      const int row0 = mi * kGemmBM + q4 * 32;  // the warp's first row
+      const int nrow = min(32, p.M - row0);     // its rows inside the product (warp-uniform)
+      if constexpr (SPLIT) {  // float32 storage: the SwiGLU epilogues through the staging rows
+        if (p.mode != 0) {
+          if (p.mode == 1) {
+            // SwiGLU forward: b 128 columns beside a; writes a, b and act's planes
+#pragma unroll 1
+            for (int c = ch * 2; c < ch * 2 + 2; ++c) {
+              float a[32], b[32];
+              load_chunk(ab * acc_cols + c * 32, a);
+              load_chunk(ab * acc_cols + 128 + c * 32, b);
+              const int col = ni * 128 + c * 32 + lane;
+              if (col < p.N) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {  // full unroll: static indices keep the arrays in registers
+                  if (i >= nrow) break;
+                  const size_t o = size_t(row0 + i) * p.ldo + col;
+                  if (p.seg[0].out) elem_store(p.seg[0].out, o, p.out_f32, a[i]);
+                  if (p.seg[1].out) elem_store(p.seg[1].out, o, p.out_f32, b[i]);
+                  elem_planes(p.pl[0], p.pl[1], o, a[i] * sigmoid_f(a[i]) * b[i]);
+                }
+              }
+            }
+          } else {
+            // SwiGLU backward: dact with the forward's a and b -> planes of da, db, act
+#pragma unroll 1
+            for (int c = ch * (BN / 64); c < (ch + 1) * (BN / 64); ++c) {
+              float d[32], a[32], b[32];
+              load_chunk(ab * acc_cols + c * 32, d);
+              const int col = ni * BN + c * 32 + lane;
+              if (col < p.N) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {  // all of the chunk's loads in flight together
+                  const size_t o = size_t(row0 + min(i, nrow - 1)) * p.ldo + col;
+                  a[i] = elem_load(p.ab[0], o, p.out_f32);
+                  b[i] = elem_load(p.ab[1], o, p.out_f32);
+                }
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {  // full unroll: static indices keep the arrays in registers
+                  if (i >= nrow) break;
+                  const size_t o = size_t(row0 + i) * p.ldo + col;
+                  const float sg = sigmoid_f(a[i]), si = a[i] * sg;
+                  elem_planes(p.pl[0], p.pl[1], o, d[i] * b[i] * sg * (1.f + a[i] * (1.f - sg)));  // da
+                  elem_planes(p.pl[2], p.pl[3], o, d[i] * si);                                     // db
+                  elem_planes(p.pl[4], p.pl[5], o, si * b[i]);                                     // act
+                }
+              }
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[ab]);
+          continue;
+        }
+      }
+      const int row = row0 + lane;
+      if (!SPLIT && p.mode != 0) {  // bfloat16 storage: the SwiGLU epilogues, 32 columns of a row per pass, 8 at a time
         const int nc = p.mode == 1 ? 2 : BN / 64;  // 32-column chunks per warp
 #pragma unroll 1
         for (int c = ch * nc; c < ch * nc + nc; ++c) {
