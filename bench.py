@@ -636,9 +636,10 @@ def block_launches(w):
     rows, dWq|dWk|dWv GEMM + reduce, dy GEMM, norm backward, dg sum (12).
     Feed-forward: norm rows, gate|up and down GEMMs; norm rows, dact, dWd,
     dWg|dWu and dy GEMMs, norm backward, dg sum (10).  Float32 storage adds
-    one operand-plane launch per call (4 and 2)."""
+    one operand-plane launch per call (4 and 2) and, for the feed-forward,
+    the split-K reduces of the down and dy products (2)."""
     if w.ffn:
-        return 12 if w.dtype == "f32" else 10
+        return 14 if w.dtype == "f32" else 10
     return 16 if w.dtype == "f32" else 12
 
 
