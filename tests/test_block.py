@@ -167,6 +167,8 @@ FFN_CASES = [
     (2, 100, 256, 320, "f32"),      # M = 200 and F = 320: ragged token and width tiles
     (2, 100, 256, 320, "bf16"),
     (1, 64, 64, 64, "f32"),         # one partial tile everywhere
+    (1, 1000, 768, 3072, "f32"),    # ragged token tiles in split-K products of 256-wide tiles
+    (1, 1000, 768, 3072, "bf16"),
     (8, 512, 768, 3072, "f32"),     # the GPU model layer, F = 4 C
     (8, 512, 768, 3072, "bf16"),
 ]
