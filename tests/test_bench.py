@@ -101,3 +101,20 @@ def test_clock_sampler_without_nvidia_smi_reports_it(tmp_path, monkeypatch):
     assert c.summary()["reasons"] == ["nvidia-smi unavailable"]
     assert c.f.closed
     assert not bench.ClockSampler(3).path.startswith(ROOT)  # raw samples go to a temporary file by default
+
+
+def test_reference_arm_under_torchrun_prints_once():
+    """Launched as the driver launches N > 1 (torchrun, one process per rank),
+    the reference arm runs on rank 0 alone: one JSON line, every rank exits 0."""
+    import socket
+
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2", "--master-addr",
+           "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus",
+           "2", "--workload", "tiny", "--steps", "1", "--warmup", "3"]
+    out = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [json.loads(l) for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1 and lines[0]["impl"] == "reference" and lines[0]["n_gpus"] == 2
