@@ -87,17 +87,19 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // Descriptor of a [B][T][H][D] tensor read as 128-row tiles of one head:
-// dimensions (innermost first) {D, H, T, B}, box {D, 1, 128, 1}; rows past T
-// read as zero.  bf16 tiles land in the operand swizzle (row = atom).
+// dimensions (innermost first) {D, H, T, B}, box {min(D, 64), 1, 128, 1};
+// rows past T read as zero.  bf16 tiles land in the operand swizzle (row =
+// atom); D = 128 takes two boxes per tile, one per 64-column block.
 int make_tile_map(CUtensorMap* m, const void* base, int B, int T, int H, int D) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (!enc) return NEA_ERR_CUDA;
   const cuuint64_t e = 2;
+  const cuuint32_t bx = D < 64 ? cuuint32_t(D) : 64u;
   const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(H), cuuint64_t(T), cuuint64_t(B)};
   const cuuint64_t strides[3] = {D * e, cuuint64_t(H) * D * e, cuuint64_t(T) * H * D * e};
-  const cuuint32_t box[4] = {cuuint32_t(D), 1, cuuint32_t(nea::kTileRows), 1};
+  const cuuint32_t box[4] = {bx, 1, cuuint32_t(nea::kTileRows), 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
-  const CUtensorMapSwizzle sw = D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  const CUtensorMapSwizzle sw = bx == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -235,10 +237,11 @@ int ensure_ws(DeviceState& st, size_t bytes) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Shape/dtype checks shared by the entry points.  `empty` is set when
-// B*T == 0 (nothing to do, pointers may be null).
-int check_shape(int B, int T, int Hq, int Hkv, int D, int dtype, int causal, bool* empty) {
+// B*T == 0 (nothing to do, pointers may be null).  D = 128 only where
+// `d128` is set (the forward, bfloat16 storage).
+int check_shape(int B, int T, int Hq, int Hkv, int D, int dtype, int causal, bool* empty, bool d128 = false) {
   if (B < 0 || T < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return NEA_ERR_ARG;
-  if (D != 32 && D != 64) return NEA_ERR_ARG;
+  if (D != 32 && D != 64 && !(D == 128 && d128 && dtype == NEA_BF16)) return NEA_ERR_ARG;
   if (dtype != NEA_F32 && dtype != NEA_BF16) return NEA_ERR_ARG;
   if (causal != 0 && causal != 1) return NEA_ERR_ARG;
   // 32-bit grid and tile indices: keep every launch well inside them
@@ -358,15 +361,17 @@ int launch_prep(const nea::PrepJob* jobs, const bool* run, int n, int T, int D, 
     pp.job[pp.n_jobs++] = j;
     pp.total += j.chunks;
   }
-  const long long rt_blocks = D == 64 ? (f32 ? nea::rowterm_blocks<64, true>(pp.rt_rows)
-                                                : nea::rowterm_blocks<64, false>(pp.rt_rows))
-                                      : (f32 ? nea::rowterm_blocks<32, true>(pp.rt_rows)
-                                             : nea::rowterm_blocks<32, false>(pp.rt_rows));
+  const long long rt_blocks = D == 128  ? 0  // the forward alone (no row terms)
+                              : D == 64 ? (f32 ? nea::rowterm_blocks<64, true>(pp.rt_rows)
+                                               : nea::rowterm_blocks<64, false>(pp.rt_rows))
+                                        : (f32 ? nea::rowterm_blocks<32, true>(pp.rt_rows)
+                                               : nea::rowterm_blocks<32, false>(pp.rt_rows));
   const long long blocks = pp.prep_blocks + rt_blocks;
   if (blocks == 0) return NEA_OK;
   const unsigned g = unsigned(blocks);
-  auto kern = D == 64 ? (f32 ? nea::attn_prep_kernel<64, true> : nea::attn_prep_kernel<64, false>)
-                      : (f32 ? nea::attn_prep_kernel<32, true> : nea::attn_prep_kernel<32, false>);
+  auto kern = D == 128  ? nea::attn_prep_kernel<128, false>
+              : D == 64 ? (f32 ? nea::attn_prep_kernel<64, true> : nea::attn_prep_kernel<64, false>)
+                        : (f32 ? nea::attn_prep_kernel<32, true> : nea::attn_prep_kernel<32, false>);
   const cudaError_t e = launch_dependent(kern, g, 256, 0, stream, pp);
   return e == cudaSuccess ? NEA_OK : cuda_fail(e);
 }
@@ -385,7 +390,7 @@ template <int D, bool F32IO>
 int launch_fwd(uint32_t& attr_done, const nea::FwdParams& p, cudaStream_t stream) {
   using L = nea::FwdSmem<D, F32IO>;
   auto kern = nea::attn_fwd_kernel<D, F32IO>;
-  int rc = set_smem(attr_done, (D == 64) * 2 + F32IO, kern, L::kAlloc);
+  int rc = set_smem(attr_done, D == 128 ? 8 : (D == 64) * 2 + F32IO, kern, L::kAlloc);
   if (rc) return rc;
   const cudaError_t e = launch_dependent(kern, unsigned(p.B * p.Hq * p.n_pairs), L::kThreads, L::kAlloc, stream, p);
   return e == cudaSuccess ? NEA_OK : cuda_fail(e);
@@ -531,8 +536,8 @@ size_t fwd_plane_bytes(int B, int T, int Hq, int Hkv, int D, bool f32, bool rope
 }
 
 int check_fwd_args(const void* Q, const void* K, const void* V, const void* O, const float* LSE, int B, int T,
-                   int Hq, int Hkv, int D, int dtype, float rope_base, int causal, bool* empty) {
-  int rc = check_shape(B, T, Hq, Hkv, D, dtype, causal, empty);
+                   int Hq, int Hkv, int D, int dtype, float rope_base, int causal, bool* empty, bool d128 = false) {
+  int rc = check_shape(B, T, Hq, Hkv, D, dtype, causal, empty, d128);
   if (rc || *empty) return rc;
   if (!Q || !K || !V || !O || !LSE) return NEA_ERR_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE)) return NEA_ERR_ARG;
@@ -595,9 +600,10 @@ int run_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, in
 #ifdef NEA_TRACE
   p.trace = t_trace;
 #endif
-  rc = dispatch(D, dtype, [&](auto d, auto f) {
-    return launch_fwd<decltype(d)::value, decltype(f)::value>(st->attr_done, p, stream);
-  });
+  rc = D == 128 ? launch_fwd<128, false>(st->attr_done, p, stream)  // bfloat16 storage only
+                : dispatch(D, dtype, [&](auto d, auto f) {
+                    return launch_fwd<decltype(d)::value, decltype(f)::value>(st->attr_done, p, stream);
+                  });
   prof_record(1, stream);
   return rc;
 }
@@ -625,7 +631,7 @@ extern "C" {
 int nea_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int T, int Hq, int Hkv,
                  int D, int dtype, float rope_base, int causal, void* stream) {
   bool empty = false;
-  int rc = check_fwd_args(Q, K, V, O, LSE, B, T, Hq, Hkv, D, dtype, rope_base, causal, &empty);
+  int rc = check_fwd_args(Q, K, V, O, LSE, B, T, Hq, Hkv, D, dtype, rope_base, causal, &empty, true);
   if (rc || empty) return rc;
   return run_fwd(Q, K, V, O, LSE, B, T, Hq, Hkv, D, dtype, rope_base, causal, static_cast<cudaStream_t>(stream),
                  nullptr);

@@ -74,8 +74,9 @@ struct FwdParams {
 
 template <int D, bool F32IO>
 struct FwdSmem {
-  static constexpr int kNK = F32IO ? 3 : 4;    // K ring stages
-  static constexpr int kNV = F32IO ? 2 : 3;    // V ring stages
+  // K and V ring stages (D = 128, bf16 only: 32 KB tiles, two of each)
+  static constexpr int kNK = F32IO ? 3 : (D == 128 ? 2 : 4);
+  static constexpr int kNV = F32IO ? 2 : (D == 128 ? 2 : 3);
   static constexpr uint32_t kTile = Stage<D, F32IO>::kBytes;  // one tile: hi (+ lo)
   static constexpr uint32_t kQA = 0;
   static constexpr uint32_t kQB = kTile;
@@ -106,7 +107,10 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
   constexpr uint32_t OPB = TileGeom<D>::kOpBytes;
   constexpr int NK = L::kNK, NV = L::kNV;
   constexpr int kTerms = F32IO ? 3 : 1;
-  constexpr bool kSepP = !F32IO;  // P in its own TMEM columns
+  // P in its own TMEM columns; float32 storage (P hi over S, lo apart) and
+  // D = 128 (O takes the columns P would) write P over S
+  constexpr bool kSepP = !F32IO && D <= 64;
+  static_assert(D <= 64 || !F32IO, "D = 128 runs with bfloat16 storage");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
@@ -218,7 +222,7 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
           tmem_st32(ocol + 32 * c, rr);
         }
       };
-      if constexpr (kSepP) {
+      if constexpr (!F32IO) {
         // P = exp2(s * scale_log2 - m) -> bf16, all 128 columns in registers;
         // one pair in four on the FMA pipe, the rest on the exponential unit
         uint32_t pk[64];
@@ -238,6 +242,7 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
           pk[i] = pack_bf16(p0, p1);
         }
         // PV_X(j-1) has read P_X(j-1) and updated O before both are touched
+        // (P over S: S_X(j) was issued after PV_X(j-1) completed)
         if (j > 0 && !wait_warp(&bar_o[x], (j - 1) & 1, wc, kErrWaitMma)) { ok = false; break; }
         tc_fence_after();
         if (__any_sync(kFullMask, alpha != 1.f && j > 0)) rescale_o();
@@ -246,7 +251,7 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
           uint32_t part[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) part[i] = pk[16 * c + i];
-          tmem_st16(pcol + 16 * c, part);
+          tmem_st16((kSepP ? pcol : scol) + 16 * c, part);
         }
       } else {
         // P = exp2(s * scale_log2 - m) -> bf16 hi over S, lo apart
@@ -317,7 +322,9 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
         // a load of `row0` of tensor X: the tile (bf16) or its hi and lo planes
         auto load_tile = [&](uint8_t* dst, const CUtensorMap* hi, const CUtensorMap* lo, int head, int row0,
                              uint64_t* bar) {
-          tma_load_4d(dst, hi, 0, head, row0, b, bar);
+#pragma unroll
+          for (uint32_t cb = 0; cb < TileGeom<D>::kBlocks; ++cb)  // column blocks of 64 elements (D = 128)
+            tma_load_4d(dst + cb * TileGeom<D>::kBlockBytes, hi, int(cb) * 64, head, row0, b, bar);
           if (F32IO) tma_load_4d(dst + OPB, lo, 0, head, row0, b, bar);
         };
         // fault-injection hook: withhold the query tiles so every wait on them
@@ -374,8 +381,8 @@ __global__ void __launch_bounds__(FwdSmem<D, F32IO>::kThreads, 1)
 #pragma unroll
             for (int term = 0; term < kTerms; ++term) {
               // float32 storage: hi*hi + hi*lo + lo*hi
-              const uint32_t qa = sQ + (term == 2 ? OPB : 0) + kk * 32;
-              const uint32_t kb = sK + (term == 1 ? OPB : 0) + kk * 32;
+              const uint32_t qa = sQ + (term == 2 ? OPB : 0) + TileGeom<D>::kslice(kk);
+              const uint32_t kb = sK + (term == 1 ? OPB : 0) + TileGeom<D>::kslice(kk);
               mma_ss(dS, smem_desc(qa, RB, 16), smem_desc(kb, RB, 16), idS, (kk | term) != 0);
             }
           }

@@ -3,8 +3,11 @@
 // A [128 rows][D] tile of one head of a [B][T][H][D] tensor arrives in shared
 // memory by TMA (rows at or beyond T read as zero), already in the bf16
 // operand layout the tcgen05 MMAs read: rows of 2*D bytes with the hardware
-// swizzle whose atom equals the row.  Float32 storage stages two such tiles
-// per tensor tile (the hi and lo planes of the operand prologue).
+// swizzle whose atom equals the row.  Rows longer than the widest swizzle
+// (D = 128: 256 bytes) are cut into column blocks of 64 elements, each a
+// [128][64] tile of its own, kBlockBytes apart (two TMA boxes per tile).
+// Float32 storage stages two such tiles per tensor tile (the hi and lo planes
+// of the operand prologue).
 #pragma once
 
 #include "nea_device.cuh"
@@ -15,8 +18,14 @@ constexpr int kTileRows = 128;
 
 template <int D>
 struct TileGeom {
-  static constexpr uint32_t kRowBytes = 2 * D;                      // bf16 operand row
-  static constexpr uint32_t kOpBytes = kTileRows * kRowBytes;       // one bf16 operand tile
+  static constexpr uint32_t kRowBytes = 2 * D <= 128 ? 2 * D : 128;  // swizzle atom row of a column block
+  static constexpr uint32_t kBlocks = 2 * D / kRowBytes;             // column blocks of a row
+  static constexpr uint32_t kBlockBytes = kTileRows * kRowBytes;     // one column block of a tile
+  static constexpr uint32_t kOpBytes = kTileRows * 2 * D;            // one bf16 operand tile
+  // byte offset of the 16-column K slice kk of a K-major tile
+  __host__ __device__ static constexpr uint32_t kslice(int kk) {
+    return (kk * 32) % kRowBytes + (kk * 32) / kRowBytes * kBlockBytes;
+  }
 };
 
 // Bytes a TMA tile occupies, and the operand tiles it becomes: fp32 storage
