@@ -238,7 +238,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 // Shape/dtype checks shared by the entry points.  `empty` is set when
 // B*T == 0 (nothing to do, pointers may be null).  D = 128 only where
-// `d128` is set (the forward, bfloat16 storage).
+// `d128` is set (bfloat16 storage; not the allocation-free backward).
 int check_shape(int B, int T, int Hq, int Hkv, int D, int dtype, int causal, bool* empty, bool d128 = false) {
   if (B < 0 || T < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return NEA_ERR_ARG;
   if (D != 32 && D != 64 && !(D == 128 && d128 && dtype == NEA_BF16)) return NEA_ERR_ARG;
@@ -361,7 +361,7 @@ int launch_prep(const nea::PrepJob* jobs, const bool* run, int n, int T, int D, 
     pp.job[pp.n_jobs++] = j;
     pp.total += j.chunks;
   }
-  const long long rt_blocks = D == 128  ? 0  // the forward alone (no row terms)
+  const long long rt_blocks = D == 128  ? nea::rowterm_blocks<128, false>(pp.rt_rows)  // bfloat16 only
                               : D == 64 ? (f32 ? nea::rowterm_blocks<64, true>(pp.rt_rows)
                                                : nea::rowterm_blocks<64, false>(pp.rt_rows))
                                         : (f32 ? nea::rowterm_blocks<32, true>(pp.rt_rows)
@@ -405,8 +405,11 @@ template <int D, bool F32IO>
 int launch_bwd(uint32_t& attr_done, const nea::BwdParams& p, cudaStream_t stream, bool ev) {
   cudaError_t e;
   using L = std::conditional_t<F32IO, nea::Bwd32Smem<D>, nea::BwdSmem<D>>;
-  auto kern = F32IO ? nea::attn_bwd_f32_kernel<D> : nea::attn_bwd_kernel<D>;
-  int rc = set_smem(attr_done, 4 + (D == 64) * 2 + F32IO, kern, L::kAlloc);
+  auto kern = [] {
+    if constexpr (F32IO) return nea::attn_bwd_f32_kernel<D>;
+    else return nea::attn_bwd_kernel<D>;
+  }();
+  int rc = set_smem(attr_done, D == 128 ? 9 : 4 + (D == 64) * 2 + F32IO, kern, L::kAlloc);
   if (rc) return rc;
   e = launch_dependent(kern, unsigned(p.n_dkdv + p.B * p.Hq * p.n_tiles), L::kThreads, L::kAlloc, stream, p);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -417,8 +420,8 @@ int launch_bwd(uint32_t& attr_done, const nea::BwdParams& p, cudaStream_t stream
 
 int check_bwd_args(const void* Q, const void* K, const void* V, const void* O, const float* LSE, const void* dO,
                    void* dQ, void* dK, void* dV, int B, int T, int Hq, int Hkv, int D, int dtype, float rope_base,
-                   int causal, bool* empty) {
-  int rc = check_shape(B, T, Hq, Hkv, D, dtype, causal, empty);
+                   int causal, bool* empty, bool d128 = false) {
+  int rc = check_shape(B, T, Hq, Hkv, D, dtype, causal, empty, d128);
   if (rc || *empty) return rc;
   if (!Q || !K || !V || !O || !LSE || !dO || !dQ || !dK || !dV) return NEA_ERR_ARG;
   for (const void* ptr : {Q, K, V, O, static_cast<const void*>(LSE), dO, static_cast<const void*>(dQ),
@@ -520,6 +523,7 @@ int run_bwd(uint32_t& attr_done, uint8_t* ws, const float2* rope, int* status, c
 #ifdef NEA_TRACE
   p.trace = t_trace_bwd;
 #endif
+  if (D == 128) return launch_bwd<128, false>(attr_done, p, stream, ev);  // bfloat16 storage only
   return dispatch(D, dtype, [&](auto d, auto f) {
     return launch_bwd<decltype(d)::value, decltype(f)::value>(attr_done, p, stream, ev);
   });
@@ -639,7 +643,7 @@ int nea_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
 
 long long nea_attn_saved_bytes(int B, int T, int Hq, int Hkv, int D, int dtype, float rope_base) {
   bool empty = false;
-  if (check_shape(B, T, Hq, Hkv, D, dtype, 1, &empty) || !std::isfinite(rope_base)) return -1;
+  if (check_shape(B, T, Hq, Hkv, D, dtype, 1, &empty, true) || !std::isfinite(rope_base)) return -1;
   if (empty) return 0;
   return static_cast<long long>(fwd_plane_bytes(B, T, Hq, Hkv, D, dtype == NEA_F32, rope_base > 0.f));
 }
@@ -647,7 +651,7 @@ long long nea_attn_saved_bytes(int B, int T, int Hq, int Hkv, int D, int dtype, 
 int nea_attn_fwd_save(const void* Q, const void* K, const void* V, void* O, float* LSE, void* saved, int B, int T,
                       int Hq, int Hkv, int D, int dtype, float rope_base, int causal, void* stream) {
   bool empty = false;
-  int rc = check_fwd_args(Q, K, V, O, LSE, B, T, Hq, Hkv, D, dtype, rope_base, causal, &empty);
+  int rc = check_fwd_args(Q, K, V, O, LSE, B, T, Hq, Hkv, D, dtype, rope_base, causal, &empty, true);
   if (rc || empty) return rc;
   const bool need = fwd_plane_bytes(B, T, Hq, Hkv, D, dtype == NEA_F32, rope_base > 0.f) > 0;
   if (need && (!saved || !aligned16(saved))) return NEA_ERR_ARG;
@@ -659,7 +663,8 @@ int nea_attn_bwd(const void* Q, const void* K, const void* V, const void* O, con
                  void* dQ, void* dK, void* dV, int B, int T, int Hq, int Hkv, int D, int dtype, float rope_base,
                  int causal, void* stream_) {
   bool empty = false;
-  int rc = check_bwd_args(Q, K, V, O, LSE, dO, dQ, dK, dV, B, T, Hq, Hkv, D, dtype, rope_base, causal, &empty);
+  int rc = check_bwd_args(Q, K, V, O, LSE, dO, dQ, dK, dV, B, T, Hq, Hkv, D, dtype, rope_base, causal, &empty,
+                          true);
   if (rc || empty) return rc;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
 
@@ -679,7 +684,8 @@ int nea_attn_bwd_saved(const void* Q, const void* K, const void* V, const void* 
                        const void* saved, void* dQ, void* dK, void* dV, int B, int T, int Hq, int Hkv, int D,
                        int dtype, float rope_base, int causal, void* stream_) {
   bool empty = false;
-  int rc = check_bwd_args(Q, K, V, O, LSE, dO, dQ, dK, dV, B, T, Hq, Hkv, D, dtype, rope_base, causal, &empty);
+  int rc = check_bwd_args(Q, K, V, O, LSE, dO, dQ, dK, dV, B, T, Hq, Hkv, D, dtype, rope_base, causal, &empty,
+                          true);
   if (rc || empty) return rc;
   const bool f32 = dtype == NEA_F32, rope_on = rope_base > 0.f;
   if (fwd_plane_bytes(B, T, Hq, Hkv, D, f32, rope_on) == 0)  // nothing was saved: the regular backward

@@ -36,6 +36,11 @@
 // registers; dV(k) once P(k) is written; dK/dQ(k) once dS(k) is written.  The
 // rows overwrite P and dS of item k-1 only after the commit that follows
 // dK/dQ(k-1) (which covers every earlier MMA).
+// D = 128: the two accumulators take TMEM [256,512), so P goes over S and dS
+// over dP, each warp half writing its 64 columns' bf16 pairs into the first
+// 32 of its own 64 columns (no half overwrites scores the other still
+// reads); S(k+1) and dP(k+1) then wait for the commit after dK/dQ(k), and the
+// rings hold two stages (32 KB tiles).
 #pragma once
 
 #include <cuda.h>
@@ -82,7 +87,7 @@ struct BwdParams {
 
 template <int D>
 struct BwdSmem {
-  static constexpr int kStages = 3;
+  static constexpr int kStages = D == 128 ? 2 : 3;
   static constexpr uint32_t kTile = TileGeom<D>::kOpBytes;
   static constexpr uint32_t kR1 = 0;
   static constexpr uint32_t kR2 = kR1 + kTile;
@@ -207,6 +212,10 @@ __device__ __forceinline__ void attn_bwd_unit(const BwdParams& p, int bid) {
   grid_dep_wait();  // operand planes and row terms come from the prologue grid
   grid_dep_launch();
   constexpr uint32_t kColS = 0, kColDP = 128, kColAcc1 = 256, kColAcc2 = 256 + D, kColP = 384, kColDS = 448;
+  constexpr bool kOver = D == 128;  // P over S, dS over dP (see the header)
+  // TMEM column of the 16-column slice kk of P or dS (bf16 pairs)
+  auto p_col = [](int kk) -> uint32_t { return kOver ? kColS + 64 * (kk / 4) + 8 * (kk % 4) : kColP + 8 * kk; };
+  auto ds_col = [](int kk) -> uint32_t { return kOver ? kColDP + 64 * (kk / 4) + 8 * (kk % 4) : kColDS + 8 * kk; };
 
   if (warp == 9) {
     // ------------------------------------------------------------ TMA
@@ -220,7 +229,9 @@ __device__ __forceinline__ void attn_bwd_unit(const BwdParams& p, int bid) {
       prefetch_tmap(m_c1);
       prefetch_tmap(m_c2);
       auto load_tile = [&](uint8_t* dst, const CUtensorMap* m, int head, int row0, uint64_t* bar) {
-        tma_load_4d(dst, m, 0, head, row0, b, bar);
+#pragma unroll
+        for (uint32_t cb = 0; cb < TileGeom<D>::kBlocks; ++cb)  // column blocks of 64 elements (D = 128)
+          tma_load_4d(dst + cb * TileGeom<D>::kBlockBytes, m, int(cb) * 64, head, row0, b, bar);
       };
       // fault-injection hook: withhold the resident tiles so every wait on
       // them runs into its limit
@@ -261,7 +272,8 @@ __device__ __forceinline__ void attn_bwd_unit(const BwdParams& p, int bid) {
         const uint32_t sC1 = stage_c1(k);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tbase + kColS, smem_desc(sR1 + kk * 32, RB, 16), smem_desc(sC1 + kk * 32, RB, 16), idSS, kk != 0);
+          mma_ss(tbase + kColS, smem_desc(sR1 + TileGeom<D>::kslice(kk), RB, 16),
+                 smem_desc(sC1 + TileGeom<D>::kslice(kk), RB, 16), idSS, kk != 0);
         tc_commit(bar_s);
       };
       bool ok = wait_thread(bar_rtma, 0, wc, kErrWaitProducer) &&
@@ -275,10 +287,11 @@ __device__ __forceinline__ void attn_bwd_unit(const BwdParams& p, int bid) {
         // dP(k) overwrites dP(k-1), which the rows read before dS(k-1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tbase + kColDP, smem_desc(sR2 + kk * 32, RB, 16), smem_desc(sC2 + kk * 32, RB, 16), idSS, kk != 0);
+          mma_ss(tbase + kColDP, smem_desc(sR2 + TileGeom<D>::kslice(kk), RB, 16),
+                 smem_desc(sC2 + TileGeom<D>::kslice(kk), RB, 16), idSS, kk != 0);
         tc_commit(bar_dp);
         NEA_TRACE_STAMP(p, 36 + min(k, 7), true);
-        if (k + 1 < n_items) {
+        if (!kOver && k + 1 < n_items) {
           // S(k+1) overwrites S(k): the rows must hold it in registers
           if (!wait_thread(bar_sread, k & 1, wc, kErrWaitSoftmax) ||
               !wait_thread(&bar_tma[(k + 1) % NS], ((k + 1) / NS) & 1, wc, kErrWaitProducer)) {
@@ -294,7 +307,7 @@ __device__ __forceinline__ void attn_bwd_unit(const BwdParams& p, int bid) {
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kTileRows / 16; ++kk)
-            mma_ts(tbase + kColAcc1, tbase + kColP + kk * 8, smem_desc(sC2 + kk * 16 * RB, RB, kTileRows * RB),
+            mma_ts(tbase + kColAcc1, tbase + p_col(kk), smem_desc(sC2 + kk * 16 * RB, RB, kTileRows * RB),
                    idAcc, (k | kk) != 0);
           NEA_TRACE_STAMP(p, 52 + min(k, 7), true);
         }
@@ -303,11 +316,21 @@ __device__ __forceinline__ void attn_bwd_unit(const BwdParams& p, int bid) {
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kTileRows / 16; ++kk)
-          mma_ts(tbase + accG, tbase + kColDS + kk * 8, smem_desc(sC1 + kk * 16 * RB, RB, kTileRows * RB), idAcc,
+          mma_ts(tbase + accG, tbase + ds_col(kk), smem_desc(sC1 + kk * 16 * RB, RB, kTileRows * RB), idAcc,
                  (k | kk) != 0);
         tc_commit(&bar_empty[k % NS]);
         tc_commit(bar_dk);
         NEA_TRACE_STAMP(p, 60 + min(k, 7), true);
+        if (kOver && k + 1 < n_items) {
+          // S(k+1) and dP(k+1) overwrite P(k) and dS(k): after dV(k) and dK/dQ(k)
+          if (!wait_thread(bar_dk, k & 1, wc, kErrWaitMma) ||
+              !wait_thread(&bar_tma[(k + 1) % NS], ((k + 1) / NS) & 1, wc, kErrWaitProducer)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_s(k + 1);
+        }
       }
       tc_commit(bar_fin);
       drain_wait(bar_fin, 0, wc);
@@ -378,7 +401,7 @@ __device__ __forceinline__ void attn_bwd_unit(const BwdParams& p, int bid) {
         uint32_t ph[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) ph[i] = pack_bf16(pv[2 * i], pv[2 * i + 1]);
-        tmem_st32(lane_base + kColP + 32 * hf, ph);
+        tmem_st32(lane_base + (kOver ? kColS + 64 * hf : kColP + 32 * hf), ph);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(bar_p);
@@ -411,7 +434,7 @@ __device__ __forceinline__ void attn_bwd_unit(const BwdParams& p, int bid) {
           pk[2 * i] = pack_bf16(a0, a1);
           pk[2 * i + 1] = pack_bf16(a2, a3);
         }
-        tmem_st16(lane_base + kColDS + 32 * hf + 16 * c, pk);
+        tmem_st16(lane_base + (kOver ? kColDP + 64 * hf : kColDS + 32 * hf) + 16 * c, pk);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -425,7 +448,9 @@ __device__ __forceinline__ void attn_bwd_unit(const BwdParams& p, int bid) {
       if (DKDV) {
         // half 0 writes the row of dV, half 1 the row of dK
         float acc[D];
-        tmem_ld_n<D>(lane_base + (hf ? kColAcc2 : kColAcc1), acc);
+        constexpr int NL = D < 64 ? D : 64;  // columns per TMEM load
+#pragma unroll
+        for (int c = 0; c < D / NL; ++c) tmem_ld_n<NL>(lane_base + (hf ? kColAcc2 : kColAcc1) + NL * c, acc + NL * c);
         if (hf) {
 #pragma unroll
           for (int i = 0; i < D; ++i) acc[i] *= p.scale;

@@ -74,9 +74,9 @@ enum {
  *               scaled, masked scores of each query row
  *   B, T        batch and sequence length, >= 0 (B*T == 0 is a no-op)
  *   Hq, Hkv     query and key/value heads, Hq % Hkv == 0
- *   D           head dimension, 32 or 64; nea_attn_fwd also takes 128 with NEA_BF16
- *               (a forward-only variant: the backward, the save-for-backward pair
- *               and float32 storage return NEA_ERR_ARG for D = 128)
+ *   D           head dimension, 32 or 64; also 128 with NEA_BF16 (forward, backward
+ *               and the save-for-backward pair; float32 storage and
+ *               nea_attn_bwd_noalloc return NEA_ERR_ARG for D = 128)
  *   dtype       NEA_F32 or NEA_BF16
  *   rope_base   rotary base (10000 for the workloads here); <= 0 disables
  *               the rotation

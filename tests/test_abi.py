@@ -62,14 +62,17 @@ def test_bad_arguments_are_rejected_without_launch(lib, kw):
     assert _bwd(lib, **kw) == 1
 
 
-def test_d128_is_a_bf16_forward_only_variant(lib):
-    """D = 128 passes the forward's checks with bfloat16 storage only; the
-    backward, the save-for-backward pair and float32 storage reject it."""
+def test_d128_is_a_bf16_variant(lib):
+    """D = 128 passes the checks with bfloat16 storage only."""
     assert _fwd(lib, D=128, dtype=1, B=0, ptr=None) == 0  # accepted: the empty problem is a no-op
+    assert _bwd(lib, D=128, dtype=1, B=0, ptr=None) == 0
     assert _fwd(lib, D=128, dtype=1, ptr=None) == 1       # and its pointers are checked
+    assert _bwd(lib, D=128, dtype=1, ptr=None) == 1
     assert _fwd(lib, D=128, dtype=0) == 1
-    assert _bwd(lib, D=128, dtype=1) == 1
-    assert _saved_bytes(lib, D=128, dtype=1) == -1
+    assert _bwd(lib, D=128, dtype=0) == 1
+    nq, nk = 2 * 100 * 6 * 128, 2 * 100 * 2 * 128  # bf16 with the rotation: rotated Q and K
+    assert _saved_bytes(lib, D=128, dtype=1) == (2 * nq + 255) // 256 * 256 + (2 * nk + 255) // 256 * 256
+    assert _saved_bytes(lib, D=128, dtype=0) == -1
 
 
 def test_nonfinite_rope_base_rejected(lib):
