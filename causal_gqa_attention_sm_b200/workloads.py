@@ -84,6 +84,8 @@ WORKLOADS = {
     "sweep1024": Workload("sweep1024", 16, 1024, 12, 4, 64, "bf16", seed=5001),
     "sweep2048": Workload("sweep2048", 8, 2048, 12, 4, 64, "bf16", seed=5002),
     "sweep4096": Workload("sweep4096", 4, 4096, 12, 4, 64, "bf16", seed=5003),
+    # head dimension 128 (bf16 storage): 8 query heads over 2 kv heads, context 4096
+    "d128": Workload("d128", 4, 4096, 8, 2, 128, "bf16", seed=5004),
     # generation over a key/value cache: 16 sequences, one new token each
     "decode1024": Workload("decode1024", 16, 1024, 12, 4, 64, "f32", seed=6000, decode=True),
     "decode4096": Workload("decode4096", 16, 4096, 12, 4, 64, "bf16", seed=6001, decode=True),

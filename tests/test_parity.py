@@ -200,7 +200,7 @@ def oracle_slices(w, inp, pairs):
             for i in range(len(pairs))]
 
 
-@pytest.mark.parametrize("name", ["layer", "long", "sweep512", "sweep1024", "sweep2048", "sweep4096"])
+@pytest.mark.parametrize("name", ["layer", "long", "sweep512", "sweep1024", "sweep2048", "sweep4096", "d128"])
 def test_full_size_sampled(cuda_lib, name):
     w = WORKLOADS[name]
     inp = make_inputs(w)
