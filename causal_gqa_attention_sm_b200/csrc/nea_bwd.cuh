@@ -39,8 +39,10 @@
 // D = 128: the two accumulators take TMEM [256,512), so P goes over S and dS
 // over dP, each warp half writing its 64 columns' bf16 pairs into the first
 // 32 of its own 64 columns (no half overwrites scores the other still
-// reads); S(k+1) and dP(k+1) then wait for the commit after dK/dQ(k), and the
-// rings hold two stages (32 KB tiles).
+// reads); S(k+1) is issued right after dV(k) (dK/dV units) and dP(k+1) right
+// after dK/dQ(k): the tensor core runs one thread's MMAs in issue order, so
+// each reads P or dS before the next product overwrites it.  The rings hold
+// two stages (32 KB tiles).
 #pragma once
 
 #include <cuda.h>
@@ -291,7 +293,7 @@ __device__ __forceinline__ void attn_bwd_unit(const BwdParams& p, int bid) {
                  smem_desc(sC2 + TileGeom<D>::kslice(kk), RB, 16), idSS, kk != 0);
         tc_commit(bar_dp);
         NEA_TRACE_STAMP(p, 36 + min(k, 7), true);
-        if (!kOver && k + 1 < n_items) {
+        if ((!kOver || !DKDV) && k + 1 < n_items) {
           // S(k+1) overwrites S(k): the rows must hold it in registers
           if (!wait_thread(bar_sread, k & 1, wc, kErrWaitSoftmax) ||
               !wait_thread(&bar_tma[(k + 1) % NS], ((k + 1) / NS) & 1, wc, kErrWaitProducer)) {
@@ -310,6 +312,16 @@ __device__ __forceinline__ void attn_bwd_unit(const BwdParams& p, int bid) {
             mma_ts(tbase + kColAcc1, tbase + p_col(kk), smem_desc(sC2 + kk * 16 * RB, RB, kTileRows * RB),
                    idAcc, (k | kk) != 0);
           NEA_TRACE_STAMP(p, 52 + min(k, 7), true);
+          if (kOver && k + 1 < n_items) {
+            // S(k+1) overwrites P(k): issued after dV(k), which reads it first
+            // (the tensor core runs this thread's MMAs in issue order)
+            if (!wait_thread(&bar_tma[(k + 1) % NS], ((k + 1) / NS) & 1, wc, kErrWaitProducer)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_s(k + 1);
+          }
         }
         // acc += dS(k) C1(k), then release the stage of item k
         if (!wait_thread(bar_ds, k & 1, wc, kErrWaitSoftmax)) { ok = false; break; }
@@ -321,16 +333,8 @@ __device__ __forceinline__ void attn_bwd_unit(const BwdParams& p, int bid) {
         tc_commit(&bar_empty[k % NS]);
         tc_commit(bar_dk);
         NEA_TRACE_STAMP(p, 60 + min(k, 7), true);
-        if (kOver && k + 1 < n_items) {
-          // S(k+1) and dP(k+1) overwrite P(k) and dS(k): after dV(k) and dK/dQ(k)
-          if (!wait_thread(bar_dk, k & 1, wc, kErrWaitMma) ||
-              !wait_thread(&bar_tma[(k + 1) % NS], ((k + 1) / NS) & 1, wc, kErrWaitProducer)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          issue_s(k + 1);
-        }
+        // (D = 128: dP(k+1), next, overwrites dS(k) after dK/dQ(k) has read it,
+        // in issue order)
       }
       tc_commit(bar_fin);
       drain_wait(bar_fin, 0, wc);
@@ -395,7 +399,9 @@ __device__ __forceinline__ void attn_bwd_unit(const BwdParams& p, int bid) {
         pv[4 * i + 3] = ex2(t3);
       }
       // P(k-1) and dS(k-1) stay in TMEM until dV/dK/dQ(k-1) have read them
-      if (k > 0 && !wait_warp(bar_dk, (k - 1) & 1, wc, kErrWaitMma)) { ok = false; break; }
+      // (D = 128: they lie under S(k) and dP(k), whose commits cover those
+      // products)
+      if (!kOver && k > 0 && !wait_warp(bar_dk, (k - 1) & 1, wc, kErrWaitMma)) { ok = false; break; }
       if (DKDV) {  // bf16 P for the dV product
         tc_fence_after();
         uint32_t ph[32];
