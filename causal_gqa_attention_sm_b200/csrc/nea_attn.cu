@@ -292,6 +292,15 @@ int dispatch(int D, int dtype, F&& f) {
              : f(std::integral_constant<int, 32>{}, std::false_type{});
 }
 
+// The decode kernels' dispatch: D = 32, 64 or 128, either storage type.
+template <typename F>
+int dispatch_dec(int D, int dtype, F&& f) {
+  if (D == 128)
+    return dtype == NEA_F32 ? f(std::integral_constant<int, 128>{}, std::true_type{})
+                            : f(std::integral_constant<int, 128>{}, std::false_type{});
+  return dispatch(D, dtype, f);
+}
+
 // ----------------------------------------------------------------- operand prologue
 // Workspace bytes the prologue writes for `n` tensors of `elems[i]` elements:
 // float32 storage, hi and lo planes of every tensor; bfloat16 storage, a
@@ -707,7 +716,7 @@ int nea_attn_bwd_saved(const void* Q, const void* K, const void* V, const void* 
 int nea_attn_decode(const void* Q, const void* Kc, const void* Vc, const int* lens, void* O, float* LSE, int B,
                     int Tc, int Hq, int Hkv, int D, int dtype, float rope_base, void* stream_) {
   if (B < 0 || Tc < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return NEA_ERR_ARG;
-  if (D != 32 && D != 64) return NEA_ERR_ARG;
+  if (D != 32 && D != 64 && D != 128) return NEA_ERR_ARG;
   if (dtype != NEA_F32 && dtype != NEA_BF16) return NEA_ERR_ARG;
   if (Hq / Hkv > nea::kDecMaxG || Hkv > 65535 || B > 65535) return NEA_ERR_ARG;
   if (!std::isfinite(rope_base)) return NEA_ERR_ARG;
@@ -756,14 +765,14 @@ int nea_attn_decode(const void* Q, const void* Kc, const void* Vc, const int* le
   if ((rc = make_cache_map(&p.tm_k, Kc, B, Tc, Hkv, D, dtype == NEA_F32, HP, R)) ||
       (rc = make_cache_map(&p.tm_v, Vc, B, Tc, Hkv, D, dtype == NEA_F32, HP, R)))
     return rc;
-  rc = dispatch(D, dtype, [&](auto d, auto f) {
+  rc = dispatch_dec(D, dtype, [&](auto d, auto f) {
     constexpr int DD = decltype(d)::value;
     constexpr bool FF = decltype(f)::value;
     auto launch = [&](auto gtag) -> int {
       constexpr int GG = decltype(gtag)::value;
       using L = nea::DecLayout<DD, FF, GG>;
       auto kern = nea::attn_decode_kernel<DD, FF, GG>;
-      const int bit = ((DD == 64) * 2 + FF) * 8 + (GG - 1);
+      const int bit = ((DD == 128 ? 2 : DD == 64 ? 1 : 0) * 2 + FF) * 8 + (GG - 1);
       if (!(st->attr_dec >> bit & 1)) {
         // both kernels ask for the largest shared-memory carveout, so that
         // the SMs keep one configuration from the stream to the merge

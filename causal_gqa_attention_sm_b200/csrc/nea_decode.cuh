@@ -386,19 +386,25 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
         for (int j = 0; j < D / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
         // ldmatrix line addresses (line = kv head R + row, so the 8 rows of
         // a matrix take 8 different swizzle phases): K (non-transposed) per
-        // 8-row block nt and column half h; V (transposed) per pair of
-        // 8-column blocks
+        // 8-row block nt and 32-column block h; V (transposed) per pair of
+        // 8-column blocks.  Columns past a line of one array (D = 128: 64
+        // per array) sit in the next array, kArray on.
         const int line0 = hh * p.R + 16 * rb;
+        constexpr int HPA = L::EPA / 32;  // 32-column blocks per array
         uint32_t koff[2][D / 32], voff[D / 16];
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
           for (int h = 0; h < D / 32; ++h)
-            koff[nt][h] = swizzle(uint32_t(line0 + 8 * nt + (lane & 7)) * L::RB + (4 * h + (lane >> 3)) * 16, L::RB);
+            koff[nt][h] = (h / HPA) * L::kArray +
+                          swizzle(uint32_t(line0 + 8 * nt + (lane & 7)) * L::RB + (4 * (h % HPA) + (lane >> 3)) * 16,
+                                  L::RB);
 #pragma unroll
         for (int jj = 0; jj < D / 16; ++jj)
-          voff[jj] = swizzle(uint32_t(line0 + 8 * ((lane >> 3) & 1) + (lane & 7)) * L::RB +
-                                 (2 * jj + (lane >> 4)) * 16, L::RB);
+          voff[jj] = (jj / (2 * HPA)) * L::kArray +
+                     swizzle(uint32_t(line0 + 8 * ((lane >> 3) & 1) + (lane & 7)) * L::RB +
+                                 (2 * (jj % (2 * HPA)) + (lane >> 4)) * 16,
+                             L::RB);
         for (int k = k0; k < kv; ++k, ++it) {
           const int s = it % L::ST;
           ok = ok && wait_warp(&full[s], (it / L::ST) & 1, wc, kErrWaitProducer);
@@ -416,7 +422,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attn_decode_kernel(const __gri
                   qa[ks][h2] = pack_bf16(x0, x1);
                 }
             }
-            const uint32_t kb = smem_u32(st), vb = smem_u32(st + L::kArray);
+            const uint32_t kb = smem_u32(st), vb = smem_u32(st + L::NA * L::kArray);
             float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)

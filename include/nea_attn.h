@@ -333,7 +333,7 @@ int nea_attn_bwd_noalloc(const void* Q, const void* K, const void* V, const void
  *   O      output [B][Hq][D], same dtype as Q
  *   LSE    output float32 [B][Hq], natural-log log-sum-exp of the scores
  *   Tc     cache capacity (positions), 1 <= Tc <= 2^24
- *   Hq / Hkv <= 8; D 32 or 64; dtype NEA_F32 or NEA_BF16 (all arithmetic in
+ *   Hq / Hkv <= 8; D 32, 64 or 128; dtype NEA_F32 or NEA_BF16 (all arithmetic in
  *   fp32); rope_base <= 0 disables the rotation of the query.
  *
  *   q' = R_{lens[b]-1} q, s_j = q' . k_j / sqrt(D) for j < lens[b],

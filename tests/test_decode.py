@@ -98,6 +98,13 @@ CASES = [
     # many short sequences: one CTA's range crosses several (sequence, kv head) pairs
     (300, 70, 6, 2, 32, "bf16", [(7 * i) % 71 for i in range(300)]),
     (40, 5, 8, 2, 64, "f32", [i % 6 for i in range(40)]),
+    # head dimension 128 (two 64-column arrays per cached line for bf16, four for fp32)
+    (3, 300, 8, 2, 128, "bf16", [300, 129, 1]),
+    (3, 300, 8, 2, 128, "f32", [1, 257, 300]),
+    (2, 190, 8, 8, 128, "bf16", [190, 64]),
+    (2, 190, 16, 2, 128, "bf16", [33, 190]),
+    (2, 190, 16, 2, 128, "f32", [190, 2]),
+    (1, 9000, 4, 1, 128, "bf16", [8999]),
 ]
 
 
