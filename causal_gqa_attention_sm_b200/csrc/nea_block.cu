@@ -469,7 +469,7 @@ int nea_block_qkv_bwd(const void* x, const void* g, const void* Wq, const void* 
   if ((rc = setup(c, dtype, stream))) return rc;
   const int Nq = Hq * D, Nk = Hkv * D;
   const int e = c.f32 ? 4 : 2;
-  const int n_part = std::min((M + 7) / 8, c.n_sm * 2);
+  const int n_part = std::min((M + 7) / 8, c.n_sm * 4);
   const size_t need = part_reserve(c.n_sm) + rup(size_t(M) * 4) + rup(size_t(M) * C * e) + rup(size_t(M) * C * 4) +
                       rup(size_t(n_part) * C * 4) +
                       (c.f32 ? rup(size_t(C) * Nq * 4) + 2 * rup(size_t(C) * Nk * 4) + rup(size_t(M) * Nq * 4) +
@@ -614,7 +614,7 @@ int nea_block_ffn_bwd(const void* x, const void* g, const void* Wg, const void* 
   Ctx c;
   if ((rc = setup(c, dtype, stream))) return rc;
   const int e = c.f32 ? 4 : 2;
-  const int n_part = std::min((M + 7) / 8, c.n_sm * 2);
+  const int n_part = std::min((M + 7) / 8, c.n_sm * 4);
   const size_t need = part_reserve(c.n_sm) + rup(size_t(M) * 4) + rup(size_t(M) * C * e) + rup(size_t(M) * C * 4) +
                       rup(size_t(n_part) * C * 4) + 3 * rup(size_t(M) * F * e) +
                       (c.f32 ? 3 * rup(size_t(C) * F * 4) + rup(size_t(M) * C * 4) : 0) + 4096;
